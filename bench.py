@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV decode hot path on B200.
+
+One step = slot mapping (new token's position -> cache slot) -> cache write of
+the new K/V -> paged decode attention (one pass, or partition kernel + LSE
+reduce, as the library chooses), over one batch of the GQA 70B-style layer
+workload: 128 sequences, 64 query / 8 KV heads, head_dim 128, block_size 16,
+lengths lognormal (median 1024, sigma 0.8) clipped to [16, 4096], shuffled
+block pool 1.2x.  Inputs are seeded synthetic data already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  `value` = KV GB/s: the decode's algorithmic
+bytes per step (KV blocks touched + queries + block tables + outputs) over the
+step time, summed over ranks / max over ranks.  The oracle (plain fp64 CPU
+code) is timed on a bounded sample as `cpu_baseline`; `--impl reference`
+times it as the reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged-decode KV GB/s (% of B200 HBM peak) and seqs/s, GQA 64q/8kv d128 b128"
+WORKLOAD = "gqa"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_gqa_ncu.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_379_b200", "csrc", f)
+                  for f in ("decode.cuh", "common.cuh", "pagedkv.cu")]
+
+
+def workload_description(w) -> str:
+    return (f"{w.num_seqs} seqs, {w.num_heads} query / {w.num_kv_heads} KV heads, head_dim {w.head_dim}, "
+            f"block_size {w.block_size}, lengths lognormal(median 1024, sigma 0.8) clipped [16, 4096], "
+            f"shuffled pool of {w.num_blocks} blocks (1.2x)")
+
+
+def algorithmic_bytes(seq_lens, block_size, num_heads, num_kv_heads, head_dim) -> int:
+    """KV blocks touched (K and V) + queries + outputs + block-table entries read + seq_lens."""
+    blocks = -(-np.asarray(seq_lens, dtype=np.int64) // block_size)
+    kv = int(blocks.sum()) * block_size * num_kv_heads * head_dim * 2 * 2
+    qo = 2 * len(seq_lens) * num_heads * head_dim * 2
+    tables = int(blocks.sum()) * 4 + 4 * len(seq_lens)
+    return kv + qo + tables
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_sha256_16\s*=\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_decode_call\s*=\s*([0-9]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
+# ------------------------------------------------------------------ clocks
+
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event reasons through NVML (the data
+    nvidia-smi reports) every 10 ms on a background thread."""
+
+    def __init__(self, cuda_index: int):
+        import torch
+        self.samples = []
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            handle = None
+            try:
+                props = torch.cuda.get_device_properties(cuda_index)
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                handle = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                handle = nv.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.nv, self.h = nv, handle
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _reasons(self):
+        nv = self.nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return int(getattr(nv, fn)(self.h))
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(), float(self.nv.nvmlDeviceGetClockInfo(
+                    self.h, self.nv.NVML_CLOCK_SM)), self._reasons()))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def window(self, t0: float, t1: float) -> dict:
+        s = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not s:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": "no NVML samples in the timed window" if self.ok else getattr(self, "err", "")}
+        bits = 0
+        for x in s:
+            bits |= x[2]
+        reasons = sorted(name for b, name in REASON_BITS.items() if bits & b and name != "gpu_idle")
+        return {"sm_mhz": statistics.median(x[1] for x in s), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(s)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+
+    from paged_kv_cache_379_b200 import ops
+    from paged_kv_cache_379_b200 import workload as wlmod
+    from paged_kv_cache_379_b200.step import DecodeBatch, bf16_to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    # independent batch per rank (weak scaling): same shape, own seed
+    seed = wlmod.SEED_BASE + wlmod.NAMES.index(WORKLOAD) + 1000 * rank
+    w = wlmod.make(WORKLOAD, seed=seed)
+    batch = DecodeBatch(w, dev)
+    stream = torch.cuda.current_stream(dev)
+    ws_bytes = 0 if batch.workspace is None else batch.workspace.numel()
+    plan = ops.decode_plan(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, batch.max_seq_len, ws_bytes)
+    launches_per_step = 2 + (2 if plan else 1) + (1 if batch.pairs is not None else 0)
+    step_bytes = algorithmic_bytes(w.seq_lens, w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
+
+    K, W = args.steps, args.warmup
+    ev_d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def decode_timed(i):
+        def fn(b):
+            ev_d0[i].record(stream)
+            ops.decode(b.query, b.key_cache, b.value_cache, b.block_tables, b.seq_lens, w.scale, b.max_seq_len,
+                       out=b.out, workspace=b.workspace, stream=stream)
+            ev_d1[i].record(stream)
+        return fn
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    for _ in range(W):
+        batch.run_step(stream=stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+
+    def timed_region():
+        barrier()
+        t0 = time.perf_counter()
+        e0.record(stream)
+        for i in range(K):
+            batch.run_step(stream=stream, decode_fn=decode_timed(i))
+        e1.record(stream)
+        barrier()
+        t1 = time.perf_counter()
+        return t0, t1
+
+    t0, t1 = timed_region()
+    clocks = sampler.window(t0, t1)
+    remeasured = False
+    if set(clocks["reasons"]) & BAD_REASONS:
+        first = clocks
+        t0, t1 = timed_region()
+        clocks = sampler.window(t0, t1)
+        clocks["first_attempt"] = first
+        remeasured = True
+    total_ms = e0.elapsed_time(e1)
+    dec_ms = [ev_d0[i].elapsed_time(ev_d1[i]) for i in range(K)]
+
+    # e2e: the same step through the C ABI with host buffers; the per-step inputs
+    # (query, new K/V, block tables, lengths) come from pinned host memory and the
+    # output goes back to pinned host memory inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        h_q = torch.from_numpy(w.query.view(np.int16)).pin_memory()
+        h_k = torch.from_numpy(w.new_key.view(np.int16)).pin_memory()
+        h_v = torch.from_numpy(w.new_value.view(np.int16)).pin_memory()
+        h_bt = torch.from_numpy(np.ascontiguousarray(w.block_tables, np.int32)).pin_memory()
+        h_sl = torch.from_numpy(w.seq_lens.astype(np.int32)).pin_memory()
+        h_out = torch.empty(batch.out.shape, dtype=torch.int16).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_bt, h_sl))
+        d2h = h_out.numel() * h_out.element_size()
+
+        def e2e_step():
+            batch.query.view(torch.int16).copy_(h_q, non_blocking=True)
+            batch.new_key.view(torch.int16).copy_(h_k, non_blocking=True)
+            batch.new_value.view(torch.int16).copy_(h_v, non_blocking=True)
+            batch.block_tables.copy_(h_bt, non_blocking=True)
+            batch.seq_lens.copy_(h_sl, non_blocking=True)
+            batch.run_step(stream=stream)
+            h_out.copy_(batch.out.view(torch.int16), non_blocking=True)
+
+        for _ in range(W):
+            e2e_step()
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        f1.record(stream)
+        barrier()
+        e2e_ms = f0.elapsed_time(f1)
+        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+    sampler.stop()
+
+    # aggregate over ranks: bytes summed, time = max over ranks
+    res = torch.tensor([total_ms, e2e["ms"] if e2e else 0.0], dtype=torch.float64, device=dev)
+    tot = torch.tensor([float(step_bytes), float(w.num_seqs)], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(res, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+    total_ms, e2e_max_ms = res.tolist()
+    all_bytes, all_seqs = tot.tolist()
+    if rank != 0:
+        return None
+
+    ms_per_step = total_ms / K
+    gbs = all_bytes * K / (total_ms * 1e-3) / 1e9
+    dec_avg_ms = float(np.mean(dec_ms))
+    achieved = step_bytes / (dec_avg_ms * 1e-3) / 1e9
+    peak, peak_src = measured_peak()
+    traffic = profiled_traffic()
+    line = {
+        "metric": METRIC,
+        "value": round(gbs, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 values, lognormal lengths, shuffled block pool)",
+        "config": {
+            "workload": f"{WORKLOAD}: {workload_description(w)}",
+            "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": w.block_size, "sum_seq_len": int(w.seq_lens.sum()),
+            "max_seq_len": w.max_seq_len, "algorithmic_bytes_per_step": step_bytes,
+            "decode_path": f"split, partition {plan} (partition kernel + LSE reduce)" if plan else "one pass",
+            "step": "slot_mapping -> reshape_and_cache -> decode",
+            "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB read per step vs 126 MB L2); no flush",
+            "parallelism": f"dp{world}: independent batch per GPU, no collective on the data path",
+        },
+        "seqs_per_s": round(all_seqs * K / (total_ms * 1e-3), 1),
+        "frac_of_spec_hbm": round(gbs / world / SPEC_HBM_GBS, 4),
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * K,
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "pa_decode (partition kernel + LSE reduce)" if plan else "pa_decode (one-pass kernel)",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
+            "traffic": traffic,
+            "algorithmic_bytes": step_bytes,
+            "avg_launch_ms": round(dec_avg_ms, 5),
+        },
+    }
+    if remeasured:
+        line["clocks_note"] = "first timed region saw a thermal/hw slowdown reason; re-measured once"
+    if e2e:
+        line["e2e"] = {"value": round(all_bytes * K / (e2e_max_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e_max_ms / K, 5)}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    return line
+
+
+# ---------------------------------------------------------------- the oracle
+
+def cpu_baseline(w, budget_s: float = 15.0) -> dict:
+    """The oracle (fp64 CPU, as it stands) on a bounded sample of the same workload."""
+    import oracle
+    threads = oracle.num_threads()
+    order = np.arange(w.num_seqs)
+    done_bytes, done_seqs, elapsed = 0, 0, 0.0
+    i = 0
+    chunk = 8
+    while elapsed < budget_s and i < w.num_seqs:
+        idx = order[i:i + chunk]
+        t = time.perf_counter()
+        oracle.paged_decode(w.query[idx], w.key_cache, w.value_cache, w.block_tables[idx], w.seq_lens[idx],
+                            w.scale, threads=threads)
+        elapsed += time.perf_counter() - t
+        done_bytes += algorithmic_bytes(w.seq_lens[idx], w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
+        done_seqs += len(idx)
+        i += chunk
+    return {"value": round(done_bytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done_seqs} of {w.num_seqs} sequences of the {WORKLOAD} batch (decode only), "
+                      f"{elapsed:.1f} s, fp64, OpenMP over (sequence, head)",
+            "seqs_per_s": round(done_seqs / elapsed, 2)}
+
+
+def run_reference(args, rank: int) -> dict | None:
+    """Reference arm: the oracle timed as it stands, each step a bounded sample."""
+    if rank != 0:
+        return None
+    import oracle
+    from paged_kv_cache_379_b200 import workload as wlmod
+
+    oracle.build()
+    w = wlmod.make(WORKLOAD)
+    threads = oracle.num_threads()
+    # sample size per step: one sequence, or more while a step stays short
+    per_step_budget = max(0.02, 120.0 / max(args.steps + args.warmup, 1))
+    t = time.perf_counter()
+    oracle.paged_decode(w.query[:1], w.key_cache, w.value_cache, w.block_tables[:1], w.seq_lens[:1], w.scale,
+                        threads=threads)
+    one = time.perf_counter() - t
+    mean_len = float(w.seq_lens.mean())
+    per_seq = one * mean_len / max(int(w.seq_lens[0]), 1)
+    S = int(max(1, min(w.num_seqs, per_step_budget // max(per_seq, 1e-9))))
+
+    def step(j):
+        idx = (np.arange(S) + j * S) % w.num_seqs
+        oracle.paged_decode(w.query[idx], w.key_cache, w.value_cache, w.block_tables[idx], w.seq_lens[idx],
+                            w.scale, threads=threads)
+        return algorithmic_bytes(w.seq_lens[idx], w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
+
+    for j in range(args.warmup):
+        step(j)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for j in range(args.steps):
+        nbytes += step(args.warmup + j)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    sample = f"{S} sequence(s) of the {WORKLOAD} batch per step, cycling; fp64 oracle decode"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": f"{WORKLOAD}: {workload_description(w)}"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from paged_kv_cache_379_b200.build import build as build_lib
+    if rank == 0 or world == 1:
+        build_lib()
+    if world > 1:
+        dist.barrier()
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,262 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: paged-KV decode attention for B200 (sm_100a).
+ *
+ * Pages cited (by title and section):
+ *   [源码解析]  "vLLM 源码解析：PagedAttention 如何让大模型推理提速 10 倍"
+ *   [深度解析]  "vLLM 核心源码深度解析：PagedAttention 的 KV Cache 管理、Scheduler
+ *               调度引擎与 Continuous Batching 实现全解"
+ *   [论文专题]  "论文专题讲解：vLLM / PagedAttention：为什么 KV cache 需要分页管理"
+ *
+ * Common conventions
+ * ------------------
+ * - Every pointer argument named *_cache, query, key, value, out, block_tables,
+ *   seq_lens, slot_mapping, src_dst_pairs, positions, seq_ids or workspace is
+ *   DEVICE memory owned by the caller.  The library allocates no device memory
+ *   and keeps no per-call state; all launches are asynchronous on `stream`
+ *   (a cudaStream_t passed as void*, NULL = the legacy default stream).
+ * - bf16 tensors are passed as void* and hold IEEE bfloat16 bit patterns.
+ * - KV cache layout ([源码解析 §四]): key_cache and value_cache are each
+ *   bf16 [num_blocks, block_size, num_kv_heads, head_dim], row-major; the page's
+ *   `num_heads` is read as the number of KV heads.
+ * - Block tables ([深度解析 «Block Table 数据结构»], [源码解析 §三]): int32
+ *   [num_seqs, max_blocks_per_seq], row s lists the physical block of each of
+ *   sequence s's logical blocks in order; entries past ceil(seq_len/block_size)
+ *   are never read.  A position pos lives in physical block
+ *   block_tables[s][pos / block_size] at offset pos % block_size.
+ * - Supported shapes: head_dim in {64, 128}; block_size in {4, 8, 16};
+ *   num_heads = G * num_kv_heads with G in 1..16.  Query head h reads KV head
+ *   h / G.
+ * - Return value: PA_OK (0) on success, a negative PA_ERR_* code otherwise.
+ *   Argument errors are detected on the host before any launch and nothing is
+ *   launched.  A launch failure returns PA_ERR_CUDA (pa_last_cuda_error() gives
+ *   the cudaError_t).  The library never aborts the process and never traps on
+ *   the device.
+ * - Preconditions NOT checked in the launch path (pa_validate_tables checks
+ *   them on the device): table entries below num_blocks for the blocks a
+ *   sequence uses; ceil(seq_len/block_size) <= max_blocks_per_seq;
+ *   0 <= seq_len <= max_seq_len; copy pairs with distinct destinations that are
+ *   not also sources.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_OK 0
+#define PA_ERR_NULL_POINTER (-1)   /* a required pointer is NULL                     */
+#define PA_ERR_BAD_SHAPE (-2)      /* a size is <= 0, inconsistent or too large      */
+#define PA_ERR_UNSUPPORTED (-3)    /* head_dim / block_size / group not compiled in  */
+#define PA_ERR_WORKSPACE (-4)      /* workspace missing or smaller than required     */
+#define PA_ERR_CUDA (-5)           /* a CUDA runtime or driver call failed           */
+#define PA_ERR_POOL_EXHAUSTED (-6) /* the host block pool has too few free blocks    */
+#define PA_ERR_BAD_BLOCK (-7)      /* a block id outside the pool / not allocated    */
+#define PA_ERR_ALIGNMENT (-8)      /* a device pointer is not 16-byte aligned         */
+#define PA_ERR_DEVICE_TIMEOUT (-9) /* a bounded on-device wait gave up (see below)   */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *pa_status_string(int status);
+
+/* cudaError_t of the last failing CUDA call in this thread (0 if none). */
+int pa_last_cuda_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int pa_version(void);
+
+/* --------------------------------------------------------------------------
+ * a1. Address translation / slot mapping ([深度解析 «Block Table 数据结构»]):
+ *     slot_mapping[t] = block_tables[seq][pos / block_size] * block_size
+ *                       + pos % block_size
+ * for token t of sequence seq at logical position pos.
+ *   seq_ids   int32 [num_tokens] or NULL (token t belongs to sequence t);
+ *   positions int64 [num_tokens] or NULL (decode: pos = seq_lens[seq] - 1);
+ *   seq_lens  int32 [num_seqs], read only when positions is NULL.
+ * block_tables has num_seqs rows.  A negative position, a seq_id outside
+ * [0, num_seqs), a position past the table row, a negative table entry, or
+ * seq_len == 0 in decode form yields slot -1.  Without seq_ids, num_tokens
+ * must not exceed num_seqs.
+ * Output slot_mapping: int64 [num_tokens].
+ * ------------------------------------------------------------------------ */
+int pa_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables, int num_seqs,
+                    int max_blocks_per_seq, const int32_t *seq_ids, const int64_t *positions,
+                    const int32_t *seq_lens, int num_tokens, int block_size, void *stream);
+
+/* --------------------------------------------------------------------------
+ * a2. Cache write ("reshape_and_cache"): the new tokens' K and V rows are
+ * stored at their slots ([论文专题 «Continuous batching 为什么离不开内存管理»]:
+ * generated K/V are written back into the owning block).
+ *   key, value: bf16 [num_tokens, num_kv_heads, head_dim], contiguous;
+ *   key_cache[slot / bs][slot % bs][h][:] = key[t][h][:] (same for value);
+ *   slot_mapping: int64 [num_tokens]; a negative slot skips the token.
+ * Slots must be < num_blocks * block_size and distinct among non-negative ones.
+ * ------------------------------------------------------------------------ */
+int pa_reshape_and_cache(const void *key, const void *value, void *key_cache, void *value_cache,
+                         const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, void *stream);
+
+/* --------------------------------------------------------------------------
+ * a3. Copy-on-write block copy ([源码解析 §五] allocate_or_get_cow: a new block
+ * receives a copy of the shared one; [深度解析 «Copy-on-Write 与 Prefix Caching»]).
+ *   src_dst_pairs: int64 [num_pairs, 2] (device), pair i copies the whole
+ *   physical block src -> dst in both caches (all heads, all slots).
+ * num_pairs == 0 is a no-op.  Destinations must be distinct and not sources;
+ * a pair naming a block outside [0, num_blocks) is skipped.
+ * ------------------------------------------------------------------------ */
+int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pairs, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int num_blocks, void *stream);
+
+/* --------------------------------------------------------------------------
+ * a4-a6. Single-query paged decode attention ([源码解析 §四] paged_attention;
+ * [论文专题 «PagedAttention：逻辑连续，物理不必连续»]): for sequence s and query
+ * head h, with L = seq_lens[s] and K_s, V_s read block by block through the
+ * table,
+ *     out[s][h] = sum_{p<L} softmax_p(scale * query[s][h] . K_s[p]) V_s[p].
+ * query, out: bf16 [num_seqs, num_heads, head_dim]; accumulation in fp32,
+ * output rounded to bf16 (round to nearest even).  L == 0 gives zeros.
+ * max_seq_len: a host-known upper bound of seq_lens (sizes the grid; no
+ * device-to-host read).
+ *
+ * pa_decode picks the one-pass kernel or the split form by max_seq_len and the
+ * number of (sequence, KV head) units; it needs a workspace of at least
+ * pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len, 0)
+ * bytes (16-byte aligned, caller-owned, contents need no initialisation) or
+ * may be given none (workspace NULL), in which case it runs one pass.
+ * ------------------------------------------------------------------------ */
+int pa_decode(void *out, const void *query, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
+              int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+              int num_blocks, int max_seq_len, void *workspace, size_t workspace_bytes,
+              void *stream);
+
+/* The plan pa_decode follows for these sizes: 0 = the one-pass kernel (one
+ * launch), otherwise the partition size of the split form (partition kernel +
+ * reduce kernel, two launches).  No device work. */
+int pa_decode_plan(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_seq_len,
+                   size_t workspace_bytes);
+
+/* Workspace bytes pa_decode / pa_decode_split need.  partition_size <= 0 means
+ * the partition size pa_decode would choose. */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len,
+                                int partition_size);
+
+/* a4 alone: one CTA per (sequence, KV head) walks all of the sequence's blocks
+ * with an online softmax ("逐块计算局部 Attention，最后合并结果", [源码解析 §四]).
+ * No workspace. */
+int pa_decode_one_pass(void *out, const void *query, const void *key_cache,
+                       const void *value_cache, const int32_t *block_tables,
+                       const int32_t *seq_lens, float scale, int block_size, int num_kv_heads,
+                       int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                       int num_blocks, int max_seq_len, void *stream);
+
+/* a5 + a6: positions are cut into partitions of partition_size tokens (a
+ * multiple of 16, >= 16); one CTA per (sequence, KV head, partition) computes
+ * the partition's local result, and a log-sum-exp reduce kernel merges them.
+ * A sequence that fits in one partition is written directly by its CTA. */
+int pa_decode_split(void *out, const void *query, const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, const int32_t *seq_lens, float scale,
+                    int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                    int max_blocks_per_seq, int num_blocks, int max_seq_len, int partition_size,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* a5 alone, for inspection: every partition p < ceil(max_seq_len/partition_size)
+ * of every (s, h) writes its local result into the workspace, laid out as
+ *   float o[num_seqs][num_heads][max_parts][head_dim]  at byte 0,
+ *   float m[num_seqs][num_heads][max_parts]           after o,
+ *   float l[num_seqs][num_heads][max_parts]           after m,
+ * with max_parts = ceil(max_seq_len / partition_size) (at least 1):
+ *   m = max_p scale*q.k_p (natural-log units), l = sum_p exp(x_p - m),
+ *   o = sum_p exp(x_p - m) v_p (not normalised).
+ * Partitions holding no position of their sequence get m = -inf, l = 0, o = 0. */
+int pa_decode_partitions(const void *query, const void *key_cache, const void *value_cache,
+                         const int32_t *block_tables, const int32_t *seq_lens, float scale,
+                         int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                         int head_dim, int max_blocks_per_seq, int num_blocks, int max_seq_len,
+                         int partition_size, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* a6 alone: merge the partitions that pa_decode_partitions wrote
+ * (out = sum_p e^{m_p-M} o_p / sum_p e^{m_p-M} l_p, M = max_p m_p) into bf16 out. */
+int pa_lse_reduce(void *out, const void *workspace, const int32_t *seq_lens, int num_seqs,
+                  int num_heads, int head_dim, int max_seq_len, int partition_size,
+                  void *stream);
+
+/* --------------------------------------------------------------------------
+ * Precondition check on the device: counts, into *bad_count (device int32,
+ * overwritten), the sequences whose seq_len is negative or above max_seq_len,
+ * whose ceil(seq_len/block_size) exceeds max_blocks_per_seq, or whose used
+ * table entries fall outside [0, num_blocks).
+ * ------------------------------------------------------------------------ */
+int pa_validate_tables(const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                       int max_blocks_per_seq, int block_size, int num_blocks, int max_seq_len,
+                       int32_t *bad_count, void *stream);
+
+/* Bounded waits.  Every wait inside the kernels (on TMA completion or on a
+ * pipeline stage being released) gives up after about one second, records a
+ * nonzero code in a device word and lets the kernel return.  This call reads
+ * and clears that word for the current device (synchronising the device);
+ * 0 means no wait ever gave up, otherwise PA_ERR_DEVICE_TIMEOUT. */
+int pa_device_status(void);
+
+/* --------------------------------------------------------------------------
+ * a7. Host block pool (host memory only; it generates block tables, slots and
+ * copy pairs, it never touches the GPU):
+ *   - a free list popped from its end in O(1) ([深度解析 «内存分配与回收流程»,
+ *     «核心方法 allocate»]; [源码解析 §三] allocate / free / get_num_free_blocks);
+ *   - per-block reference counts; fork() adds an owner to every block of a
+ *     table (parallel sampling / beam search share prompt blocks,
+ *     [论文专题 «共享前缀和 copy-on-write»]);
+ *   - copy-on-write: a write into a block with reference count > 1 takes a
+ *     fresh block, records (src, dst) and decrements src ([源码解析 §五]);
+ *   - on-demand growth: a new block only when the last one is full
+ *     ([源码解析 §六]; [论文专题 «Block table：为什么它能减少碎片»], Figure 6).
+ * Not thread-safe: one pool per host thread, or external locking.
+ * ------------------------------------------------------------------------ */
+typedef struct pa_pool pa_pool;
+
+/* free_order: int32 [num_blocks] permutation giving the initial free list
+ * (the LAST entry is handed out first), or NULL for 0..num_blocks-1.
+ * Returns NULL on bad arguments or out of host memory. */
+pa_pool *pa_pool_create(int num_blocks, int block_size, const int32_t *free_order);
+void pa_pool_destroy(pa_pool *pool);
+int pa_pool_num_free(const pa_pool *pool);
+int pa_pool_num_blocks(const pa_pool *pool);
+/* Reference count of a block (0 = free), or PA_ERR_BAD_BLOCK. */
+int pa_pool_refcount(const pa_pool *pool, int block);
+/* Take n blocks (refcount 1 each) into out_ids[n]; PA_ERR_POOL_EXHAUSTED and
+ * no change if fewer than n are free. */
+int pa_pool_allocate(pa_pool *pool, int n, int32_t *out_ids);
+/* Drop one owner; the block returns to the free list at refcount 0. */
+int pa_pool_free(pa_pool *pool, int block);
+/* Add one owner to each of ids[0..n). */
+int pa_pool_fork(pa_pool *pool, const int32_t *ids, int n);
+/* Copy-on-write decision for a write into `block`: *out_block is the block to
+ * write; *copied is 1 if a fresh block was taken (then copy block -> *out_block). */
+int pa_pool_cow(pa_pool *pool, int block, int32_t *out_block, int32_t *copied);
+/* Adopt existing tables (host int32 [num_seqs, max_blocks], first
+ * num_table_blocks[s] entries of row s valid): every reference adds an owner and
+ * referenced blocks leave the free list (the others keep their order). */
+int pa_pool_import(pa_pool *pool, const int32_t *block_tables, int num_seqs, int max_blocks,
+                   const int32_t *num_table_blocks);
+/* One decode step's host work for a batch (all arrays host memory):
+ * sequence s has context_lens[s] cached tokens and appends one at position
+ * context_lens[s].  If that position opens a new logical block, a fresh block is
+ * appended to row s (num_table_blocks[s] += 1); otherwise the copy-on-write
+ * decision is taken for the block being written.  Outputs slot_mapping[s] and
+ * the (src, dst) pairs (int64 [num_seqs, 2], *num_pairs of them).  Returns
+ * PA_ERR_POOL_EXHAUSTED if the pool runs dry (sequences before the failing
+ * one keep their updates) or PA_ERR_BAD_SHAPE if a row would overflow. */
+int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, int max_blocks,
+                           int32_t *num_table_blocks, const int32_t *context_lens,
+                           int64_t *slot_mapping, int64_t *src_dst_pairs, int *num_pairs);
+/* Release every block of the first n entries of a table row. */
+int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

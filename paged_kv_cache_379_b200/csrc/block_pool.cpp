@@ -1,0 +1,212 @@
+// block_pool.cpp -- host-side KV block pool behind the pa_pool_* C ABI.
+//
+// The pool owns no device memory: it hands out physical block ids, keeps their
+// reference counts and decides copy-on-write, so that a serving loop (or the
+// benchmark) can build the block tables, slot mappings and copy pairs that the
+// kernels consume.
+//
+// Pages followed:
+//   "vLLM 源码解析：PagedAttention 如何让大模型推理提速 10 倍", §三 (BlockAllocator:
+//     allocate / free / get_num_free_blocks), §五 (allocate_or_get_cow), §六 (only
+//     the next page is reserved, when the last one is full);
+//   "vLLM 核心源码深度解析 …", «内存分配与回收流程» (free_list with O(1) pop and
+//     push), «核心方法 allocate» (free_list.pop()), «Copy-on-Write 与 Prefix Caching»
+//     (shared prompt blocks carry a reference count; a write copies the block,
+//     writes the new value and decrements the count);
+//   "论文专题讲解：vLLM / PagedAttention …", «共享前缀和 copy-on-write» and
+//     «Block table：为什么它能减少碎片» (Figure 6).
+//
+// The free list is a vector used as a stack: the last entry is handed out first,
+// freed blocks are pushed on the end.  Both are O(1).
+
+#include <cstdint>
+#include <new>
+#include <vector>
+
+#include "../../include/pagedkv.h"
+
+struct pa_pool {
+    int num_blocks;
+    int block_size;
+    std::vector<int32_t> free_stack;   // top = back()
+    std::vector<int32_t> refcount;
+};
+
+extern "C" {
+
+pa_pool *pa_pool_create(int num_blocks, int block_size, const int32_t *free_order)
+{
+    if (num_blocks <= 0 || block_size <= 0) return nullptr;
+    pa_pool *p = new (std::nothrow) pa_pool;
+    if (!p) return nullptr;
+    try {
+        p->num_blocks = num_blocks;
+        p->block_size = block_size;
+        p->refcount.assign(num_blocks, 0);
+        p->free_stack.resize(num_blocks);
+        if (free_order) {
+            std::vector<char> seen(num_blocks, 0);
+            for (int i = 0; i < num_blocks; ++i) {
+                int32_t b = free_order[i];
+                if (b < 0 || b >= num_blocks || seen[b]) { delete p; return nullptr; }
+                seen[b] = 1;
+                p->free_stack[i] = b;
+            }
+        } else {
+            for (int i = 0; i < num_blocks; ++i) p->free_stack[i] = i;
+        }
+    } catch (...) {
+        delete p;
+        return nullptr;
+    }
+    return p;
+}
+
+void pa_pool_destroy(pa_pool *pool) { delete pool; }
+
+int pa_pool_num_free(const pa_pool *pool)
+{
+    if (!pool) return PA_ERR_NULL_POINTER;
+    return (int)pool->free_stack.size();
+}
+
+int pa_pool_num_blocks(const pa_pool *pool)
+{
+    if (!pool) return PA_ERR_NULL_POINTER;
+    return pool->num_blocks;
+}
+
+int pa_pool_refcount(const pa_pool *pool, int block)
+{
+    if (!pool) return PA_ERR_NULL_POINTER;
+    if (block < 0 || block >= pool->num_blocks) return PA_ERR_BAD_BLOCK;
+    return pool->refcount[block];
+}
+
+int pa_pool_allocate(pa_pool *pool, int n, int32_t *out_ids)
+{
+    if (!pool || (n > 0 && !out_ids)) return PA_ERR_NULL_POINTER;
+    if (n < 0) return PA_ERR_BAD_SHAPE;
+    if ((size_t)n > pool->free_stack.size()) return PA_ERR_POOL_EXHAUSTED;
+    for (int i = 0; i < n; ++i) {
+        int32_t b = pool->free_stack.back();
+        pool->free_stack.pop_back();
+        pool->refcount[b] = 1;
+        out_ids[i] = b;
+    }
+    return PA_OK;
+}
+
+int pa_pool_free(pa_pool *pool, int block)
+{
+    if (!pool) return PA_ERR_NULL_POINTER;
+    if (block < 0 || block >= pool->num_blocks || pool->refcount[block] <= 0) return PA_ERR_BAD_BLOCK;
+    if (--pool->refcount[block] == 0) pool->free_stack.push_back(block);
+    return PA_OK;
+}
+
+int pa_pool_fork(pa_pool *pool, const int32_t *ids, int n)
+{
+    if (!pool || (n > 0 && !ids)) return PA_ERR_NULL_POINTER;
+    for (int i = 0; i < n; ++i)
+        if (ids[i] < 0 || ids[i] >= pool->num_blocks || pool->refcount[ids[i]] <= 0) return PA_ERR_BAD_BLOCK;
+    for (int i = 0; i < n; ++i) ++pool->refcount[ids[i]];
+    return PA_OK;
+}
+
+int pa_pool_cow(pa_pool *pool, int block, int32_t *out_block, int32_t *copied)
+{
+    if (!pool || !out_block || !copied) return PA_ERR_NULL_POINTER;
+    if (block < 0 || block >= pool->num_blocks || pool->refcount[block] <= 0) return PA_ERR_BAD_BLOCK;
+    if (pool->refcount[block] > 1) {
+        if (pool->free_stack.empty()) return PA_ERR_POOL_EXHAUSTED;
+        int32_t fresh = pool->free_stack.back();
+        pool->free_stack.pop_back();
+        pool->refcount[fresh] = 1;
+        --pool->refcount[block];
+        *out_block = fresh;
+        *copied = 1;
+    } else {
+        *out_block = block;
+        *copied = 0;
+    }
+    return PA_OK;
+}
+
+int pa_pool_import(pa_pool *pool, const int32_t *block_tables, int num_seqs, int max_blocks,
+                   const int32_t *num_table_blocks)
+{
+    if (!pool || (num_seqs > 0 && (!block_tables || !num_table_blocks))) return PA_ERR_NULL_POINTER;
+    if (num_seqs < 0 || max_blocks < 0) return PA_ERR_BAD_SHAPE;
+    for (int s = 0; s < num_seqs; ++s) {
+        if (num_table_blocks[s] < 0 || num_table_blocks[s] > max_blocks) return PA_ERR_BAD_SHAPE;
+        for (int j = 0; j < num_table_blocks[s]; ++j) {
+            int32_t b = block_tables[(int64_t)s * max_blocks + j];
+            if (b < 0 || b >= pool->num_blocks) return PA_ERR_BAD_BLOCK;
+        }
+    }
+    for (int s = 0; s < num_seqs; ++s)
+        for (int j = 0; j < num_table_blocks[s]; ++j) ++pool->refcount[block_tables[(int64_t)s * max_blocks + j]];
+    std::vector<int32_t> kept;
+    kept.reserve(pool->free_stack.size());
+    for (int32_t b : pool->free_stack)
+        if (pool->refcount[b] == 0) kept.push_back(b);
+    pool->free_stack.swap(kept);
+    return PA_OK;
+}
+
+int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, int max_blocks,
+                           int32_t *num_table_blocks, const int32_t *context_lens,
+                           int64_t *slot_mapping, int64_t *src_dst_pairs, int *num_pairs)
+{
+    if (!pool || !num_pairs) return PA_ERR_NULL_POINTER;
+    if (num_seqs > 0 && (!block_tables || !num_table_blocks || !context_lens || !slot_mapping || !src_dst_pairs))
+        return PA_ERR_NULL_POINTER;
+    if (num_seqs < 0 || max_blocks <= 0) return PA_ERR_BAD_SHAPE;
+    const int bs = pool->block_size;
+    *num_pairs = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t pos = context_lens[s];
+        if (pos < 0) return PA_ERR_BAD_SHAPE;
+        int64_t logical = pos / bs;
+        int64_t offset = pos % bs;
+        int32_t *row = block_tables + (int64_t)s * max_blocks;
+        int32_t have = num_table_blocks[s];
+        if (logical == have) {
+            // the last page is full (or there is none): reserve the next page
+            if (offset != 0) return PA_ERR_BAD_SHAPE;
+            if (have >= max_blocks) return PA_ERR_BAD_SHAPE;
+            int32_t fresh;
+            int rc = pa_pool_allocate(pool, 1, &fresh);
+            if (rc != PA_OK) return rc;
+            row[have] = fresh;
+            num_table_blocks[s] = have + 1;
+        } else if (logical < have) {
+            int32_t target, copied;
+            int rc = pa_pool_cow(pool, row[logical], &target, &copied);
+            if (rc != PA_OK) return rc;
+            if (copied) {
+                src_dst_pairs[2 * (*num_pairs)] = row[logical];
+                src_dst_pairs[2 * (*num_pairs) + 1] = target;
+                ++*num_pairs;
+                row[logical] = target;
+            }
+        } else {
+            return PA_ERR_BAD_SHAPE;
+        }
+        slot_mapping[s] = (int64_t)row[logical] * bs + offset;
+    }
+    return PA_OK;
+}
+
+int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n)
+{
+    if (!pool || (n > 0 && !table)) return PA_ERR_NULL_POINTER;
+    for (int i = 0; i < n; ++i) {
+        int rc = pa_pool_free(pool, table[i]);
+        if (rc != PA_OK) return rc;
+    }
+    return PA_OK;
+}
+
+}  // extern "C"

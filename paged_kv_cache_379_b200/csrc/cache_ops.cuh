@@ -1,0 +1,134 @@
+// cache_ops.cuh -- the integer / byte-moving kernels of the decode step:
+//   slot mapping   (address translation of a new token's position),
+//   reshape_and_cache (write the new K/V rows at their slots),
+//   copy_blocks    (copy-on-write block copies),
+//   validate_tables (device-side precondition check).
+// All of them are HBM- or launch-bound copies: 16-byte vector accesses, grid
+// sized from the work, no shared memory.  Included once, by pagedkv.cu.
+#pragma once
+
+#include "common.cuh"
+
+namespace pakv {
+
+// Address translation ("vLLM 核心源码深度解析 …", «Block Table 数据结构»):
+//   block_number = pos / block_size, offset = pos % block_size,
+//   slot = block_table[block_number] * block_size + offset.
+__global__ void slot_mapping_kernel(int64_t *__restrict__ slots, const int32_t *__restrict__ block_tables,
+                                    int num_seqs, int max_blocks, const int32_t *__restrict__ seq_ids,
+                                    const int64_t *__restrict__ positions,
+                                    const int32_t *__restrict__ seq_lens, int num_tokens, int block_size)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= num_tokens) return;
+    const int seq = seq_ids ? seq_ids[t] : t;
+    int64_t slot = -1;
+    if (seq < 0 || seq >= num_seqs) {  // out-of-range sequence id: treated as padding
+        slots[t] = slot;
+        return;
+    }
+    const int64_t pos = positions ? positions[t] : (int64_t)seq_lens[seq] - 1;
+    if (pos >= 0) {
+        const int64_t block_number = pos / block_size;
+        const int64_t offset = pos - block_number * block_size;
+        if (block_number < max_blocks) {
+            const int32_t physical = block_tables[(int64_t)seq * max_blocks + block_number];
+            if (physical >= 0) slot = (int64_t)physical * block_size + offset;
+        }
+    }
+    slots[t] = slot;
+}
+
+// One thread per 16-byte chunk of a token's [num_kv_heads, head_dim] row (the
+// row is contiguous both in `key` and at its slot in the cache, because the
+// cache is [num_blocks, block_size, num_kv_heads, head_dim]).
+__global__ void reshape_and_cache_kernel(const uint4 *__restrict__ key, const uint4 *__restrict__ value,
+                                         uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache,
+                                         const int64_t *__restrict__ slot_mapping, int num_tokens,
+                                         int chunks_per_token, int64_t num_slots)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)num_tokens * chunks_per_token) return;
+    const int64_t t = i / chunks_per_token;
+    const int64_t c = i - t * chunks_per_token;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0 || slot >= num_slots) return;
+    const int64_t dst = slot * chunks_per_token + c;
+    const uint4 k = key[i];
+    const uint4 v = value[i];
+    key_cache[dst] = k;
+    value_cache[dst] = v;
+}
+
+// One CTA per (pair, slice): copies `per_cta` 16-byte chunks of the source block
+// into the destination block, in both caches, with 4 loads in flight per thread.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ key_cache,
+                                                          uint4 *__restrict__ value_cache,
+                                                          const int64_t *__restrict__ pairs,
+                                                          int64_t chunks_per_block, int slices, int64_t num_blocks)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int pair = blockIdx.x / slices;
+    const int slice = blockIdx.x - pair * slices;
+    const int64_t src = pairs[2 * pair];
+    const int64_t dst = pairs[2 * pair + 1];
+    if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) return;  // ids outside the pool
+    const int64_t per_cta = (chunks_per_block + slices - 1) / slices;
+    const int64_t begin = slice * per_cta;
+    const int64_t end = min(chunks_per_block, begin + per_cta);
+    const uint4 *ks = key_cache + src * chunks_per_block;
+    const uint4 *vs = value_cache + src * chunks_per_block;
+    uint4 *kd = key_cache + dst * chunks_per_block;
+    uint4 *vd = value_cache + dst * chunks_per_block;
+    constexpr int U = 2;
+    int64_t c = begin + threadIdx.x;
+    for (; c + (U - 1) * blockDim.x < end; c += U * blockDim.x) {
+        uint4 k[U], v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            k[u] = ks[c + u * blockDim.x];
+            v[u] = vs[c + u * blockDim.x];
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            kd[c + u * blockDim.x] = k[u];
+            vd[c + u * blockDim.x] = v[u];
+        }
+    }
+    for (; c < end; c += blockDim.x) {
+        kd[c] = ks[c];
+        vd[c] = vs[c];
+    }
+}
+
+// Counts sequences that break a precondition of the decode kernels.
+__global__ void validate_tables_kernel(const int32_t *__restrict__ block_tables,
+                                       const int32_t *__restrict__ seq_lens, int num_seqs, int max_blocks,
+                                       int block_size, int num_blocks, int max_seq_len, int32_t *bad_count)
+{
+    pdl_wait();
+    const int s = blockIdx.x;
+    if (s >= num_seqs) return;
+    const int L = seq_lens[s];
+    __shared__ int bad;
+    if (threadIdx.x == 0) bad = (L < 0 || L > max_seq_len) ? 1 : 0;
+    __syncthreads();
+    const int64_t used = L > 0 ? ((int64_t)L + block_size - 1) / block_size : 0;
+    if (used > max_blocks) {
+        if (threadIdx.x == 0) bad = 1;
+    } else {
+        for (int64_t j = threadIdx.x; j < used; j += blockDim.x) {
+            const int32_t b = block_tables[(int64_t)s * max_blocks + j];
+            if (b < 0 || b >= num_blocks) bad = 1;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && bad) atomicAdd(bad_count, 1);
+}
+
+}  // namespace pakv

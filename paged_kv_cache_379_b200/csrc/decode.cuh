@@ -1,0 +1,597 @@
+// decode.cuh -- single-query paged decode attention for sm_100a.
+//
+// What is computed ("vLLM 源码解析：PagedAttention 如何让大模型推理提速 10 倍", §四;
+// "论文专题讲解：vLLM / PagedAttention …", «PagedAttention：逻辑连续，物理不必连续»):
+// for sequence s and query head h, with L = seq_lens[s],
+//     out[s][h] = sum_{p<L} softmax_p(scale * q[s][h] . k_p) v_p,
+// where k_p, v_p live in physical block block_tables[s][p / bs] at offset p % bs
+// of the cache [num_blocks, bs, num_kv_heads, head_dim].  The kernel walks the
+// sequence block by block and merges the per-block results with an online
+// softmax -- the "compute locally per block, merge at the end" pattern of §四.
+//
+// Work unit: one CTA per (sequence, KV head, partition).  All G = Hq/Hkv query
+// heads of the KV head are handled by the same CTA, so every K/V byte crosses
+// HBM once.  A partition is a run of `part_tokens` positions; the one-pass form
+// is a single partition covering the whole sequence.
+//
+// CTA = 4 consumer warps + 1 producer warp.
+//  * Producer: one coalesced warp load of up to 32 table entries, then for each
+//    16-token tile one elected lane issues TMA tile loads of the tile's K and V
+//    blocks (box = [bs tokens x 1 head x head_dim], 128B-swizzled) into an
+//    8-stage shared-memory ring guarded by mbarriers.  Nothing else touches HBM.
+//  * Consumers: tile i goes to warp i % 4 (each warp owns 2 stages).  Every warp
+//    keeps its own running max m, sum l and fp32 accumulator; the four states
+//    are merged through shared memory at the end.
+//    - G >= 3 (grouped heads: a dense [G x D] . [D x 16] contraction per tile):
+//      bf16 mma.sync m16n8k16, S = Q K^T with Q as the A operand (rows = heads),
+//      K tiles through ldmatrix, then O += P V with P taken straight from the S
+//      accumulators and V through ldmatrix.trans.
+//    - G <= 2 (MHA-like, a matrix-vector product): CUDA cores, 16-byte shared
+//      loads, warp-shuffle reductions for the dot products, max and sum.
+//  * Masking selects (-inf logits, zeroed V rows) instead of multiplying by 0,
+//    so stale or NaN data in unused slots of a partial block is never mixed in.
+//  * Every mbarrier wait is bounded in time (about 1 s); on expiry the kernel
+//    records a code in the device status word, drains its own TMA copies and
+//    returns.
+// Split form: a partition's (m, l, o) go to a workspace and lse_reduce_kernel
+// merges them; a sequence with a single partition is finished in place.
+#pragma once
+
+#include "common.cuh"
+
+namespace pakv {
+
+struct DecodeParams {
+    __nv_bfloat16 *out;               // [B, Hq, D]
+    const __nv_bfloat16 *query;       // [B, Hq, D]
+    const int32_t *block_tables;      // [B, max_blocks]
+    const int32_t *seq_lens;          // [B]
+    float *ws_o;                      // [B, Hq, max_parts, D]   (split form)
+    float *ws_m;                      // [B, Hq, max_parts]      natural-log units
+    float *ws_l;                      // [B, Hq, max_parts]
+    float scale_log2;                 // scale * log2(e)
+    int num_seqs, num_heads, num_kv_heads, group, max_blocks;
+    int part_tokens;                  // positions per partition (multiple of 16)
+    int max_parts;                    // partitions per sequence in the grid; 1 = one pass
+    int direct_single;                // a sequence with one partition writes `out`
+};
+
+struct ReduceParams {
+    __nv_bfloat16 *out;
+    const float *ws_o, *ws_m, *ws_l;
+    const int32_t *seq_lens;
+    int num_seqs, num_heads, head_dim, part_tokens, max_parts;
+    int skip_single;                  // sequences with one partition are already done
+};
+
+constexpr int kConsumerWarps = 4;
+constexpr int kStages = 8;
+constexpr int kTileTokens = 16;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr float kLn2 = 0.693147180559945309f;
+
+template <int D, int BS>
+struct TileGeom {
+    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(BS == 4 || BS == 8 || BS == 16, "block_size");
+    static constexpr int kRows128 = D / 64;                       // 128-byte rows per token
+    static constexpr int kBlkBytes = BS * D * 2;                  // one block of one head
+    static constexpr int kBlkSmem = kBlkBytes < 1024 ? 1024 : kBlkBytes;  // keep 1024-B phase
+    static constexpr int kBlocksPerTile = kTileTokens / BS;
+    static constexpr int kTileSmem = kBlocksPerTile * kBlkSmem;
+    static constexpr int kStageSmem = 2 * kTileSmem;              // K tile, then V tile
+    static constexpr int kPipeSmem = kStages * kStageSmem;
+    static constexpr int kSmemBytes = kPipeSmem + 1024 /* alignment slack */ + 2 * kStages * 8 + 16;
+
+    // Byte offset inside a K or V tile of the 16-byte chunk c (0..D/8-1) of
+    // token t (0..15), as the 128B-swizzled TMA box stores it: chunk index XOR
+    // (128-byte row index mod 8), every block slot starting 1024-B aligned.
+    __device__ static __forceinline__ uint32_t chunk_offset(int t, int c)
+    {
+        const uint32_t row = (uint32_t)((t % BS) * kRows128 + (c >> 3));
+        return (uint32_t)((t / BS) * kBlkSmem) + row * 128u + ((((uint32_t)c & 7u) ^ (row & 7u)) << 4);
+    }
+    __device__ static __forceinline__ uint32_t token_offset(int t)
+    {
+        return (uint32_t)((t / BS) * kBlkSmem + (t % BS) * kRows128 * 128);
+    }
+};
+
+// Merge scratch (reuses the drained pipeline ring): per consumer warp, the
+// running max (log2 units), sum and accumulator of up to 16 heads.
+template <int D>
+struct MergeScratch {
+    float o[kConsumerWarps][16][D];
+    float m[kConsumerWarps][16];
+    float l[kConsumerWarps][16];
+};
+
+template <int D, int BS, int MODE, int GC>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+    paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v)
+{
+    // MODE 0: CUDA cores, GC (1 or 2) query heads per KV head.
+    // MODE 1: tensor cores, up to 8 query heads per KV head.
+    // MODE 2: tensor cores, up to 16 query heads per KV head.
+    using Geo = TileGeom<D, BS>;
+    static_assert(sizeof(MergeScratch<D>) <= Geo::kPipeSmem, "merge scratch must fit the ring");
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *const base_ptr = smem_raw + (base - raw);
+    const uint32_t full_bar = base + Geo::kPipeSmem;
+    const uint32_t empty_bar = full_bar + kStages * 8;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Geo::kPipeSmem + 2 * kStages * 8);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    int bid = blockIdx.x;
+    const int g = bid % p.num_kv_heads;
+    bid /= p.num_kv_heads;
+    const int s = bid % p.num_seqs;
+    const int part = bid / p.num_seqs;
+
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(full_bar + 8 * i, 1);
+            mbar_init(empty_bar + 8 * i, 1);
+        }
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (threadIdx.x == kConsumerWarps * 32) {
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
+
+    const int L = min(p.seq_lens[s], p.max_blocks * BS);
+    int nparts = 1;
+    int t_begin = 0, t_end = L;
+    if (p.max_parts > 1) {
+        nparts = L > 0 ? min((L + p.part_tokens - 1) / p.part_tokens, p.max_parts) : 1;
+        t_begin = part * p.part_tokens;
+        t_end = min(L, t_begin + p.part_tokens);
+    }
+    const int G = (MODE == 0) ? GC : p.group;
+    if (part >= nparts) {  // uniform over the CTA
+        if (!p.direct_single) {
+            // partitions-only form: an empty partition reports m = -inf, l = 0, o = 0
+            for (int idx = threadIdx.x; idx < G * D; idx += kDecodeThreads) {
+                const int row = idx / D;
+                const int64_t wi = ((int64_t)s * p.num_heads + (int64_t)g * G + row) * p.max_parts + part;
+                p.ws_o[wi * D + (idx - row * D)] = 0.f;
+                if (idx - row * D == 0) {
+                    p.ws_m[wi] = -INFINITY;
+                    p.ws_l[wi] = 0.f;
+                }
+            }
+        }
+        return;
+    }
+    const int n_tiles = t_end > t_begin ? (t_end - t_begin + kTileTokens - 1) / kTileTokens : 0;
+    const bool direct = p.direct_single && nparts == 1;
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        const int32_t *table = p.block_tables + (int64_t)s * p.max_blocks;
+        const int first_blk = t_begin / BS;
+        const int end_blk = (t_end + BS - 1) / BS;
+        int issued = 0;
+        bool stop = false;
+        for (int cb = first_blk; cb < end_blk && !stop; cb += 32) {
+            const int nchunk = min(32, end_blk - cb);
+            const int my = lane < nchunk ? __ldg(table + cb + lane) : 0;
+            for (int j = 0; j < nchunk; j += Geo::kBlocksPerTile) {
+                int phys[Geo::kBlocksPerTile];
+#pragma unroll
+                for (int k = 0; k < Geo::kBlocksPerTile; ++k) phys[k] = __shfl_sync(0xffffffffu, my, (j + k) & 31);
+                const int valid = min(Geo::kBlocksPerTile, nchunk - j);
+                if (lane == 0) {
+                    const int stage = issued % kStages;
+                    const uint32_t parity = ((issued / kStages) & 1) ^ 1;
+                    if (*abort_flag) {
+                        stop = true;
+                    } else if (!mbar_wait_bounded(empty_bar + 8 * stage, parity)) {
+                        record_timeout(kTimeoutEmptyBarrier);
+                        *abort_flag = 1;
+                        stop = true;
+                    } else {
+                        const uint32_t kdst = base + stage * Geo::kStageSmem;
+                        const uint32_t vdst = kdst + Geo::kTileSmem;
+                        const uint32_t bar = full_bar + 8 * stage;
+                        mbar_arrive_expect_tx(bar, (uint32_t)(valid * Geo::kBlkBytes * 2));
+#pragma unroll
+                        for (int k = 0; k < Geo::kBlocksPerTile; ++k) {
+                            if (k < valid) {
+                                tma_load_4d(kdst + k * Geo::kBlkSmem, &tmap_k, bar, 0, 0, g, phys[k] * BS);
+                                tma_load_4d(vdst + k * Geo::kBlkSmem, &tmap_v, bar, 0, 0, g, phys[k] * BS);
+                            }
+                        }
+                        ++issued;
+                    }
+                }
+                stop = __shfl_sync(0xffffffffu, stop, 0);
+                if (stop) break;
+            }
+        }
+        // On an abort, wait for the copies already in flight before the ring is
+        // reused or the CTA exits.
+        if (lane == 0 && *abort_flag && issued > 0) {
+            for (int st = 0; st < kStages && st < issued; ++st) {
+                const int last = issued - 1 - ((issued - 1 - st) % kStages);
+                if (!mbar_wait_bounded(full_bar + 8 * st, (last / kStages) & 1)) record_timeout(kTimeoutDrain);
+            }
+        }
+    } else {
+        // ----------------------------------------------------------- consumers
+        MergeScratch<D> *ms = reinterpret_cast<MergeScratch<D> *>(base_ptr);
+        const int64_t q_off = ((int64_t)s * p.num_heads + (int64_t)g * G) * D;
+
+        // Zero the V rows of tokens [valid, 16) so masked positions contribute
+        // exactly 0 (stale or NaN data is never multiplied).
+        auto zero_tail = [&](uint32_t vt, int valid) {
+            constexpr int kChunksPerTok = Geo::kRows128 * 8;
+            for (int i = lane; i < (kTileTokens - valid) * kChunksPerTok; i += 32) {
+                const int t = valid + i / kChunksPerTok;
+                const int c = i % kChunksPerTok;
+                *reinterpret_cast<uint4 *>(base_ptr + (vt - base) + Geo::token_offset(t) + c * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        };
+
+        if constexpr (MODE == 0) {
+            constexpr int CPT = D / 8;              // lanes per token in the dot products
+            constexpr int TPP = 32 / CPT;           // tokens per pass
+            constexpr int PASSES = kTileTokens / TPP;
+            constexpr int DPL = D / 32;             // accumulator columns per lane
+            const int qc = lane % CPT;
+            const int qt = lane / CPT;
+            float q[GC][8];
+#pragma unroll
+            for (int h = 0; h < GC; ++h) {
+                const uint4 raw_q = *reinterpret_cast<const uint4 *>(p.query + q_off + (int64_t)h * D + qc * 8);
+                const uint32_t w[4] = {raw_q.x, raw_q.y, raw_q.z, raw_q.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = unpack_bf16x2(w[e]);
+                    q[h][2 * e] = f.x * p.scale_log2;
+                    q[h][2 * e + 1] = f.y * p.scale_log2;
+                }
+            }
+            float o[GC][DPL];
+            float m[GC], l[GC];
+#pragma unroll
+            for (int h = 0; h < GC; ++h) {
+                m[h] = -INFINITY;
+                l[h] = 0.f;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
+            }
+            for (int tile = warp; tile < n_tiles; tile += kConsumerWarps) {
+                const int stage = tile % kStages;
+                if (*abort_flag) break;
+                const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar + 8 * stage, (tile / kStages) & 1));
+                if (!ok) {
+                    if (lane == 0) { record_timeout(kTimeoutFullBarrier); *abort_flag = 1; }
+                    break;
+                }
+                const uint32_t kt = base + stage * Geo::kStageSmem;
+                const uint32_t vt = kt + Geo::kTileSmem;
+                const int valid = min(kTileTokens, t_end - (t_begin + tile * kTileTokens));
+                if (valid < kTileTokens) zero_tail(vt, valid);
+
+                float sv[GC][PASSES];
+#pragma unroll
+                for (int j = 0; j < PASSES; ++j) {
+                    const int tok = j * TPP + qt;
+                    const uint4 kr = *reinterpret_cast<const uint4 *>(base_ptr + (kt - base) + Geo::chunk_offset(tok, qc));
+                    const uint32_t w[4] = {kr.x, kr.y, kr.z, kr.w};
+                    float kf[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = unpack_bf16x2(w[e]);
+                        kf[2 * e] = f.x;
+                        kf[2 * e + 1] = f.y;
+                    }
+#pragma unroll
+                    for (int h = 0; h < GC; ++h) {
+                        float dot = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dot = fmaf(q[h][e], kf[e], dot);
+#pragma unroll
+                        for (int off = CPT / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+                        sv[h][j] = tok < valid ? dot : -INFINITY;
+                    }
+                }
+                float pr[GC][PASSES];
+#pragma unroll
+                for (int h = 0; h < GC; ++h) {
+                    float mx = sv[h][0];
+#pragma unroll
+                    for (int j = 1; j < PASSES; ++j) mx = fmaxf(mx, sv[h][j]);
+#pragma unroll
+                    for (int off = CPT; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                    const float m_new = fmaxf(m[h], mx);
+                    const float corr = exp2f(m[h] - m_new);
+                    m[h] = m_new;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int j = 0; j < PASSES; ++j) {
+                        pr[h][j] = exp2f(sv[h][j] - m_new);
+                        sum += pr[h][j];
+                    }
+#pragma unroll
+                    for (int off = CPT; off < 32; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                    l[h] = l[h] * corr + sum;
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) o[h][e] *= corr;
+                }
+#pragma unroll
+                for (int tok = 0; tok < kTileTokens; ++tok) {
+                    const int c = (DPL * lane) >> 3;
+                    const uint32_t off = Geo::chunk_offset(tok, c) + ((DPL * lane) & 7) * 2;
+                    float vf[DPL];
+                    if constexpr (DPL == 4) {
+                        const uint2 vr = *reinterpret_cast<const uint2 *>(base_ptr + (vt - base) + off);
+                        const float2 a = unpack_bf16x2(vr.x), b = unpack_bf16x2(vr.y);
+                        vf[0] = a.x; vf[1] = a.y; vf[2] = b.x; vf[3] = b.y;
+                    } else {
+                        const uint32_t vr = *reinterpret_cast<const uint32_t *>(base_ptr + (vt - base) + off);
+                        const float2 a = unpack_bf16x2(vr);
+                        vf[0] = a.x; vf[1] = a.y;
+                    }
+#pragma unroll
+                    for (int h = 0; h < GC; ++h) {
+                        const float pt = __shfl_sync(0xffffffffu, pr[h][tok / TPP], (tok % TPP) * CPT);
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(pt, vf[e], o[h][e]);
+                    }
+                }
+                if (valid < kTileTokens) fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar + 8 * stage);
+            }
+            __syncthreads();  // ring drained (all consumers and the producer are past it)
+#pragma unroll
+            for (int h = 0; h < GC; ++h) {
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) ms->o[warp][h][DPL * lane + e] = o[h][e];
+                if (lane == 0) {
+                    ms->m[warp][h] = m[h];
+                    ms->l[warp][h] = l[h];
+                }
+            }
+        } else {
+            constexpr bool HI = (MODE == 2);
+            constexpr int KSTEPS = D / 16;
+            constexpr int NT = D / 8;
+            const int r = lane >> 2;
+            const int tq = lane & 3;
+            uint32_t qlo[KSTEPS][2], qhi[KSTEPS][2];
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int col = kk * 16 + hh * 8 + tq * 2;
+                    qlo[kk][hh] = r < G ? *reinterpret_cast<const uint32_t *>(p.query + q_off + (int64_t)r * D + col) : 0u;
+                    qhi[kk][hh] = (HI && r + 8 < G)
+                                      ? *reinterpret_cast<const uint32_t *>(p.query + q_off + (int64_t)(r + 8) * D + col)
+                                      : 0u;
+                }
+            }
+            float o[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+            float m_lo = -INFINITY, l_lo = 0.f, m_hi = -INFINITY, l_hi = 0.f;
+            // ldmatrix lane roles: K (B operand of S = Q K^T) and V (B operand of O += P V, transposed)
+            const int ktok = (lane & 7) + ((lane >> 4) << 3);
+            const int kpar = (lane >> 3) & 1;
+            const int vtok = (lane & 7) + (((lane >> 3) & 1) << 3);
+            const int vpar = lane >> 4;
+
+            for (int tile = warp; tile < n_tiles; tile += kConsumerWarps) {
+                const int stage = tile % kStages;
+                if (*abort_flag) break;
+                const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar + 8 * stage, (tile / kStages) & 1));
+                if (!ok) {
+                    if (lane == 0) { record_timeout(kTimeoutFullBarrier); *abort_flag = 1; }
+                    break;
+                }
+                const uint32_t kt = base + stage * Geo::kStageSmem;
+                const uint32_t vt = kt + Geo::kTileSmem;
+                const int valid = min(kTileTokens, t_end - (t_begin + tile * kTileTokens));
+                if (valid < kTileTokens) zero_tail(vt, valid);
+
+                // S[16 rows = heads][16 tokens] = Q K^T
+                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), b0, b1, b2, b3);
+                    mma_bf16_16816(sc[0], qlo[kk][0], qhi[kk][0], qlo[kk][1], qhi[kk][1], b0, b1);
+                    mma_bf16_16816(sc[1], qlo[kk][0], qhi[kk][0], qlo[kk][1], qhi[kk][1], b2, b3);
+                }
+                // scale to log2 units, mask positions past the end
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const bool in = nt * 8 + tq * 2 + j < valid;
+                        sc[nt][j] = in ? sc[nt][j] * p.scale_log2 : -INFINITY;
+                        if (HI) sc[nt][2 + j] = in ? sc[nt][2 + j] * p.scale_log2 : -INFINITY;
+                    }
+                }
+                // online softmax, rows r (and r + 8)
+                uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;
+                {
+                    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float m_new = fmaxf(m_lo, mx);
+                    const float corr = exp2f(m_lo - m_new);
+                    m_lo = m_new;
+                    pa0 = pack_bf16x2(exp2f(sc[0][0] - m_new), exp2f(sc[0][1] - m_new));
+                    pa2 = pack_bf16x2(exp2f(sc[1][0] - m_new), exp2f(sc[1][1] - m_new));
+                    const float2 f0 = unpack_bf16x2(pa0), f2 = unpack_bf16x2(pa2);
+                    l_lo = l_lo * corr + ((f0.x + f0.y) + (f2.x + f2.y));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        o[nt][0] *= corr;
+                        o[nt][1] *= corr;
+                    }
+                }
+                if (HI) {
+                    float mx = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float m_new = fmaxf(m_hi, mx);
+                    const float corr = exp2f(m_hi - m_new);
+                    m_hi = m_new;
+                    pa1 = pack_bf16x2(exp2f(sc[0][2] - m_new), exp2f(sc[0][3] - m_new));
+                    pa3 = pack_bf16x2(exp2f(sc[1][2] - m_new), exp2f(sc[1][3] - m_new));
+                    const float2 f1 = unpack_bf16x2(pa1), f3 = unpack_bf16x2(pa3);
+                    l_hi = l_hi * corr + ((f1.x + f1.y) + (f3.x + f3.y));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        o[nt][2] *= corr;
+                        o[nt][3] *= corr;
+                    }
+                }
+                // O[16 rows][D] += P[16 x 16 tokens] V[16 tokens x D]
+#pragma unroll
+                for (int nc = 0; nc < KSTEPS; ++nc) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * nc + vpar), b0, b1, b2, b3);
+                    mma_bf16_16816(o[2 * nc], pa0, pa1, pa2, pa3, b0, b1);
+                    mma_bf16_16816(o[2 * nc + 1], pa0, pa1, pa2, pa3, b2, b3);
+                }
+                if (valid < kTileTokens) fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar + 8 * stage);
+            }
+            l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+            l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+            if (HI) {
+                l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+                l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+            }
+            __syncthreads();  // ring drained
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int d = nt * 8 + tq * 2;
+                if (r < G) {
+                    ms->o[warp][r][d] = o[nt][0];
+                    ms->o[warp][r][d + 1] = o[nt][1];
+                }
+                if (HI && r + 8 < G) {
+                    ms->o[warp][r + 8][d] = o[nt][2];
+                    ms->o[warp][r + 8][d + 1] = o[nt][3];
+                }
+            }
+            if (tq == 0) {
+                ms->m[warp][r] = m_lo;
+                ms->l[warp][r] = l_lo;
+                if (HI) {
+                    ms->m[warp][r + 8] = m_hi;
+                    ms->l[warp][r + 8] = l_hi;
+                }
+            }
+        }
+    }
+    if (warp == kConsumerWarps) __syncthreads();  // pairs with the consumers' "ring drained"
+    __syncthreads();                              // merge scratch written
+
+    // ------------------------------------------------ merge the four warps
+    if (*abort_flag) return;
+    const MergeScratch<D> *ms = reinterpret_cast<const MergeScratch<D> *>(base_ptr);
+    for (int idx = threadIdx.x; idx < G * D; idx += kDecodeThreads) {
+        const int row = idx / D;
+        const int d = idx - row * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->m[w][row]);
+        float num = 0.f, den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = ms->m[w][row];
+                if (mw != -INFINITY) {
+                    const float c = exp2f(mw - M);
+                    num = fmaf(c, ms->o[w][row][d], num);
+                    den = fmaf(c, ms->l[w][row], den);
+                }
+            }
+        }
+        const int64_t hrow = (int64_t)s * p.num_heads + (int64_t)g * G + row;
+        if (direct) {
+            p.out[hrow * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+        } else {
+            const int64_t wi = hrow * p.max_parts + part;
+            p.ws_o[wi * D + d] = num;
+            if (d == 0) {
+                p.ws_m[wi] = M == -INFINITY ? -INFINITY : M * kLn2;
+                p.ws_l[wi] = den;
+            }
+        }
+    }
+}
+
+// Log-sum-exp merge of the partitions of one (sequence, head) per CTA:
+//   M = max_p m_p,  out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p.
+__global__ void __launch_bounds__(128) lse_reduce_kernel(const ReduceParams r)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int h = blockIdx.x % r.num_heads;
+    const int s = blockIdx.x / r.num_heads;
+    const int L = r.seq_lens[s];
+    int nparts = L > 0 ? (L + r.part_tokens - 1) / r.part_tokens : 1;
+    nparts = min(nparts, r.max_parts);
+    if (r.skip_single && nparts == 1) return;
+    const int64_t row = (int64_t)s * r.num_heads + h;
+    const float *m = r.ws_m + row * r.max_parts;
+    const float *l = r.ws_l + row * r.max_parts;
+    const float *o = r.ws_o + row * r.max_parts * r.head_dim;
+    __shared__ float red[4];
+    __shared__ float bcast[2];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    float mx = -INFINITY;
+    for (int i = threadIdx.x; i < nparts; i += blockDim.x) mx = fmaxf(mx, m[i]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) bcast[0] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    const float M = bcast[0];
+
+    float den = 0.f;
+    if (M != -INFINITY)
+        for (int i = threadIdx.x; i < nparts; i += blockDim.x)
+            if (m[i] != -INFINITY) den += expf(m[i] - M) * l[i];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    __syncthreads();
+    if (lane == 0) red[warp] = den;
+    __syncthreads();
+    if (threadIdx.x == 0) bcast[1] = (red[0] + red[1]) + (red[2] + red[3]);
+    __syncthreads();
+    den = bcast[1];
+
+    for (int d = threadIdx.x; d < r.head_dim; d += blockDim.x) {
+        float num = 0.f;
+        if (M != -INFINITY)
+            for (int i = 0; i < nparts; ++i)
+                if (m[i] != -INFINITY) num = fmaf(expf(m[i] - M), o[(int64_t)i * r.head_dim + d], num);
+        r.out[row * r.head_dim + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+    }
+}
+
+}  // namespace pakv

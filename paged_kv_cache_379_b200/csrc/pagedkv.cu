@@ -1,0 +1,430 @@
+// pagedkv.cu -- the C ABI of libpagedkv.so (declared in include/pagedkv.h):
+// argument checks, TMA tensor-map encoding, kernel selection and launch.
+// The kernels themselves are in cache_ops.cuh and decode.cuh.
+#include <atomic>
+#include <climits>
+#include <mutex>
+
+#include "cache_ops.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace pakv {
+
+static thread_local int t_last_cuda_error = 0;
+void set_last_cuda_error(cudaError_t e) { t_last_cuda_error = (int)e; }
+
+// ----------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// The cache [num_blocks, bs, Hkv, D] seen by TMA as 4-D (innermost first):
+//   {64 elements = 128 B, D/64, Hkv, num_blocks*bs slots}
+// with a box of one block of one head: {64, D/64, 1, bs}, 128-byte swizzle.
+static int make_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int bs, int hkv, int d)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return check_cuda(cudaErrorNotSupported);
+    const cuuint64_t dims[4] = {64, (cuuint64_t)(d / 64), (cuuint64_t)hkv, (cuuint64_t)(num_blocks * bs)};
+    const cuuint64_t strides[3] = {128, (cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)(d / 64), 1, (cuuint32_t)bs};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(cache), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_last_cuda_error(cudaErrorInvalidValue);
+        return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
+// --------------------------------------------------------------- decode launch
+
+// Sets the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+static int ensure_smem(K kernel, size_t bytes, std::atomic<uint64_t> &done)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return check_cuda(e);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return PA_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return check_cuda(e);
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return PA_OK;
+}
+
+template <int D, int BS, int MODE, int GC>
+static int launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int64_t grid,
+                           cudaStream_t st)
+{
+    static std::atomic<uint64_t> smem_done{0};
+    auto kernel = paged_decode_kernel<D, BS, MODE, GC>;
+    constexpr size_t smem = TileGeom<D, BS>::kSmemBytes;
+    int rc = ensure_smem(kernel, smem, smem_done);
+    if (rc != PA_OK) return rc;
+    return launch_pdl(kernel, dim3((unsigned)grid), dim3(kDecodeThreads), smem, st, p, tk, tv);
+}
+
+template <int D, int BS>
+static int launch_decode_bs(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int64_t grid,
+                            cudaStream_t st)
+{
+    const int G = p.group;
+    if (G == 1) return launch_decode_t<D, BS, 0, 1>(p, tk, tv, grid, st);
+    if (G == 2) return launch_decode_t<D, BS, 0, 2>(p, tk, tv, grid, st);
+    if (G <= 8) return launch_decode_t<D, BS, 1, 0>(p, tk, tv, grid, st);
+    if (G <= 16) return launch_decode_t<D, BS, 2, 0>(p, tk, tv, grid, st);
+    return PA_ERR_UNSUPPORTED;
+}
+
+template <int D>
+static int launch_decode_d(int bs, const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
+                           int64_t grid, cudaStream_t st)
+{
+    switch (bs) {
+    case 4: return launch_decode_bs<D, 4>(p, tk, tv, grid, st);
+    case 8: return launch_decode_bs<D, 8>(p, tk, tv, grid, st);
+    case 16: return launch_decode_bs<D, 16>(p, tk, tv, grid, st);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+struct DecodeArgs {
+    void *out;
+    const void *query, *key_cache, *value_cache;
+    const int32_t *block_tables, *seq_lens;
+    float scale;
+    int block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks, num_blocks, max_seq_len;
+};
+
+static int check_decode_args(const DecodeArgs &a, bool need_out)
+{
+    if ((need_out && !a.out) || !a.query || !a.key_cache || !a.value_cache || !a.block_tables || !a.seq_lens)
+        return PA_ERR_NULL_POINTER;
+    if (a.num_seqs < 0 || a.num_heads <= 0 || a.num_kv_heads <= 0 || a.head_dim <= 0 || a.block_size <= 0 ||
+        a.max_blocks <= 0 || a.num_blocks <= 0 || a.max_seq_len < 0)
+        return PA_ERR_BAD_SHAPE;
+    if (a.num_heads % a.num_kv_heads != 0) return PA_ERR_BAD_SHAPE;
+    if (a.head_dim != 64 && a.head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (a.block_size != 4 && a.block_size != 8 && a.block_size != 16) return PA_ERR_UNSUPPORTED;
+    if (a.num_heads / a.num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+    if ((int64_t)a.num_blocks * a.block_size > INT_MAX) return PA_ERR_BAD_SHAPE;
+    if ((int64_t)a.max_blocks * a.block_size > INT_MAX) return PA_ERR_BAD_SHAPE;
+    if (!aligned16(a.query) || !aligned16(a.key_cache) || !aligned16(a.value_cache) ||
+        (need_out && !aligned16(a.out)))
+        return PA_ERR_ALIGNMENT;
+    return PA_OK;
+}
+
+static constexpr int kDefaultPartition = 512;
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int max_parts_for(int max_seq_len, int part) { return max_seq_len > 0 ? (int)cdiv64(max_seq_len, part) : 1; }
+
+static size_t workspace_bytes_for(int num_seqs, int num_heads, int head_dim, int max_parts)
+{
+    const size_t rows = (size_t)num_seqs * num_heads * max_parts;
+    return align256(rows * head_dim * sizeof(float)) + 2 * align256(rows * sizeof(float));
+}
+
+// mode: 0 = one pass, 1 = split (direct singles + reduce), 2 = partitions only
+static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t ws_bytes, cudaStream_t st)
+{
+    int rc = check_decode_args(a, mode != 2);
+    if (rc != PA_OK) return rc;
+    if (a.num_seqs == 0) return PA_OK;
+    DecodeParams p = {};
+    p.out = static_cast<__nv_bfloat16 *>(a.out);
+    p.query = static_cast<const __nv_bfloat16 *>(a.query);
+    p.block_tables = a.block_tables;
+    p.seq_lens = a.seq_lens;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.num_seqs = a.num_seqs;
+    p.num_heads = a.num_heads;
+    p.num_kv_heads = a.num_kv_heads;
+    p.group = a.num_heads / a.num_kv_heads;
+    p.max_blocks = a.max_blocks;
+    if (mode == 0) {
+        p.part_tokens = 0;
+        p.max_parts = 1;
+        p.direct_single = 1;
+    } else {
+        if (part < kTileTokens || part % kTileTokens != 0) return PA_ERR_BAD_SHAPE;
+        p.part_tokens = part;
+        p.max_parts = max_parts_for(a.max_seq_len, part);
+        p.direct_single = mode == 1 ? 1 : 0;
+        const size_t need = workspace_bytes_for(a.num_seqs, a.num_heads, a.head_dim, p.max_parts);
+        if (!ws || ws_bytes < need || !aligned16(ws)) return PA_ERR_WORKSPACE;
+        const size_t rows = (size_t)a.num_seqs * a.num_heads * p.max_parts;
+        char *w = static_cast<char *>(ws);
+        p.ws_o = reinterpret_cast<float *>(w);
+        p.ws_m = reinterpret_cast<float *>(w + align256(rows * a.head_dim * sizeof(float)));
+        p.ws_l = reinterpret_cast<float *>(w + align256(rows * a.head_dim * sizeof(float)) +
+                                           align256(rows * sizeof(float)));
+    }
+    const int64_t grid = (int64_t)p.max_parts * a.num_seqs * a.num_kv_heads;
+    if (grid > INT_MAX) return PA_ERR_BAD_SHAPE;
+    CUtensorMap tk, tv;
+    rc = make_cache_map(&tk, a.key_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim);
+    if (rc != PA_OK) return rc;
+    rc = make_cache_map(&tv, a.value_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim);
+    if (rc != PA_OK) return rc;
+    rc = a.head_dim == 64 ? launch_decode_d<64>(a.block_size, p, tk, tv, grid, st)
+                          : launch_decode_d<128>(a.block_size, p, tk, tv, grid, st);
+    if (rc != PA_OK || mode != 1) return rc;
+    ReduceParams r = {};
+    r.out = p.out;
+    r.ws_o = p.ws_o;
+    r.ws_m = p.ws_m;
+    r.ws_l = p.ws_l;
+    r.seq_lens = a.seq_lens;
+    r.num_seqs = a.num_seqs;
+    r.num_heads = a.num_heads;
+    r.head_dim = a.head_dim;
+    r.part_tokens = part;
+    r.max_parts = p.max_parts;
+    r.skip_single = 1;
+    return launch_pdl(lse_reduce_kernel, dim3((unsigned)(a.num_seqs * a.num_heads)), dim3(128), 0, st, r);
+}
+
+// Partition size the dispatcher uses for a split run.
+static int choose_partition(int num_seqs, int num_kv_heads, int max_seq_len)
+{
+    (void)num_seqs;
+    (void)num_kv_heads;
+    (void)max_seq_len;
+    return kDefaultPartition;
+}
+
+// One pass when every (sequence, KV head) unit is short enough and there are
+// enough units to fill the GPU; otherwise split into partitions.
+static bool prefer_split(int num_seqs, int num_kv_heads, int max_seq_len)
+{
+    const int64_t units = (int64_t)num_seqs * num_kv_heads;
+    if (max_seq_len > 1024) return true;
+    if (units < 2 * 148 && max_seq_len > 256) return true;
+    return false;
+}
+
+}  // namespace pakv
+
+using namespace pakv;
+
+extern "C" {
+
+const char *pa_status_string(int status)
+{
+    switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_NULL_POINTER: return "null pointer";
+    case PA_ERR_BAD_SHAPE: return "bad shape";
+    case PA_ERR_UNSUPPORTED: return "unsupported head_dim / block_size / group";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_POOL_EXHAUSTED: return "block pool exhausted";
+    case PA_ERR_BAD_BLOCK: return "bad block id";
+    case PA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case PA_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
+    default: return "unknown status";
+    }
+}
+
+int pa_last_cuda_error(void) { return t_last_cuda_error; }
+
+int pa_version(void) { return 10000; }
+
+int pa_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables, int num_seqs, int max_blocks_per_seq,
+                    const int32_t *seq_ids, const int64_t *positions, const int32_t *seq_lens, int num_tokens,
+                    int block_size, void *stream)
+{
+    if (num_tokens < 0 || num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0) return PA_ERR_BAD_SHAPE;
+    if (!seq_ids && num_tokens > num_seqs) return PA_ERR_BAD_SHAPE;
+    if (num_tokens == 0) return PA_OK;
+    if (!slot_mapping || !block_tables || (!positions && !seq_lens)) return PA_ERR_NULL_POINTER;
+    const int threads = 256;
+    return launch_pdl(slot_mapping_kernel, dim3((unsigned)cdiv64(num_tokens, threads)), dim3(threads), 0,
+                      static_cast<cudaStream_t>(stream), slot_mapping, block_tables, num_seqs, max_blocks_per_seq, seq_ids,
+                      positions, seq_lens, num_tokens, block_size);
+}
+
+int pa_reshape_and_cache(const void *key, const void *value, void *key_cache, void *value_cache,
+                         const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                         int block_size, int num_blocks, void *stream)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PA_ERR_BAD_SHAPE;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL_POINTER;
+    if (((int64_t)num_kv_heads * head_dim) % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return PA_ERR_ALIGNMENT;
+    const int chunks = (int)((int64_t)num_kv_heads * head_dim / 8);
+    const int64_t total = (int64_t)num_tokens * chunks;
+    const int threads = 256;
+    if (cdiv64(total, threads) > INT_MAX) return PA_ERR_BAD_SHAPE;
+    return launch_pdl(reshape_and_cache_kernel, dim3((unsigned)cdiv64(total, threads)), dim3(threads), 0,
+                      static_cast<cudaStream_t>(stream), static_cast<const uint4 *>(key),
+                      static_cast<const uint4 *>(value), static_cast<uint4 *>(key_cache),
+                      static_cast<uint4 *>(value_cache), slot_mapping, num_tokens, chunks,
+                      (int64_t)num_blocks * block_size);
+}
+
+int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pairs, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int num_blocks, void *stream)
+{
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PA_ERR_BAD_SHAPE;
+    if (num_pairs == 0) return PA_OK;
+    if (!key_cache || !value_cache || !src_dst_pairs) return PA_ERR_NULL_POINTER;
+    const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+    if (block_elems % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_ALIGNMENT;
+    const int64_t chunks = block_elems / 8;
+    // 2048 chunks (32 KB) per CTA slice keeps ~16 KB of loads in flight per CTA.
+    const int slices = (int)std::max<int64_t>(1, std::min<int64_t>(64, cdiv64(chunks, 2048)));
+    if ((int64_t)num_pairs * slices > INT_MAX) return PA_ERR_BAD_SHAPE;
+    return launch_pdl(copy_blocks_kernel, dim3((unsigned)(num_pairs * slices)), dim3(256), 0,
+                      static_cast<cudaStream_t>(stream), static_cast<uint4 *>(key_cache),
+                      static_cast<uint4 *>(value_cache), src_dst_pairs, chunks, slices, (int64_t)num_blocks);
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len, int partition_size)
+{
+    if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return 0;
+    const int part = partition_size > 0 ? partition_size : kDefaultPartition;
+    return workspace_bytes_for(num_seqs, num_heads, head_dim, max_parts_for(max_seq_len, part));
+}
+
+int pa_decode_plan(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_seq_len,
+                   size_t workspace_bytes)
+{
+    if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return 0;
+    if (!prefer_split(num_seqs, num_kv_heads, max_seq_len)) return 0;
+    const int part = choose_partition(num_seqs, num_kv_heads, max_seq_len);
+    const size_t need = workspace_bytes_for(num_seqs, num_heads, head_dim, max_parts_for(max_seq_len, part));
+    return workspace_bytes >= need ? part : 0;
+}
+
+int pa_decode(void *out, const void *query, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size, int num_kv_heads,
+              int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq, int num_blocks, int max_seq_len,
+              void *workspace, size_t workspace_bytes, void *stream)
+{
+    const DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                          num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int part = workspace ? pa_decode_plan(num_seqs, num_heads, num_kv_heads, head_dim, max_seq_len,
+                                                workspace_bytes)
+                               : 0;
+    if (part > 0) return run_decode(a, 1, part, workspace, workspace_bytes, st);
+    return run_decode(a, 0, 0, nullptr, 0, st);
+}
+
+int pa_decode_one_pass(void *out, const void *query, const void *key_cache, const void *value_cache,
+                       const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
+                       int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                       int num_blocks, int max_seq_len, void *stream)
+{
+    const DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                          num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    return run_decode(a, 0, 0, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+int pa_decode_split(void *out, const void *query, const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
+                    int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                    int num_blocks, int max_seq_len, int partition_size, void *workspace, size_t workspace_bytes,
+                    void *stream)
+{
+    const DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                          num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    return run_decode(a, 1, partition_size, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pa_decode_partitions(const void *query, const void *key_cache, const void *value_cache,
+                         const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
+                         int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                         int num_blocks, int max_seq_len, int partition_size, void *workspace,
+                         size_t workspace_bytes, void *stream)
+{
+    const DecodeArgs a = {nullptr, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                          num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    return run_decode(a, 2, partition_size, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pa_lse_reduce(void *out, const void *workspace, const int32_t *seq_lens, int num_seqs, int num_heads,
+                  int head_dim, int max_seq_len, int partition_size, void *stream)
+{
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return PA_ERR_BAD_SHAPE;
+    if (partition_size < kTileTokens || partition_size % kTileTokens != 0) return PA_ERR_BAD_SHAPE;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !workspace || !seq_lens) return PA_ERR_NULL_POINTER;
+    const int max_parts = max_parts_for(max_seq_len, partition_size);
+    const size_t rows = (size_t)num_seqs * num_heads * max_parts;
+    const char *w = static_cast<const char *>(workspace);
+    ReduceParams r = {};
+    r.out = static_cast<__nv_bfloat16 *>(out);
+    r.ws_o = reinterpret_cast<const float *>(w);
+    r.ws_m = reinterpret_cast<const float *>(w + align256(rows * head_dim * sizeof(float)));
+    r.ws_l = reinterpret_cast<const float *>(w + align256(rows * head_dim * sizeof(float)) +
+                                             align256(rows * sizeof(float)));
+    r.seq_lens = seq_lens;
+    r.num_seqs = num_seqs;
+    r.num_heads = num_heads;
+    r.head_dim = head_dim;
+    r.part_tokens = partition_size;
+    r.max_parts = max_parts;
+    r.skip_single = 0;
+    return launch_pdl(lse_reduce_kernel, dim3((unsigned)(num_seqs * num_heads)), dim3(128), 0,
+                      static_cast<cudaStream_t>(stream), r);
+}
+
+int pa_validate_tables(const int32_t *block_tables, const int32_t *seq_lens, int num_seqs, int max_blocks_per_seq,
+                       int block_size, int num_blocks, int max_seq_len, int32_t *bad_count, void *stream)
+{
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || num_blocks <= 0) return PA_ERR_BAD_SHAPE;
+    if (!bad_count || (num_seqs > 0 && (!block_tables || !seq_lens))) return PA_ERR_NULL_POINTER;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = check_cuda(cudaMemsetAsync(bad_count, 0, sizeof(int32_t), st));
+    if (rc != PA_OK || num_seqs == 0) return rc;
+    return launch_pdl(validate_tables_kernel, dim3((unsigned)num_seqs), dim3(128), 0, st, block_tables, seq_lens,
+                      num_seqs, max_blocks_per_seq, block_size, num_blocks, max_seq_len, bad_count);
+}
+
+int pa_device_status(void)
+{
+    int rc = check_cuda(cudaDeviceSynchronize());
+    if (rc != PA_OK) return rc;
+    int v = 0;
+    rc = check_cuda(cudaMemcpyFromSymbol(&v, g_pa_device_status, sizeof(int)));
+    if (rc != PA_OK) return rc;
+    if (v != 0) {
+        const int zero = 0;
+        rc = check_cuda(cudaMemcpyToSymbol(g_pa_device_status, &zero, sizeof(int)));
+        if (rc != PA_OK) return rc;
+        return PA_ERR_DEVICE_TIMEOUT;
+    }
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,228 @@
+"""Python binding of the C ABI: the same names, argument marshalling only.
+
+Each function checks dtypes / devices / contiguity of the torch tensors it is
+given, passes their device pointers and the current CUDA stream to the
+library, and raises :class:`PagedKVError` on a negative status.  Every step of
+the computation runs in the library's CUDA kernels; nothing here computes.
+
+Tensor conventions (see include/pagedkv.h):
+  key_cache, value_cache : bf16 [num_blocks, block_size, num_kv_heads, head_dim]
+  query, out             : bf16 [num_seqs, num_heads, head_dim]
+  block_tables           : int32 [num_seqs, max_blocks_per_seq]
+  seq_lens               : int32 [num_seqs]
+  slot_mapping           : int64 [num_tokens]
+  src_dst_pairs          : int64 [num_pairs, 2]
+"""
+
+from __future__ import annotations
+
+import torch
+
+from ._lib import PagedKVError, check, load  # noqa: F401
+
+__all__ = [
+    "slot_mapping", "reshape_and_cache", "copy_blocks", "decode", "decode_one_pass",
+    "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
+    "validate_tables", "device_status", "PagedKVError",
+]
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor | None, dtype, name: str, ndim: int | None = None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _cache_dims(key_cache, value_cache):
+    _dev(key_cache, torch.bfloat16, "key_cache", 4)
+    _dev(value_cache, torch.bfloat16, "value_cache", 4)
+    if key_cache.shape != value_cache.shape:
+        raise ValueError("key_cache and value_cache shapes differ")
+    nb, bs, hkv, d = key_cache.shape
+    return nb, bs, hkv, d
+
+
+def slot_mapping(block_tables, block_size: int, *, seq_lens=None, positions=None, seq_ids=None,
+                 out=None, stream=None):
+    """Device address translation; decode form (positions=None) uses pos = seq_len - 1."""
+    lib = load()
+    bt = _dev(block_tables, torch.int32, "block_tables", 2)
+    n = positions.shape[0] if positions is not None else (
+        seq_ids.shape[0] if seq_ids is not None else seq_lens.shape[0])
+    if out is None:
+        out = torch.empty(n, dtype=torch.int64, device=block_tables.device)
+    check("pa_slot_mapping", lib.pa_slot_mapping(
+        _dev(out, torch.int64, "out", 1), bt, block_tables.shape[0], block_tables.shape[1],
+        _dev(seq_ids, torch.int32, "seq_ids", 1),
+        _dev(positions, torch.int64, "positions", 1), _dev(seq_lens, torch.int32, "seq_lens", 1),
+        n, int(block_size), _stream(stream)))
+    return out
+
+
+def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, stream=None) -> None:
+    lib = load()
+    nb, bs, hkv, d = _cache_dims(key_cache, value_cache)
+    k = _dev(key, torch.bfloat16, "key", 3)
+    v = _dev(value, torch.bfloat16, "value", 3)
+    if tuple(key.shape[1:]) != (hkv, d) or key.shape != value.shape:
+        raise ValueError("key/value must be [num_tokens, num_kv_heads, head_dim] matching the cache")
+    sm = _dev(slot_mapping, torch.int64, "slot_mapping", 1)
+    if slot_mapping.shape[0] != key.shape[0]:
+        raise ValueError("slot_mapping length != num_tokens")
+    check("pa_reshape_and_cache", lib.pa_reshape_and_cache(
+        k, v, key_cache.data_ptr(), value_cache.data_ptr(), sm, key.shape[0], hkv, d, bs, nb,
+        _stream(stream)))
+
+
+def copy_blocks(key_cache, value_cache, src_dst_pairs, stream=None) -> None:
+    lib = load()
+    nb, bs, hkv, d = _cache_dims(key_cache, value_cache)
+    pr = _dev(src_dst_pairs, torch.int64, "src_dst_pairs", 2)
+    if src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [num_pairs, 2]")
+    check("pa_copy_blocks", lib.pa_copy_blocks(
+        key_cache.data_ptr(), value_cache.data_ptr(), pr, src_dst_pairs.shape[0], hkv, d, bs, nb,
+        _stream(stream)))
+
+
+def _decode_common(query, key_cache, value_cache, block_tables, seq_lens):
+    nb, bs, hkv, d = _cache_dims(key_cache, value_cache)
+    q = _dev(query, torch.bfloat16, "query", 3)
+    B, hq, dq = query.shape
+    if dq != d:
+        raise ValueError("query head_dim != cache head_dim")
+    bt = _dev(block_tables, torch.int32, "block_tables", 2)
+    sl = _dev(seq_lens, torch.int32, "seq_lens", 1)
+    if block_tables.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_tables / seq_lens batch size != query batch size")
+    return q, bt, sl, B, hq, hkv, d, bs, nb, block_tables.shape[1]
+
+
+def decode_workspace_size(num_seqs: int, num_heads: int, head_dim: int, max_seq_len: int,
+                          partition_size: int = 0) -> int:
+    return int(load().pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len, partition_size))
+
+
+def decode_plan(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, max_seq_len: int,
+                workspace_bytes: int) -> int:
+    """0 if pa_decode runs one pass for these sizes, else the split partition size."""
+    return int(load().pa_decode_plan(num_seqs, num_heads, num_kv_heads, head_dim, max_seq_len,
+                                     int(workspace_bytes)))
+
+
+def _out(out, query):
+    if out is None:
+        out = torch.empty_like(query)
+    return _dev(out, torch.bfloat16, "out", 3), out
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def decode(query, key_cache, value_cache, block_tables, seq_lens, scale: float, max_seq_len: int,
+           *, out=None, workspace=None, stream=None):
+    """pa_decode: one pass or split, chosen by the library."""
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens)
+    o, out = _out(out, query)
+    wp, wb = _ws(workspace)
+    check("pa_decode", lib.pa_decode(o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale),
+                                     bs, hkv, B, hq, d, mb, nb, int(max_seq_len), wp, wb, _stream(stream)))
+    return out
+
+
+def decode_one_pass(query, key_cache, value_cache, block_tables, seq_lens, scale: float, max_seq_len: int,
+                    *, out=None, stream=None):
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens)
+    o, out = _out(out, query)
+    check("pa_decode_one_pass", lib.pa_decode_one_pass(
+        o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), bs, hkv, B, hq, d, mb, nb,
+        int(max_seq_len), _stream(stream)))
+    return out
+
+
+def decode_split(query, key_cache, value_cache, block_tables, seq_lens, scale: float, max_seq_len: int,
+                 partition_size: int, workspace, *, out=None, stream=None):
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens)
+    o, out = _out(out, query)
+    wp, wb = _ws(workspace)
+    check("pa_decode_split", lib.pa_decode_split(
+        o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), bs, hkv, B, hq, d, mb, nb,
+        int(max_seq_len), int(partition_size), wp, wb, _stream(stream)))
+    return out
+
+
+def decode_partitions(query, key_cache, value_cache, block_tables, seq_lens, scale: float, max_seq_len: int,
+                      partition_size: int, workspace, stream=None):
+    """pa_decode_partitions; returns views (o, m, l) into the workspace."""
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens)
+    wp, wb = _ws(workspace)
+    check("pa_decode_partitions", lib.pa_decode_partitions(
+        q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), bs, hkv, B, hq, d, mb, nb,
+        int(max_seq_len), int(partition_size), wp, wb, _stream(stream)))
+    return workspace_views(workspace, B, hq, d, max_seq_len, partition_size)
+
+
+def workspace_views(workspace, num_seqs, num_heads, head_dim, max_seq_len, partition_size):
+    """(o, m, l) float32 views of a split-form workspace (layout of include/pagedkv.h)."""
+    parts = max(1, -(-int(max_seq_len) // int(partition_size)))
+    rows = num_seqs * num_heads * parts
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    raw = workspace.view(torch.uint8)
+    ob = rows * head_dim * 4
+    o = raw[:ob].view(torch.float32).view(num_seqs, num_heads, parts, head_dim)
+    m = raw[a256(ob):a256(ob) + rows * 4].view(torch.float32).view(num_seqs, num_heads, parts)
+    lo = a256(ob) + a256(rows * 4)
+    l = raw[lo:lo + rows * 4].view(torch.float32).view(num_seqs, num_heads, parts)
+    return o, m, l
+
+
+def lse_reduce(out, workspace, seq_lens, max_seq_len: int, partition_size: int, stream=None):
+    lib = load()
+    o = _dev(out, torch.bfloat16, "out", 3)
+    B, hq, d = out.shape
+    wp, _ = _ws(workspace)
+    check("pa_lse_reduce", lib.pa_lse_reduce(o, wp, _dev(seq_lens, torch.int32, "seq_lens", 1), B, hq, d,
+                                             int(max_seq_len), int(partition_size), _stream(stream)))
+    return out
+
+
+def validate_tables(block_tables, seq_lens, block_size: int, num_blocks: int, max_seq_len: int,
+                    stream=None) -> int:
+    """Number of sequences breaking a decode precondition (synchronises)."""
+    lib = load()
+    bad = torch.zeros(1, dtype=torch.int32, device=block_tables.device)
+    check("pa_validate_tables", lib.pa_validate_tables(
+        _dev(block_tables, torch.int32, "block_tables", 2), _dev(seq_lens, torch.int32, "seq_lens", 1),
+        block_tables.shape[0], block_tables.shape[1], int(block_size), int(num_blocks), int(max_seq_len),
+        bad.data_ptr(), _stream(stream)))
+    return int(bad.item())
+
+
+def device_status() -> int:
+    """0, or the negative status PA_ERR_DEVICE_TIMEOUT if a bounded device wait gave up."""
+    return int(load().pa_device_status())

@@ -31,6 +31,8 @@ so that a read of a wrong block shows up.
 
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -51,14 +53,43 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return rounded
 
 
-def bf16_normal(rng: np.random.Generator, shape, chunk: int = 1 << 24) -> np.ndarray:
-    """N(0, 1) values rounded to bf16, generated in chunks to bound host memory."""
+def bf16_normal(rng: np.random.Generator, shape, chunk: int = 1 << 22) -> np.ndarray:
+    """N(0, 1) values rounded to bf16.
+
+    The values are drawn in fixed-size chunks, each from its own PCG64 stream
+    seeded from `rng`, on a thread pool; the result depends only on `rng`'s
+    state, not on the number of threads.
+    """
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
-    for start in range(0, n, chunk):
+    starts = list(range(0, n, chunk))
+    seeds = rng.integers(0, 2**63 - 1, size=max(len(starts), 1), dtype=np.int64)
+
+    def fill(i):
+        start = starts[i]
         stop = min(n, start + chunk)
-        out[start:stop] = f32_to_bf16_bits(rng.standard_normal(stop - start, dtype=np.float32))
+        g = np.random.Generator(np.random.PCG64(int(seeds[i])))
+        out[start:stop] = f32_to_bf16_bits(g.standard_normal(stop - start, dtype=np.float32))
+
+    if len(starts) <= 1:
+        for i in range(len(starts)):
+            fill(i)
+    else:
+        workers = min(len(starts), os.cpu_count() or 1, 32)
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(fill, range(len(starts))))
     return out.reshape(shape)
+
+
+def _fill_cache(rng, num_blocks, bs, hkv, d, free):
+    """Cache contents: random bf16 in owned blocks, bf16 NaN in unowned ones."""
+    cache = np.empty((num_blocks, bs, hkv, d), dtype=np.uint16)
+    is_free = np.zeros(num_blocks, dtype=bool)
+    is_free[np.asarray(free, dtype=np.int64)] = True
+    owned = np.flatnonzero(~is_free)
+    cache[is_free] = BF16_NAN
+    cache[owned] = bf16_normal(rng, (owned.size, bs, hkv, d))
+    return cache
 
 
 @dataclass
@@ -195,11 +226,8 @@ def make(name: str, seed: int | None = None, *, num_seqs: int | None = None,
     new_value = bf16_normal(rng, (B, Hkv, D))
     cache_shape = (num_blocks, bs, Hkv, D)
     if fill_cache:
-        key_cache = bf16_normal(rng, cache_shape)
-        value_cache = bf16_normal(rng, cache_shape)
-        if free.size:
-            key_cache[free] = BF16_NAN
-            value_cache[free] = BF16_NAN
+        key_cache = _fill_cache(rng, num_blocks, bs, Hkv, D, free)
+        value_cache = _fill_cache(rng, num_blocks, bs, Hkv, D, free)
     else:
         key_cache = np.zeros(cache_shape, dtype=np.uint16)
         value_cache = np.zeros(cache_shape, dtype=np.uint16)
@@ -233,11 +261,8 @@ def random_decode_case(seed: int, *, num_seqs: int, num_heads: int, num_kv_heads
     query = bf16_normal(rng, (num_seqs, Hq, D))
     new_key = bf16_normal(rng, (num_seqs, Hkv, D))
     new_value = bf16_normal(rng, (num_seqs, Hkv, D))
-    key_cache = bf16_normal(rng, (num_blocks, block_size, Hkv, D))
-    value_cache = bf16_normal(rng, (num_blocks, block_size, Hkv, D))
-    if free.size:
-        key_cache[free] = BF16_NAN
-        value_cache[free] = BF16_NAN
+    key_cache = _fill_cache(rng, num_blocks, block_size, Hkv, D, free)
+    value_cache = _fill_cache(rng, num_blocks, block_size, Hkv, D, free)
     return Workload(name="custom", seed=seed, num_seqs=num_seqs, num_heads=Hq, num_kv_heads=Hkv,
                     head_dim=D, block_size=block_size, num_blocks=num_blocks,
                     scale=float(1.0 / np.sqrt(D)), seq_lens=seq_lens, block_tables=tables,

@@ -1,0 +1,85 @@
+"""The C-ABI library loads and exports every symbol include/pagedkv.h declares;
+argument checks answer on the host without touching a GPU (CPU only)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_379_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("pa_reshape_and_cache", "pa_decode", "pa_copy_blocks", "pa_slot_mapping",
+                     "pa_decode_one_pass", "pa_decode_split", "pa_lse_reduce", "pa_pool_create"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(_lib.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(raw, n)]
+    assert not missing, missing
+    # and the binding knows every one of them
+    assert set(_declared()) <= set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert _lib.status_string(0) == "ok"
+    for code in range(-1, -10, -1):
+        assert _lib.status_string(code) != "unknown status"
+    assert lib.pa_version() >= 10000
+
+
+def test_argument_errors_without_gpu(lib):
+    P = ctypes.c_void_p
+    # null pointers
+    assert lib.pa_decode(None, None, None, None, None, None, 1.0, 16, 8, 4, 64, 128, 8, 100, 128,
+                         None, 0, None) == -1
+    fake = P(4096)
+    # num_heads not a multiple of num_kv_heads
+    assert lib.pa_decode(fake, fake, fake, fake, fake, fake, 1.0, 16, 8, 4, 63, 128, 8, 100, 128,
+                         None, 0, None) == -2
+    # unsupported head_dim / block_size / group
+    assert lib.pa_decode_one_pass(fake, fake, fake, fake, fake, fake, 1.0, 16, 8, 4, 64, 96, 8, 100,
+                                  128, None) == -3
+    assert lib.pa_decode_one_pass(fake, fake, fake, fake, fake, fake, 1.0, 32, 8, 4, 64, 128, 8, 100,
+                                  128, None) == -3
+    assert lib.pa_decode_one_pass(fake, fake, fake, fake, fake, fake, 1.0, 16, 2, 4, 64, 128, 8, 100,
+                                  128, None) == -3
+    # misaligned pointer
+    assert lib.pa_decode_one_pass(P(4100), fake, fake, fake, fake, fake, 1.0, 16, 8, 4, 64, 128, 8,
+                                  100, 128, None) == -8
+    # split without workspace, bad partition size
+    assert lib.pa_decode_split(fake, fake, fake, fake, fake, fake, 1.0, 16, 8, 4, 64, 128, 8, 100,
+                               128, 512, None, 0, None) == -4
+    assert lib.pa_decode_split(fake, fake, fake, fake, fake, fake, 1.0, 16, 8, 4, 64, 128, 8, 100,
+                               128, 100, fake, 1 << 30, None) == -2
+    # empty work is a no-op
+    assert lib.pa_slot_mapping(None, None, 4, 1, None, None, None, 0, 16, None) == 0
+    assert lib.pa_slot_mapping(fake, fake, 4, 1, None, None, fake, 5, 16, None) == -2
+    assert lib.pa_copy_blocks(fake, fake, None, 0, 8, 128, 16, 10, None) == 0
+    assert lib.pa_reshape_and_cache(None, None, None, None, None, 0, 8, 128, 16, 10, None) == 0
+    assert lib.pa_reshape_and_cache(fake, fake, fake, fake, fake, 3, 8, 128, 16, 0, None) == -2
+
+
+def test_workspace_size(lib):
+    # 4 seqs x 8 heads x ceil(1000/512)=2 parts: o = 64*128*4 B, m and l = 64*4 B each (256-aligned)
+    assert lib.pa_decode_workspace_size(4, 8, 128, 1000, 512) == 64 * 128 * 4 + 2 * 256
+    assert lib.pa_decode_workspace_size(4, 8, 128, 0, 512) == 32 * 128 * 4 + 2 * 256
+    assert lib.pa_decode_workspace_size(0, 8, 128, 10, 512) == 0

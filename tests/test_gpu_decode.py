@@ -1,0 +1,177 @@
+"""GPU parity of paged decode attention (one-pass, split + reduce, and the
+library's own choice) against the fp64 oracle, element by element."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _helpers import assert_close, oracle_step, poison_tail_slots
+from paged_kv_cache_379_b200 import ops
+from paged_kv_cache_379_b200 import workload as wl
+from paged_kv_cache_379_b200.step import DecodeBatch, bf16_to_device, bf16_to_host_bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _dev_inputs(w):
+    return dict(
+        query=bf16_to_device(w.query, DEV),
+        key_cache=bf16_to_device(w.key_cache, DEV),
+        value_cache=bf16_to_device(w.value_cache, DEV),
+        block_tables=torch.from_numpy(np.ascontiguousarray(w.block_tables, np.int32)).to(DEV),
+        seq_lens=torch.from_numpy(w.seq_lens.astype(np.int32)).to(DEV),
+    )
+
+
+def _run(w, kind, partition=512):
+    d = _dev_inputs(w)
+    args = (d["query"], d["key_cache"], d["value_cache"], d["block_tables"], d["seq_lens"], w.scale,
+            w.max_seq_len)
+    if kind == "one_pass":
+        out = ops.decode_one_pass(*args)
+    elif kind == "split":
+        nbytes = ops.decode_workspace_size(w.num_seqs, w.num_heads, w.head_dim, w.max_seq_len, partition)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+        out = ops.decode_split(*args, partition, ws)
+    else:
+        nbytes = ops.decode_workspace_size(w.num_seqs, w.num_heads, w.head_dim, w.max_seq_len)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+        out = ops.decode(*args, workspace=ws)
+    torch.cuda.synchronize()
+    return bf16_to_host_bits(out)
+
+
+# ---- the five workloads, whole step, in the benchmark's launch configuration --------
+
+@pytest.mark.parametrize("name", ["tiny", "mha", "gqa", "long", "shared"])
+def test_workload_step_matches_oracle(name):
+    w = wl.make(name)
+    tables, pairs = w.block_tables, None
+    if name == "shared":
+        from paged_kv_cache_379_b200.step import host_step
+        _, tables, _, _, pairs = host_step(w, fork_all=True)
+    poison_tail_slots(w, tables)
+    batch = DecodeBatch(w, DEV, tables=tables, pairs=pairs)
+    out = batch.run_step()
+    torch.cuda.synchronize()
+    ref_k, ref_v, ref_slots, ref_out = oracle_step(w, tables, pairs)
+    assert np.array_equal(batch.slots.cpu().numpy(), ref_slots)
+    assert np.array_equal(bf16_to_host_bits(batch.key_cache), ref_k)
+    assert np.array_equal(bf16_to_host_bits(batch.value_cache), ref_v)
+    assert_close(bf16_to_host_bits(out), ref_out, name)
+    assert ops.device_status() == 0
+
+
+# ---- kernel variants over shapes, groups, block sizes and ragged lengths ------------
+
+LENS = [1, 2, 15, 16, 17, 31, 33, 64, 100, 255, 256, 257, 511, 512, 513, 700, 1025, 2000]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [4, 8, 16])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (8, 2), (16, 2), (16, 1), (6, 2)])
+def test_variants_match_oracle(D, bs, Hq, Hkv):
+    seed = 1000 + D + 7 * bs + Hq * 31 + Hkv
+    w = wl.random_decode_case(seed, num_seqs=len(LENS), num_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                              block_size=bs, lengths=LENS)
+    poison_tail_slots(w)
+    # tail slots of positions >= L are poison; the token at L-1 is the cache's own
+    for s, L in enumerate(w.seq_lens):
+        blk = w.block_tables[s, (L - 1) // bs]
+        w.key_cache[blk, (L - 1) % bs] = w.new_key[s]
+        w.value_cache[blk, (L - 1) % bs] = w.new_value[s]
+    ref = oracle.paged_decode(w.query, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, w.scale,
+                              threads=0)
+    for kind, part in (("one_pass", 0), ("split", 16), ("split", 64), ("split", 512), ("auto", 0)):
+        assert_close(_run(w, kind, part), ref, f"{kind}/{part}")
+
+
+def test_zero_length_and_single_token():
+    lens = [0, 1, 0, 5, 1]
+    w = wl.random_decode_case(77, num_seqs=5, num_heads=8, num_kv_heads=1, head_dim=128, block_size=16,
+                              lengths=lens, spare_blocks=2)
+    for kind, part in (("one_pass", 0), ("split", 16), ("auto", 0)):
+        got = _run(w, kind, part)
+        assert np.all(got[0] == 0) and np.all(got[2] == 0)
+        for s in (1, 4):   # L = 1: the value row itself, bit for bit
+            blk = w.block_tables[s, 0]
+            assert np.array_equal(got[s], np.broadcast_to(w.value_cache[blk, 0, 0], got[s].shape))
+
+
+def test_permutation_of_physical_blocks_is_bitwise_invariant():
+    w = wl.random_decode_case(5, num_seqs=6, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                              lengths=[33, 200, 1000, 17, 512, 1500])
+    rng = np.random.default_rng(1)
+    perm = rng.permutation(w.num_blocks)
+    w2 = wl.random_decode_case(5, num_seqs=6, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                               lengths=[33, 200, 1000, 17, 512, 1500])
+    w2.key_cache[perm] = w.key_cache
+    w2.value_cache[perm] = w.value_cache
+    w2.block_tables = np.where(w.block_tables >= 0, perm[np.maximum(w.block_tables, 0)], -1).astype(np.int32)
+    for kind, part in (("one_pass", 0), ("split", 128), ("auto", 0)):
+        assert np.array_equal(_run(w, kind, part), _run(w2, kind, part))
+
+
+def test_shared_prefix_identical_outputs():
+    w = wl.random_decode_case(6, num_seqs=4, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                              lengths=[700, 700, 700, 700])
+    w.block_tables[1:] = w.block_tables[0]
+    w.query[1:] = w.query[0]
+    for kind, part in (("one_pass", 0), ("split", 256)):
+        got = _run(w, kind, part)
+        assert all(np.array_equal(got[0], got[i]) for i in range(1, 4))
+
+
+@pytest.mark.parametrize("Hq,Hkv,part", [(32, 8, 512), (8, 8, 64), (16, 1, 32)])
+def test_partitions_and_reduce_match_oracle(Hq, Hkv, part):
+    lens = [1, 40, 511, 512, 513, 1300, 0, 2047]
+    w = wl.random_decode_case(88, num_seqs=len(lens), num_heads=Hq, num_kv_heads=Hkv, head_dim=128,
+                              block_size=16, lengths=lens, spare_blocks=1)
+    d = _dev_inputs(w)
+    nbytes = ops.decode_workspace_size(w.num_seqs, Hq, 128, w.max_seq_len, part)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
+    o, m, l = ops.decode_partitions(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
+                                    d["seq_lens"], w.scale, w.max_seq_len, part, ws)
+    torch.cuda.synchronize()
+    parts = o.shape[2]
+    rm, rl, ro = oracle.paged_decode_partials(w.query, w.key_cache, w.value_cache, w.block_tables,
+                                              w.seq_lens, w.scale, part, parts)
+    gm, gl, go = m.double().cpu().numpy(), l.double().cpu().numpy(), o.double().cpu().numpy()
+    empty = np.isneginf(rm)
+    assert np.array_equal(np.isneginf(gm), empty)
+    assert np.all(gl[empty] == 0) and np.all(go[empty] == 0)
+    full = ~empty
+    np.testing.assert_allclose(gm[full], rm[full], rtol=1e-5, atol=1e-4)
+    np.testing.assert_allclose(gl[full], rl[full], rtol=1e-2)
+    norm_ref = ro[full] / rl[full][:, None]
+    norm_gpu = go[full] / gl[full][:, None]
+    ok, max_abs, _, _ = oracle.allclose_report(norm_gpu, norm_ref, 2e-3, 1e-2)
+    assert ok, max_abs
+    out = torch.empty_like(d["query"])
+    ops.lse_reduce(out, ws, d["seq_lens"], w.max_seq_len, part)
+    torch.cuda.synchronize()
+    ref = oracle.paged_decode(w.query, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(bf16_to_host_bits(out), ref, "lse_reduce")
+
+
+def test_split_and_one_pass_agree_on_long_sequences():
+    w = wl.make("gqa", num_seqs=16)
+    one = _run(w, "one_pass")
+    for part in (256, 512, 1024):
+        split = _run(w, "split", part)
+        a, b = oracle.bf16_bits_to_f64(one), oracle.bf16_bits_to_f64(split)
+        assert np.max(np.abs(a - b)) <= 4e-3
+
+
+def test_validate_tables():
+    w = wl.make("tiny", fill_cache=False)
+    d = _dev_inputs(w)
+    assert ops.validate_tables(d["block_tables"], d["seq_lens"], w.block_size, w.num_blocks, w.max_seq_len) == 0
+    bad = w.block_tables.copy()
+    bad[1, 0] = w.num_blocks
+    bt = torch.from_numpy(bad).to(DEV)
+    assert ops.validate_tables(bt, d["seq_lens"], w.block_size, w.num_blocks, w.max_seq_len) == 1
+    assert ops.validate_tables(d["block_tables"], d["seq_lens"], w.block_size, w.num_blocks, 40) == 1
+    assert ops.device_status() == 0

@@ -1,0 +1,124 @@
+"""The native host block pool (C++ behind the C ABI) against the oracle's plain
+Python pool: identical ids, reference counts, slots and copy pairs, bit for bit
+(CPU only)."""
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.pool import OraclePool, PoolExhausted
+from paged_kv_cache_379_b200 import workload as wl
+from paged_kv_cache_379_b200._lib import PagedKVError
+from paged_kv_cache_379_b200.pool import BlockPool
+from paged_kv_cache_379_b200.step import host_step
+
+
+def test_random_operation_sequences_match():
+    rng = np.random.default_rng(17)
+    n, bs = 96, 4
+    order = rng.permutation(n)
+    a = BlockPool(n, bs, free_order=order)
+    b = OraclePool(n, bs, free_order=order.tolist())
+    seqs_a, seqs_b = [], []
+    for _ in range(600):
+        op = int(rng.integers(0, 5))
+        if op == 0 or not seqs_a:
+            k = int(rng.integers(1, 6))
+            try:
+                ta = a.allocate(k)
+            except PagedKVError as e:
+                assert e.status == -6
+                with pytest.raises(PoolExhausted):
+                    b.allocate(k)
+                continue
+            assert ta == b.allocate(k)
+            seqs_a.append(ta)
+            seqs_b.append(list(ta))
+        elif op == 1:
+            i = int(rng.integers(len(seqs_a)))
+            seqs_a.append(a.fork(seqs_a[i]))
+            seqs_b.append(b.fork(seqs_b[i]))
+        elif op == 2:
+            i = int(rng.integers(len(seqs_a)))
+            j = int(rng.integers(len(seqs_a[i])))
+            try:
+                ra = a.allocate_or_get_cow(seqs_a[i][j])
+            except PagedKVError:
+                with pytest.raises(PoolExhausted):
+                    b.allocate_or_get_cow(seqs_b[i][j])
+                continue
+            rb = b.allocate_or_get_cow(seqs_b[i][j])
+            assert ra == rb
+            seqs_a[i][j] = ra[0]
+            seqs_b[i][j] = rb[0]
+        else:
+            i = int(rng.integers(len(seqs_a)))
+            a.free_table(seqs_a.pop(i))
+            b.free_sequence(seqs_b.pop(i))
+        assert a.get_num_free_blocks() == b.get_num_free_blocks()
+    assert a.refcounts() == b.refcount
+
+
+def test_bad_block_ids_are_rejected():
+    p = BlockPool(4, 16)
+    with pytest.raises(PagedKVError):
+        p.free(2)                       # not allocated
+    with pytest.raises(PagedKVError):
+        p.fork([7])
+    with pytest.raises(ValueError):
+        BlockPool(4, 16, free_order=[0, 1, 1, 2])
+
+
+def _oracle_host_step(w, fork_all):
+    """The same step with the oracle pool: adopt tables, optional fork, append a token."""
+    tables = [list(w.block_tables[s, :w.blocks_per_seq[s]]) for s in range(w.num_seqs)]
+    unowned = list(w.free_blocks)
+    owned = sorted(set(range(w.num_blocks)) - set(unowned))
+    pool = OraclePool(w.num_blocks, w.block_size, free_order=owned + unowned[::-1])
+    # adoption: every table reference is an owner; adopted blocks leave the free list
+    for t in tables:
+        for blk in t:
+            pool.refcount[blk] += 1
+    pool.free_list = [x for x in pool.free_list if pool.refcount[x] == 0]
+    if fork_all:
+        for t in tables:
+            pool.fork(t)
+    slots, pairs = [], []
+    for s, t in enumerate(tables):
+        slot, pair, _ = pool.append_token(t, int(w.seq_lens[s]) - 1)
+        slots.append(slot)
+        if pair:
+            pairs.append(pair)
+    return pool, tables, slots, pairs
+
+
+@pytest.mark.parametrize("name,kw,fork_all", [
+    ("tiny", {}, False),
+    ("shared", {"num_seqs": 64}, True),
+    ("shared", {"num_seqs": 8, "shared_prompt_len": 1020, "lengths": [1] * 8}, False),
+])
+def test_host_step_matches_oracle_pool(name, kw, fork_all):
+    w = wl.make(name, fill_cache=False, **kw)
+    pool, tables, nblk, slots, pairs = host_step(w, fork_all=fork_all)
+    opool, otables, oslots, opairs = _oracle_host_step(w, fork_all)
+    assert slots.tolist() == oslots
+    assert [tuple(p) for p in pairs.tolist()] == opairs
+    for s in range(w.num_seqs):
+        assert tables[s, :nblk[s]].tolist() == otables[s]
+    assert pool.refcounts() == opool.refcount
+    # the device-side address translation agrees with the pool's slots (oracle form)
+    got = oracle.slot_mapping(tables, np.arange(w.num_seqs, dtype=np.int32),
+                              w.seq_lens.astype(np.int64) - 1, w.block_size)
+    assert got.tolist() == oslots
+    if name == "shared" and not fork_all:
+        assert len(pairs) == 7          # 8 samples write into their shared partial block
+
+
+def test_shared_workload_pair_count():
+    """Fork snapshot + one token: a copy per sequence unless its token opens a new block."""
+    w = wl.make("shared", fill_cache=False)
+    _, tables, nblk, slots, pairs = host_step(w, fork_all=True)
+    opening = int(np.sum((w.seq_lens - 1) % w.block_size == 0))
+    assert len(pairs) == w.num_seqs - opening
+    assert len(set(pairs[:, 1].tolist())) == len(pairs)
+    assert not set(pairs[:, 1].tolist()) & set(pairs[:, 0].tolist())
