@@ -3,6 +3,8 @@ whole decode step, and the tolerance check."""
 
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 import oracle
@@ -31,7 +33,7 @@ def poison_tail_slots(w: wl.Workload, tables=None) -> None:
         w.value_cache[last, off:] = wl.BF16_NAN
 
 
-def oracle_step(w: wl.Workload, tables=None, pairs=None, threads: int = 0):
+def oracle_step(w: wl.Workload, tables=None, pairs=None, threads: int = min(32, os.cpu_count() or 1)):
     """The oracle's step: copy pairs, slots of position L-1, cache write, decode.
 
     Returns (key_cache, value_cache, slots, out fp64)."""
