@@ -22,10 +22,11 @@
 //  * Consumers: tile i goes to warp i % 4 (each warp owns 2 stages).  Every warp
 //    keeps its own running max m, sum l and fp32 accumulator; the four states
 //    are merged through shared memory at the end.
-//    - G >= 3 (grouped heads: a dense [G x D] . [D x 16] contraction per tile):
-//      bf16 mma.sync m16n8k16, S = Q K^T with Q as the A operand (rows = heads),
-//      K tiles through ldmatrix, then O += P V with P taken straight from the S
-//      accumulators and V through ldmatrix.trans.
+//    - G >= 3 (grouped heads: a dense [16 x D] . [D x G] contraction per tile):
+//      bf16 mma.sync m16n8k16 in transposed form, S^T = K Q^T with the K tile as
+//      the A operand (rows = tokens, via ldmatrix) and Q^T in registers, then
+//      O^T += V^T P^T with V^T through ldmatrix.trans and P^T moved out of the
+//      S^T accumulators by movmatrix.trans; P goes in as bf16 hi + residual.
 //    - G <= 2 (MHA-like, a matrix-vector product): CUDA cores, 16-byte shared
 //      loads, warp-shuffle reductions for the dot products, max and sum.
 //  * Masking selects (-inf logits, zeroed V rows) instead of multiplying by 0,
@@ -112,8 +113,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         const __grid_constant__ CUtensorMap tmap_v)
 {
     // MODE 0: CUDA cores, GC (1 or 2) query heads per KV head.
-    // MODE 1: tensor cores, up to 8 query heads per KV head.
-    // MODE 2: tensor cores, up to 16 query heads per KV head.
+    // MODE 1: tensor cores, up to 8 query heads per KV head (one 8-head tile).
+    // MODE 2: tensor cores, up to 16 query heads per KV head (two 8-head tiles).
     using Geo = TileGeom<D, BS>;
     static_assert(sizeof(MergeScratch<D>) <= Geo::kPipeSmem, "merge scratch must fit the ring");
     extern __shared__ uint8_t smem_raw[];
@@ -368,32 +369,46 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 }
             }
         } else {
-            constexpr bool HI = (MODE == 2);
-            constexpr int KSTEPS = D / 16;
-            constexpr int NT = D / 8;
-            const int r = lane >> 2;
-            const int tq = lane & 3;
-            uint32_t qlo[KSTEPS][2], qhi[KSTEPS][2];
+            // Tensor cores, transposed form: S^T[16 tokens x 8*NH heads] = K Q^T,
+            // then O^T[D x heads] += V^T P^T.  Tokens are the MMA's M dimension,
+            // so no accumulator row is wasted when G <= 8; P^T is taken from the
+            // S^T accumulators by an in-register 8x8 transpose (movmatrix).
+            constexpr int NH = (MODE == 2) ? 2 : 1;  // 8-head column tiles
+            constexpr int KSTEPS = D / 16;           // k-steps of S^T = K Q^T
+            constexpr int MT = D / 16;               // 16-row d tiles of O^T
+            const int gq = lane >> 2;                // MMA groupID
+            const int tq = lane & 3;                 // MMA thread-in-group
+            // B operand of S^T = K Q^T: b0 = Q[head][d 16kk+2tq..+1], b1 = Q[head][d 16kk+8+2tq..+1]
+            uint32_t qb[NH][KSTEPS][2];
 #pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk) {
+            for (int nh = 0; nh < NH; ++nh) {
+                const int head = nh * 8 + gq;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int col = kk * 16 + hh * 8 + tq * 2;
-                    qlo[kk][hh] = r < G ? *reinterpret_cast<const uint32_t *>(p.query + q_off + (int64_t)r * D + col) : 0u;
-                    qhi[kk][hh] = (HI && r + 8 < G)
-                                      ? *reinterpret_cast<const uint32_t *>(p.query + q_off + (int64_t)(r + 8) * D + col)
-                                      : 0u;
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int col = kk * 16 + hh * 8 + tq * 2;
+                        qb[nh][kk][hh] = head < G
+                                             ? *reinterpret_cast<const uint32_t *>(p.query + q_off + (int64_t)head * D + col)
+                                             : 0u;
+                    }
                 }
             }
-            float o[NT][4];
+            float o[MT][NH][4];
+            float m[NH][2], l[NH][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-            float m_lo = -INFINITY, l_lo = 0.f, m_hi = -INFINITY, l_hi = 0.f;
-            // ldmatrix lane roles: K (B operand of S = Q K^T) and V (B operand of O += P V, transposed)
-            const int ktok = (lane & 7) + ((lane >> 4) << 3);
-            const int kpar = (lane >> 3) & 1;
-            const int vtok = (lane & 7) + (((lane >> 3) & 1) << 3);
-            const int vpar = lane >> 4;
+            for (int nh = 0; nh < NH; ++nh) {
+                m[nh][0] = m[nh][1] = -INFINITY;
+                l[nh][0] = l[nh][1] = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) o[mt][nh][0] = o[mt][nh][1] = o[mt][nh][2] = o[mt][nh][3] = 0.f;
+            }
+            // ldmatrix lane roles: K as the A operand (rows = tokens), V^T as the A
+            // operand through the transposing load (rows = d)
+            const int ktok = (lane & 7) + (((lane >> 3) & 1) << 3);
+            const int kpar = lane >> 4;
+            const int vtok = (lane & 7) + ((lane >> 4) << 3);
+            const int vpar = (lane >> 3) & 1;
 
             for (int tile = warp; tile < n_tiles; tile += kConsumerWarps) {
                 const int stage = tile % kStages;
@@ -408,98 +423,95 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 const int valid = min(kTileTokens, t_end - (t_begin + tile * kTileTokens));
                 if (valid < kTileTokens) zero_tail(vt, valid);
 
-                // S[16 rows = heads][16 tokens] = Q K^T
-                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                // S^T[token][head] = K Q^T
+                float sc[NH][4];
+#pragma unroll
+                for (int nh = 0; nh < NH; ++nh) sc[nh][0] = sc[nh][1] = sc[nh][2] = sc[nh][3] = 0.f;
 #pragma unroll
                 for (int kk = 0; kk < KSTEPS; ++kk) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), b0, b1, b2, b3);
-                    mma_bf16_16816(sc[0], qlo[kk][0], qhi[kk][0], qlo[kk][1], qhi[kk][1], b0, b1);
-                    mma_bf16_16816(sc[1], qlo[kk][0], qhi[kk][0], qlo[kk][1], qhi[kk][1], b2, b3);
-                }
-                // scale to log2 units, mask positions past the end
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
+                    for (int nh = 0; nh < NH; ++nh) mma_bf16_16816(sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                }
+                // online softmax per head column; this lane holds tokens gq and gq+8
+                // of heads 2tq and 2tq+1.  P enters the PV product as a bf16 high
+                // part plus a bf16 residual (two MMAs): ~16 significant bits.
+                const bool in0 = gq < valid, in1 = gq + 8 < valid;
+                uint32_t bh[NH][2], bl[NH][2];
+#pragma unroll
+                for (int nh = 0; nh < NH; ++nh) {
+                    float pr[2][2];  // [head j][token row]
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const bool in = nt * 8 + tq * 2 + j < valid;
-                        sc[nt][j] = in ? sc[nt][j] * p.scale_log2 : -INFINITY;
-                        if (HI) sc[nt][2 + j] = in ? sc[nt][2 + j] * p.scale_log2 : -INFINITY;
+                        const float x0 = in0 ? sc[nh][j] * p.scale_log2 : -INFINITY;
+                        const float x1 = in1 ? sc[nh][2 + j] * p.scale_log2 : -INFINITY;
+                        float mx = fmaxf(x0, x1);
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                        const float m_new = fmaxf(m[nh][j], mx);
+                        const float corr = exp2f(m[nh][j] - m_new);
+                        m[nh][j] = m_new;
+                        pr[j][0] = exp2f(x0 - m_new);
+                        pr[j][1] = exp2f(x1 - m_new);
+                        l[nh][j] = l[nh][j] * corr + (pr[j][0] + pr[j][1]);
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            o[mt][nh][j] *= corr;
+                            o[mt][nh][2 + j] *= corr;
+                        }
+                    }
+#pragma unroll
+                    for (int row = 0; row < 2; ++row) {
+                        const uint32_t hi = pack_bf16x2(pr[0][row], pr[1][row]);
+                        const float2 hf = unpack_bf16x2(hi);
+                        const uint32_t lo = pack_bf16x2(pr[0][row] - hf.x, pr[1][row] - hf.y);
+                        bh[nh][row] = movmatrix_trans(hi);
+                        bl[nh][row] = movmatrix_trans(lo);
                     }
                 }
-                // online softmax, rows r (and r + 8)
-                uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;
-                {
-                    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float m_new = fmaxf(m_lo, mx);
-                    const float corr = exp2f(m_lo - m_new);
-                    m_lo = m_new;
-                    pa0 = pack_bf16x2(exp2f(sc[0][0] - m_new), exp2f(sc[0][1] - m_new));
-                    pa2 = pack_bf16x2(exp2f(sc[1][0] - m_new), exp2f(sc[1][1] - m_new));
-                    const float2 f0 = unpack_bf16x2(pa0), f2 = unpack_bf16x2(pa2);
-                    l_lo = l_lo * corr + ((f0.x + f0.y) + (f2.x + f2.y));
+                // O^T[d][head] += V^T P^T
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        o[nt][0] *= corr;
-                        o[nt][1] *= corr;
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * mt + vpar), a0, a1, a2, a3);
+#pragma unroll
+                    for (int nh = 0; nh < NH; ++nh) {
+                        mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
+                        mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
                     }
-                }
-                if (HI) {
-                    float mx = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float m_new = fmaxf(m_hi, mx);
-                    const float corr = exp2f(m_hi - m_new);
-                    m_hi = m_new;
-                    pa1 = pack_bf16x2(exp2f(sc[0][2] - m_new), exp2f(sc[0][3] - m_new));
-                    pa3 = pack_bf16x2(exp2f(sc[1][2] - m_new), exp2f(sc[1][3] - m_new));
-                    const float2 f1 = unpack_bf16x2(pa1), f3 = unpack_bf16x2(pa3);
-                    l_hi = l_hi * corr + ((f1.x + f1.y) + (f3.x + f3.y));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        o[nt][2] *= corr;
-                        o[nt][3] *= corr;
-                    }
-                }
-                // O[16 rows][D] += P[16 x 16 tokens] V[16 tokens x D]
-#pragma unroll
-                for (int nc = 0; nc < KSTEPS; ++nc) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * nc + vpar), b0, b1, b2, b3);
-                    mma_bf16_16816(o[2 * nc], pa0, pa1, pa2, pa3, b0, b1);
-                    mma_bf16_16816(o[2 * nc + 1], pa0, pa1, pa2, pa3, b2, b3);
                 }
                 if (valid < kTileTokens) fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty_bar + 8 * stage);
             }
-            l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
-            l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
-            if (HI) {
-                l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
-                l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+#pragma unroll
+            for (int nh = 0; nh < NH; ++nh) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    l[nh][j] += __shfl_xor_sync(0xffffffffu, l[nh][j], 4);
+                    l[nh][j] += __shfl_xor_sync(0xffffffffu, l[nh][j], 8);
+                    l[nh][j] += __shfl_xor_sync(0xffffffffu, l[nh][j], 16);
+                }
             }
             __syncthreads();  // ring drained
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int d = nt * 8 + tq * 2;
-                if (r < G) {
-                    ms->o[warp][r][d] = o[nt][0];
-                    ms->o[warp][r][d + 1] = o[nt][1];
-                }
-                if (HI && r + 8 < G) {
-                    ms->o[warp][r + 8][d] = o[nt][2];
-                    ms->o[warp][r + 8][d + 1] = o[nt][3];
-                }
-            }
-            if (tq == 0) {
-                ms->m[warp][r] = m_lo;
-                ms->l[warp][r] = l_lo;
-                if (HI) {
-                    ms->m[warp][r + 8] = m_hi;
-                    ms->l[warp][r + 8] = l_hi;
+            for (int nh = 0; nh < NH; ++nh) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int head = nh * 8 + 2 * tq + j;
+                    if (head < G) {
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            ms->o[warp][head][mt * 16 + gq] = o[mt][nh][j];
+                            ms->o[warp][head][mt * 16 + gq + 8] = o[mt][nh][2 + j];
+                        }
+                        if (gq == 0) {
+                            ms->m[warp][head] = m[nh][j];
+                            ms->l[warp][head] = l[nh][j];
+                        }
+                    }
                 }
             }
         }
