@@ -75,26 +75,38 @@ template <int D, int BS>
 struct TileGeom {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(BS == 4 || BS == 8 || BS == 16, "block_size");
-    static constexpr int kRows128 = D / 64;                       // 128-byte rows per token
-    static constexpr int kBlkBytes = BS * D * 2;                  // one block of one head
-    static constexpr int kBlkSmem = kBlkBytes < 1024 ? 1024 : kBlkBytes;  // keep 1024-B phase
+    // A K (or V) tile of 16 tokens is stored as D/64 planes; plane h holds
+    // d in [64h, 64h+64) of every token as one 128-byte row per token.  TMA
+    // writes one box {64 elements, 1, 1 head, bs tokens} per (block, plane),
+    // 128B-swizzled, at a 1024-byte aligned slot.  With bs >= 8, 8 consecutive
+    // tokens occupy 8 consecutive rows, so every ldmatrix phase touches 8
+    // distinct swizzle rows: no bank conflicts.
+    static constexpr int kHalves = D / 64;
+    static constexpr int kBlkBytes = BS * D * 2;                  // bytes TMA delivers per block
+    static constexpr int kSlotRows = BS < 8 ? 8 : BS;             // 128-B rows reserved per block per plane
     static constexpr int kBlocksPerTile = kTileTokens / BS;
-    static constexpr int kTileSmem = kBlocksPerTile * kBlkSmem;
+    static constexpr int kPlaneSmem = kBlocksPerTile * kSlotRows * 128;
+    static constexpr int kTileSmem = kHalves * kPlaneSmem;
     static constexpr int kStageSmem = 2 * kTileSmem;              // K tile, then V tile
     static constexpr int kPipeSmem = kStages * kStageSmem;
     static constexpr int kSmemBytes = kPipeSmem + 1024 /* alignment slack */ + 2 * kStages * 8 + 16;
 
-    // Byte offset inside a K or V tile of the 16-byte chunk c (0..D/8-1) of
-    // token t (0..15), as the 128B-swizzled TMA box stores it: chunk index XOR
-    // (128-byte row index mod 8), every block slot starting 1024-B aligned.
+    // Offset, inside a plane, of token t's 128-byte row.
+    __device__ static __forceinline__ uint32_t row_offset(int t)
+    {
+        return (uint32_t)((t / BS) * kSlotRows * 128 + (t % BS) * 128);
+    }
+    // Offset inside a tile of the 16-byte chunk c (0..D/8-1) of token t (0..15):
+    // chunk index XOR (row index mod 8), the 128-byte swizzle.
     __device__ static __forceinline__ uint32_t chunk_offset(int t, int c)
     {
-        const uint32_t row = (uint32_t)((t % BS) * kRows128 + (c >> 3));
-        return (uint32_t)((t / BS) * kBlkSmem) + row * 128u + ((((uint32_t)c & 7u) ^ (row & 7u)) << 4);
+        const uint32_t ro = row_offset(t);
+        return (uint32_t)((c >> 3) * kPlaneSmem) + ro + ((((uint32_t)c & 7u) ^ ((ro >> 7) & 7u)) << 4);
     }
-    __device__ static __forceinline__ uint32_t token_offset(int t)
+    // Destination of the TMA box of block k (within the tile), plane h.
+    __device__ static __forceinline__ uint32_t box_offset(int k, int h)
     {
-        return (uint32_t)((t / BS) * kBlkSmem + (t % BS) * kRows128 * 128);
+        return (uint32_t)(h * kPlaneSmem + k * kSlotRows * 128);
     }
 };
 
@@ -102,7 +114,7 @@ struct TileGeom {
 // running max (log2 units), sum and accumulator of up to 16 heads.
 template <int D>
 struct MergeScratch {
-    float o[kConsumerWarps][16][D];
+    float o[kConsumerWarps][16][D + 4];  // +4: heads 2tq+j land in distinct banks
     float m[kConsumerWarps][16];
     float l[kConsumerWarps][16];
 };
@@ -209,8 +221,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 #pragma unroll
                         for (int k = 0; k < Geo::kBlocksPerTile; ++k) {
                             if (k < valid) {
-                                tma_load_4d(kdst + k * Geo::kBlkSmem, &tmap_k, bar, 0, 0, g, phys[k] * BS);
-                                tma_load_4d(vdst + k * Geo::kBlkSmem, &tmap_v, bar, 0, 0, g, phys[k] * BS);
+#pragma unroll
+                                for (int h = 0; h < Geo::kHalves; ++h) {
+                                    tma_load_4d(kdst + Geo::box_offset(k, h), &tmap_k, bar, 0, h, g, phys[k] * BS);
+                                    tma_load_4d(vdst + Geo::box_offset(k, h), &tmap_v, bar, 0, h, g, phys[k] * BS);
+                                }
                             }
                         }
                         ++issued;
@@ -236,12 +251,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         // Zero the V rows of tokens [valid, 16) so masked positions contribute
         // exactly 0 (stale or NaN data is never multiplied).
         auto zero_tail = [&](uint32_t vt, int valid) {
-            constexpr int kChunksPerTok = Geo::kRows128 * 8;
+            constexpr int kChunksPerTok = Geo::kHalves * 8;
             for (int i = lane; i < (kTileTokens - valid) * kChunksPerTok; i += 32) {
                 const int t = valid + i / kChunksPerTok;
-                const int c = i % kChunksPerTok;
-                *reinterpret_cast<uint4 *>(base_ptr + (vt - base) + Geo::token_offset(t) + c * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
+                const int c = i % kChunksPerTok;  // whole rows are zeroed, so the swizzle does not matter
+                *reinterpret_cast<uint4 *>(base_ptr + (vt - base) + (c >> 3) * Geo::kPlaneSmem +
+                                           Geo::row_offset(t) + (c & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
             }
             __syncwarp();
         };
@@ -554,56 +569,78 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     }
 }
 
-// Log-sum-exp merge of the partitions of one (sequence, head) per CTA:
+// Log-sum-exp merge of the partitions of one (sequence, head) per warp:
 //   M = max_p m_p,  out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p.
-__global__ void __launch_bounds__(128) lse_reduce_kernel(const ReduceParams r)
+// Lane p computes the weight of partition p; the weighted sum over partitions
+// reads each partition's o row as one coalesced 16-byte (D = 128) or 8-byte
+// (D = 64) vector per lane.
+constexpr int kReduceWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const ReduceParams r)
 {
+    constexpr int VEC = D / 32;
     pdl_wait();
     pdl_launch_dependents();
-    const int h = blockIdx.x % r.num_heads;
-    const int s = blockIdx.x / r.num_heads;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
+    if (row >= (int64_t)r.num_seqs * r.num_heads) return;
+    const int s = (int)(row / r.num_heads);
     const int L = r.seq_lens[s];
     int nparts = L > 0 ? (L + r.part_tokens - 1) / r.part_tokens : 1;
     nparts = min(nparts, r.max_parts);
     if (r.skip_single && nparts == 1) return;
-    const int64_t row = (int64_t)s * r.num_heads + h;
     const float *m = r.ws_m + row * r.max_parts;
     const float *l = r.ws_l + row * r.max_parts;
-    const float *o = r.ws_o + row * r.max_parts * r.head_dim;
-    __shared__ float red[4];
-    __shared__ float bcast[2];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float *o = r.ws_o + row * r.max_parts * D + lane * VEC;
 
-    float mx = -INFINITY;
-    for (int i = threadIdx.x; i < nparts; i += blockDim.x) mx = fmaxf(mx, m[i]);
+    float M = -INFINITY;
+    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, m[i]);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (lane == 0) red[warp] = mx;
-    __syncthreads();
-    if (threadIdx.x == 0) bcast[0] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    const float M = bcast[0];
-
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float acc[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
     float den = 0.f;
-    if (M != -INFINITY)
-        for (int i = threadIdx.x; i < nparts; i += blockDim.x)
-            if (m[i] != -INFINITY) den += expf(m[i] - M) * l[i];
+    if (M != -INFINITY) {
+        for (int i0 = 0; i0 < nparts; i0 += 32) {
+            const int i = i0 + lane;
+            const float w = (i < nparts) ? expf(m[i] - M) : 0.f;  // an empty partition has m = -inf: weight 0
+            den += (i < nparts) ? w * l[i] : 0.f;
+            const int cnt = min(32, nparts - i0);
+            int j = 0;
+            for (; j + 4 <= cnt; j += 4) {
+                float wj[4], v[4][VEC];
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-    __syncthreads();
-    if (lane == 0) red[warp] = den;
-    __syncthreads();
-    if (threadIdx.x == 0) bcast[1] = (red[0] + red[1]) + (red[2] + red[3]);
-    __syncthreads();
-    den = bcast[1];
-
-    for (int d = threadIdx.x; d < r.head_dim; d += blockDim.x) {
-        float num = 0.f;
-        if (M != -INFINITY)
-            for (int i = 0; i < nparts; ++i)
-                if (m[i] != -INFINITY) num = fmaf(expf(m[i] - M), o[(int64_t)i * r.head_dim + d], num);
-        r.out[row * r.head_dim + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+                for (int u = 0; u < 4; ++u) {
+                    wj[u] = __shfl_sync(0xffffffffu, w, j + u);
+                    const float *src = o + (int64_t)(i0 + j + u) * D;
+                    if constexpr (VEC == 4) {
+                        const float4 f = *reinterpret_cast<const float4 *>(src);
+                        v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+                    } else {
+                        const float2 f = *reinterpret_cast<const float2 *>(src);
+                        v[u][0] = f.x; v[u][1] = f.y;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[e] = fmaf(wj[u], v[u][e], acc[e]);
+            }
+            for (; j < cnt; ++j) {
+                const float wj = __shfl_sync(0xffffffffu, w, j);
+                const float *src = o + (int64_t)(i0 + j) * D;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[e] = fmaf(wj, src[e], acc[e]);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
     }
+    __nv_bfloat16 *dst = r.out + row * D + lane * VEC;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) dst[e] = __float2bfloat16_rn(den > 0.f ? acc[e] / den : 0.f);
 }
 
 }  // namespace pakv

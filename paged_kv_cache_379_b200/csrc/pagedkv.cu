@@ -37,14 +37,15 @@ static EncodeTiledFn encode_fn()
 
 // The cache [num_blocks, bs, Hkv, D] seen by TMA as 4-D (innermost first):
 //   {64 elements = 128 B, D/64, Hkv, num_blocks*bs slots}
-// with a box of one block of one head: {64, D/64, 1, bs}, 128-byte swizzle.
+// with a box of one 64-wide d-plane of one block of one head: {64, 1, 1, bs},
+// 128-byte swizzle.
 static int make_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int bs, int hkv, int d)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return check_cuda(cudaErrorNotSupported);
     const cuuint64_t dims[4] = {64, (cuuint64_t)(d / 64), (cuuint64_t)hkv, (cuuint64_t)(num_blocks * bs)};
     const cuuint64_t strides[3] = {128, (cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)(d / 64), 1, (cuuint32_t)bs};
+    const cuuint32_t box[4] = {64, 1, 1, (cuuint32_t)bs};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(cache), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -107,6 +108,14 @@ static int launch_decode_d(int bs, const DecodeParams &p, const CUtensorMap &tk,
     case 16: return launch_decode_bs<D, 16>(p, tk, tv, grid, st);
     default: return PA_ERR_UNSUPPORTED;
     }
+}
+
+static int launch_reduce(const ReduceParams &r, cudaStream_t st)
+{
+    const int64_t rows = (int64_t)r.num_seqs * r.num_heads;
+    const dim3 grid((unsigned)cdiv64(rows, kReduceWarps));
+    if (r.head_dim == 64) return launch_pdl(lse_reduce_kernel<64>, grid, dim3(kReduceWarps * 32), 0, st, r);
+    return launch_pdl(lse_reduce_kernel<128>, grid, dim3(kReduceWarps * 32), 0, st, r);
 }
 
 struct DecodeArgs {
@@ -204,7 +213,7 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
     r.part_tokens = part;
     r.max_parts = p.max_parts;
     r.skip_single = 1;
-    return launch_pdl(lse_reduce_kernel, dim3((unsigned)(a.num_seqs * a.num_heads)), dim3(128), 0, st, r);
+    return launch_reduce(r, st);
 }
 
 // Partition size the dispatcher uses for a split run.
@@ -395,8 +404,9 @@ int pa_lse_reduce(void *out, const void *workspace, const int32_t *seq_lens, int
     r.part_tokens = partition_size;
     r.max_parts = max_parts;
     r.skip_single = 0;
-    return launch_pdl(lse_reduce_kernel, dim3((unsigned)(num_seqs * num_heads)), dim3(128), 0,
-                      static_cast<cudaStream_t>(stream), r);
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(workspace) || !aligned16(out)) return PA_ERR_ALIGNMENT;
+    return launch_reduce(r, static_cast<cudaStream_t>(stream));
 }
 
 int pa_validate_tables(const int32_t *block_tables, const int32_t *seq_lens, int num_seqs, int max_blocks_per_seq,
