@@ -121,10 +121,23 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pa
  * device-to-host read).
  *
  * pa_decode picks the one-pass kernel or the split form by max_seq_len and the
- * number of (sequence, KV head) units; it needs a workspace of at least
+ * number of (sequence, KV head) units.  It takes a workspace of at least
  * pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len, 0)
- * bytes (16-byte aligned, caller-owned, contents need no initialisation) or
- * may be given none (workspace NULL), in which case it runs one pass.
+ * bytes, or none (workspace NULL: one pass, work handed out round-robin).
+ *
+ * Workspace contract (all decode entry points that take one): caller-owned
+ * device memory, 16-byte aligned.  Its first 256 bytes hold the counters of
+ * the kernels' dynamic work scheduler: ZERO-FILL THE WORKSPACE ONCE after
+ * allocating it (e.g. cudaMemsetAsync); every call leaves those bytes zero
+ * again when it completes.  The rest is scratch (no initialisation needed).
+ * Calls that may run concurrently must not share a workspace.  After
+ * pa_device_status() has reported a timeout, zero the workspace again.
+ *
+ * The decode kernel is persistent: (resident CTAs per SM) x (SMs) CTAs loop
+ * over (sequence, partition, KV head) work items.  Sequence count limit of the
+ * split form: the per-CTA prefix table of num_seqs+1 ints must fit in shared
+ * memory next to the pipeline (num_seqs up to about 35000); beyond that the
+ * call returns PA_ERR_BAD_SHAPE.
  * ------------------------------------------------------------------------ */
 int pa_decode(void *out, const void *query, const void *key_cache, const void *value_cache,
               const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
@@ -143,9 +156,9 @@ int pa_decode_plan(int num_seqs, int num_heads, int num_kv_heads, int head_dim, 
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len,
                                 int partition_size);
 
-/* a4 alone: one CTA per (sequence, KV head) walks all of the sequence's blocks
- * with an online softmax ("逐块计算局部 Attention，最后合并结果", [源码解析 §四]).
- * No workspace. */
+/* a4 alone: each (sequence, KV head) work item walks all of the sequence's
+ * blocks with an online softmax ("逐块计算局部 Attention，最后合并结果",
+ * [源码解析 §四]).  No workspace: items are handed out round-robin. */
 int pa_decode_one_pass(void *out, const void *query, const void *key_cache,
                        const void *value_cache, const int32_t *block_tables,
                        const int32_t *seq_lens, float scale, int block_size, int num_kv_heads,
@@ -153,9 +166,9 @@ int pa_decode_one_pass(void *out, const void *query, const void *key_cache,
                        int num_blocks, int max_seq_len, void *stream);
 
 /* a5 + a6: positions are cut into partitions of partition_size tokens (a
- * multiple of 16, >= 16); one CTA per (sequence, KV head, partition) computes
- * the partition's local result, and a log-sum-exp reduce kernel merges them.
- * A sequence that fits in one partition is written directly by its CTA. */
+ * multiple of 16, >= 16); each (sequence, partition, KV head) work item
+ * computes the partition's local result, and a log-sum-exp reduce kernel
+ * merges them.  A sequence that fits in one partition is written directly. */
 int pa_decode_split(void *out, const void *query, const void *key_cache, const void *value_cache,
                     const int32_t *block_tables, const int32_t *seq_lens, float scale,
                     int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
@@ -164,9 +177,10 @@ int pa_decode_split(void *out, const void *query, const void *key_cache, const v
 
 /* a5 alone, for inspection: every partition p < ceil(max_seq_len/partition_size)
  * of every (s, h) writes its local result into the workspace, laid out as
- *   float o[num_seqs][num_heads][max_parts][head_dim]  at byte 0,
- *   float m[num_seqs][num_heads][max_parts]           after o,
- *   float l[num_seqs][num_heads][max_parts]           after m,
+ *   the 256-byte scheduler header,
+ *   float o[num_seqs][num_heads][max_parts][head_dim]  at byte 256,
+ *   float m[num_seqs][num_heads][max_parts]           after o (256-B aligned),
+ *   float l[num_seqs][num_heads][max_parts]           after m (256-B aligned),
  * with max_parts = ceil(max_seq_len / partition_size) (at least 1):
  *   m = max_p scale*q.k_p (natural-log units), l = sum_p exp(x_p - m),
  *   o = sum_p exp(x_p - m) v_p (not normalised).

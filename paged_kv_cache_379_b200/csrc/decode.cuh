@@ -9,19 +9,28 @@
 // sequence block by block and merges the per-block results with an online
 // softmax -- the "compute locally per block, merge at the end" pattern of §四.
 //
-// Work unit: one CTA per (sequence, KV head, partition).  All G = Hq/Hkv query
-// heads of the KV head are handled by the same CTA, so every K/V byte crosses
-// HBM once.  A partition is a run of `part_tokens` positions; the one-pass form
-// is a single partition covering the whole sequence.
+// Work item: (sequence, partition, KV head).  All G = Hq/Hkv query heads of the
+// KV head are handled together, so every K/V byte crosses HBM once.  A
+// partition is a run of `part_tokens` positions; the one-pass form has one
+// partition per sequence.
 //
-// CTA = 4 consumer warps + 1 producer warp.
-//  * Producer: one coalesced warp load of up to 32 table entries, then for each
-//    16-token tile one elected lane issues TMA tile loads of the tile's K and V
-//    blocks (box = [bs tokens x 1 head x head_dim], 128B-swizzled) into an
-//    8-stage shared-memory ring guarded by mbarriers.  Nothing else touches HBM.
-//  * Consumers: tile i goes to warp i % 4 (each warp owns 2 stages).  Every warp
+// Persistent kernel: a grid of (CTAs per SM) x (SM count) CTAs loops over the
+// work items.  The items of a launch are enumerated compactly (a prefix sum of
+// partitions per sequence, in shared memory), sequence-major with the KV head
+// fastest, and handed out by an atomic counter in the workspace (or round-robin
+// when there is no workspace).  A CTA is six warps:
+//  * Scheduler warp: takes the next item, decodes it, bulk-copies the item's G
+//    query rows into an item slot, and loads the item's block-table entries in
+//    chunks of 32 into a chunk queue -- running ahead of the other warps, so
+//    their latency is hidden.
+//  * Producer warp: for each chunk, one elected lane issues TMA tile loads of the
+//    K and V blocks (one box {64 d, 1 head, bs tokens} per 64-wide d-plane,
+//    128B-swizzled) into an 8-stage shared-memory ring guarded by mbarriers.  The
+//    ring runs continuously across items.
+//  * 4 consumer warps: 16-token tile i of an item goes to warp i % 4.  Every warp
 //    keeps its own running max m, sum l and fp32 accumulator; the four states
-//    are merged through shared memory at the end.
+//    are merged through shared memory at the end of the item (consumer-only
+//    named barriers, so the loads of the next item keep flowing meanwhile).
 //    - G >= 3 (grouped heads: a dense [16 x D] . [D x G] contraction per tile):
 //      bf16 mma.sync m16n8k16 in transposed form, S^T = K Q^T with the K tile as
 //      the A operand (rows = tokens, via ldmatrix) and Q^T in registers, then
@@ -34,7 +43,7 @@
 //  * Every mbarrier wait is bounded in time (about 1 s); on expiry the kernel
 //    records a code in the device status word, drains its own TMA copies and
 //    returns.
-// Split form: a partition's (m, l, o) go to a workspace and lse_reduce_kernel
+// Split form: a partition's (m, l, o) go to the workspace and lse_reduce_kernel
 // merges them; a sequence with a single partition is finished in place.
 #pragma once
 
@@ -50,10 +59,11 @@ struct DecodeParams {
     float *ws_o;                      // [B, Hq, max_parts, D]   (split form)
     float *ws_m;                      // [B, Hq, max_parts]      natural-log units
     float *ws_l;                      // [B, Hq, max_parts]
+    int *sched;                       // [2] item counter, finished-CTA counter; nullptr = round robin
     float scale_log2;                 // scale * log2(e)
     int num_seqs, num_heads, num_kv_heads, group, max_blocks;
-    int part_tokens;                  // positions per partition (multiple of 16)
-    int max_parts;                    // partitions per sequence in the grid; 1 = one pass
+    int part_tokens;                  // positions per partition (multiple of 16); 0 = one pass
+    int max_parts;                    // partitions per sequence (workspace stride); 1 = one pass
     int direct_single;                // a sequence with one partition writes `out`
 };
 
@@ -66,9 +76,14 @@ struct ReduceParams {
 };
 
 constexpr int kConsumerWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kSchedulerWarp = 5;
+constexpr int kDecodeThreads = 6 * 32;
 constexpr int kStages = 8;
 constexpr int kTileTokens = 16;
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kItemSlots = 2;
+constexpr int kChunkSlots = 4;
+constexpr int kChunkBlocks = 32;
 constexpr float kLn2 = 0.693147180559945309f;
 
 template <int D, int BS>
@@ -89,7 +104,6 @@ struct TileGeom {
     static constexpr int kTileSmem = kHalves * kPlaneSmem;
     static constexpr int kStageSmem = 2 * kTileSmem;              // K tile, then V tile
     static constexpr int kPipeSmem = kStages * kStageSmem;
-    static constexpr int kSmemBytes = kPipeSmem + 1024 /* alignment slack */ + 2 * kStages * 8 + 16;
 
     // Offset, inside a plane, of token t's 128-byte row.
     __device__ static __forceinline__ uint32_t row_offset(int t)
@@ -110,13 +124,72 @@ struct TileGeom {
     }
 };
 
-// Merge scratch (reuses the drained pipeline ring): per consumer warp, the
-// running max (log2 units), sum and accumulator of up to 16 heads.
-template <int D>
+// Per-item merge scratch: each consumer warp's running max (log2 units), sum
+// and accumulator of up to ROWS heads.
+template <int D, int ROWS>
 struct MergeScratch {
-    float o[kConsumerWarps][16][D + 4];  // +4: heads 2tq+j land in distinct banks
-    float m[kConsumerWarps][16];
-    float l[kConsumerWarps][16];
+    float o[kConsumerWarps][ROWS][D + 4];  // +4: the heads a warp writes at once land in distinct banks
+    float m[kConsumerWarps][ROWS];
+    float l[kConsumerWarps][ROWS];
+};
+
+// A work item as the scheduler publishes it.
+struct ItemInfo {
+    int s, g, part, nparts;
+    int t_begin, t_end, n_tiles;
+    int ring_base;                    // ring position of the item's first tile
+    int stop;                         // 1: no more items
+};
+
+// A run of up to 32 blocks of one item for the producer.
+struct ChunkInfo {
+    int g, n_blocks, stop, pad;
+    int phys[kChunkBlocks];
+};
+
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Named barrier over the 4 consumer warps that also ORs a predicate across them,
+// so every consumer warp takes the same decision after it.
+__device__ __forceinline__ bool consumer_bar_or(bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, 128, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
+}
+
+// Bulk copy global -> this CTA's shared memory, completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+template <int D, int BS, int MODE, int GC>
+struct DecodeSmem {
+    static constexpr int ROWS = MODE == 0 ? GC : (MODE == 1 ? 8 : 16);
+    using Geo = TileGeom<D, BS>;
+    using Merge = MergeScratch<D, ROWS>;
+    static constexpr int kMergeOff = Geo::kPipeSmem;
+    static constexpr int kQOff = (kMergeOff + (int)sizeof(Merge) + 127) & ~127;
+    static constexpr int kQBytes = ROWS * D * 2;                  // one item's query rows
+    static constexpr int kItemOff = kQOff + kItemSlots * kQBytes;
+    static constexpr int kChunkOff = kItemOff + kItemSlots * (int)sizeof(ItemInfo);
+    static constexpr int kBarOff = (kChunkOff + kChunkSlots * (int)sizeof(ChunkInfo) + 7) & ~7;
+    // barriers: full[kStages], empty[kStages], item_full, item_empty, chunk_full, chunk_empty
+    static constexpr int kNumBars = 2 * kStages + 2 * kItemSlots + 2 * kChunkSlots;
+    static constexpr int kFlagOff = kBarOff + kNumBars * 8;
+    static constexpr int kPrefixOff = kFlagOff + 16;
+    // bytes of dynamic shared memory for a launch with prefix_entries prefix ints
+    static constexpr int bytes(int prefix_entries) { return 1024 + kPrefixOff + 4 * prefix_entries; }
 };
 
 template <int D, int BS, int MODE, int GC>
@@ -128,126 +201,259 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     // MODE 1: tensor cores, up to 8 query heads per KV head (one 8-head tile).
     // MODE 2: tensor cores, up to 16 query heads per KV head (two 8-head tiles).
     using Geo = TileGeom<D, BS>;
-    static_assert(sizeof(MergeScratch<D>) <= Geo::kPipeSmem, "merge scratch must fit the ring");
+    using Lay = DecodeSmem<D, BS, MODE, GC>;
+    using Merge = typename Lay::Merge;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const base_ptr = smem_raw + (base - raw);
-    const uint32_t full_bar = base + Geo::kPipeSmem;
+    Merge *const ms = reinterpret_cast<Merge *>(base_ptr + Lay::kMergeOff);
+    ItemInfo *const items = reinterpret_cast<ItemInfo *>(base_ptr + Lay::kItemOff);
+    ChunkInfo *const chunks = reinterpret_cast<ChunkInfo *>(base_ptr + Lay::kChunkOff);
+    const uint32_t full_bar = base + Lay::kBarOff;
     const uint32_t empty_bar = full_bar + kStages * 8;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Geo::kPipeSmem + 2 * kStages * 8);
+    const uint32_t ifull_bar = empty_bar + kStages * 8;
+    const uint32_t iempty_bar = ifull_bar + kItemSlots * 8;
+    const uint32_t cfull_bar = iempty_bar + kItemSlots * 8;
+    const uint32_t cempty_bar = cfull_bar + kChunkSlots * 8;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Lay::kFlagOff);
+    int *const prefix = reinterpret_cast<int *>(base_ptr + Lay::kPrefixOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    int bid = blockIdx.x;
-    const int g = bid % p.num_kv_heads;
-    bid /= p.num_kv_heads;
-    const int s = bid % p.num_seqs;
-    const int part = bid / p.num_seqs;
+    const int G = (MODE == 0) ? GC : p.group;
+    const int B = p.num_seqs;
+    const int Hkv = p.num_kv_heads;
+    const bool split = p.max_parts > 1;
 
     if (threadIdx.x == 0) {
-#pragma unroll
         for (int i = 0; i < kStages; ++i) {
             mbar_init(full_bar + 8 * i, 1);
             mbar_init(empty_bar + 8 * i, 1);
         }
+        for (int i = 0; i < kItemSlots; ++i) {
+            mbar_init(ifull_bar + 8 * i, 1);
+            mbar_init(iempty_bar + 8 * i, 1);
+        }
+        for (int i = 0; i < kChunkSlots; ++i) {
+            mbar_init(cfull_bar + 8 * i, 1);
+            mbar_init(cempty_bar + 8 * i, 1);
+        }
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (threadIdx.x == kConsumerWarps * 32) {
+    if (threadIdx.x == kProducerWarp * 32) {
         prefetch_tensormap(&tmap_k);
         prefetch_tensormap(&tmap_v);
     }
-    __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
 
-    const int L = min(p.seq_lens[s], p.max_blocks * BS);
-    int nparts = 1;
-    int t_begin = 0, t_end = L;
-    if (p.max_parts > 1) {
-        nparts = L > 0 ? min((L + p.part_tokens - 1) / p.part_tokens, p.max_parts) : 1;
-        t_begin = part * p.part_tokens;
-        t_end = min(L, t_begin + p.part_tokens);
+    // ---- compact enumeration of the items: prefix[s] = partitions before sequence s
+    auto nparts_of = [&](int L) {
+        return (split && L > 0) ? min((L + p.part_tokens - 1) / p.part_tokens, p.max_parts) : 1;
+    };
+    __shared__ int warp_tot[kDecodeThreads / 32];
+    if (split) {
+        const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
+        const int s0 = min(B, (int)threadIdx.x * per);
+        const int s1 = min(B, s0 + per);
+        int local = 0;
+        for (int s = s0; s < s1; ++s) local += nparts_of(p.seq_lens[s]);
+        // block-wide exclusive scan of `local`
+        int incl = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        int run = incl - local;
+        for (int w = 0; w < warp; ++w) run += warp_tot[w];
+        for (int s = s0; s < s1; ++s) {
+            prefix[s] = run;
+            run += nparts_of(p.seq_lens[s]);
+        }
+        if (threadIdx.x == kDecodeThreads - 1) prefix[B] = run;
     }
-    const int G = (MODE == 0) ? GC : p.group;
-    if (part >= nparts) {  // uniform over the CTA
-        if (!p.direct_single) {
-            // partitions-only form: an empty partition reports m = -inf, l = 0, o = 0
-            for (int idx = threadIdx.x; idx < G * D; idx += kDecodeThreads) {
-                const int row = idx / D;
-                const int64_t wi = ((int64_t)s * p.num_heads + (int64_t)g * G + row) * p.max_parts + part;
-                p.ws_o[wi * D + (idx - row * D)] = 0.f;
-                if (idx - row * D == 0) {
-                    p.ws_m[wi] = -INFINITY;
-                    p.ws_l[wi] = 0.f;
+    __syncthreads();
+    const int total_sp = split ? prefix[B] : B;
+    const int total_items = total_sp * Hkv;
+
+    if (warp == kSchedulerWarp) {
+        // ------------------------------------------------------------ scheduler
+        int rr_next = blockIdx.x;
+        auto grab = [&]() -> int {
+            int v = 0;
+            if (lane == 0) {
+                if (p.sched) {
+                    v = atomicAdd(&p.sched[0], 1);
+                } else {
+                    v = rr_next;
+                    rr_next += gridDim.x;
                 }
             }
-        }
-        return;
-    }
-    const int n_tiles = t_end > t_begin ? (t_end - t_begin + kTileTokens - 1) / kTileTokens : 0;
-    const bool direct = p.direct_single && nparts == 1;
-
-    if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        const int32_t *table = p.block_tables + (int64_t)s * p.max_blocks;
-        const int first_blk = t_begin / BS;
-        const int end_blk = (t_end + BS - 1) / BS;
-        int issued = 0;
-        bool stop = false;
-        for (int cb = first_blk; cb < end_blk && !stop; cb += 32) {
-            const int nchunk = min(32, end_blk - cb);
-            const int my = lane < nchunk ? __ldg(table + cb + lane) : 0;
-            for (int j = 0; j < nchunk; j += Geo::kBlocksPerTile) {
-                int phys[Geo::kBlocksPerTile];
-#pragma unroll
-                for (int k = 0; k < Geo::kBlocksPerTile; ++k) phys[k] = __shfl_sync(0xffffffffu, my, (j + k) & 31);
-                const int valid = min(Geo::kBlocksPerTile, nchunk - j);
+            return __shfl_sync(0xffffffffu, v, 0);
+        };
+        int idx = grab();
+        int item_seq = 0, chunk_seq = 0, ring_base = 0;
+        while (true) {
+            const bool have = idx < total_items;
+            const int next_idx = have ? grab() : idx;  // one item ahead
+            // item slot
+            const int islot = item_seq % kItemSlots;
+            bool ok = true;
+            if (lane == 0) {
+                if (*abort_flag || !mbar_wait_bounded(iempty_bar + 8 * islot, ((item_seq / kItemSlots) & 1) ^ 1)) {
+                    if (!*abort_flag) record_timeout(kTimeoutEmptyBarrier);
+                    *abort_flag = 1;
+                    ok = false;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            ItemInfo it = {};
+            int first_blk = 0, end_blk = 0;
+            if (have) {
+                const int sp = idx / Hkv;
+                it.g = idx - sp * Hkv;
+                if (split) {
+                    int lo = 0, hi = B;  // largest s with prefix[s] <= sp
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if (prefix[mid] <= sp) lo = mid; else hi = mid;
+                    }
+                    it.s = lo;
+                    it.part = sp - prefix[lo];
+                    it.nparts = prefix[lo + 1] - prefix[lo];
+                } else {
+                    it.s = sp;
+                    it.part = 0;
+                    it.nparts = 1;
+                }
+                const int L = min(p.seq_lens[it.s], p.max_blocks * BS);
+                it.t_begin = split ? it.part * p.part_tokens : 0;
+                it.t_end = split ? min(L, it.t_begin + p.part_tokens) : L;
+                it.n_tiles = it.t_end > it.t_begin ? (it.t_end - it.t_begin + kTileTokens - 1) / kTileTokens : 0;
+                it.ring_base = ring_base;
+                it.stop = 0;
+                first_blk = it.t_begin / BS;
+                end_blk = it.n_tiles > 0 ? (it.t_end + BS - 1) / BS : first_blk;
+            } else {
+                it.stop = 1;
+            }
+            if (lane == 0) {
+                items[islot] = it;
+                const uint32_t bar = ifull_bar + 8 * islot;
+                if (!it.stop) {
+                    const uint32_t qbytes = (uint32_t)(G * D * 2);
+                    mbar_arrive_expect_tx(bar, qbytes);
+                    bulk_load(base + Lay::kQOff + islot * Lay::kQBytes,
+                              p.query + ((int64_t)it.s * p.num_heads + (int64_t)it.g * G) * D, qbytes, bar);
+                } else {
+                    mbar_arrive(bar);
+                }
+            }
+            // chunks of the item's block table (and a stop marker after the last item)
+            for (int cb = first_blk; ok && (cb < end_blk || it.stop); cb += kChunkBlocks) {
+                const int cslot = chunk_seq % kChunkSlots;
+                bool cok = true;
                 if (lane == 0) {
-                    const int stage = issued % kStages;
-                    const uint32_t parity = ((issued / kStages) & 1) ^ 1;
-                    if (*abort_flag) {
-                        stop = true;
-                    } else if (!mbar_wait_bounded(empty_bar + 8 * stage, parity)) {
-                        record_timeout(kTimeoutEmptyBarrier);
+                    if (*abort_flag ||
+                        !mbar_wait_bounded(cempty_bar + 8 * cslot, ((chunk_seq / kChunkSlots) & 1) ^ 1)) {
+                        if (!*abort_flag) record_timeout(kTimeoutEmptyBarrier);
                         *abort_flag = 1;
-                        stop = true;
-                    } else {
-                        const uint32_t kdst = base + stage * Geo::kStageSmem;
-                        const uint32_t vdst = kdst + Geo::kTileSmem;
-                        const uint32_t bar = full_bar + 8 * stage;
-                        mbar_arrive_expect_tx(bar, (uint32_t)(valid * Geo::kBlkBytes * 2));
-#pragma unroll
-                        for (int k = 0; k < Geo::kBlocksPerTile; ++k) {
-                            if (k < valid) {
-#pragma unroll
-                                for (int h = 0; h < Geo::kHalves; ++h) {
-                                    tma_load_4d(kdst + Geo::box_offset(k, h), &tmap_k, bar, 0, h, g, phys[k] * BS);
-                                    tma_load_4d(vdst + Geo::box_offset(k, h), &tmap_v, bar, 0, h, g, phys[k] * BS);
-                                }
-                            }
-                        }
-                        ++issued;
+                        cok = false;
                     }
                 }
-                stop = __shfl_sync(0xffffffffu, stop, 0);
-                if (stop) break;
+                cok = __shfl_sync(0xffffffffu, cok, 0);
+                if (!cok) {
+                    ok = false;
+                    break;
+                }
+                ChunkInfo *c = chunks + cslot;
+                if (it.stop) {
+                    if (lane == 0) c->stop = 1;
+                } else {
+                    const int n = min(kChunkBlocks, end_blk - cb);
+                    c->phys[lane] = lane < n ? __ldg(p.block_tables + (int64_t)it.s * p.max_blocks + cb + lane) : 0;
+                    if (lane == 0) {
+                        c->g = it.g;
+                        c->n_blocks = n;
+                        c->stop = 0;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(cfull_bar + 8 * cslot);
+                ++chunk_seq;
+                if (it.stop) break;
             }
+            if (!ok || it.stop) break;
+            ring_base += it.n_tiles;
+            ++item_seq;
+            idx = next_idx;
         }
-        // On an abort, wait for the copies already in flight before the ring is
-        // reused or the CTA exits.
-        if (lane == 0 && *abort_flag && issued > 0) {
-            for (int st = 0; st < kStages && st < issued; ++st) {
-                const int last = issued - 1 - ((issued - 1 - st) % kStages);
+    } else if (warp == kProducerWarp) {
+        // ------------------------------------------------------------- producer
+        int chunk_seq = 0, ring = 0;
+        while (true) {
+            const int cslot = chunk_seq % kChunkSlots;
+            bool ok = true;
+            if (lane == 0 && (*abort_flag || !mbar_wait_bounded(cfull_bar + 8 * cslot, (chunk_seq / kChunkSlots) & 1))) {
+                if (!*abort_flag) record_timeout(kTimeoutFullBarrier);
+                *abort_flag = 1;
+                ok = false;
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            const ChunkInfo *c = chunks + cslot;
+            if (c->stop) break;
+            if (lane == 0) {
+                const int n = c->n_blocks;
+                const int g = c->g;
+                for (int j = 0; j < n; j += Geo::kBlocksPerTile) {
+                    const int valid = min(Geo::kBlocksPerTile, n - j);
+                    const int stage = ring % kStages;
+                    if (*abort_flag || !mbar_wait_bounded(empty_bar + 8 * stage, ((ring / kStages) & 1) ^ 1)) {
+                        if (!*abort_flag) record_timeout(kTimeoutEmptyBarrier);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t kdst = base + stage * Geo::kStageSmem;
+                    const uint32_t vdst = kdst + Geo::kTileSmem;
+                    const uint32_t bar = full_bar + 8 * stage;
+                    mbar_arrive_expect_tx(bar, (uint32_t)(valid * Geo::kBlkBytes * 2));
+#pragma unroll
+                    for (int k = 0; k < Geo::kBlocksPerTile; ++k) {
+                        if (k < valid) {
+                            const int row = c->phys[j + k] * BS;
+#pragma unroll
+                            for (int h = 0; h < Geo::kHalves; ++h) {
+                                tma_load_4d(kdst + Geo::box_offset(k, h), &tmap_k, bar, 0, h, g, row);
+                                tma_load_4d(vdst + Geo::box_offset(k, h), &tmap_v, bar, 0, h, g, row);
+                            }
+                        }
+                    }
+                    ++ring;
+                }
+                if (ok) mbar_arrive(cempty_bar + 8 * cslot);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            ring = __shfl_sync(0xffffffffu, ring, 0);
+            if (!ok) break;
+            ++chunk_seq;
+        }
+        // On an abort, wait for the copies already in flight before the CTA exits.
+        if (lane == 0 && *abort_flag && ring > 0) {
+            for (int st = 0; st < kStages && st < ring; ++st) {
+                const int last = ring - 1 - ((ring - 1 - st) % kStages);
                 if (!mbar_wait_bounded(full_bar + 8 * st, (last / kStages) & 1)) record_timeout(kTimeoutDrain);
             }
         }
     } else {
-        // ----------------------------------------------------------- consumers
-        MergeScratch<D> *ms = reinterpret_cast<MergeScratch<D> *>(base_ptr);
-        const int64_t q_off = ((int64_t)s * p.num_heads + (int64_t)g * G) * D;
-
+        // ------------------------------------------------------------ consumers
         // Zero the V rows of tokens [valid, 16) so masked positions contribute
         // exactly 0 (stale or NaN data is never multiplied).
         auto zero_tail = [&](uint32_t vt, int valid) {
@@ -260,311 +466,351 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             }
             __syncwarp();
         };
-
-        if constexpr (MODE == 0) {
-            constexpr int CPT = D / 8;              // lanes per token in the dot products
-            constexpr int TPP = 32 / CPT;           // tokens per pass
-            constexpr int PASSES = kTileTokens / TPP;
-            constexpr int DPL = D / 32;             // accumulator columns per lane
-            const int qc = lane % CPT;
-            const int qt = lane / CPT;
-            float q[GC][8];
-#pragma unroll
-            for (int h = 0; h < GC; ++h) {
-                const uint4 raw_q = *reinterpret_cast<const uint4 *>(p.query + q_off + (int64_t)h * D + qc * 8);
-                const uint32_t w[4] = {raw_q.x, raw_q.y, raw_q.z, raw_q.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = unpack_bf16x2(w[e]);
-                    q[h][2 * e] = f.x * p.scale_log2;
-                    q[h][2 * e + 1] = f.y * p.scale_log2;
-                }
+        // Wait for a ring stage; false (and the abort flag set) if the wait gave up.
+        auto wait_full = [&](int ring) -> bool {
+            if (*abort_flag) return false;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar + 8 * (ring % kStages), (ring / kStages) & 1));
+            if (!ok && lane == 0) {
+                record_timeout(kTimeoutFullBarrier);
+                *abort_flag = 1;
             }
-            float o[GC][DPL];
-            float m[GC], l[GC];
-#pragma unroll
-            for (int h = 0; h < GC; ++h) {
-                m[h] = -INFINITY;
-                l[h] = 0.f;
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
-            }
-            for (int tile = warp; tile < n_tiles; tile += kConsumerWarps) {
-                const int stage = tile % kStages;
-                if (*abort_flag) break;
-                const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar + 8 * stage, (tile / kStages) & 1));
-                if (!ok) {
-                    if (lane == 0) { record_timeout(kTimeoutFullBarrier); *abort_flag = 1; }
-                    break;
-                }
-                const uint32_t kt = base + stage * Geo::kStageSmem;
-                const uint32_t vt = kt + Geo::kTileSmem;
-                const int valid = min(kTileTokens, t_end - (t_begin + tile * kTileTokens));
-                if (valid < kTileTokens) zero_tail(vt, valid);
+            return ok;
+        };
+        auto release = [&](int ring, int valid) {
+            if (valid < kTileTokens) fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar + 8 * (ring % kStages));
+        };
 
-                float sv[GC][PASSES];
+        int item_seq = 0;
+        while (true) {
+            const int islot = item_seq % kItemSlots;
+            bool ok = !*abort_flag;
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(ifull_bar + 8 * islot, (item_seq / kItemSlots) & 1));
+            if (!ok && lane == 0 && !*abort_flag) {
+                record_timeout(kTimeoutFullBarrier);
+                *abort_flag = 1;
+            }
+            // all four consumer warps leave together, or none does
+            if (consumer_bar_or(!ok || *abort_flag)) break;
+            const ItemInfo it = items[islot];
+            if (it.stop) break;
+            const uint8_t *qsm = base_ptr + Lay::kQOff + islot * Lay::kQBytes;
+
+            if constexpr (MODE == 0) {
+                constexpr int CPT = D / 8;              // lanes per token in the dot products
+                constexpr int TPP = 32 / CPT;           // tokens per pass
+                constexpr int PASSES = kTileTokens / TPP;
+                constexpr int DPL = D / 32;             // accumulator columns per lane
+                const int qc = lane % CPT;
+                const int qt = lane / CPT;
+                float q[GC][8];
 #pragma unroll
-                for (int j = 0; j < PASSES; ++j) {
-                    const int tok = j * TPP + qt;
-                    const uint4 kr = *reinterpret_cast<const uint4 *>(base_ptr + (kt - base) + Geo::chunk_offset(tok, qc));
-                    const uint32_t w[4] = {kr.x, kr.y, kr.z, kr.w};
-                    float kf[8];
+                for (int h = 0; h < GC; ++h) {
+                    const uint4 rq = *reinterpret_cast<const uint4 *>(qsm + (h * D + qc * 8) * 2);
+                    const uint32_t w[4] = {rq.x, rq.y, rq.z, rq.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 f = unpack_bf16x2(w[e]);
-                        kf[2 * e] = f.x;
-                        kf[2 * e + 1] = f.y;
-                    }
-#pragma unroll
-                    for (int h = 0; h < GC; ++h) {
-                        float dot = 0.f;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) dot = fmaf(q[h][e], kf[e], dot);
-#pragma unroll
-                        for (int off = CPT / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-                        sv[h][j] = tok < valid ? dot : -INFINITY;
+                        q[h][2 * e] = f.x * p.scale_log2;
+                        q[h][2 * e + 1] = f.y * p.scale_log2;
                     }
                 }
-                float pr[GC][PASSES];
+                float o[GC][DPL];
+                float m[GC], l[GC];
 #pragma unroll
                 for (int h = 0; h < GC; ++h) {
-                    float mx = sv[h][0];
+                    m[h] = -INFINITY;
+                    l[h] = 0.f;
 #pragma unroll
-                    for (int j = 1; j < PASSES; ++j) mx = fmaxf(mx, sv[h][j]);
-#pragma unroll
-                    for (int off = CPT; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                    const float m_new = fmaxf(m[h], mx);
-                    const float corr = exp2f(m[h] - m_new);
-                    m[h] = m_new;
-                    float sum = 0.f;
-#pragma unroll
-                    for (int j = 0; j < PASSES; ++j) {
-                        pr[h][j] = exp2f(sv[h][j] - m_new);
-                        sum += pr[h][j];
-                    }
-#pragma unroll
-                    for (int off = CPT; off < 32; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-                    l[h] = l[h] * corr + sum;
-#pragma unroll
-                    for (int e = 0; e < DPL; ++e) o[h][e] *= corr;
+                    for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
                 }
+                for (int j = warp; j < it.n_tiles; j += kConsumerWarps) {
+                    const int ring = it.ring_base + j;
+                    if (!wait_full(ring)) break;
+                    const uint32_t kt = base + (ring % kStages) * Geo::kStageSmem;
+                    const uint32_t vt = kt + Geo::kTileSmem;
+                    const int valid = min(kTileTokens, it.t_end - (it.t_begin + j * kTileTokens));
+                    if (valid < kTileTokens) zero_tail(vt, valid);
+
+                    float sv[GC][PASSES];
 #pragma unroll
-                for (int tok = 0; tok < kTileTokens; ++tok) {
-                    const int c = (DPL * lane) >> 3;
-                    const uint32_t off = Geo::chunk_offset(tok, c) + ((DPL * lane) & 7) * 2;
-                    float vf[DPL];
-                    if constexpr (DPL == 4) {
-                        const uint2 vr = *reinterpret_cast<const uint2 *>(base_ptr + (vt - base) + off);
-                        const float2 a = unpack_bf16x2(vr.x), b = unpack_bf16x2(vr.y);
-                        vf[0] = a.x; vf[1] = a.y; vf[2] = b.x; vf[3] = b.y;
-                    } else {
-                        const uint32_t vr = *reinterpret_cast<const uint32_t *>(base_ptr + (vt - base) + off);
-                        const float2 a = unpack_bf16x2(vr);
-                        vf[0] = a.x; vf[1] = a.y;
+                    for (int jj = 0; jj < PASSES; ++jj) {
+                        const int tok = jj * TPP + qt;
+                        const uint4 kr = *reinterpret_cast<const uint4 *>(base_ptr + (kt - base) + Geo::chunk_offset(tok, qc));
+                        const uint32_t w[4] = {kr.x, kr.y, kr.z, kr.w};
+                        float kf[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = unpack_bf16x2(w[e]);
+                            kf[2 * e] = f.x;
+                            kf[2 * e + 1] = f.y;
+                        }
+#pragma unroll
+                        for (int h = 0; h < GC; ++h) {
+                            float dot = 0.f;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) dot = fmaf(q[h][e], kf[e], dot);
+#pragma unroll
+                            for (int off = CPT / 2; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+                            sv[h][jj] = tok < valid ? dot : -INFINITY;
+                        }
                     }
+                    float pr[GC][PASSES];
 #pragma unroll
                     for (int h = 0; h < GC; ++h) {
-                        const float pt = __shfl_sync(0xffffffffu, pr[h][tok / TPP], (tok % TPP) * CPT);
+                        float mx = sv[h][0];
 #pragma unroll
-                        for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(pt, vf[e], o[h][e]);
+                        for (int jj = 1; jj < PASSES; ++jj) mx = fmaxf(mx, sv[h][jj]);
+#pragma unroll
+                        for (int off = CPT; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                        const float m_new = fmaxf(m[h], mx);
+                        const float corr = exp2f(m[h] - m_new);
+                        m[h] = m_new;
+                        float sum = 0.f;
+#pragma unroll
+                        for (int jj = 0; jj < PASSES; ++jj) {
+                            pr[h][jj] = exp2f(sv[h][jj] - m_new);
+                            sum += pr[h][jj];
+                        }
+#pragma unroll
+                        for (int off = CPT; off < 32; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                        l[h] = l[h] * corr + sum;
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) o[h][e] *= corr;
+                    }
+#pragma unroll
+                    for (int tok = 0; tok < kTileTokens; ++tok) {
+                        const int c = (DPL * lane) >> 3;
+                        const uint32_t off = Geo::chunk_offset(tok, c) + ((DPL * lane) & 7) * 2;
+                        float vf[DPL];
+                        if constexpr (DPL == 4) {
+                            const uint2 vr = *reinterpret_cast<const uint2 *>(base_ptr + (vt - base) + off);
+                            const float2 a = unpack_bf16x2(vr.x), b = unpack_bf16x2(vr.y);
+                            vf[0] = a.x; vf[1] = a.y; vf[2] = b.x; vf[3] = b.y;
+                        } else {
+                            const uint32_t vr = *reinterpret_cast<const uint32_t *>(base_ptr + (vt - base) + off);
+                            const float2 a = unpack_bf16x2(vr);
+                            vf[0] = a.x; vf[1] = a.y;
+                        }
+#pragma unroll
+                        for (int h = 0; h < GC; ++h) {
+                            const float pt = __shfl_sync(0xffffffffu, pr[h][tok / TPP], (tok % TPP) * CPT);
+#pragma unroll
+                            for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(pt, vf[e], o[h][e]);
+                        }
+                    }
+                    release(ring, valid);
+                }
+#pragma unroll
+                for (int h = 0; h < GC; ++h) {
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) ms->o[warp][h][DPL * lane + e] = o[h][e];
+                    if (lane == 0) {
+                        ms->m[warp][h] = m[h];
+                        ms->l[warp][h] = l[h];
                     }
                 }
-                if (valid < kTileTokens) fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar + 8 * stage);
-            }
-            __syncthreads();  // ring drained (all consumers and the producer are past it)
-#pragma unroll
-            for (int h = 0; h < GC; ++h) {
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) ms->o[warp][h][DPL * lane + e] = o[h][e];
-                if (lane == 0) {
-                    ms->m[warp][h] = m[h];
-                    ms->l[warp][h] = l[h];
-                }
-            }
-        } else {
-            // Tensor cores, transposed form: S^T[16 tokens x 8*NH heads] = K Q^T,
-            // then O^T[D x heads] += V^T P^T.  Tokens are the MMA's M dimension,
-            // so no accumulator row is wasted when G <= 8; P^T is taken from the
-            // S^T accumulators by an in-register 8x8 transpose (movmatrix).
-            constexpr int NH = (MODE == 2) ? 2 : 1;  // 8-head column tiles
-            constexpr int KSTEPS = D / 16;           // k-steps of S^T = K Q^T
-            constexpr int MT = D / 16;               // 16-row d tiles of O^T
-            const int gq = lane >> 2;                // MMA groupID
-            const int tq = lane & 3;                 // MMA thread-in-group
-            // B operand of S^T = K Q^T: b0 = Q[head][d 16kk+2tq..+1], b1 = Q[head][d 16kk+8+2tq..+1]
-            uint32_t qb[NH][KSTEPS][2];
-#pragma unroll
-            for (int nh = 0; nh < NH; ++nh) {
-                const int head = nh * 8 + gq;
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk) {
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int col = kk * 16 + hh * 8 + tq * 2;
-                        qb[nh][kk][hh] = head < G
-                                             ? *reinterpret_cast<const uint32_t *>(p.query + q_off + (int64_t)head * D + col)
-                                             : 0u;
-                    }
-                }
-            }
-            float o[MT][NH][4];
-            float m[NH][2], l[NH][2];
-#pragma unroll
-            for (int nh = 0; nh < NH; ++nh) {
-                m[nh][0] = m[nh][1] = -INFINITY;
-                l[nh][0] = l[nh][1] = 0.f;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) o[mt][nh][0] = o[mt][nh][1] = o[mt][nh][2] = o[mt][nh][3] = 0.f;
-            }
-            // ldmatrix lane roles: K as the A operand (rows = tokens), V^T as the A
-            // operand through the transposing load (rows = d)
-            const int ktok = (lane & 7) + (((lane >> 3) & 1) << 3);
-            const int kpar = lane >> 4;
-            const int vtok = (lane & 7) + ((lane >> 4) << 3);
-            const int vpar = (lane >> 3) & 1;
-
-            for (int tile = warp; tile < n_tiles; tile += kConsumerWarps) {
-                const int stage = tile % kStages;
-                if (*abort_flag) break;
-                const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar + 8 * stage, (tile / kStages) & 1));
-                if (!ok) {
-                    if (lane == 0) { record_timeout(kTimeoutFullBarrier); *abort_flag = 1; }
-                    break;
-                }
-                const uint32_t kt = base + stage * Geo::kStageSmem;
-                const uint32_t vt = kt + Geo::kTileSmem;
-                const int valid = min(kTileTokens, t_end - (t_begin + tile * kTileTokens));
-                if (valid < kTileTokens) zero_tail(vt, valid);
-
-                // S^T[token][head] = K Q^T
-                float sc[NH][4];
-#pragma unroll
-                for (int nh = 0; nh < NH; ++nh) sc[nh][0] = sc[nh][1] = sc[nh][2] = sc[nh][3] = 0.f;
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk) {
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
-#pragma unroll
-                    for (int nh = 0; nh < NH; ++nh) mma_bf16_16816(sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
-                }
-                // online softmax per head column; this lane holds tokens gq and gq+8
-                // of heads 2tq and 2tq+1.  P enters the PV product as a bf16 high
-                // part plus a bf16 residual (two MMAs): ~16 significant bits.
-                const bool in0 = gq < valid, in1 = gq + 8 < valid;
-                uint32_t bh[NH][2], bl[NH][2];
+            } else {
+                // Tensor cores, transposed form: S^T[16 tokens x 8*NH heads] = K Q^T,
+                // then O^T[D x heads] += V^T P^T.  Tokens are the MMA's M dimension,
+                // so no accumulator row is wasted when G <= 8; P^T is taken from the
+                // S^T accumulators by an in-register 8x8 transpose (movmatrix).
+                constexpr int NH = (MODE == 2) ? 2 : 1;  // 8-head column tiles
+                constexpr int KSTEPS = D / 16;           // k-steps of S^T = K Q^T
+                constexpr int MT = D / 16;               // 16-row d tiles of O^T
+                const int gq = lane >> 2;                // MMA groupID
+                const int tq = lane & 3;                 // MMA thread-in-group
+                // B operand of S^T = K Q^T: b0 = Q[head][d 16kk+2tq..+1], b1 = Q[head][d 16kk+8+2tq..+1]
+                uint32_t qb[NH][KSTEPS][2];
 #pragma unroll
                 for (int nh = 0; nh < NH; ++nh) {
-                    float pr[2][2];  // [head j][token row]
+                    const int head = nh * 8 + gq;
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const float x0 = in0 ? sc[nh][j] * p.scale_log2 : -INFINITY;
-                        const float x1 = in1 ? sc[nh][2 + j] * p.scale_log2 : -INFINITY;
-                        float mx = fmaxf(x0, x1);
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                        const float m_new = fmaxf(m[nh][j], mx);
-                        const float corr = exp2f(m[nh][j] - m_new);
-                        m[nh][j] = m_new;
-                        pr[j][0] = exp2f(x0 - m_new);
-                        pr[j][1] = exp2f(x1 - m_new);
-                        l[nh][j] = l[nh][j] * corr + (pr[j][0] + pr[j][1]);
+                    for (int kk = 0; kk < KSTEPS; ++kk) {
 #pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            o[mt][nh][j] *= corr;
-                            o[mt][nh][2 + j] *= corr;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int col = kk * 16 + hh * 8 + tq * 2;
+                            qb[nh][kk][hh] = head < G ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
                         }
                     }
-#pragma unroll
-                    for (int row = 0; row < 2; ++row) {
-                        const uint32_t hi = pack_bf16x2(pr[0][row], pr[1][row]);
-                        const float2 hf = unpack_bf16x2(hi);
-                        const uint32_t lo = pack_bf16x2(pr[0][row] - hf.x, pr[1][row] - hf.y);
-                        bh[nh][row] = movmatrix_trans(hi);
-                        bl[nh][row] = movmatrix_trans(lo);
-                    }
                 }
-                // O^T[d][head] += V^T P^T
+                float o[MT][NH][4];
+                float m[NH][2], l[NH][2];
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * mt + vpar), a0, a1, a2, a3);
+                for (int nh = 0; nh < NH; ++nh) {
+                    m[nh][0] = m[nh][1] = -INFINITY;
+                    l[nh][0] = l[nh][1] = 0.f;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) o[mt][nh][0] = o[mt][nh][1] = o[mt][nh][2] = o[mt][nh][3] = 0.f;
+                }
+                // ldmatrix lane roles: K as the A operand (rows = tokens), V^T as the A
+                // operand through the transposing load (rows = d)
+                const int ktok = (lane & 7) + (((lane >> 3) & 1) << 3);
+                const int kpar = lane >> 4;
+                const int vtok = (lane & 7) + ((lane >> 4) << 3);
+                const int vpar = (lane >> 3) & 1;
+
+                for (int j = warp; j < it.n_tiles; j += kConsumerWarps) {
+                    const int ring = it.ring_base + j;
+                    if (!wait_full(ring)) break;
+                    const uint32_t kt = base + (ring % kStages) * Geo::kStageSmem;
+                    const uint32_t vt = kt + Geo::kTileSmem;
+                    const int valid = min(kTileTokens, it.t_end - (it.t_begin + j * kTileTokens));
+                    if (valid < kTileTokens) zero_tail(vt, valid);
+
+                    // S^T[token][head] = K Q^T
+                    float sc[NH][4];
+#pragma unroll
+                    for (int nh = 0; nh < NH; ++nh) sc[nh][0] = sc[nh][1] = sc[nh][2] = sc[nh][3] = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < KSTEPS; ++kk) {
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
+#pragma unroll
+                        for (int nh = 0; nh < NH; ++nh) mma_bf16_16816(sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                    }
+                    // online softmax per head column; this lane holds tokens gq and gq+8
+                    // of heads 2tq and 2tq+1.  P enters the PV product as a bf16 high
+                    // part plus a bf16 residual (two MMAs): ~16 significant bits.
+                    const bool in0 = gq < valid, in1 = gq + 8 < valid;
+                    uint32_t bh[NH][2], bl[NH][2];
 #pragma unroll
                     for (int nh = 0; nh < NH; ++nh) {
-                        mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
-                        mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
-                    }
-                }
-                if (valid < kTileTokens) fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar + 8 * stage);
-            }
+                        float pr[2][2];  // [head j][token row]
 #pragma unroll
-            for (int nh = 0; nh < NH; ++nh) {
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const float x0 = in0 ? sc[nh][jj] * p.scale_log2 : -INFINITY;
+                            const float x1 = in1 ? sc[nh][2 + jj] * p.scale_log2 : -INFINITY;
+                            float mx = fmaxf(x0, x1);
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                            const float m_new = fmaxf(m[nh][jj], mx);
+                            const float corr = exp2f(m[nh][jj] - m_new);
+                            m[nh][jj] = m_new;
+                            pr[jj][0] = exp2f(x0 - m_new);
+                            pr[jj][1] = exp2f(x1 - m_new);
+                            l[nh][jj] = l[nh][jj] * corr + (pr[jj][0] + pr[jj][1]);
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    l[nh][j] += __shfl_xor_sync(0xffffffffu, l[nh][j], 4);
-                    l[nh][j] += __shfl_xor_sync(0xffffffffu, l[nh][j], 8);
-                    l[nh][j] += __shfl_xor_sync(0xffffffffu, l[nh][j], 16);
-                }
-            }
-            __syncthreads();  // ring drained
-#pragma unroll
-            for (int nh = 0; nh < NH; ++nh) {
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int head = nh * 8 + 2 * tq + j;
-                    if (head < G) {
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            ms->o[warp][head][mt * 16 + gq] = o[mt][nh][j];
-                            ms->o[warp][head][mt * 16 + gq + 8] = o[mt][nh][2 + j];
+                            for (int mt = 0; mt < MT; ++mt) {
+                                o[mt][nh][jj] *= corr;
+                                o[mt][nh][2 + jj] *= corr;
+                            }
                         }
-                        if (gq == 0) {
-                            ms->m[warp][head] = m[nh][j];
-                            ms->l[warp][head] = l[nh][j];
+#pragma unroll
+                        for (int row = 0; row < 2; ++row) {
+                            const uint32_t hi = pack_bf16x2(pr[0][row], pr[1][row]);
+                            const float2 hf = unpack_bf16x2(hi);
+                            const uint32_t lo = pack_bf16x2(pr[0][row] - hf.x, pr[1][row] - hf.y);
+                            bh[nh][row] = movmatrix_trans(hi);
+                            bl[nh][row] = movmatrix_trans(lo);
                         }
                     }
+                    // O^T[d][head] += V^T P^T
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * mt + vpar), a0, a1, a2, a3);
+#pragma unroll
+                        for (int nh = 0; nh < NH; ++nh) {
+                            mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
+                            mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
+                        }
+                    }
+                    release(ring, valid);
+                }
+#pragma unroll
+                for (int nh = 0; nh < NH; ++nh) {
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        l[nh][jj] += __shfl_xor_sync(0xffffffffu, l[nh][jj], 4);
+                        l[nh][jj] += __shfl_xor_sync(0xffffffffu, l[nh][jj], 8);
+                        l[nh][jj] += __shfl_xor_sync(0xffffffffu, l[nh][jj], 16);
+                    }
+                }
+#pragma unroll
+                for (int nh = 0; nh < NH; ++nh) {
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int head = nh * 8 + 2 * tq + jj;
+                        if (head < G) {
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt) {
+                                ms->o[warp][head][mt * 16 + gq] = o[mt][nh][jj];
+                                ms->o[warp][head][mt * 16 + gq + 8] = o[mt][nh][2 + jj];
+                            }
+                            if (gq == 0) {
+                                ms->m[warp][head] = m[nh][jj];
+                                ms->l[warp][head] = l[nh][jj];
+                            }
+                        }
+                    }
                 }
             }
+            consumer_bar();  // every warp's state is in the merge scratch
+            // ---- merge the four warps of this item (after an abort the values are
+            // meaningless but harmless; the next item check stops every warp)
+            const bool direct = p.direct_single && it.nparts == 1;
+            for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+                const int row = idx / D;
+                const int d = idx - row * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->m[w][row]);
+                float num = 0.f, den = 0.f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        const float mw = ms->m[w][row];
+                        if (mw != -INFINITY) {
+                            const float c = exp2f(mw - M);
+                            num = fmaf(c, ms->o[w][row][d], num);
+                            den = fmaf(c, ms->l[w][row], den);
+                        }
+                    }
+                }
+                const int64_t hrow = (int64_t)it.s * p.num_heads + (int64_t)it.g * G + row;
+                if (direct) {
+                    p.out[hrow * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+                } else {
+                    const int64_t wi = hrow * p.max_parts + it.part;
+                    p.ws_o[wi * D + d] = num;
+                    if (d == 0) {
+                        p.ws_m[wi] = M == -INFINITY ? -INFINITY : M * kLn2;
+                        p.ws_l[wi] = den;
+                    }
+                }
+            }
+            consumer_bar();  // merge scratch and the item slot may be reused
+            if (threadIdx.x == 0) mbar_arrive(iempty_bar + 8 * islot);
+            ++item_seq;
         }
     }
-    if (warp == kConsumerWarps) __syncthreads();  // pairs with the consumers' "ring drained"
-    __syncthreads();                              // merge scratch written
 
-    // ------------------------------------------------ merge the four warps
-    if (*abort_flag) return;
-    const MergeScratch<D> *ms = reinterpret_cast<const MergeScratch<D> *>(base_ptr);
-    for (int idx = threadIdx.x; idx < G * D; idx += kDecodeThreads) {
-        const int row = idx / D;
-        const int d = idx - row * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->m[w][row]);
-        float num = 0.f, den = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float mw = ms->m[w][row];
-                if (mw != -INFINITY) {
-                    const float c = exp2f(mw - M);
-                    num = fmaf(c, ms->o[w][row][d], num);
-                    den = fmaf(c, ms->l[w][row], den);
-                }
-            }
+    // Partitions-only form: partitions that hold no position (past the end of
+    // their sequence) report m = -inf, l = 0, o = 0.  Grid-strided over all
+    // (sequence, head, partition) triples, after the CTA's items.
+    if (split && !p.direct_single) {
+        const int64_t triples = (int64_t)B * p.num_heads * p.max_parts;
+        for (int64_t t = (int64_t)blockIdx.x * kDecodeThreads + threadIdx.x; t < triples;
+             t += (int64_t)gridDim.x * kDecodeThreads) {
+            const int part = (int)(t % p.max_parts);
+            const int s = (int)(t / ((int64_t)p.num_heads * p.max_parts));
+            if (part < prefix[s + 1] - prefix[s]) continue;
+            p.ws_m[t] = -INFINITY;
+            p.ws_l[t] = 0.f;
+            for (int d = 0; d < D; ++d) p.ws_o[t * D + d] = 0.f;
         }
-        const int64_t hrow = (int64_t)s * p.num_heads + (int64_t)g * G + row;
-        if (direct) {
-            p.out[hrow * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
-        } else {
-            const int64_t wi = hrow * p.max_parts + part;
-            p.ws_o[wi * D + d] = num;
-            if (d == 0) {
-                p.ws_m[wi] = M == -INFINITY ? -INFINITY : M * kLn2;
-                p.ws_l[wi] = den;
-            }
+    }
+
+    __syncthreads();
+    // The last CTA to finish leaves the scheduler counters at zero for the next launch.
+    if (threadIdx.x == 0 && p.sched) {
+        __threadfence();
+        if (atomicAdd(&p.sched[1], 1) == (int)gridDim.x - 1) {
+            atomicExch(&p.sched[0], 0);
+            atomicExch(&p.sched[1], 0);
         }
     }
 }

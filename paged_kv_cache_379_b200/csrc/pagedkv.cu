@@ -1,9 +1,12 @@
 // pagedkv.cu -- the C ABI of libpagedkv.so (declared in include/pagedkv.h):
 // argument checks, TMA tensor-map encoding, kernel selection and launch.
 // The kernels themselves are in cache_ops.cuh and decode.cuh.
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <mutex>
+#include <tuple>
+#include <vector>
 
 #include "cache_ops.cuh"
 #include "common.cuh"
@@ -59,30 +62,55 @@ static int make_cache_map(CUtensorMap *map, const void *cache, int64_t num_block
 
 // --------------------------------------------------------------- decode launch
 
-// Sets the dynamic shared-memory limit of a kernel once per device.
-template <typename K>
-static int ensure_smem(K kernel, size_t bytes, std::atomic<uint64_t> &done)
+// Raises a kernel's dynamic shared-memory limit (per device) when a launch
+// needs more than was set before.
+static int ensure_smem(const void *kernel, size_t bytes)
 {
+    static std::mutex mu;
+    static std::vector<std::tuple<const void *, int, size_t>> done;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return check_cuda(e);
-    const uint64_t bit = 1ull << (dev & 63);
-    if (done.load(std::memory_order_acquire) & bit) return PA_OK;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto &t : done)
+        if (std::get<0>(t) == kernel && std::get<1>(t) == dev && std::get<2>(t) >= bytes) return PA_OK;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return check_cuda(e);
-    done.fetch_or(bit, std::memory_order_acq_rel);
+    done.emplace_back(kernel, dev, bytes);
     return PA_OK;
 }
 
+static int sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const int slot = dev & 63;
+    int n = cache[slot].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[slot].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// Persistent launch: (resident CTAs per SM) x (SM count) CTAs, at most one per item.
 template <int D, int BS, int MODE, int GC>
-static int launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int64_t grid,
+static int launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int64_t max_items,
                            cudaStream_t st)
 {
-    static std::atomic<uint64_t> smem_done{0};
+    using Lay = DecodeSmem<D, BS, MODE, GC>;
     auto kernel = paged_decode_kernel<D, BS, MODE, GC>;
-    constexpr size_t smem = TileGeom<D, BS>::kSmemBytes;
-    int rc = ensure_smem(kernel, smem, smem_done);
+    const int prefix_entries = p.max_parts > 1 ? p.num_seqs + 1 : 0;
+    const size_t smem = (size_t)Lay::bytes(prefix_entries);
+    if (smem > 227 * 1024) return PA_ERR_BAD_SHAPE;  // too many sequences for the split form
+    int rc = ensure_smem(reinterpret_cast<const void *>(kernel), smem);
     if (rc != PA_OK) return rc;
+    int occ = 0;
+    rc = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kDecodeThreads, smem));
+    if (rc != PA_OK) return rc;
+    const int sms = sm_count();
+    if (occ < 1 || sms < 1) return check_cuda(cudaErrorInvalidConfiguration);
+    const int64_t grid = std::min<int64_t>(max_items, (int64_t)occ * sms);
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kDecodeThreads), smem, st, p, tk, tv);
 }
 
@@ -146,6 +174,7 @@ static int check_decode_args(const DecodeArgs &a, bool need_out)
 }
 
 static constexpr int kDefaultPartition = 512;
+static constexpr size_t kSchedBytes = 256;  // workspace header: the scheduler counters
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 static int max_parts_for(int max_seq_len, int part) { return max_seq_len > 0 ? (int)cdiv64(max_seq_len, part) : 1; }
@@ -153,10 +182,27 @@ static int max_parts_for(int max_seq_len, int part) { return max_seq_len > 0 ? (
 static size_t workspace_bytes_for(int num_seqs, int num_heads, int head_dim, int max_parts)
 {
     const size_t rows = (size_t)num_seqs * num_heads * max_parts;
-    return align256(rows * head_dim * sizeof(float)) + 2 * align256(rows * sizeof(float));
+    return kSchedBytes + align256(rows * head_dim * sizeof(float)) + 2 * align256(rows * sizeof(float));
 }
 
-// mode: 0 = one pass, 1 = split (direct singles + reduce), 2 = partitions only
+// Partial-result sections of a split-form workspace (after the header).
+struct WsLayout {
+    float *o, *m, *l;
+};
+static WsLayout ws_layout(void *ws, int num_seqs, int num_heads, int head_dim, int max_parts)
+{
+    const size_t rows = (size_t)num_seqs * num_heads * max_parts;
+    char *w = static_cast<char *>(ws) + kSchedBytes;
+    WsLayout L;
+    L.o = reinterpret_cast<float *>(w);
+    L.m = reinterpret_cast<float *>(w + align256(rows * head_dim * sizeof(float)));
+    L.l = reinterpret_cast<float *>(w + align256(rows * head_dim * sizeof(float)) + align256(rows * sizeof(float)));
+    return L;
+}
+
+// mode: 0 = one pass, 1 = split (direct singles + reduce), 2 = partitions only.
+// A workspace (when given) supplies the scheduler counters for every mode and
+// the partial results for modes 1 and 2.
 static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t ws_bytes, cudaStream_t st)
 {
     int rc = check_decode_args(a, mode != 2);
@@ -173,6 +219,8 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
     p.num_kv_heads = a.num_kv_heads;
     p.group = a.num_heads / a.num_kv_heads;
     p.max_blocks = a.max_blocks;
+    if (ws && (!aligned16(ws) || ws_bytes < kSchedBytes)) return PA_ERR_WORKSPACE;
+    p.sched = ws ? static_cast<int *>(ws) : nullptr;
     if (mode == 0) {
         p.part_tokens = 0;
         p.max_parts = 1;
@@ -183,23 +231,21 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
         p.max_parts = max_parts_for(a.max_seq_len, part);
         p.direct_single = mode == 1 ? 1 : 0;
         const size_t need = workspace_bytes_for(a.num_seqs, a.num_heads, a.head_dim, p.max_parts);
-        if (!ws || ws_bytes < need || !aligned16(ws)) return PA_ERR_WORKSPACE;
-        const size_t rows = (size_t)a.num_seqs * a.num_heads * p.max_parts;
-        char *w = static_cast<char *>(ws);
-        p.ws_o = reinterpret_cast<float *>(w);
-        p.ws_m = reinterpret_cast<float *>(w + align256(rows * a.head_dim * sizeof(float)));
-        p.ws_l = reinterpret_cast<float *>(w + align256(rows * a.head_dim * sizeof(float)) +
-                                           align256(rows * sizeof(float)));
+        if (!ws || ws_bytes < need) return PA_ERR_WORKSPACE;
+        const WsLayout L = ws_layout(ws, a.num_seqs, a.num_heads, a.head_dim, p.max_parts);
+        p.ws_o = L.o;
+        p.ws_m = L.m;
+        p.ws_l = L.l;
     }
-    const int64_t grid = (int64_t)p.max_parts * a.num_seqs * a.num_kv_heads;
-    if (grid > INT_MAX) return PA_ERR_BAD_SHAPE;
+    const int64_t max_items = (int64_t)p.max_parts * a.num_seqs * a.num_kv_heads;
+    if (max_items > INT_MAX) return PA_ERR_BAD_SHAPE;
     CUtensorMap tk, tv;
     rc = make_cache_map(&tk, a.key_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim);
     if (rc != PA_OK) return rc;
     rc = make_cache_map(&tv, a.value_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim);
     if (rc != PA_OK) return rc;
-    rc = a.head_dim == 64 ? launch_decode_d<64>(a.block_size, p, tk, tv, grid, st)
-                          : launch_decode_d<128>(a.block_size, p, tk, tv, grid, st);
+    rc = a.head_dim == 64 ? launch_decode_d<64>(a.block_size, p, tk, tv, max_items, st)
+                          : launch_decode_d<128>(a.block_size, p, tk, tv, max_items, st);
     if (rc != PA_OK || mode != 1) return rc;
     ReduceParams r = {};
     r.out = p.out;
@@ -346,7 +392,8 @@ int pa_decode(void *out, const void *query, const void *key_cache, const void *v
                                                 workspace_bytes)
                                : 0;
     if (part > 0) return run_decode(a, 1, part, workspace, workspace_bytes, st);
-    return run_decode(a, 0, 0, nullptr, 0, st);
+    const bool counters = workspace && workspace_bytes >= kSchedBytes;
+    return run_decode(a, 0, 0, counters ? workspace : nullptr, counters ? workspace_bytes : 0, st);
 }
 
 int pa_decode_one_pass(void *out, const void *query, const void *key_cache, const void *value_cache,
@@ -389,14 +436,12 @@ int pa_lse_reduce(void *out, const void *workspace, const int32_t *seq_lens, int
     if (num_seqs == 0) return PA_OK;
     if (!out || !workspace || !seq_lens) return PA_ERR_NULL_POINTER;
     const int max_parts = max_parts_for(max_seq_len, partition_size);
-    const size_t rows = (size_t)num_seqs * num_heads * max_parts;
-    const char *w = static_cast<const char *>(workspace);
+    const WsLayout L = ws_layout(const_cast<void *>(workspace), num_seqs, num_heads, head_dim, max_parts);
     ReduceParams r = {};
     r.out = static_cast<__nv_bfloat16 *>(out);
-    r.ws_o = reinterpret_cast<const float *>(w);
-    r.ws_m = reinterpret_cast<const float *>(w + align256(rows * head_dim * sizeof(float)));
-    r.ws_l = reinterpret_cast<const float *>(w + align256(rows * head_dim * sizeof(float)) +
-                                             align256(rows * sizeof(float)));
+    r.ws_o = L.o;
+    r.ws_m = L.m;
+    r.ws_l = L.l;
     r.seq_lens = seq_lens;
     r.num_seqs = num_seqs;
     r.num_heads = num_heads;

@@ -20,10 +20,13 @@ import torch
 
 from ._lib import PagedKVError, check, load  # noqa: F401
 
+# First bytes of every decode workspace: the dynamic scheduler's counters.
+WORKSPACE_HEADER_BYTES = 256
+
 __all__ = [
     "slot_mapping", "reshape_and_cache", "copy_blocks", "decode", "decode_one_pass",
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
-    "validate_tables", "device_status", "PagedKVError",
+    "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
 ]
 
 
@@ -192,13 +195,20 @@ def workspace_views(workspace, num_seqs, num_heads, head_dim, max_seq_len, parti
     parts = max(1, -(-int(max_seq_len) // int(partition_size)))
     rows = num_seqs * num_heads * parts
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    raw = workspace.view(torch.uint8)
+    raw = workspace.view(torch.uint8)[WORKSPACE_HEADER_BYTES:]
     ob = rows * head_dim * 4
     o = raw[:ob].view(torch.float32).view(num_seqs, num_heads, parts, head_dim)
     m = raw[a256(ob):a256(ob) + rows * 4].view(torch.float32).view(num_seqs, num_heads, parts)
     lo = a256(ob) + a256(rows * 4)
     l = raw[lo:lo + rows * 4].view(torch.float32).view(num_seqs, num_heads, parts)
     return o, m, l
+
+
+def new_workspace(num_seqs: int, num_heads: int, head_dim: int, max_seq_len: int, partition_size: int = 0,
+                  device="cuda"):
+    """A zero-filled decode workspace (the scheduler counters must start at zero)."""
+    nbytes = decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len, partition_size)
+    return torch.zeros(max(nbytes, WORKSPACE_HEADER_BYTES), dtype=torch.uint8, device=device)
 
 
 def lse_reduce(out, workspace, seq_lens, max_seq_len: int, partition_size: int, stream=None):

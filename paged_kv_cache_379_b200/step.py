@@ -77,8 +77,8 @@ class DecodeBatch:
         self.max_seq_len = wl.max_seq_len
         self.workspace = None
         if workspace:
-            nbytes = ops.decode_workspace_size(wl.num_seqs, wl.num_heads, wl.head_dim, self.max_seq_len)
-            self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
+            self.workspace = ops.new_workspace(wl.num_seqs, wl.num_heads, wl.head_dim, self.max_seq_len,
+                                               device=self.device)
 
     def run_step(self, stream=None, decode_fn=None):
         wl = self.wl
