@@ -57,6 +57,7 @@ extern "C" {
 #define PA_ERR_BAD_BLOCK (-7)      /* a block id outside the pool / not allocated    */
 #define PA_ERR_ALIGNMENT (-8)      /* a device pointer is not 16-byte aligned         */
 #define PA_ERR_DEVICE_TIMEOUT (-9) /* a bounded on-device wait gave up (see below)   */
+#define PA_ERR_SCRATCH_TOO_SMALL (-10) /* the built-in scratch of the no-allocation call is too small */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *pa_status_string(int status);
@@ -207,6 +208,42 @@ int pa_lse_reduce(void *out, const void *workspace, const int32_t *seq_lens, int
 int pa_validate_tables(const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
                        int max_blocks_per_seq, int block_size, int num_blocks, int max_seq_len,
                        int32_t *bad_count, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Split-form decode that allocates nothing and takes no workspace.
+ * (The pages have no counterpart of this call; it exists for callers of this
+ * library, not for the method.)
+ *
+ * Some callers cannot hand the library a workspace: code that must not call
+ * cudaMalloc on its decode path (cudaMalloc can synchronise the device and
+ * stall a latency-critical serving loop), code that runs inside another
+ * framework's memory arena with no way to allocate from it, or plugin hosts
+ * that fix the device memory a component may own up front.  This call keeps
+ * the split form's scratch -- the scheduler counters and the per-partition
+ * partial results -- in one fixed array inside the library instead:
+ * PA_NOALLOC_SCRATCH_BYTES of device memory that every GPU which loads the
+ * library holds until the process exits.
+ *
+ * Arguments and results are those of pa_decode_split without the workspace;
+ * the caller still owns and passes query, caches, tables, lengths and out.
+ * A problem whose split workspace (pa_decode_workspace_size with the same
+ * sizes and partition_size) exceeds PA_NOALLOC_SCRATCH_BYTES is rejected with
+ * PA_ERR_SCRATCH_TOO_SMALL before any launch; a larger partition_size shrinks it.
+ * The call allocates no device memory and calls no allocating routine.
+ * The first call on each device looks up the array's device address on that
+ * device (with the device current); make that first call before any stream
+ * capture.  Each call clears the scheduler counters (an asynchronous memset on
+ * `stream`) and leaves its partial results in the array.  All calls share the
+ * one array: calls that may overlap on the GPU (different streams, or other
+ * host threads) race on it and must be serialised by the caller.
+ * ------------------------------------------------------------------------ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int pa_decode_split_noalloc(void *out, const void *query, const void *key_cache,
+                            const void *value_cache, const int32_t *block_tables,
+                            const int32_t *seq_lens, float scale, int block_size,
+                            int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                            int max_blocks_per_seq, int num_blocks, int max_seq_len,
+                            int partition_size, void *stream);
 
 /* Bounded waits.  Every wait inside the kernels (on TMA completion or on a
  * pipeline stage being released) gives up after about one second, records a

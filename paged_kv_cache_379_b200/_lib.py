@@ -31,6 +31,7 @@ SIGNATURES = {
     "pa_decode_plan": (_I, [_I, _I, _I, _I, _I, _SZ]),
     "pa_decode_one_pass": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "pa_decode_split": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "pa_decode_split_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "pa_decode_partitions": (_I, [_P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "pa_lse_reduce": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_validate_tables": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),

@@ -300,6 +300,9 @@ const char *pa_status_string(int status)
     case PA_ERR_BAD_BLOCK: return "bad block id";
     case PA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case PA_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
+    case PA_ERR_SCRATCH_TOO_SMALL:
+        return "split workspace exceeds the built-in scratch of pa_decode_split_noalloc (use a larger "
+               "partition_size, or pa_decode_split with a caller workspace)";
     default: return "unknown status";
     }
 }
@@ -415,6 +418,55 @@ int pa_decode_split(void *out, const void *query, const void *key_cache, const v
     const DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
                           num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
     return run_decode(a, 1, partition_size, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// Scratch of pa_decode_split_noalloc: one fixed array per device, part of the
+// library image, so that the call needs no allocation by anyone.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up on the
+// first call per device (host code may not use the symbol itself as a pointer).
+static int noalloc_scratch(void **ptr)
+{
+    static std::mutex mu;
+    static void *addr[64] = {};
+    int dev = 0;
+    int rc = check_cuda(cudaGetDevice(&dev));
+    if (rc != PA_OK) return rc;
+    if (dev < 0 || dev >= 64) return check_cuda(cudaErrorInvalidDevice);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        rc = check_cuda(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+        if (rc != PA_OK) return rc;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return PA_OK;
+}
+
+int pa_decode_split_noalloc(void *out, const void *query, const void *key_cache, const void *value_cache,
+                            const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
+                            int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                            int num_blocks, int max_seq_len, int partition_size, void *stream)
+{
+    const DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                          num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    int rc = check_decode_args(a, true);
+    if (rc != PA_OK) return rc;
+    if (partition_size < kTileTokens || partition_size % kTileTokens != 0) return PA_ERR_BAD_SHAPE;
+    if (num_seqs == 0) return PA_OK;
+    const size_t need =
+        workspace_bytes_for(num_seqs, num_heads, head_dim, max_parts_for(max_seq_len, partition_size));
+    if (need > (size_t)PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_SCRATCH_TOO_SMALL;
+    void *scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc != PA_OK) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the scheduler counters must start at zero; the array keeps whatever the last call left
+    rc = check_cuda(cudaMemsetAsync(scratch, 0, kSchedBytes, st));
+    if (rc != PA_OK) return rc;
+    return run_decode(a, 1, partition_size, scratch, PA_NOALLOC_SCRATCH_BYTES, st);
 }
 
 int pa_decode_partitions(const void *query, const void *key_cache, const void *value_cache,

@@ -27,6 +27,7 @@ __all__ = [
     "slot_mapping", "reshape_and_cache", "copy_blocks", "decode", "decode_one_pass",
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
+    "decode_split_noalloc",
 ]
 
 
@@ -175,6 +176,27 @@ def decode_split(query, key_cache, value_cache, block_tables, seq_lens, scale: f
     check("pa_decode_split", lib.pa_decode_split(
         o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), bs, hkv, B, hq, d, mb, nb,
         int(max_seq_len), int(partition_size), wp, wb, _stream(stream)))
+    return out
+
+
+# Bytes of the fixed scratch array inside the library (PA_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_split_noalloc(query, key_cache, value_cache, block_tables, seq_lens, scale: float, max_seq_len: int,
+                         partition_size: int, *, out=None, stream=None):
+    """pa_decode_split_noalloc: the split form with the library's own fixed scratch.
+
+    For callers that cannot provide a workspace (see include/pagedkv.h).  Raises
+    PagedKVError(PA_ERR_SCRATCH_TOO_SMALL) if the problem needs more than
+    NOALLOC_SCRATCH_BYTES of split workspace.  Calls must not overlap on the GPU.
+    """
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens)
+    o, out = _out(out, query)
+    check("pa_decode_split_noalloc", lib.pa_decode_split_noalloc(
+        o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), bs, hkv, B, hq, d, mb, nb,
+        int(max_seq_len), int(partition_size), _stream(stream)))
     return out
 
 
