@@ -43,8 +43,11 @@
 //  * Every mbarrier wait is bounded in time (about 1 s); on expiry the kernel
 //    records a code in the device status word, drains its own TMA copies and
 //    returns.
-// Split form: a partition's (m, l, o) go to the workspace and lse_reduce_kernel
-// merges them; a sequence with a single partition is finished in place.
+// Split form: a partition's (m, l, o) go to the workspace; a sequence with a
+// single partition is finished in place.  With few partitions per sequence the
+// CTA that completes the last partition of a (sequence, KV head) merges them by
+// log-sum-exp right away (a counter per pair in the workspace); otherwise
+// lse_reduce_kernel merges them, one warp per (sequence, head).
 #pragma once
 
 #include "common.cuh"
@@ -60,6 +63,8 @@ struct DecodeParams {
     float *ws_m;                      // [B, Hq, max_parts]      natural-log units
     float *ws_l;                      // [B, Hq, max_parts]
     int *sched;                       // [2] item counter, finished-CTA counter; nullptr = round robin
+    int *merge_cnt;                   // [B * Hkv] partitions finished per (sequence, KV head); nullptr =
+                                      // partitions are merged by lse_reduce_kernel instead
     float scale_log2;                 // scale * log2(e)
     int num_seqs, num_heads, num_kv_heads, group, max_blocks;
     int part_tokens;                  // positions per partition (multiple of 16); 0 = one pass
@@ -79,7 +84,7 @@ constexpr int kConsumerWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kSchedulerWarp = 5;
 constexpr int kDecodeThreads = 6 * 32;
-constexpr int kStages = 8;
+constexpr int kRingBudget = 80 * 1024;  // shared memory for the K/V ring per CTA (2 CTAs per SM)
 constexpr int kTileTokens = 16;
 constexpr int kItemSlots = 2;
 constexpr int kChunkSlots = 4;
@@ -103,6 +108,9 @@ struct TileGeom {
     static constexpr int kPlaneSmem = kBlocksPerTile * kSlotRows * 128;
     static constexpr int kTileSmem = kHalves * kPlaneSmem;
     static constexpr int kStageSmem = 2 * kTileSmem;              // K tile, then V tile
+    // ring depth: as many stages as the budget holds (10 at head_dim 128, bs 16)
+    static constexpr int kStages = kRingBudget / kStageSmem > 16 ? 16
+                                   : (kRingBudget / kStageSmem < 4 ? 4 : kRingBudget / kStageSmem);
     static constexpr int kPipeSmem = kStages * kStageSmem;
 
     // Offset, inside a plane, of token t's 128-byte row.
@@ -185,7 +193,7 @@ struct DecodeSmem {
     static constexpr int kChunkOff = kItemOff + kItemSlots * (int)sizeof(ItemInfo);
     static constexpr int kBarOff = (kChunkOff + kChunkSlots * (int)sizeof(ChunkInfo) + 7) & ~7;
     // barriers: full[kStages], empty[kStages], item_full, item_empty, chunk_full, chunk_empty
-    static constexpr int kNumBars = 2 * kStages + 2 * kItemSlots + 2 * kChunkSlots;
+    static constexpr int kNumBars = 2 * Geo::kStages + 2 * kItemSlots + 2 * kChunkSlots;
     static constexpr int kFlagOff = kBarOff + kNumBars * 8;
     static constexpr int kPrefixOff = kFlagOff + 16;
     // bytes of dynamic shared memory for a launch with prefix_entries prefix ints
@@ -203,6 +211,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     using Geo = TileGeom<D, BS>;
     using Lay = DecodeSmem<D, BS, MODE, GC>;
     using Merge = typename Lay::Merge;
+    constexpr int kStages = Geo::kStages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -217,6 +226,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     const uint32_t cfull_bar = iempty_bar + kItemSlots * 8;
     const uint32_t cempty_bar = cfull_bar + kChunkSlots * 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Lay::kFlagOff);
+    volatile int *merge_flag = abort_flag + 1;
     int *const prefix = reinterpret_cast<int *>(base_ptr + Lay::kPrefixOff);
 
     const int warp = threadIdx.x >> 5;
@@ -780,6 +790,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         p.ws_m[wi] = M == -INFINITY ? -INFINITY : M * kLn2;
                         p.ws_l[wi] = den;
                     }
+                }
+            }
+            if (!direct && p.merge_cnt) {
+                // Log-sum-exp merge in place: the CTA that finishes the last
+                // partition of (s, g) merges all of them.  Writers publish their
+                // partials (fence, then count); the last one reads them from L2.
+                __threadfence();
+                consumer_bar();
+                int *cnt = p.merge_cnt + (int64_t)it.s * Hkv + it.g;
+                if (threadIdx.x == 0) *merge_flag = (atomicAdd(cnt, 1) == it.nparts - 1);
+                consumer_bar();
+                if (*merge_flag) {
+                    __threadfence();
+                    const int np = it.nparts;
+                    for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+                        const int row = idx / D;
+                        const int d = idx - row * D;
+                        const int64_t hrow = (int64_t)it.s * p.num_heads + (int64_t)it.g * G + row;
+                        const int64_t wb = hrow * p.max_parts;
+                        float M = -INFINITY;
+                        for (int q = 0; q < np; ++q) M = fmaxf(M, __ldcg(p.ws_m + wb + q));
+                        float num = 0.f, den = 0.f;
+                        if (M != -INFINITY) {
+                            for (int q = 0; q < np; ++q) {
+                                const float mq = __ldcg(p.ws_m + wb + q);
+                                if (mq == -INFINITY) continue;
+                                const float w = expf(mq - M);
+                                num = fmaf(w, __ldcg(p.ws_o + (wb + q) * D + d), num);
+                                den = fmaf(w, __ldcg(p.ws_l + wb + q), den);
+                            }
+                        }
+                        p.out[hrow * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+                    }
+                    if (threadIdx.x == 0) atomicExch(cnt, 0);  // left at zero for the next launch
                 }
             }
             consumer_bar();  // merge scratch and the item slot may be reused
