@@ -84,7 +84,7 @@ constexpr int kConsumerWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kSchedulerWarp = 5;
 constexpr int kDecodeThreads = 6 * 32;
-constexpr int kRingBudget = 80 * 1024;  // shared memory for the K/V ring per CTA (2 CTAs per SM)
+constexpr int kRingBudget = 80 * 1024;  // shared memory budget for the K/V ring per CTA (2 CTAs per SM)
 constexpr int kTileTokens = 16;
 constexpr int kItemSlots = 2;
 constexpr int kChunkSlots = 4;
@@ -108,9 +108,16 @@ struct TileGeom {
     static constexpr int kPlaneSmem = kBlocksPerTile * kSlotRows * 128;
     static constexpr int kTileSmem = kHalves * kPlaneSmem;
     static constexpr int kStageSmem = 2 * kTileSmem;              // K tile, then V tile
-    // ring depth: as many stages as the budget holds (10 at head_dim 128, bs 16)
-    static constexpr int kStages = kRingBudget / kStageSmem > 16 ? 16
-                                   : (kRingBudget / kStageSmem < 4 ? 4 : kRingBudget / kStageSmem);
+    // Ring depth: as many stages as the budget holds, rounded down to a multiple
+    // of the consumer-warp count (8 at head_dim 128, bs 16).  The multiple is
+    // required: tile j of an item goes to warp j % 4 and sits at ring position
+    // base + j, so a stage's previous tile (position - kStages) then belongs to
+    // the same warp, which has consumed it before it waits on the stage again.
+    // Otherwise a warp could wait on a stage whose previous phase is still
+    // pending, and an mbarrier parity wait cannot tell that phase from the next.
+    static constexpr int kStagesRaw = kRingBudget / kStageSmem > 16 ? 16 : kRingBudget / kStageSmem;
+    static constexpr int kStages = kStagesRaw / kConsumerWarps * kConsumerWarps;
+    static_assert(kStages >= kConsumerWarps && kStages % kConsumerWarps == 0, "ring depth");
     static constexpr int kPipeSmem = kStages * kStageSmem;
 
     // Offset, inside a plane, of token t's 128-byte row.

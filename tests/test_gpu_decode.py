@@ -153,6 +153,28 @@ def test_partitions_and_reduce_match_oracle(Hq, Hkv, part):
     assert_close(bf16_to_host_bits(out), ref, "lse_reduce")
 
 
+@pytest.mark.parametrize("sched", ["round_robin", "dynamic"])
+def test_one_pass_full_gqa_batch_matches_oracle(sched):
+    """One pass over the whole GQA batch: every CTA runs several long items of
+    many table chunks (up to 256 tiles each), so the consumer warps drift apart
+    and the ring wraps many times within one item."""
+    w = wl.make("gqa")
+    d = _dev_inputs(w)
+    args = (d["query"], d["key_cache"], d["value_cache"], d["block_tables"], d["seq_lens"], w.scale, w.max_seq_len)
+    if sched == "round_robin":
+        out = ops.decode_one_pass(*args)
+    else:
+        counters = torch.zeros(256, dtype=torch.uint8, device=DEV)   # too small to split: one pass, dynamic
+        assert ops.decode_plan(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, 256) == 0
+        out = ops.decode(*args, workspace=counters)
+        out = ops.decode(*args, workspace=counters)                    # counters were left at zero
+        assert int(counters.view(torch.int32)[:2].abs().sum().item()) == 0
+    torch.cuda.synchronize()
+    ref = oracle.paged_decode(w.query, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, w.scale, threads=0)
+    assert_close(bf16_to_host_bits(out), ref, f"one pass, {sched}")
+    assert ops.device_status() == 0
+
+
 def test_split_and_one_pass_agree_on_long_sequences():
     w = wl.make("gqa", num_seqs=16)
     one = _run(w, "one_pass")
