@@ -129,9 +129,8 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pa
  * Workspace contract (all decode entry points that take one): caller-owned
  * device memory, 16-byte aligned.  Its first 256 bytes hold the counters of
  * the kernels' dynamic work scheduler: ZERO-FILL THE WORKSPACE ONCE after
- * allocating it (e.g. cudaMemsetAsync); every call leaves those bytes, and
- * the per-(sequence, head) merge counters at the workspace's end, zero again
- * when it completes.  The rest is scratch (no initialisation needed).
+ * allocating it (e.g. cudaMemsetAsync); every call leaves those bytes zero
+ * again when it completes.  The rest is scratch (no initialisation needed).
  * Calls that may run concurrently must not share a workspace.  After
  * pa_device_status() has reported a timeout, zero the workspace again.
  *
@@ -169,10 +168,8 @@ int pa_decode_one_pass(void *out, const void *query, const void *key_cache,
 
 /* a5 + a6: positions are cut into partitions of partition_size tokens (a
  * multiple of 16, >= 16); each (sequence, partition, KV head) work item
- * computes the partition's local result, and the results are merged by
- * log-sum-exp: inside the same kernel by the work item that finishes last when
- * a sequence has at most 16 partitions, else by a separate reduce kernel.  A
- * sequence that fits in one partition is written directly. */
+ * computes the partition's local result, and a log-sum-exp reduce kernel
+ * merges them.  A sequence that fits in one partition is written directly. */
 int pa_decode_split(void *out, const void *query, const void *key_cache, const void *value_cache,
                     const int32_t *block_tables, const int32_t *seq_lens, float scale,
                     int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
@@ -185,7 +182,6 @@ int pa_decode_split(void *out, const void *query, const void *key_cache, const v
  *   float o[num_seqs][num_heads][max_parts][head_dim]  at byte 256,
  *   float m[num_seqs][num_heads][max_parts]           after o (256-B aligned),
  *   float l[num_seqs][num_heads][max_parts]           after m (256-B aligned),
- *   int   merge counters[num_seqs][num_heads]          after l (256-B aligned),
  * with max_parts = ceil(max_seq_len / partition_size) (at least 1):
  *   m = max_p scale*q.k_p (natural-log units), l = sum_p exp(x_p - m),
  *   o = sum_p exp(x_p - m) v_p (not normalised).

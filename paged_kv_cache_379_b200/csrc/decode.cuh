@@ -43,11 +43,9 @@
 //  * Every mbarrier wait is bounded in time (about 1 s); on expiry the kernel
 //    records a code in the device status word, drains its own TMA copies and
 //    returns.
-// Split form: a partition's (m, l, o) go to the workspace; a sequence with a
-// single partition is finished in place.  With few partitions per sequence the
-// CTA that completes the last partition of a (sequence, KV head) merges them by
-// log-sum-exp right away (a counter per pair in the workspace); otherwise
-// lse_reduce_kernel merges them, one warp per (sequence, head).
+// Split form: a partition's (m, l, o) go to the workspace and lse_reduce_kernel
+// merges them, one warp per (sequence, head); a sequence with a single
+// partition is finished in place.
 #pragma once
 
 #include "common.cuh"
@@ -63,8 +61,6 @@ struct DecodeParams {
     float *ws_m;                      // [B, Hq, max_parts]      natural-log units
     float *ws_l;                      // [B, Hq, max_parts]
     int *sched;                       // [2] item counter, finished-CTA counter; nullptr = round robin
-    int *merge_cnt;                   // [B * Hkv] partitions finished per (sequence, KV head); nullptr =
-                                      // partitions are merged by lse_reduce_kernel instead
     float scale_log2;                 // scale * log2(e)
     int num_seqs, num_heads, num_kv_heads, group, max_blocks;
     int part_tokens;                  // positions per partition (multiple of 16); 0 = one pass
@@ -233,7 +229,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     const uint32_t cfull_bar = iempty_bar + kItemSlots * 8;
     const uint32_t cempty_bar = cfull_bar + kChunkSlots * 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Lay::kFlagOff);
-    volatile int *merge_flag = abort_flag + 1;
     int *const prefix = reinterpret_cast<int *>(base_ptr + Lay::kPrefixOff);
 
     const int warp = threadIdx.x >> 5;
@@ -799,40 +794,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     }
                 }
             }
-            if (!direct && p.merge_cnt) {
-                // Log-sum-exp merge in place: the CTA that finishes the last
-                // partition of (s, g) merges all of them.  Writers publish their
-                // partials (fence, then count); the last one reads them from L2.
-                __threadfence();
-                consumer_bar();
-                int *cnt = p.merge_cnt + (int64_t)it.s * Hkv + it.g;
-                if (threadIdx.x == 0) *merge_flag = (atomicAdd(cnt, 1) == it.nparts - 1);
-                consumer_bar();
-                if (*merge_flag) {
-                    __threadfence();
-                    const int np = it.nparts;
-                    for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
-                        const int row = idx / D;
-                        const int d = idx - row * D;
-                        const int64_t hrow = (int64_t)it.s * p.num_heads + (int64_t)it.g * G + row;
-                        const int64_t wb = hrow * p.max_parts;
-                        float M = -INFINITY;
-                        for (int q = 0; q < np; ++q) M = fmaxf(M, __ldcg(p.ws_m + wb + q));
-                        float num = 0.f, den = 0.f;
-                        if (M != -INFINITY) {
-                            for (int q = 0; q < np; ++q) {
-                                const float mq = __ldcg(p.ws_m + wb + q);
-                                if (mq == -INFINITY) continue;
-                                const float w = expf(mq - M);
-                                num = fmaf(w, __ldcg(p.ws_o + (wb + q) * D + d), num);
-                                den = fmaf(w, __ldcg(p.ws_l + wb + q), den);
-                            }
-                        }
-                        p.out[hrow * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
-                    }
-                    if (threadIdx.x == 0) atomicExch(cnt, 0);  // left at zero for the next launch
-                }
-            }
             consumer_bar();  // merge scratch and the item slot may be reused
             if (threadIdx.x == 0) mbar_arrive(iempty_bar + 8 * islot);
             ++item_seq;
@@ -868,15 +829,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 
 // Log-sum-exp merge of the partitions of one (sequence, head) per warp:
 //   M = max_p m_p,  out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p.
-// Lane p computes the weight of partition p; the weighted sum over partitions
-// reads each partition's o row as one coalesced 16-byte (D = 128) or 8-byte
-// (D = 64) vector per lane.
+// The partials were just written and sit in L2; the kernel is bound by load
+// latency, so it keeps many loads in flight: lane p reads m_p and l_p (one
+// round), then the o rows of 8 partitions at a time are read together, each as
+// one coalesced 16-byte (D = 128) or 8-byte (D = 64) vector per lane.
 constexpr int kReduceWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const ReduceParams r)
 {
     constexpr int VEC = D / 32;
+    constexpr int U = 8;  // partitions whose o rows are in flight together
     pdl_wait();
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
@@ -900,18 +863,24 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Red
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
     float den = 0.f;
     if (M != -INFINITY) {
-        for (int i0 = 0; i0 < nparts; i0 += 32) {
-            const int i = i0 + lane;
-            const float w = (i < nparts) ? expf(m[i] - M) : 0.f;  // an empty partition has m = -inf: weight 0
-            den += (i < nparts) ? w * l[i] : 0.f;
-            const int cnt = min(32, nparts - i0);
-            int j = 0;
-            for (; j + 4 <= cnt; j += 4) {
-                float wj[4], v[4][VEC];
+        for (int i = lane; i < nparts; i += 32) {
+            const float mi = m[i];
+            if (mi != -INFINITY) den = fmaf(expf(mi - M), l[i], den);  // an empty partition weighs 0
+        }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    wj[u] = __shfl_sync(0xffffffffu, w, j + u);
-                    const float *src = o + (int64_t)(i0 + j + u) * D;
+        for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+        for (int j0 = 0; j0 < nparts; j0 += U) {
+            float v[U][VEC], w[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = j0 + u;
+                w[u] = 0.f;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
+                if (j < nparts) {
+                    const float mj = m[j];
+                    w[u] = mj != -INFINITY ? expf(mj - M) : 0.f;
+                    const float *src = o + (int64_t)j * D;
                     if constexpr (VEC == 4) {
                         const float4 f = *reinterpret_cast<const float4 *>(src);
                         v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
@@ -920,20 +889,12 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Red
                         v[u][0] = f.x; v[u][1] = f.y;
                     }
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                    for (int e = 0; e < VEC; ++e) acc[e] = fmaf(wj[u], v[u][e], acc[e]);
             }
-            for (; j < cnt; ++j) {
-                const float wj = __shfl_sync(0xffffffffu, w, j);
-                const float *src = o + (int64_t)(i0 + j) * D;
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[e] = fmaf(wj, src[e], acc[e]);
-            }
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[e] = fmaf(w[u], v[u][e], acc[e]);
         }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
     }
     __nv_bfloat16 *dst = r.out + row * D + lane * VEC;
 #pragma unroll

@@ -179,21 +179,16 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 static int max_parts_for(int max_seq_len, int part) { return max_seq_len > 0 ? (int)cdiv64(max_seq_len, part) : 1; }
 
-// Split-form workspace: [scheduler counters, 256 B][partial results o, m, l]
-// [merge counters: one int per (sequence, head), zero between calls], every
-// section 256-byte aligned.
-static size_t counter_bytes(int num_seqs, int num_heads) { return align256((size_t)num_seqs * num_heads * sizeof(int)); }
-
+// Split-form workspace: [scheduler counters, 256 B][partial results o, m, l],
+// every section 256-byte aligned.
 static size_t workspace_bytes_for(int num_seqs, int num_heads, int head_dim, int max_parts)
 {
     const size_t rows = (size_t)num_seqs * num_heads * max_parts;
-    return kSchedBytes + align256(rows * head_dim * sizeof(float)) + 2 * align256(rows * sizeof(float)) +
-           counter_bytes(num_seqs, num_heads);
+    return kSchedBytes + align256(rows * head_dim * sizeof(float)) + 2 * align256(rows * sizeof(float));
 }
 
 struct WsLayout {
     float *o, *m, *l;
-    int *cnt;  // merge counters, [num_seqs * num_heads] (only num_seqs * num_kv_heads used)
 };
 static WsLayout ws_layout(void *ws, int num_seqs, int num_heads, int head_dim, int max_parts)
 {
@@ -204,12 +199,8 @@ static WsLayout ws_layout(void *ws, int num_seqs, int num_heads, int head_dim, i
     L.o = reinterpret_cast<float *>(w);
     L.m = reinterpret_cast<float *>(w + ob);
     L.l = reinterpret_cast<float *>(w + ob + mb);
-    L.cnt = reinterpret_cast<int *>(w + ob + 2 * mb);
     return L;
 }
-
-// Partitions per sequence up to which the partition kernel merges in place.
-static constexpr int kMaxFusedParts = 16;
 
 // mode: 0 = one pass, 1 = split (direct singles + reduce), 2 = partitions only.
 // A workspace (when given) supplies the scheduler counters for every mode and
@@ -247,7 +238,6 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
         p.ws_o = L.o;
         p.ws_m = L.m;
         p.ws_l = L.l;
-        p.merge_cnt = (mode == 1 && p.max_parts <= kMaxFusedParts) ? L.cnt : nullptr;
     }
     const int64_t max_items = (int64_t)p.max_parts * a.num_seqs * a.num_kv_heads;
     if (max_items > INT_MAX) return PA_ERR_BAD_SHAPE;
@@ -258,7 +248,7 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
     if (rc != PA_OK) return rc;
     rc = a.head_dim == 64 ? launch_decode_d<64>(a.block_size, p, tk, tv, max_items, st)
                           : launch_decode_d<128>(a.block_size, p, tk, tv, max_items, st);
-    if (rc != PA_OK || mode != 1 || p.merge_cnt) return rc;
+    if (rc != PA_OK || mode != 1) return rc;
     ReduceParams r = {};
     r.out = p.out;
     r.ws_o = p.ws_o;
@@ -475,11 +465,8 @@ int pa_decode_split_noalloc(void *out, const void *query, const void *key_cache,
     rc = noalloc_scratch(&scratch);
     if (rc != PA_OK) return rc;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the scheduler and merge counters must start at zero; the array keeps whatever the last call left
-    const WsLayout L = ws_layout(scratch, num_seqs, num_heads, head_dim, max_parts_for(max_seq_len, partition_size));
+    // the scheduler counters must start at zero; the array keeps whatever the last call left
     rc = check_cuda(cudaMemsetAsync(scratch, 0, kSchedBytes, st));
-    if (rc != PA_OK) return rc;
-    rc = check_cuda(cudaMemsetAsync(L.cnt, 0, counter_bytes(num_seqs, num_heads), st));
     if (rc != PA_OK) return rc;
     return run_decode(a, 1, partition_size, scratch, PA_NOALLOC_SCRATCH_BYTES, st);
 }
