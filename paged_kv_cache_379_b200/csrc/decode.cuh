@@ -86,6 +86,9 @@ constexpr int kItemSlots = 2;
 constexpr int kChunkSlots = 4;
 constexpr int kChunkBlocks = 32;
 constexpr float kLn2 = 0.693147180559945309f;
+// A column's softmax reference max moves only when a logit exceeds it by more
+// than this (log2 units), so unnormalised weights stay below 2^8.
+constexpr float kRescaleSlack = 8.f;
 
 template <int D, int BS>
 struct TileGeom {
@@ -140,7 +143,8 @@ struct TileGeom {
 template <int D, int ROWS>
 struct MergeScratch {
     float o[kConsumerWarps][ROWS][D + 4];  // +4: the heads a warp writes at once land in distinct banks
-    float m[kConsumerWarps][ROWS];
+    float m[kConsumerWarps][ROWS];         // reference max that o and l are relative to (log2 units)
+    float mt[kConsumerWarps][ROWS];        // true max of the logits seen (log2 units), >= m
     float l[kConsumerWarps][ROWS];
 };
 
@@ -620,6 +624,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     for (int e = 0; e < DPL; ++e) ms->o[warp][h][DPL * lane + e] = o[h][e];
                     if (lane == 0) {
                         ms->m[warp][h] = m[h];
+                        ms->mt[warp][h] = m[h];
                         ms->l[warp][h] = l[h];
                     }
                 }
@@ -648,10 +653,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     }
                 }
                 float o[MT][NH][4];
-                float m[NH][2], l[NH][2];
+                float m[NH][2], mtrue[NH][2], l[NH][2];
 #pragma unroll
                 for (int nh = 0; nh < NH; ++nh) {
                     m[nh][0] = m[nh][1] = -INFINITY;
+                    mtrue[nh][0] = mtrue[nh][1] = -INFINITY;
                     l[nh][0] = l[nh][1] = 0.f;
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) o[mt][nh][0] = o[mt][nh][1] = o[mt][nh][2] = o[mt][nh][3] = 0.f;
@@ -671,44 +677,70 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     const int valid = min(kTileTokens, it.t_end - (it.t_begin + j * kTileTokens));
                     if (valid < kTileTokens) zero_tail(vt, valid);
 
-                    // S^T[token][head] = K Q^T
-                    float sc[NH][4];
+                    // S^T[token][head] = K Q^T, as two independent MMA chains (even and
+                    // odd k-steps) summed at the end: half the dependent latency
+                    float sc[NH][4], sd[NH][4];
 #pragma unroll
-                    for (int nh = 0; nh < NH; ++nh) sc[nh][0] = sc[nh][1] = sc[nh][2] = sc[nh][3] = 0.f;
+                    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) sc[nh][c] = sd[nh][c] = 0.f;
 #pragma unroll
                     for (int kk = 0; kk < KSTEPS; ++kk) {
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
 #pragma unroll
-                        for (int nh = 0; nh < NH; ++nh) mma_bf16_16816(sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                        for (int nh = 0; nh < NH; ++nh)
+                            mma_bf16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
                     }
-                    // online softmax per head column; this lane holds tokens gq and gq+8
-                    // of heads 2tq and 2tq+1.  P enters the PV product as a bf16 high
-                    // part plus a bf16 residual (two MMAs): ~16 significant bits.
+#pragma unroll
+                    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) sc[nh][c] += sd[nh][c];
+                    // Online softmax per head column; this lane holds tokens gq and gq+8
+                    // of heads 2tq and 2tq+1.  The reference max m of a column moves
+                    // only when a logit exceeds it by more than kRescaleSlack (log2
+                    // units): weights stay <= 2^kRescaleSlack, and o and l keep one
+                    // common reference, so the result is the same softmax while the
+                    // rescale of o is almost never taken.  P enters the PV product as a
+                    // bf16 high part plus a bf16 residual (two MMAs): ~16 significant bits.
                     const bool in0 = gq < valid, in1 = gq + 8 < valid;
                     uint32_t bh[NH][2], bl[NH][2];
 #pragma unroll
                     for (int nh = 0; nh < NH; ++nh) {
-                        float pr[2][2];  // [head j][token row]
+                        float x[2][2], mx[2];  // [head j][token row]
+                        bool bump = false;
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
-                            const float x0 = in0 ? sc[nh][jj] * p.scale_log2 : -INFINITY;
-                            const float x1 = in1 ? sc[nh][2 + jj] * p.scale_log2 : -INFINITY;
-                            float mx = fmaxf(x0, x1);
-                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                            const float m_new = fmaxf(m[nh][jj], mx);
-                            const float corr = exp2f(m[nh][jj] - m_new);
-                            m[nh][jj] = m_new;
-                            pr[jj][0] = exp2f(x0 - m_new);
-                            pr[jj][1] = exp2f(x1 - m_new);
-                            l[nh][jj] = l[nh][jj] * corr + (pr[jj][0] + pr[jj][1]);
+                            x[jj][0] = in0 ? sc[nh][jj] * p.scale_log2 : -INFINITY;
+                            x[jj][1] = in1 ? sc[nh][2 + jj] * p.scale_log2 : -INFINITY;
+                            float v = fmaxf(x[jj][0], x[jj][1]);
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                            mx[jj] = v;
+                            mtrue[nh][jj] = fmaxf(mtrue[nh][jj], v);
+                            bump |= v > m[nh][jj] + kRescaleSlack;
+                        }
+                        if (__any_sync(0xffffffffu, bump)) {
 #pragma unroll
-                            for (int mt = 0; mt < MT; ++mt) {
-                                o[mt][nh][jj] *= corr;
-                                o[mt][nh][2 + jj] *= corr;
+                            for (int jj = 0; jj < 2; ++jj) {
+                                const float m_new = mx[jj] > m[nh][jj] + kRescaleSlack ? mx[jj] : m[nh][jj];
+                                const float corr = exp2f(m[nh][jj] - m_new);  // 1 for an unmoved column
+                                m[nh][jj] = m_new;
+                                l[nh][jj] *= corr;
+#pragma unroll
+                                for (int mt = 0; mt < MT; ++mt) {
+                                    o[mt][nh][jj] *= corr;
+                                    o[mt][nh][2 + jj] *= corr;
+                                }
                             }
+                        }
+                        float pr[2][2];
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            pr[jj][0] = exp2f(x[jj][0] - m[nh][jj]);
+                            pr[jj][1] = exp2f(x[jj][1] - m[nh][jj]);
+                            l[nh][jj] += pr[jj][0] + pr[jj][1];
                         }
 #pragma unroll
                         for (int row = 0; row < 2; ++row) {
@@ -754,6 +786,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             }
                             if (gq == 0) {
                                 ms->m[warp][head] = m[nh][jj];
+                                ms->mt[warp][head] = mtrue[nh][jj];
                                 ms->l[warp][head] = l[nh][jj];
                             }
                         }
@@ -767,9 +800,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
                 const int row = idx / D;
                 const int d = idx - row * D;
+                // the combined true max is the common reference: every warp's own
+                // reference is <= it, so the weights below are <= 1
                 float M = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->m[w][row]);
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->mt[w][row]);
                 float num = 0.f, den = 0.f;
                 if (M != -INFINITY) {
 #pragma unroll
