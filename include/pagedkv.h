@@ -123,7 +123,7 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pa
  *
  * pa_decode picks the one-pass kernel or the split form by max_seq_len and the
  * number of (sequence, KV head) units.  It takes a workspace of at least
- * pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len, 0)
+ * pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_seq_len, 0)
  * bytes, or none (workspace NULL: one pass, work handed out round-robin).
  *
  * Workspace contract (all decode entry points that take one): caller-owned
@@ -146,16 +146,21 @@ int pa_decode(void *out, const void *query, const void *key_cache, const void *v
               int num_blocks, int max_seq_len, void *workspace, size_t workspace_bytes,
               void *stream);
 
-/* The plan pa_decode follows for these sizes: 0 = the one-pass kernel (one
- * launch), otherwise the partition size of the split form (partition kernel +
- * reduce kernel, two launches).  No device work. */
+/* The plan pa_decode follows for these sizes: 0 = one pass (one launch),
+ * otherwise the partition size of the split form (partition kernel + reduce
+ * kernel, two launches).  One pass when max_seq_len <= 1536 and the
+ * (sequence, KV head) units give every SM several items; else partitions of
+ * 512 positions (2048 beyond 16384), halved while the batch is too small to
+ * give every SM several items.  A workspace smaller than the split form needs
+ * gives one pass.  No device work. */
 int pa_decode_plan(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_seq_len,
                    size_t workspace_bytes);
 
 /* Workspace bytes pa_decode / pa_decode_split need.  partition_size <= 0 means
- * the partition size pa_decode would choose. */
-size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len,
-                                int partition_size);
+ * the plan pa_decode would choose for these sizes (256 bytes when that plan is
+ * one pass).  0 for invalid sizes. */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                int max_seq_len, int partition_size);
 
 /* a4 alone: each (sequence, KV head) work item walks all of the sequence's
  * blocks with an online softmax ("逐块计算局部 Attention，最后合并结果",

@@ -27,7 +27,7 @@ SIGNATURES = {
     "pa_reshape_and_cache": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_decode": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
-    "pa_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "pa_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "pa_decode_plan": (_I, [_I, _I, _I, _I, _I, _SZ]),
     "pa_decode_one_pass": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "pa_decode_split": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),

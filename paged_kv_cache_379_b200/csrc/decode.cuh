@@ -146,6 +146,9 @@ struct MergeScratch {
     float m[kConsumerWarps][ROWS];         // reference max that o and l are relative to (log2 units)
     float mt[kConsumerWarps][ROWS];        // true max of the logits seen (log2 units), >= m
     float l[kConsumerWarps][ROWS];
+    float cw[kConsumerWarps][ROWS];        // merge weight of each warp's state
+    float den[ROWS];                       // merged sum of weights
+    float M[ROWS];                         // merged reference max (log2 units)
 };
 
 // A work item as the scheduler publishes it.
@@ -797,33 +800,53 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             // ---- merge the four warps of this item (after an abort the values are
             // meaningless but harmless; the next item check stops every warp)
             const bool direct = p.direct_single && it.nparts == 1;
-            for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
-                const int row = idx / D;
-                const int d = idx - row * D;
-                // the combined true max is the common reference: every warp's own
-                // reference is <= it, so the weights below are <= 1
+            // per head row: the combined true max is the common reference (every
+            // warp's own reference is <= it, so the weights are <= 1)
+            if (threadIdx.x < G) {
+                const int row = threadIdx.x;
                 float M = -INFINITY;
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->mt[w][row]);
-                float num = 0.f, den = 0.f;
-                if (M != -INFINITY) {
+                float den = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w) {
-                        const float mw = ms->m[w][row];
-                        if (mw != -INFINITY) {
-                            const float c = exp2f(mw - M);
-                            num = fmaf(c, ms->o[w][row][d], num);
-                            den = fmaf(c, ms->l[w][row], den);
-                        }
-                    }
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float mw = ms->m[w][row];
+                    const float c = (M != -INFINITY && mw != -INFINITY) ? exp2f(mw - M) : 0.f;
+                    ms->cw[w][row] = c;
+                    den = fmaf(c, ms->l[w][row], den);
+                }
+                ms->den[row] = den;
+                ms->M[row] = M;
+            }
+            consumer_bar();
+            // weighted sum of the four accumulators, 4 columns per thread
+            constexpr int D4 = D / 4;
+            for (int idx = threadIdx.x; idx < G * D4; idx += kConsumerWarps * 32) {
+                const int row = idx / D4;
+                const int d = (idx - row * D4) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float c = ms->cw[w][row];
+                    const float4 v = *reinterpret_cast<const float4 *>(&ms->o[w][row][d]);
+                    acc.x = fmaf(c, v.x, acc.x);
+                    acc.y = fmaf(c, v.y, acc.y);
+                    acc.z = fmaf(c, v.z, acc.z);
+                    acc.w = fmaf(c, v.w, acc.w);
                 }
                 const int64_t hrow = (int64_t)it.s * p.num_heads + (int64_t)it.g * G + row;
+                const float den = ms->den[row];
                 if (direct) {
-                    p.out[hrow * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+                    const float inv = den > 0.f ? 1.f / den : 0.f;
+                    uint2 packed;
+                    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+                    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+                    *reinterpret_cast<uint2 *>(p.out + hrow * D + d) = packed;
                 } else {
                     const int64_t wi = hrow * p.max_parts + it.part;
-                    p.ws_o[wi * D + d] = num;
+                    *reinterpret_cast<float4 *>(p.ws_o + wi * D + d) = acc;
                     if (d == 0) {
+                        const float M = ms->M[row];
                         p.ws_m[wi] = M == -INFINITY ? -INFINITY : M * kLn2;
                         p.ws_l[wi] = den;
                     }

@@ -173,7 +173,6 @@ static int check_decode_args(const DecodeArgs &a, bool need_out)
     return PA_OK;
 }
 
-static constexpr int kDefaultPartition = 512;
 static constexpr size_t kSchedBytes = 256;  // workspace header: the scheduler counters
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -264,23 +263,24 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
     return launch_reduce(r, st);
 }
 
-// Partition size the dispatcher uses for a split run.
-static int choose_partition(int num_seqs, int num_kv_heads, int max_seq_len)
-{
-    (void)num_seqs;
-    (void)num_kv_heads;
-    (void)max_seq_len;
-    return kDefaultPartition;
-}
+// pa_decode's plan: 0 = one pass, else the partition size of the split form.
+// Chosen from measurements on B200 (head_dim 128, bs 16): one pass wins when
+// every sequence is short and the (sequence, KV head) units alone give every
+// SM several items (shared-prefix batch, max 1280 tokens: 203 us one pass vs
+// 311 us split); otherwise 512-token partitions (GQA batch 135 us, MHA batch
+// 221 us) up to 16K positions and 2048-token ones beyond (128K-context batch
+// 445 us vs 502 us at 512); partitions shrink until a small batch still yields
+// several items per resident CTA.
+static constexpr int kOnePassMaxLen = 1536;
 
-// One pass when every (sequence, KV head) unit is short enough and there are
-// enough units to fill the GPU; otherwise split into partitions.
-static bool prefer_split(int num_seqs, int num_kv_heads, int max_seq_len)
+static int choose_plan(int num_seqs, int num_kv_heads, int max_seq_len)
 {
     const int64_t units = (int64_t)num_seqs * num_kv_heads;
-    if (max_seq_len > 1024) return true;
-    if (units < 2 * 148 && max_seq_len > 256) return true;
-    return false;
+    const int64_t target = 8LL * std::max(1, sm_count());  // ~4 items per resident CTA
+    if (max_seq_len <= kOnePassMaxLen && units >= target / 2) return 0;
+    int part = max_seq_len > 16384 ? 2048 : 512;
+    while (part > 64 && units * std::max<int64_t>(1, max_seq_len / (2 * part)) < target) part /= 2;
+    return part;
 }
 
 }  // namespace pakv
@@ -368,10 +368,12 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pa
                       static_cast<uint4 *>(value_cache), src_dst_pairs, chunks, slices, (int64_t)num_blocks);
 }
 
-size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len, int partition_size)
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_seq_len,
+                                int partition_size)
 {
-    if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return 0;
-    const int part = partition_size > 0 ? partition_size : kDefaultPartition;
+    if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return 0;
+    const int part = partition_size > 0 ? partition_size : choose_plan(num_seqs, num_kv_heads, max_seq_len);
+    if (part == 0) return kSchedBytes;  // one pass: the scheduler counters only
     return workspace_bytes_for(num_seqs, num_heads, head_dim, max_parts_for(max_seq_len, part));
 }
 
@@ -379,8 +381,8 @@ int pa_decode_plan(int num_seqs, int num_heads, int num_kv_heads, int head_dim, 
                    size_t workspace_bytes)
 {
     if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return 0;
-    if (!prefer_split(num_seqs, num_kv_heads, max_seq_len)) return 0;
-    const int part = choose_partition(num_seqs, num_kv_heads, max_seq_len);
+    const int part = choose_plan(num_seqs, num_kv_heads, max_seq_len);
+    if (part == 0) return 0;
     const size_t need = workspace_bytes_for(num_seqs, num_heads, head_dim, max_parts_for(max_seq_len, part));
     return workspace_bytes >= need ? part : 0;
 }

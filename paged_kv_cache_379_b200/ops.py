@@ -118,9 +118,11 @@ def _decode_common(query, key_cache, value_cache, block_tables, seq_lens):
     return q, bt, sl, B, hq, hkv, d, bs, nb, block_tables.shape[1]
 
 
-def decode_workspace_size(num_seqs: int, num_heads: int, head_dim: int, max_seq_len: int,
+def decode_workspace_size(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, max_seq_len: int,
                           partition_size: int = 0) -> int:
-    return int(load().pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len, partition_size))
+    """Bytes of decode workspace; partition_size 0 = what pa_decode would choose."""
+    return int(load().pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_seq_len,
+                                               partition_size))
 
 
 def decode_plan(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, max_seq_len: int,
@@ -226,10 +228,10 @@ def workspace_views(workspace, num_seqs, num_heads, head_dim, max_seq_len, parti
     return o, m, l
 
 
-def new_workspace(num_seqs: int, num_heads: int, head_dim: int, max_seq_len: int, partition_size: int = 0,
-                  device="cuda"):
+def new_workspace(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, max_seq_len: int,
+                  partition_size: int = 0, device="cuda"):
     """A zero-filled decode workspace (the scheduler counters must start at zero)."""
-    nbytes = decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len, partition_size)
+    nbytes = decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_seq_len, partition_size)
     return torch.zeros(max(nbytes, WORKSPACE_HEADER_BYTES), dtype=torch.uint8, device=device)
 
 

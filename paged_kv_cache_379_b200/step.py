@@ -77,7 +77,7 @@ class DecodeBatch:
         self.max_seq_len = wl.max_seq_len
         self.workspace = None
         if workspace:
-            self.workspace = ops.new_workspace(wl.num_seqs, wl.num_heads, wl.head_dim, self.max_seq_len,
+            self.workspace = ops.new_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, self.max_seq_len,
                                                device=self.device)
 
     def run_step(self, stream=None, decode_fn=None):

@@ -81,6 +81,6 @@ def test_argument_errors_without_gpu(lib):
 def test_workspace_size(lib):
     # 256-byte scheduler header, then for 4 seqs x 8 heads x ceil(1000/512)=2 parts:
     # o = 64*128*4 B, m and l = 64*4 B each (each 256-aligned)
-    assert lib.pa_decode_workspace_size(4, 8, 128, 1000, 512) == 256 + 64 * 128 * 4 + 2 * 256
-    assert lib.pa_decode_workspace_size(4, 8, 128, 0, 512) == 256 + 32 * 128 * 4 + 2 * 256
-    assert lib.pa_decode_workspace_size(0, 8, 128, 10, 512) == 0
+    assert lib.pa_decode_workspace_size(4, 8, 2, 128, 1000, 512) == 256 + 64 * 128 * 4 + 2 * 256
+    assert lib.pa_decode_workspace_size(4, 8, 2, 128, 0, 512) == 256 + 32 * 128 * 4 + 2 * 256
+    assert lib.pa_decode_workspace_size(0, 8, 2, 128, 10, 512) == 0

@@ -32,10 +32,11 @@ def _run(w, kind, partition=512):
     if kind == "one_pass":
         out = ops.decode_one_pass(*args)
     elif kind == "split":
-        ws = ops.new_workspace(w.num_seqs, w.num_heads, w.head_dim, w.max_seq_len, partition, device=DEV)
+        ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, partition,
+                               device=DEV)
         out = ops.decode_split(*args, partition, ws)
     else:
-        ws = ops.new_workspace(w.num_seqs, w.num_heads, w.head_dim, w.max_seq_len, device=DEV)
+        ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, device=DEV)
         out = ops.decode(*args, workspace=ws)
     torch.cuda.synchronize()
     return bf16_to_host_bits(out)
@@ -128,7 +129,7 @@ def test_partitions_and_reduce_match_oracle(Hq, Hkv, part):
     w = wl.random_decode_case(88, num_seqs=len(lens), num_heads=Hq, num_kv_heads=Hkv, head_dim=128,
                               block_size=16, lengths=lens, spare_blocks=1)
     d = _dev_inputs(w)
-    ws = ops.new_workspace(w.num_seqs, Hq, 128, w.max_seq_len, part, device=DEV)
+    ws = ops.new_workspace(w.num_seqs, Hq, Hkv, 128, w.max_seq_len, part, device=DEV)
     o, m, l = ops.decode_partitions(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
                                     d["seq_lens"], w.scale, w.max_seq_len, part, ws)
     torch.cuda.synchronize()

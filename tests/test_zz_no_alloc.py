@@ -35,9 +35,10 @@ def test_noalloc_split_matches_workspace_split_on_two_calls():
     w = wl.make("gqa", num_seqs=32)
     part = 512
     q, kc, vc, bt, sl = _inputs(w)
-    need = ops.decode_workspace_size(w.num_seqs, w.num_heads, w.head_dim, w.max_seq_len, part)
+    need = ops.decode_workspace_size(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, part)
     assert need <= ops.NOALLOC_SCRATCH_BYTES
-    ws = ops.new_workspace(w.num_seqs, w.num_heads, w.head_dim, w.max_seq_len, part, device=DEV)
+    ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, part,
+                           device=DEV)
     ref = ops.decode_split(q, kc, vc, bt, sl, w.scale, w.max_seq_len, part, ws)
     torch.cuda.synchronize()
     ref_bits = bf16_to_host_bits(ref)
@@ -54,7 +55,7 @@ def test_noalloc_split_rejects_a_problem_beyond_its_scratch():
     # all 128 sequences at partition 16: ~270 MB of split workspace
     w = wl.make("gqa", fill_cache=False)
     q, kc, vc, bt, sl = _inputs(w)
-    assert ops.decode_workspace_size(w.num_seqs, w.num_heads, w.head_dim, w.max_seq_len, 16) > \
+    assert ops.decode_workspace_size(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, 16) > \
         ops.NOALLOC_SCRATCH_BYTES
     with pytest.raises(PagedKVError) as err:
         ops.decode_split_noalloc(q, kc, vc, bt, sl, w.scale, w.max_seq_len, 16)
