@@ -85,6 +85,7 @@ constexpr int kTileTokens = 16;
 constexpr int kItemSlots = 2;
 constexpr int kChunkSlots = 4;
 constexpr int kChunkBlocks = 32;
+constexpr int kSortKeys = 256;  // size classes (16-token tiles) of the largest-first item order
 constexpr float kLn2 = 0.693147180559945309f;
 // A column's softmax reference max moves only when a logit exceeds it by more
 // than this (log2 units), so unnormalised weights stay below 2^8.
@@ -206,8 +207,9 @@ struct DecodeSmem {
     static constexpr int kNumBars = 2 * Geo::kStages + 2 * kItemSlots + 2 * kChunkSlots;
     static constexpr int kFlagOff = kBarOff + kNumBars * 8;
     static constexpr int kPrefixOff = kFlagOff + 16;
-    // bytes of dynamic shared memory for a launch with prefix_entries prefix ints
-    static constexpr int bytes(int prefix_entries) { return 1024 + kPrefixOff + 4 * prefix_entries; }
+    // bytes of dynamic shared memory for a launch over num_seqs sequences
+    // (enumeration tables: pf[B + 1], rest_order[B], sort keys)
+    static constexpr int bytes(int num_seqs) { return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys); }
 };
 
 template <int D, int BS, int MODE, int GC>
@@ -268,9 +270,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     pdl_wait();
     pdl_launch_dependents();
 
-    // ---- compact enumeration of the items: prefix[s] = partitions before sequence s
-    auto nparts_of = [&](int L) {
-        return (split && L > 0) ? min((L + p.part_tokens - 1) / p.part_tokens, p.max_parts) : 1;
+    // ---- enumeration of the work items, largest first.  Per sequence (length L
+    // clamped to its table): f = number of full partitions of part_tokens
+    // positions, plus one "rest" pair for the remainder (or for an empty
+    // sequence, whose output is zeros).  Pair order: every full partition first
+    // (sequence-major), then the rest pairs by size, largest first (a stable,
+    // deterministic counting sort, so every CTA derives the same order; the
+    // tail of the launch is made of the smallest items).  One pass: no full
+    // partitions, every sequence is a rest pair, so sequences go longest first.
+    // Item = pair * Hkv + KV head.  pf[s] = full partitions before sequence s.
+    int *const pf = prefix;                    // [B + 1]
+    int *const rest_order = prefix + B + 1;    // [B]
+    int *const sort_base = rest_order + B;     // [kSortKeys]
+    const int Lcap = p.max_blocks * BS;
+    auto full_of = [&](int L) {
+        return (split && L > 0) ? min(L / p.part_tokens, p.max_parts) : 0;
+    };
+    auto rest_key = [&](int L) -> int {        // -1: no rest pair
+        const int f = full_of(L);
+        if (split && L > 0 && (f == p.max_parts || L == f * p.part_tokens)) return -1;
+        const int r = max(L, 0) - f * (split ? p.part_tokens : 0);
+        return min((r + kTileTokens - 1) / kTileTokens, kSortKeys - 1);
     };
     __shared__ int warp_tot[kDecodeThreads / 32];
     if (split) {
@@ -278,7 +298,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         const int s0 = min(B, (int)threadIdx.x * per);
         const int s1 = min(B, s0 + per);
         int local = 0;
-        for (int s = s0; s < s1; ++s) local += nparts_of(p.seq_lens[s]);
+        for (int s = s0; s < s1; ++s) local += full_of(min(p.seq_lens[s], Lcap));
         // block-wide exclusive scan of `local`
         int incl = local;
 #pragma unroll
@@ -291,28 +311,77 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         int run = incl - local;
         for (int w = 0; w < warp; ++w) run += warp_tot[w];
         for (int s = s0; s < s1; ++s) {
-            prefix[s] = run;
-            run += nparts_of(p.seq_lens[s]);
+            pf[s] = run;
+            run += full_of(min(p.seq_lens[s], Lcap));
         }
-        if (threadIdx.x == kDecodeThreads - 1) prefix[B] = run;
+        if (threadIdx.x == kDecodeThreads - 1) pf[B] = run;
     }
     __syncthreads();
-    const int total_sp = split ? prefix[B] : B;
-    const int total_items = total_sp * Hkv;
+    const int total_full = split ? pf[B] : 0;
 
     if (warp == kSchedulerWarp) {
         // ------------------------------------------------------------ scheduler
+        // rest pairs sorted by size, largest first: counting sort over kSortKeys
+        // tile-count keys, stable in sequence order (match_any ranks lanes)
+        for (int k = lane; k < kSortKeys; k += 32) sort_base[k] = 0;
+        __syncwarp();
+        for (int c = 0; c < B; c += 32) {
+            const int key = c + lane < B ? rest_key(min(p.seq_lens[c + lane], Lcap)) : -1;
+            if (key >= 0) atomicAdd(&sort_base[key], 1);
+        }
+        __syncwarp();
+        int total_rest;
+        {
+            // exclusive scan in descending key order; lane owns kSortKeys/32 keys
+            constexpr int KPL = kSortKeys / 32;
+            int cnt[KPL], sum = 0;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                cnt[i] = sort_base[kSortKeys - 1 - (lane * KPL + i)];
+                sum += cnt[i];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            total_rest = __shfl_sync(0xffffffffu, incl, 31);
+            int run = incl - sum;
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                sort_base[kSortKeys - 1 - (lane * KPL + i)] = run;
+                run += cnt[i];
+            }
+        }
+        __syncwarp();
+        for (int c = 0; c < B; c += 32) {
+            const int key = c + lane < B ? rest_key(min(p.seq_lens[c + lane], Lcap)) : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, key);
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            if (key >= 0) rest_order[sort_base[key] + rank] = c + lane;
+            __syncwarp();
+            if (key >= 0 && rank == 0) sort_base[key] += __popc(peers);
+            __syncwarp();
+        }
+        const int total_items = (total_full + total_rest) * Hkv;
+
+        // Each CTA starts on item blockIdx.x; later items come from the atomic
+        // counter (offset by the grid size) or round-robin without a workspace.
         int rr_next = blockIdx.x;
+        bool first_grab = true;
         auto grab = [&]() -> int {
             int v = 0;
             if (lane == 0) {
-                if (p.sched) {
-                    v = atomicAdd(&p.sched[0], 1);
-                } else {
+                if (first_grab || !p.sched) {
                     v = rr_next;
                     rr_next += gridDim.x;
+                } else {
+                    v = (int)gridDim.x + atomicAdd(&p.sched[0], 1);
                 }
             }
+            first_grab = false;
             return __shfl_sync(0xffffffffu, v, 0);
         };
         int idx = grab();
@@ -337,23 +406,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             if (have) {
                 const int sp = idx / Hkv;
                 it.g = idx - sp * Hkv;
-                if (split) {
-                    int lo = 0, hi = B;  // largest s with prefix[s] <= sp
+                if (sp < total_full) {
+                    int lo = 0, hi = B;  // largest s with pf[s] <= sp
                     while (hi - lo > 1) {
                         const int mid = (lo + hi) >> 1;
-                        if (prefix[mid] <= sp) lo = mid; else hi = mid;
+                        if (pf[mid] <= sp) lo = mid; else hi = mid;
                     }
                     it.s = lo;
-                    it.part = sp - prefix[lo];
-                    it.nparts = prefix[lo + 1] - prefix[lo];
+                    it.part = sp - pf[lo];
                 } else {
-                    it.s = sp;
-                    it.part = 0;
-                    it.nparts = 1;
+                    it.s = rest_order[sp - total_full];
+                    it.part = -1;  // the rest pair: after the full partitions
                 }
-                const int L = min(p.seq_lens[it.s], p.max_blocks * BS);
+                const int L = min(p.seq_lens[it.s], Lcap);
+                const int f = full_of(L);
+                it.nparts = f + (rest_key(L) >= 0 ? 1 : 0);
+                if (it.part < 0) it.part = f;
                 it.t_begin = split ? it.part * p.part_tokens : 0;
-                it.t_end = split ? min(L, it.t_begin + p.part_tokens) : L;
+                it.t_end = split ? min(L, it.t_begin + p.part_tokens) : max(L, 0);
                 it.n_tiles = it.t_end > it.t_begin ? (it.t_end - it.t_begin + kTileTokens - 1) / kTileTokens : 0;
                 it.ring_base = ring_base;
                 it.stop = 0;
@@ -867,7 +937,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
              t += (int64_t)gridDim.x * kDecodeThreads) {
             const int part = (int)(t % p.max_parts);
             const int s = (int)(t / ((int64_t)p.num_heads * p.max_parts));
-            if (part < prefix[s + 1] - prefix[s]) continue;
+            const int L = min(p.seq_lens[s], Lcap);
+            if (part < full_of(L) + (rest_key(L) >= 0 ? 1 : 0)) continue;
             p.ws_m[t] = -INFINITY;
             p.ws_l[t] = 0.f;
             for (int d = 0; d < D; ++d) p.ws_o[t * D + d] = 0.f;

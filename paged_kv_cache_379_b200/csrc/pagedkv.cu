@@ -100,9 +100,8 @@ static int launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const C
 {
     using Lay = DecodeSmem<D, BS, MODE, GC>;
     auto kernel = paged_decode_kernel<D, BS, MODE, GC>;
-    const int prefix_entries = p.max_parts > 1 ? p.num_seqs + 1 : 0;
-    const size_t smem = (size_t)Lay::bytes(prefix_entries);
-    if (smem > 227 * 1024) return PA_ERR_BAD_SHAPE;  // too many sequences for the split form
+    const size_t smem = (size_t)Lay::bytes(p.num_seqs);
+    if (smem > 227 * 1024) return PA_ERR_BAD_SHAPE;  // too many sequences for the enumeration tables
     int rc = ensure_smem(reinterpret_cast<const void *>(kernel), smem);
     if (rc != PA_OK) return rc;
     int occ = 0;
