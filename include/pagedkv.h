@@ -148,9 +148,9 @@ int pa_decode(void *out, const void *query, const void *key_cache, const void *v
 
 /* The plan pa_decode follows for these sizes: 0 = one pass (one launch),
  * otherwise the partition size of the split form (partition kernel + reduce
- * kernel, two launches).  One pass when max_seq_len <= 1536 and the
+ * kernel, two launches).  One pass when max_seq_len <= 2048 and the
  * (sequence, KV head) units give every SM several items; else partitions of
- * 512 positions (2048 beyond 16384), halved while the batch is too small to
+ * 1024 positions (2048 beyond 16384), halved while the batch is too small to
  * give every SM several items.  A workspace smaller than the split form needs
  * gives one pass.  No device work. */
 int pa_decode_plan(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_seq_len,
@@ -310,6 +310,32 @@ int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, i
                            int64_t *slot_mapping, int64_t *src_dst_pairs, int *num_pairs);
 /* Release every block of the first n entries of a table row. */
 int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n);
+
+/* --------------------------------------------------------------------------
+ * Prefix caching in the host block pool ([深度解析 «Copy-on-Write 与 Prefix
+ * Caching»]: a block is recognised by hash(token_ids[0:block_size]); a prompt
+ * that starts with the same tokens references the existing blocks, an O(1)
+ * lookup).  The hash of a full block is chained with its parent's, so equal
+ * blocks behind different prefixes do not match:
+ *   pa_block_hash(parent, tokens, n) = FNV-1a-64 over the 8 little-endian bytes
+ *   of `parent` followed by the 4 little-endian bytes of each token id;
+ *   the first block of a prompt has parent 0.
+ * pa_pool_allocate_prompt_cached builds the table of a prompt of num_tokens
+ * tokens: the leading run of full blocks whose chained hashes are registered
+ * (and alive) is referenced (refcount + 1, *num_cached_tokens = their tokens,
+ * whose K/V need no recomputation); every later block is taken from the free
+ * list, and the full ones among them are registered under their hashes.  A
+ * partly filled last block is never registered (it will be written).  A block
+ * leaves the cache when its reference count returns to 0.  PA_ERR_POOL_EXHAUSTED
+ * (no change) if the free list is too short, PA_ERR_BAD_SHAPE if the table
+ * needs more than max_blocks entries.
+ * ------------------------------------------------------------------------ */
+uint64_t pa_block_hash(uint64_t parent_hash, const int32_t *token_ids, int num_tokens);
+int pa_pool_allocate_prompt_cached(pa_pool *pool, const int32_t *token_ids, int num_tokens,
+                                   int32_t *table_out, int max_blocks, int *num_table_blocks,
+                                   int *num_cached_tokens);
+/* Number of blocks currently registered in the prefix cache. */
+int pa_pool_num_cached_blocks(const pa_pool *pool);
 
 #ifdef __cplusplus
 }

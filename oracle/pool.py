@@ -24,9 +24,33 @@ Readings where the pages are silent:
   * A block whose reference count reaches 0 returns to the free list.
   * Copy-on-write is decided per write: reference count > 1 -> take a fresh block,
     record (src, dst), decrement src.  The last remaining owner writes in place.
+  * Prefix caching ([深度解析 «Copy-on-Write 与 Prefix Caching»]: hash =
+    hash(token_ids[0:block_size]); an existing block with the same prefix is
+    referenced, O(1)).  The hash is 64-bit FNV-1a, chained: a block's hash covers
+    the previous block's hash (8 little-endian bytes; 0 for the first block) and
+    its token ids (4 little-endian bytes each).  Only the leading run of cached
+    full blocks of a prompt is reused; later full blocks are registered; a
+    partly filled block never is; a block leaves the cache when it is freed.
 """
 
 from __future__ import annotations
+
+FNV_OFFSET = 14695981039346656037
+FNV_PRIME = 1099511628211
+MASK64 = (1 << 64) - 1
+
+
+def fnv1a_64(data: bytes, h: int = FNV_OFFSET) -> int:
+    """64-bit FNV-1a: for each byte, h = (h XOR byte) * prime mod 2^64."""
+    for byte in data:
+        h = ((h ^ byte) * FNV_PRIME) & MASK64
+    return h
+
+
+def block_hash(parent_hash: int, token_ids) -> int:
+    data = (parent_hash & MASK64).to_bytes(8, "little")
+    data += b"".join((int(t) & 0xFFFFFFFF).to_bytes(4, "little") for t in token_ids)
+    return fnv1a_64(data)
 
 
 class PoolExhausted(RuntimeError):
@@ -44,6 +68,8 @@ class OraclePool:
         self.block_size = block_size
         self.free_list = list(free_order)
         self.refcount = [0] * num_blocks
+        self.cache = {}          # chained block hash -> block id
+        self.hash_of = {}        # block id -> the hash it is registered under
 
     # -- BlockAllocator ([源码解析 §三]) --------------------------------------
     def get_num_free_blocks(self) -> int:
@@ -64,6 +90,9 @@ class OraclePool:
             raise ValueError(f"block {block_id} is not allocated")
         self.refcount[block_id] -= 1
         if self.refcount[block_id] == 0:
+            h = self.hash_of.pop(block_id, None)
+            if h is not None and self.cache.get(h) == block_id:
+                del self.cache[h]
             self.free_list.append(block_id)
 
     # -- sharing and copy-on-write ([源码解析 §五], [论文专题 共享前缀和 copy-on-write]) --
@@ -124,6 +153,39 @@ class OraclePool:
         used = {b for t in tables for b in t}
         live = sum(int(x) for x in seq_lens)
         return live / (len(used) * self.block_size) if used else 0.0
+
+    # -- prefix caching ([深度解析 «Copy-on-Write 与 Prefix Caching»]) ----------------
+    def allocate_prompt_cached(self, token_ids):
+        """(table, num_cached_tokens) for a prompt, reusing the leading cached blocks."""
+        bs = self.block_size
+        toks = [int(t) for t in token_ids]
+        n_full = len(toks) // bs
+        n_all = -(-len(toks) // bs)
+        hashes, parent = [], 0
+        for j in range(n_full):
+            parent = block_hash(parent, toks[j * bs:(j + 1) * bs])
+            hashes.append(parent)
+        hits = 0
+        while hits < n_full and hashes[hits] in self.cache and self.refcount[self.cache[hashes[hits]]] > 0:
+            hits += 1
+        if n_all - hits > len(self.free_list):
+            raise PoolExhausted(f"need {n_all - hits}, {len(self.free_list)} free")
+        table = []
+        for j in range(hits):
+            b = self.cache[hashes[j]]
+            self.refcount[b] += 1
+            table.append(b)
+        for j in range(hits, n_all):
+            b = self.free_list.pop()
+            self.refcount[b] = 1
+            table.append(b)
+            if j < n_full:
+                old = self.cache.get(hashes[j])
+                if old is not None:
+                    self.hash_of.pop(old, None)
+                self.cache[hashes[j]] = b
+                self.hash_of[b] = hashes[j]
+        return table, hits * bs
 
 
 def slot_of(table, pos: int, block_size: int) -> int:

@@ -48,6 +48,9 @@ SIGNATURES = {
     "pa_pool_import": (_I, [_P, _P, _I, _I, _P]),
     "pa_pool_prepare_decode": (_I, [_P, _I, _P, _I, _P, _P, _P, _P, _P]),
     "pa_pool_free_table": (_I, [_P, _P, _I]),
+    "pa_block_hash": (ctypes.c_uint64, [ctypes.c_uint64, _P, _I]),
+    "pa_pool_allocate_prompt_cached": (_I, [_P, _P, _I, _P, _I, _P, _P]),
+    "pa_pool_num_cached_blocks": (_I, [_P]),
 }
 
 _lib = None

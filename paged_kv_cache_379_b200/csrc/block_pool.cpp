@@ -20,7 +20,9 @@
 // freed blocks are pushed on the end.  Both are O(1).
 
 #include <cstdint>
+#include <cstring>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "../../include/pagedkv.h"
@@ -30,7 +32,37 @@ struct pa_pool {
     int block_size;
     std::vector<int32_t> free_stack;   // top = back()
     std::vector<int32_t> refcount;
+    // prefix cache: chained hash of a full block's tokens -> the block holding them
+    std::unordered_map<uint64_t, int32_t> cache;
+    std::vector<uint64_t> block_hash;  // hash a block is registered under
+    std::vector<char> registered;
 };
+
+namespace {
+
+// 64-bit FNV-1a (offset basis 14695981039346656037, prime 1099511628211).
+constexpr uint64_t kFnvOffset = 14695981039346656037ull;
+constexpr uint64_t kFnvPrime = 1099511628211ull;
+
+uint64_t fnv1a(uint64_t h, const unsigned char *bytes, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) {
+        h ^= bytes[i];
+        h *= kFnvPrime;
+    }
+    return h;
+}
+
+// Drop a block's prefix-cache entry (when it returns to the free list).
+void unregister_block(pa_pool *pool, int32_t b)
+{
+    if (!pool->registered[b]) return;
+    auto it = pool->cache.find(pool->block_hash[b]);
+    if (it != pool->cache.end() && it->second == b) pool->cache.erase(it);
+    pool->registered[b] = 0;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -43,6 +75,8 @@ pa_pool *pa_pool_create(int num_blocks, int block_size, const int32_t *free_orde
         p->num_blocks = num_blocks;
         p->block_size = block_size;
         p->refcount.assign(num_blocks, 0);
+        p->block_hash.assign(num_blocks, 0);
+        p->registered.assign(num_blocks, 0);
         p->free_stack.resize(num_blocks);
         if (free_order) {
             std::vector<char> seen(num_blocks, 0);
@@ -101,7 +135,10 @@ int pa_pool_free(pa_pool *pool, int block)
 {
     if (!pool) return PA_ERR_NULL_POINTER;
     if (block < 0 || block >= pool->num_blocks || pool->refcount[block] <= 0) return PA_ERR_BAD_BLOCK;
-    if (--pool->refcount[block] == 0) pool->free_stack.push_back(block);
+    if (--pool->refcount[block] == 0) {
+        unregister_block(pool, block);
+        pool->free_stack.push_back(block);
+    }
     return PA_OK;
 }
 
@@ -207,6 +244,77 @@ int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n)
         if (rc != PA_OK) return rc;
     }
     return PA_OK;
+}
+
+// Prefix caching ("vLLM 核心源码深度解析 …", «Copy-on-Write 与 Prefix Caching»: a
+// block is identified by the hash of its tokens, so a request whose prompt
+// starts with the same tokens references the existing blocks -- an O(1)
+// lookup).  The hash is chained with the previous block's, so two equal blocks
+// behind different prefixes do not match.
+uint64_t pa_block_hash(uint64_t parent_hash, const int32_t *token_ids, int num_tokens)
+{
+    unsigned char buf[8];
+    for (int i = 0; i < 8; ++i) buf[i] = (unsigned char)(parent_hash >> (8 * i));
+    uint64_t h = fnv1a(kFnvOffset, buf, 8);
+    for (int t = 0; t < num_tokens; ++t) {
+        const uint32_t v = (uint32_t)token_ids[t];
+        unsigned char tb[4] = {(unsigned char)v, (unsigned char)(v >> 8), (unsigned char)(v >> 16),
+                               (unsigned char)(v >> 24)};
+        h = fnv1a(h, tb, 4);
+    }
+    return h;
+}
+
+int pa_pool_allocate_prompt_cached(pa_pool *pool, const int32_t *token_ids, int num_tokens, int32_t *table_out,
+                                   int max_blocks, int *num_table_blocks, int *num_cached_tokens)
+{
+    if (!pool || !table_out || !num_table_blocks || !num_cached_tokens || (num_tokens > 0 && !token_ids))
+        return PA_ERR_NULL_POINTER;
+    if (num_tokens < 0) return PA_ERR_BAD_SHAPE;
+    const int bs = pool->block_size;
+    const int n_full = num_tokens / bs;
+    const int n_all = (num_tokens + bs - 1) / bs;
+    if (n_all > max_blocks) return PA_ERR_BAD_SHAPE;
+    // blocks this prompt must take from the free list: everything after the leading cached run
+    std::vector<uint64_t> hashes(n_full);
+    uint64_t parent = 0;
+    int hits = 0;
+    for (int j = 0; j < n_full; ++j) {
+        hashes[j] = pa_block_hash(parent, token_ids + (int64_t)j * bs, bs);
+        parent = hashes[j];
+        if (hits == j) {
+            auto it = pool->cache.find(hashes[j]);
+            if (it != pool->cache.end() && pool->refcount[it->second] > 0) ++hits;
+        }
+    }
+    if ((size_t)(n_all - hits) > pool->free_stack.size()) return PA_ERR_POOL_EXHAUSTED;
+    for (int j = 0; j < hits; ++j) {
+        const int32_t b = pool->cache.find(hashes[j])->second;
+        ++pool->refcount[b];
+        table_out[j] = b;
+    }
+    for (int j = hits; j < n_all; ++j) {
+        const int32_t b = pool->free_stack.back();
+        pool->free_stack.pop_back();
+        pool->refcount[b] = 1;
+        table_out[j] = b;
+        if (j < n_full) {  // a full block: later prompts with this prefix may reuse it
+            auto it = pool->cache.find(hashes[j]);
+            if (it != pool->cache.end()) pool->registered[it->second] = 0;
+            pool->cache[hashes[j]] = b;
+            pool->block_hash[b] = hashes[j];
+            pool->registered[b] = 1;
+        }
+    }
+    *num_table_blocks = n_all;
+    *num_cached_tokens = hits * bs;
+    return PA_OK;
+}
+
+int pa_pool_num_cached_blocks(const pa_pool *pool)
+{
+    if (!pool) return PA_ERR_NULL_POINTER;
+    return (int)pool->cache.size();
 }
 
 }  // extern "C"

@@ -263,21 +263,22 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
 }
 
 // pa_decode's plan: 0 = one pass, else the partition size of the split form.
-// Chosen from measurements on B200 (head_dim 128, bs 16): one pass wins when
-// every sequence is short and the (sequence, KV head) units alone give every
-// SM several items (shared-prefix batch, max 1280 tokens: 203 us one pass vs
-// 311 us split); otherwise 512-token partitions (GQA batch 135 us, MHA batch
-// 221 us) up to 16K positions and 2048-token ones beyond (128K-context batch
-// 445 us vs 502 us at 512); partitions shrink until a small batch still yields
-// several items per resident CTA.
-static constexpr int kOnePassMaxLen = 1536;
+// Chosen from measurements on B200 (head_dim 128, bs 16, largest-first item
+// order): one pass wins when every sequence is short and the (sequence, KV
+// head) units alone give every SM several items (MHA batch, max 2048: 209 us
+// one pass vs 212 us at 512; shared-prefix batch, max 1280: 192 vs 206 us);
+// otherwise 1024-token partitions (GQA batch, max 4096: 115 us vs 118 us at 512
+// and 126 us one pass) up to 16K positions and 2048-token ones beyond (128K
+// context: 439 us vs 458 us at 1024); partitions shrink until a small batch
+// still yields several items per resident CTA.
+static constexpr int kOnePassMaxLen = 2048;
 
 static int choose_plan(int num_seqs, int num_kv_heads, int max_seq_len)
 {
     const int64_t units = (int64_t)num_seqs * num_kv_heads;
     const int64_t target = 8LL * std::max(1, sm_count());  // ~4 items per resident CTA
     if (max_seq_len <= kOnePassMaxLen && units >= target / 2) return 0;
-    int part = max_seq_len > 16384 ? 2048 : 512;
+    int part = max_seq_len > 16384 ? 2048 : 1024;
     while (part > 64 && units * std::max<int64_t>(1, max_seq_len / (2 * part)) < target) part /= 2;
     return part;
 }

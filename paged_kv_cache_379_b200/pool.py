@@ -113,3 +113,27 @@ class BlockPool:
     def free_table(self, table) -> None:
         ids = np.ascontiguousarray(table, dtype=np.int32)
         check("pa_pool_free_table", load().pa_pool_free_table(self._h, _ptr(ids), int(ids.size)))
+
+    # ---- prefix caching ----------------------------------------------------------
+    def allocate_prompt_cached(self, token_ids, max_blocks: int | None = None):
+        """Table for a prompt, reusing registered full blocks of an equal prefix.
+
+        Returns (table, num_cached_tokens)."""
+        toks = np.ascontiguousarray(token_ids, dtype=np.int32)
+        n_all = -(-toks.size // self.block_size)
+        cap = n_all if max_blocks is None else int(max_blocks)
+        table = np.empty(max(cap, 1), dtype=np.int32)
+        nb = ctypes.c_int(0)
+        cached = ctypes.c_int(0)
+        check("pa_pool_allocate_prompt_cached", load().pa_pool_allocate_prompt_cached(
+            self._h, _ptr(toks), int(toks.size), _ptr(table), cap, ctypes.byref(nb), ctypes.byref(cached)))
+        return table[:nb.value].tolist(), cached.value
+
+    def num_cached_blocks(self) -> int:
+        return int(load().pa_pool_num_cached_blocks(self._h))
+
+
+def block_hash(parent_hash: int, token_ids) -> int:
+    """pa_block_hash: chained FNV-1a-64 of a block's tokens."""
+    toks = np.ascontiguousarray(token_ids, dtype=np.int32)
+    return int(load().pa_block_hash(ctypes.c_uint64(parent_hash), _ptr(toks), int(toks.size)))
