@@ -58,6 +58,7 @@ extern "C" {
 #define PA_ERR_ALIGNMENT (-8)      /* a device pointer is not 16-byte aligned         */
 #define PA_ERR_DEVICE_TIMEOUT (-9) /* a bounded on-device wait gave up (see below)   */
 #define PA_ERR_SCRATCH_TOO_SMALL (-10) /* the built-in scratch of the no-allocation call is too small */
+#define PA_ERR_NOT_DEVICE_ACCESSIBLE (-11) /* a pointer the kernel would read is not device-accessible */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *pa_status_string(int status);
@@ -109,6 +110,26 @@ int pa_reshape_and_cache(const void *key, const void *value, void *key_cache, vo
  * ------------------------------------------------------------------------ */
 int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Swap of whole blocks between two caches in different memories -- the GPU
+ * cache and a cache in pinned host memory -- for a two-level GPU/CPU block
+ * allocator that swaps cold blocks out to host memory when the GPU runs short
+ * and back in when they are needed ([深度解析 «BlockAllocator 源码核心»],
+ * CpuGpuBlockAllocator).  Pair i copies src block src_dst_pairs[i][0] of
+ * (src_key_cache, src_value_cache) to dst block src_dst_pairs[i][1] of
+ * (dst_key_cache, dst_value_cache); both caches are [num_blocks, block_size,
+ * num_kv_heads, head_dim] bf16 with their own block counts.  A device kernel
+ * does the gather/scatter, so host-side caches and the pairs must be
+ * device-accessible: device memory or pinned, mapped host memory
+ * (cudaHostAlloc / cudaMallocHost / cudaHostRegister).  Pageable host memory
+ * is rejected with PA_ERR_NOT_DEVICE_ACCESSIBLE before any launch.  Pairs with
+ * ids outside their cache are skipped.
+ * ------------------------------------------------------------------------ */
+int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, const void *src_key_cache,
+                   const void *src_value_cache, const int64_t *src_dst_pairs, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int src_num_blocks,
+                   int dst_num_blocks, void *stream);
 
 /* --------------------------------------------------------------------------
  * a4-a6. Single-query paged decode attention ([源码解析 §四] paged_attention;
@@ -310,6 +331,16 @@ int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, i
                            int64_t *slot_mapping, int64_t *src_dst_pairs, int *num_pairs);
 /* Release every block of the first n entries of a table row. */
 int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n);
+
+/* Swap planning between two pools (GPU pool and host pool): every distinct
+ * block of table[0..n) gets a block in `dst` (reference count = its number of
+ * entries in the table), the table is rewritten to the dst ids, each source
+ * block loses those references (returning to src's free list at zero), and
+ * one (src, dst) pair per distinct block is written to src_dst_pairs
+ * (int64 [n, 2], host) for pa_swap_blocks.  PA_ERR_POOL_EXHAUSTED and no
+ * change if dst has too few free blocks. */
+int pa_pool_swap_plan(pa_pool *src, pa_pool *dst, int32_t *table, int n, int64_t *src_dst_pairs,
+                      int *num_pairs);
 
 /* --------------------------------------------------------------------------
  * Prefix caching in the host block pool ([深度解析 «Copy-on-Write 与 Prefix

@@ -12,6 +12,7 @@ Functions, each restating a passage of the pages (see ``oracle.c`` and
 * :func:`slot_mapping`      -- address translation pos -> physical slot
 * :func:`reshape_and_cache` -- write new K/V rows at their slots
 * :func:`copy_blocks`       -- copy-on-write block copies
+* :func:`swap_blocks`       -- whole-block copies between a GPU and a host cache
 * :func:`paged_decode`      -- softmax(scale * q K^T) V, K/V gathered through the table
 * :func:`paged_decode_partials`, :func:`lse_merge` -- the split form and its merge
 * :class:`pool.OraclePool`  -- free list, reference counts, fork, copy-on-write
@@ -55,6 +56,8 @@ def _load():
         lib.oracle_reshape_and_cache.restype = None
         lib.oracle_copy_blocks.argtypes = [P, P, P, I, I, I, I]
         lib.oracle_copy_blocks.restype = None
+        lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I]
+        lib.oracle_swap_blocks.restype = None
         lib.oracle_paged_decode.argtypes = [P, P, P, P, P, P, ctypes.c_double, I, I, I, I, I, I, I]
         lib.oracle_paged_decode.restype = None
         lib.oracle_paged_decode_partials.argtypes = [P, P, P, P, P, P, P, P, ctypes.c_double,
@@ -116,6 +119,19 @@ def copy_blocks(key_cache, value_cache, pairs) -> None:
     assert key_cache.dtype == np.uint16 and key_cache.flags.c_contiguous
     lib.oracle_copy_blocks(key_cache.ctypes.data_as(ctypes.c_void_p),
                            value_cache.ctypes.data_as(ctypes.c_void_p), prp, pr.shape[0], H, D, bs)
+
+
+def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, pairs) -> None:
+    """In place on dst_*: whole-block copies from the src caches."""
+    lib = _load()
+    pr, prp = _c(np.asarray(pairs, dtype=np.int64).reshape(-1, 2), np.int64)
+    sk, skp = _c(src_key_cache, np.uint16)
+    sv, svp = _c(src_value_cache, np.uint16)
+    for a in (dst_key_cache, dst_value_cache):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous
+    nb, bs, H, D = sk.shape
+    lib.oracle_swap_blocks(dst_key_cache.ctypes.data_as(ctypes.c_void_p),
+                           dst_value_cache.ctypes.data_as(ctypes.c_void_p), skp, svp, prp, pr.shape[0], H, D, bs)
 
 
 def paged_decode(query, key_cache, value_cache, block_tables, seq_lens, scale: float,

@@ -112,6 +112,26 @@ void oracle_copy_blocks(uint16_t *key_cache, uint16_t *value_cache,
 }
 
 /*
+ * Swap of whole blocks between two caches (GPU cache and host cache), the copy
+ * behind the GPU/CPU swap of "vLLM 核心源码深度解析 …", «BlockAllocator 源码核心»:
+ * pair i copies block src of (src_k, src_v) into block dst of (dst_k, dst_v).
+ */
+void oracle_swap_blocks(uint16_t *dst_k, uint16_t *dst_v, const uint16_t *src_k, const uint16_t *src_v,
+                        const int64_t *src_dst_pairs, int num_pairs, int num_kv_heads, int head_dim,
+                        int block_size)
+{
+    int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+    for (int i = 0; i < num_pairs; ++i) {
+        int64_t src = src_dst_pairs[2 * i];
+        int64_t dst = src_dst_pairs[2 * i + 1];
+        for (int64_t e = 0; e < block_elems; ++e) {
+            dst_k[dst * block_elems + e] = src_k[src * block_elems + e];
+            dst_v[dst * block_elems + e] = src_v[src * block_elems + e];
+        }
+    }
+}
+
+/*
  * Gather of one sequence's logical K (or V) rows for one KV head into a
  * contiguous [len, head_dim] double array, walking the block table exactly as
  * [论文专题 «PagedAttention：逻辑连续，物理不必连续»] describes: logical block j

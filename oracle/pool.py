@@ -188,6 +188,34 @@ class OraclePool:
         return table, hits * bs
 
 
+def swap_plan(src: OraclePool, dst: OraclePool, table):
+    """Move a table's blocks from pool `src` to pool `dst` (the swap of the GPU/CPU
+    two-level allocator, [深度解析 «BlockAllocator 源码核心»]).
+
+    Every distinct block gets one dst block, in order of first appearance; its
+    dst reference count is its number of entries in the table; every entry gives
+    up its reference on the src block.  Returns (new_table, [(src, dst), ...])."""
+    distinct = list(dict.fromkeys(int(b) for b in table))
+    for b in distinct:
+        if src.refcount[b] <= 0:
+            raise ValueError(f"block {b} is not allocated")
+    if len(distinct) > len(dst.free_list):
+        raise PoolExhausted(f"need {len(distinct)}, {len(dst.free_list)} free")
+    moved, pairs = {}, []
+    for b in distinct:
+        d = dst.free_list.pop()
+        dst.refcount[d] = 0
+        moved[b] = d
+        pairs.append((b, d))
+    new_table = []
+    for b in table:
+        d = moved[int(b)]
+        dst.refcount[d] += 1
+        new_table.append(d)
+        src.free(int(b))
+    return new_table, pairs
+
+
 def slot_of(table, pos: int, block_size: int) -> int:
     """Address translation of [深度解析 «Block Table 数据结构»]: pos -> physical slot."""
     return table[pos // block_size] * block_size + pos % block_size

@@ -26,6 +26,7 @@ SIGNATURES = {
     "pa_slot_mapping": (_I, [_P, _P, _I, _I, _P, _P, _P, _I, _I, _P]),
     "pa_reshape_and_cache": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "pa_swap_blocks": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "pa_decode": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "pa_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "pa_decode_plan": (_I, [_I, _I, _I, _I, _I, _SZ]),
@@ -51,6 +52,7 @@ SIGNATURES = {
     "pa_block_hash": (ctypes.c_uint64, [ctypes.c_uint64, _P, _I]),
     "pa_pool_allocate_prompt_cached": (_I, [_P, _P, _I, _P, _I, _P, _P]),
     "pa_pool_num_cached_blocks": (_I, [_P]),
+    "pa_pool_swap_plan": (_I, [_P, _P, _P, _I, _P, _P]),
 }
 
 _lib = None

@@ -246,6 +246,43 @@ int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n)
     return PA_OK;
 }
 
+// Swap planning between two pools (the GPU pool and a host-memory pool, as in
+// the GPU/CPU two-level allocator with swap of "vLLM 核心源码深度解析 …",
+// «BlockAllocator 源码核心»): every distinct block of `table` gets a block in
+// `dst`, the table is rewritten to the new ids, the source blocks lose the
+// table's reference, and one (src, dst) pair per distinct block is emitted.
+int pa_pool_swap_plan(pa_pool *src, pa_pool *dst, int32_t *table, int n, int64_t *src_dst_pairs, int *num_pairs)
+{
+    if (!src || !dst || !num_pairs || (n > 0 && (!table || !src_dst_pairs))) return PA_ERR_NULL_POINTER;
+    if (n < 0) return PA_ERR_BAD_SHAPE;
+    if (src->block_size != dst->block_size) return PA_ERR_BAD_SHAPE;
+    std::unordered_map<int32_t, int32_t> moved;
+    for (int i = 0; i < n; ++i) {
+        const int32_t b = table[i];
+        if (b < 0 || b >= src->num_blocks || src->refcount[b] <= 0) return PA_ERR_BAD_BLOCK;
+        moved.emplace(b, -1);
+    }
+    if (moved.size() > dst->free_stack.size()) return PA_ERR_POOL_EXHAUSTED;
+    int np = 0;
+    for (int i = 0; i < n; ++i) {
+        const int32_t b = table[i];
+        int32_t &d = moved[b];
+        if (d < 0) {
+            d = dst->free_stack.back();
+            dst->free_stack.pop_back();
+            dst->refcount[d] = 0;
+            src_dst_pairs[2 * np] = b;
+            src_dst_pairs[2 * np + 1] = d;
+            ++np;
+        }
+        ++dst->refcount[d];
+        table[i] = d;
+        pa_pool_free(src, b);
+    }
+    *num_pairs = np;
+    return PA_OK;
+}
+
 // Prefix caching ("vLLM 核心源码深度解析 …", «Copy-on-Write 与 Prefix Caching»: a
 // block is identified by the hash of its tokens, so a request whose prompt
 // starts with the same tokens references the existing blocks -- an O(1)

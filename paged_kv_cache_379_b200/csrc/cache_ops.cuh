@@ -106,6 +106,50 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ ke
     }
 }
 
+// Block copies between two caches that may live in different memories (device
+// memory and pinned, mapped host memory): swap-out / swap-in.  One CTA per
+// (pair, slice), 16-byte accesses, two loads in flight per cache per thread.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(uint4 *__restrict__ dst_key, uint4 *__restrict__ dst_value,
+                                                          const uint4 *__restrict__ src_key,
+                                                          const uint4 *__restrict__ src_value,
+                                                          const int64_t *__restrict__ pairs, int64_t chunks_per_block,
+                                                          int slices, int64_t src_blocks, int64_t dst_blocks)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int pair = blockIdx.x / slices;
+    const int slice = blockIdx.x - pair * slices;
+    const int64_t src = pairs[2 * pair];
+    const int64_t dst = pairs[2 * pair + 1];
+    if (src < 0 || dst < 0 || src >= src_blocks || dst >= dst_blocks) return;  // ids outside the caches
+    const int64_t per_cta = (chunks_per_block + slices - 1) / slices;
+    const int64_t begin = slice * per_cta;
+    const int64_t end = min(chunks_per_block, begin + per_cta);
+    const uint4 *ks = src_key + src * chunks_per_block;
+    const uint4 *vs = src_value + src * chunks_per_block;
+    uint4 *kd = dst_key + dst * chunks_per_block;
+    uint4 *vd = dst_value + dst * chunks_per_block;
+    constexpr int U = 2;
+    int64_t c = begin + threadIdx.x;
+    for (; c + (U - 1) * blockDim.x < end; c += U * blockDim.x) {
+        uint4 k[U], v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            k[u] = ks[c + u * blockDim.x];
+            v[u] = vs[c + u * blockDim.x];
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            kd[c + u * blockDim.x] = k[u];
+            vd[c + u * blockDim.x] = v[u];
+        }
+    }
+    for (; c < end; c += blockDim.x) {
+        kd[c] = ks[c];
+        vd[c] = vs[c];
+    }
+}
+
 // Counts sequences that break a precondition of the decode kernels.
 __global__ void validate_tables_kernel(const int32_t *__restrict__ block_tables,
                                        const int32_t *__restrict__ seq_lens, int num_seqs, int max_blocks,

@@ -302,6 +302,7 @@ const char *pa_status_string(int status)
     case PA_ERR_BAD_BLOCK: return "bad block id";
     case PA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case PA_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
+    case PA_ERR_NOT_DEVICE_ACCESSIBLE: return "memory not accessible from the device (pageable host memory?)";
     case PA_ERR_SCRATCH_TOO_SMALL:
         return "split workspace exceeds the built-in scratch of pa_decode_split_noalloc (use a larger "
                "partition_size, or pa_decode_split with a caller workspace)";
@@ -366,6 +367,48 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pa
     return launch_pdl(copy_blocks_kernel, dim3((unsigned)(num_pairs * slices)), dim3(256), 0,
                       static_cast<cudaStream_t>(stream), static_cast<uint4 *>(key_cache),
                       static_cast<uint4 *>(value_cache), src_dst_pairs, chunks, slices, (int64_t)num_blocks);
+}
+
+// Device-accessible memory: device allocations, or host memory that is pinned
+// and mapped into the device's address space (cudaHostAlloc / registered).
+static bool device_accessible(const void *ptr)
+{
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) return true;
+    return attr.type == cudaMemoryTypeHost && attr.devicePointer == ptr;
+}
+
+int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, const void *src_key_cache,
+                   const void *src_value_cache, const int64_t *src_dst_pairs, int num_pairs, int num_kv_heads,
+                   int head_dim, int block_size, int src_num_blocks, int dst_num_blocks, void *stream)
+{
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || src_num_blocks <= 0 ||
+        dst_num_blocks <= 0)
+        return PA_ERR_BAD_SHAPE;
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || !src_dst_pairs)
+        return PA_ERR_NULL_POINTER;
+    const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+    if (block_elems % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(dst_key_cache) || !aligned16(dst_value_cache) || !aligned16(src_key_cache) ||
+        !aligned16(src_value_cache))
+        return PA_ERR_ALIGNMENT;
+    if (!device_accessible(dst_key_cache) || !device_accessible(dst_value_cache) ||
+        !device_accessible(src_key_cache) || !device_accessible(src_value_cache) ||
+        !device_accessible(src_dst_pairs))
+        return PA_ERR_NOT_DEVICE_ACCESSIBLE;
+    const int64_t chunks = block_elems / 8;
+    const int slices = (int)std::max<int64_t>(1, std::min<int64_t>(64, cdiv64(chunks, 2048)));
+    if ((int64_t)num_pairs * slices > INT_MAX) return PA_ERR_BAD_SHAPE;
+    return launch_pdl(swap_blocks_kernel, dim3((unsigned)(num_pairs * slices)), dim3(256), 0,
+                      static_cast<cudaStream_t>(stream), static_cast<uint4 *>(dst_key_cache),
+                      static_cast<uint4 *>(dst_value_cache), static_cast<const uint4 *>(src_key_cache),
+                      static_cast<const uint4 *>(src_value_cache), src_dst_pairs, chunks, slices,
+                      (int64_t)src_num_blocks, (int64_t)dst_num_blocks);
 }
 
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_seq_len,

@@ -27,7 +27,7 @@ __all__ = [
     "slot_mapping", "reshape_and_cache", "copy_blocks", "decode", "decode_one_pass",
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
-    "decode_split_noalloc",
+    "decode_split_noalloc", "swap_blocks",
 ]
 
 
@@ -103,6 +103,31 @@ def copy_blocks(key_cache, value_cache, src_dst_pairs, stream=None) -> None:
     check("pa_copy_blocks", lib.pa_copy_blocks(
         key_cache.data_ptr(), value_cache.data_ptr(), pr, src_dst_pairs.shape[0], hkv, d, bs, nb,
         _stream(stream)))
+
+
+def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, src_dst_pairs, stream=None) -> None:
+    """pa_swap_blocks: block copies between a device cache and a pinned host cache (either way).
+
+    Host-side tensors must be pinned (``tensor.pin_memory()``); ``src_dst_pairs``
+    is an int64 [P, 2] tensor in device or pinned host memory."""
+    lib = load()
+    for name, t in (("dst_key_cache", dst_key_cache), ("dst_value_cache", dst_value_cache),
+                    ("src_key_cache", src_key_cache), ("src_value_cache", src_value_cache)):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous bf16 [num_blocks, block_size, heads, head_dim] tensor")
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if src_key_cache.shape[1:] != dst_key_cache.shape[1:] or src_key_cache.shape != src_value_cache.shape or \
+            dst_key_cache.shape != dst_value_cache.shape:
+        raise ValueError("cache shapes do not match")
+    if src_dst_pairs.dtype != torch.int64 or src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2 or \
+            not src_dst_pairs.is_contiguous():
+        raise ValueError("src_dst_pairs must be a contiguous int64 [P, 2] tensor")
+    _, bs, hkv, d = src_key_cache.shape
+    check("pa_swap_blocks", lib.pa_swap_blocks(
+        dst_key_cache.data_ptr(), dst_value_cache.data_ptr(), src_key_cache.data_ptr(), src_value_cache.data_ptr(),
+        src_dst_pairs.data_ptr(), src_dst_pairs.shape[0], hkv, d, bs, src_key_cache.shape[0],
+        dst_key_cache.shape[0], _stream(stream)))
 
 
 def _decode_common(query, key_cache, value_cache, block_tables, seq_lens):

@@ -133,6 +133,18 @@ class BlockPool:
         return int(load().pa_pool_num_cached_blocks(self._h))
 
 
+def swap_plan(src: BlockPool, dst: BlockPool, table):
+    """pa_pool_swap_plan: move a table's blocks from `src` to `dst`.
+
+    Returns (new_table, src_dst_pairs int64 [P, 2])."""
+    t = np.ascontiguousarray(table, dtype=np.int32).copy()
+    pairs = np.empty((max(t.size, 1), 2), dtype=np.int64)
+    n = ctypes.c_int(0)
+    check("pa_pool_swap_plan", load().pa_pool_swap_plan(src._h, dst._h, _ptr(t), int(t.size), _ptr(pairs),
+                                                        ctypes.byref(n)))
+    return t.tolist(), pairs[:n.value].copy()
+
+
 def block_hash(parent_hash: int, token_ids) -> int:
     """pa_block_hash: chained FNV-1a-64 of a block's tokens."""
     toks = np.ascontiguousarray(token_ids, dtype=np.int32)

@@ -279,3 +279,16 @@ def test_copy_blocks_copies_whole_blocks_only():
     assert np.array_equal(vc[[0, 1, 2, 3]], v0[[0, 1, 2, 3]])
     oracle.copy_blocks(kc, vc, np.zeros((0, 2), np.int64))
     assert np.array_equal(kc[4], k0[1])
+
+
+def test_swap_blocks_copies_between_caches():
+    rng = np.random.default_rng(2)
+    src_k = rng.integers(0, 65535, size=(5, 4, 2, 8), dtype=np.uint16)
+    src_v = rng.integers(0, 65535, size=(5, 4, 2, 8), dtype=np.uint16)
+    dst_k = rng.integers(0, 65535, size=(3, 4, 2, 8), dtype=np.uint16)
+    dst_v = rng.integers(0, 65535, size=(3, 4, 2, 8), dtype=np.uint16)
+    d0k, d0v, s0k = dst_k.copy(), dst_v.copy(), src_k.copy()
+    oracle.swap_blocks(dst_k, dst_v, src_k, src_v, [(4, 0), (1, 2)])
+    assert np.array_equal(dst_k[0], src_k[4]) and np.array_equal(dst_v[2], src_v[1])
+    assert np.array_equal(dst_k[1], d0k[1]) and np.array_equal(dst_v[1], d0v[1])
+    assert np.array_equal(src_k, s0k)

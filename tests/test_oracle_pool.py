@@ -103,3 +103,18 @@ def test_random_operations_keep_invariants():
         _check_invariants(pool, [t for t, _ in seqs])
     for t, n in seqs:
         assert len(t) == -(-n // bs)
+
+
+def test_swap_plan_moves_references_between_pools():
+    from oracle.pool import swap_plan
+    gpu, cpu = OraclePool(16, 4), OraclePool(8, 4)
+    a = gpu.allocate_prompt(10)                  # 3 blocks
+    b = gpu.fork(a[:2]) + gpu.allocate(1)        # shares 2 of them
+    host_b, pairs = swap_plan(gpu, cpu, b)
+    assert len(pairs) == 3 and [s for s, _ in pairs] == b
+    assert [gpu.refcount[x] for x in a] == [1, 1, 1]      # a keeps its blocks
+    assert gpu.get_num_free_blocks() == 16 - 3
+    assert [cpu.refcount[x] for x in host_b] == [1, 1, 1]
+    back, pairs_in = swap_plan(cpu, gpu, host_b)
+    assert cpu.get_num_free_blocks() == 8 and [d for _, d in pairs_in] == back
+    _check_invariants(gpu, [a, back])

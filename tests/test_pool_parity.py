@@ -122,3 +122,36 @@ def test_shared_workload_pair_count():
     assert len(pairs) == w.num_seqs - opening
     assert len(set(pairs[:, 1].tolist())) == len(pairs)
     assert not set(pairs[:, 1].tolist()) & set(pairs[:, 0].tolist())
+
+
+def test_swap_plan_matches_oracle_and_keeps_bookkeeping():
+    from oracle.pool import swap_plan as o_swap_plan
+    from paged_kv_cache_379_b200.pool import swap_plan
+    rng = np.random.default_rng(11)
+    gpu_order, cpu_order = rng.permutation(64), rng.permutation(32)
+    g, c = BlockPool(64, 16, free_order=gpu_order), BlockPool(32, 16, free_order=cpu_order)
+    og, oc = OraclePool(64, 16, free_order=gpu_order.tolist()), OraclePool(32, 16, free_order=cpu_order.tolist())
+    t1 = g.allocate(5)
+    assert t1 == og.allocate(5)
+    t2 = g.fork(t1[:3]) + g.allocate(2)          # shares 3 blocks with t1
+    ot2 = og.fork(t1[:3]) + og.allocate(2)
+    assert t2 == ot2
+    # swap t2 out to the host pool
+    new2, pairs = swap_plan(g, c, t2)
+    onew2, opairs = o_swap_plan(og, oc, list(t2))
+    assert new2 == onew2 and [tuple(p) for p in pairs.tolist()] == opairs
+    assert g.refcounts() == og.refcount and c.refcounts() == oc.refcount
+    assert all(g.refcount(b) == 1 for b in t1[:3])     # t1 still owns the shared blocks
+    # and back in
+    back, pairs_in = swap_plan(c, g, new2)
+    oback, opairs_in = o_swap_plan(oc, og, list(new2))
+    assert back == oback and [tuple(p) for p in pairs_in.tolist()] == opairs_in
+    assert c.get_num_free_blocks() == 32 and g.refcounts() == og.refcount
+    # a table repeating a block maps it once, with the repeat count as its refcount
+    t3 = g.allocate(1)
+    og.allocate(1)
+    g.fork(t3)
+    og.fork(list(t3))
+    new3, p3 = swap_plan(g, c, t3 + t3)
+    onew3, op3 = o_swap_plan(og, oc, list(t3 + t3))
+    assert new3 == onew3 and len(p3) == 1 and c.refcount(new3[0]) == 2
