@@ -15,6 +15,7 @@ Functions, each restating a passage of the pages (see ``oracle.c`` and
 * :func:`swap_blocks`       -- whole-block copies between a GPU and a host cache
 * :func:`paged_decode`      -- softmax(scale * q K^T) V, K/V gathered through the table
 * :func:`paged_decode_partials`, :func:`lse_merge` -- the split form and its merge
+* :func:`reshape_and_cache_fp8`, :func:`paged_decode_fp8` -- the same over an E4M3 cache
 * :class:`pool.OraclePool`  -- free list, reference counts, fork, copy-on-write
 """
 
@@ -65,6 +66,15 @@ def _load():
         lib.oracle_paged_decode_partials.restype = None
         lib.oracle_lse_merge.argtypes = [P, P, P, P, I, I, I]
         lib.oracle_lse_merge.restype = None
+        lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+        lib.oracle_f64_to_e4m3.argtypes = [ctypes.c_double]
+        lib.oracle_f64_to_e4m3.restype = ctypes.c_uint8
+        lib.oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, ctypes.c_float, ctypes.c_float]
+        lib.oracle_reshape_and_cache_fp8.restype = None
+        lib.oracle_paged_decode_fp8.argtypes = [P, P, P, P, P, P, ctypes.c_double, ctypes.c_double,
+                                                ctypes.c_double, I, I, I, I, I, I, I]
+        lib.oracle_paged_decode_fp8.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = I
         _lib = lib
@@ -171,6 +181,49 @@ def paged_decode_partials(query, key_cache, value_cache, block_tables, seq_lens,
                                      float(scale), bs, Hkv, B, Hq, D, bt.shape[1],
                                      int(partition_size), int(max_parts))
     return m, l, o
+
+
+def e4m3_to_f64(code: int) -> float:
+    return float(_load().oracle_e4m3_to_f64(int(code) & 0xFF))
+
+
+def f64_to_e4m3(x: float) -> int:
+    return int(_load().oracle_f64_to_e4m3(float(x)))
+
+
+def reshape_and_cache_fp8(key, value, key_cache, value_cache, slots, block_size: int, k_scale: float,
+                          v_scale: float) -> None:
+    """In place on uint8 E4M3 caches [nb, bs, Hkv, D]; the inverse scales are formed in fp32."""
+    lib = _load()
+    k, kp = _c(key, np.uint16)
+    v, vp = _c(value, np.uint16)
+    s, sp = _c(slots, np.int64)
+    for a in (key_cache, value_cache):
+        assert a.dtype == np.uint8 and a.flags.c_contiguous
+    T, H, D = k.shape
+    k_inv = float(np.float32(1.0) / np.float32(k_scale))
+    v_inv = float(np.float32(1.0) / np.float32(v_scale))
+    lib.oracle_reshape_and_cache_fp8(kp, vp, key_cache.ctypes.data_as(ctypes.c_void_p),
+                                     value_cache.ctypes.data_as(ctypes.c_void_p), sp, T, H, D, block_size,
+                                     k_inv, v_inv)
+
+
+def paged_decode_fp8(query, key_cache, value_cache, block_tables, seq_lens, scale: float, k_scale: float,
+                     v_scale: float, threads: int = 1) -> np.ndarray:
+    """fp64 [B, Hq, D] decode over uint8 E4M3 caches (value = e4m3(code) * scale)."""
+    lib = _load()
+    q, qp = _c(query, np.uint16)
+    kc, kcp = _c(key_cache, np.uint8)
+    vc, vcp = _c(value_cache, np.uint8)
+    bt, btp = _c(block_tables, np.int32)
+    sl, slp = _c(seq_lens, np.int32)
+    B, Hq, D = q.shape
+    nb, bs, Hkv, _ = kc.shape
+    out = np.empty((B, Hq, D), dtype=np.float64)
+    lib.oracle_paged_decode_fp8(out.ctypes.data_as(ctypes.c_void_p), qp, kcp, vcp, btp, slp, float(scale),
+                                float(np.float32(k_scale)), float(np.float32(v_scale)), bs, Hkv, B, Hq, D,
+                                bt.shape[1], int(threads))
+    return out
 
 
 def lse_merge(m, l, o) -> np.ndarray:

@@ -303,6 +303,111 @@ void oracle_lse_merge(double *out, const double *m, const double *l, const doubl
     }
 }
 
+/*
+ * FP8 KV cache ("vLLM 核心源码深度解析 …", milestone list: FP8 KV Cache).  The
+ * stored byte is an OCP FP8 E4M3 code: sign bit, 4 exponent bits (bias 7), 3
+ * mantissa bits; exponent 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN; no
+ * infinities; the largest finite magnitude is 448.  A stored code c stands for
+ * e4m3(c) * scale (one scale per cache tensor).
+ */
+double oracle_e4m3_to_f64(uint8_t c)
+{
+    int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to x (ties to the even code), finite values beyond 448 clamped
+ * to +-448, NaN to 0x7F: a linear scan over the 127 non-negative finite codes. */
+uint8_t oracle_f64_to_e4m3(double x)
+{
+    if (x != x) return 0x7F;
+    uint8_t sign = x < 0 ? 0x80 : 0;
+    double a = fabs(x);
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 126; ++c) {
+        double err = fabs(oracle_e4m3_to_f64((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* Cache write with quantisation: code = e4m3(fp32(fp32(x) * inv_scale)), the
+ * product taken in fp32 (as the kernel takes it) and then rounded to E4M3. */
+void oracle_reshape_and_cache_fp8(const uint16_t *key, const uint16_t *value, uint8_t *key_cache,
+                                  uint8_t *value_cache, const int64_t *slot_mapping, int num_tokens,
+                                  int num_kv_heads, int head_dim, int block_size, float k_inv_scale,
+                                  float v_inv_scale)
+{
+    for (int t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t block = slot / block_size;
+        int64_t offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            for (int d = 0; d < head_dim; ++d) {
+                int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * (int64_t)head_dim + d;
+                int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim + d;
+                float kx = (float)widen_bf16(key[src]) * k_inv_scale;
+                float vx = (float)widen_bf16(value[src]) * v_inv_scale;
+                key_cache[dst] = oracle_f64_to_e4m3((double)kx);
+                value_cache[dst] = oracle_f64_to_e4m3((double)vx);
+            }
+        }
+    }
+}
+
+/* Paged decode over an FP8 cache: K and V rows are e4m3(code) * k_scale and
+ * e4m3(code) * v_scale; otherwise exactly oracle_paged_decode. */
+void oracle_paged_decode_fp8(double *out, const uint16_t *query, const uint8_t *key_cache,
+                             const uint8_t *value_cache, const int32_t *block_tables,
+                             const int32_t *seq_lens, double scale, double k_scale, double v_scale,
+                             int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                             int max_blocks, int nthreads)
+{
+    int group = num_heads / num_kv_heads;
+    int64_t units = (int64_t)num_seqs * num_heads;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int64_t u = 0; u < units; ++u) {
+        int s = (int)(u / num_heads);
+        int h = (int)(u % num_heads);
+        int len = seq_lens[s];
+        double *o = out + u * head_dim;
+        if (len <= 0) {
+            for (int d = 0; d < head_dim; ++d) o[d] = 0.0;
+            continue;
+        }
+        int kv_head = h / group;
+        double *q = malloc(sizeof(double) * head_dim);
+        double *k = malloc(sizeof(double) * (size_t)len * head_dim);
+        double *v = malloc(sizeof(double) * (size_t)len * head_dim);
+        double *x = malloc(sizeof(double) * (size_t)len);
+        const uint16_t *qrow = query + u * head_dim;
+        for (int d = 0; d < head_dim; ++d) q[d] = widen_bf16(qrow[d]);
+        const int32_t *table = block_tables + (int64_t)s * max_blocks;
+        for (int i = 0; i < len; ++i) {
+            int64_t physical = table[i / block_size];
+            int64_t row = ((physical * block_size + i % block_size) * num_kv_heads + kv_head) * (int64_t)head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                k[(int64_t)i * head_dim + d] = oracle_e4m3_to_f64(key_cache[row + d]) * k_scale;
+                v[(int64_t)i * head_dim + d] = oracle_e4m3_to_f64(value_cache[row + d]) * v_scale;
+            }
+        }
+        double m, l;
+        partial_attention(&m, &l, o, q, k, v, len, head_dim, scale, x);
+        for (int d = 0; d < head_dim; ++d) o[d] /= l;
+        free(q); free(k); free(v); free(x);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -292,3 +292,63 @@ def test_swap_blocks_copies_between_caches():
     assert np.array_equal(dst_k[0], src_k[4]) and np.array_equal(dst_v[2], src_v[1])
     assert np.array_equal(dst_k[1], d0k[1]) and np.array_equal(dst_v[1], d0v[1])
     assert np.array_equal(src_k, s0k)
+
+
+# ---- FP8 (E4M3) cache: the format's definition ------------------------------------
+
+def test_e4m3_decode_fixed_points():
+    # one, the largest finite value, the smallest normal and subnormal, signed zero, NaN
+    assert oracle.e4m3_to_f64(0x38) == 1.0
+    assert oracle.e4m3_to_f64(0x7E) == 448.0
+    assert oracle.e4m3_to_f64(0x08) == 2.0 ** -6
+    assert oracle.e4m3_to_f64(0x01) == 2.0 ** -9
+    assert oracle.e4m3_to_f64(0x80) == 0.0 and oracle.e4m3_to_f64(0xB8) == -1.0
+    assert np.isnan(oracle.e4m3_to_f64(0x7F)) and np.isnan(oracle.e4m3_to_f64(0xFF))
+    vals = [oracle.e4m3_to_f64(c) for c in range(127)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))            # codes are ordered
+
+
+def test_e4m3_round_to_nearest_even_and_saturate():
+    # every code round-trips; midpoints go to the even code; overflow saturates
+    for c in range(127):
+        assert oracle.f64_to_e4m3(oracle.e4m3_to_f64(c)) == c
+        assert oracle.f64_to_e4m3(-oracle.e4m3_to_f64(c)) == (c | 0x80 if c else oracle.f64_to_e4m3(-0.0))
+    one, nxt = oracle.e4m3_to_f64(0x38), oracle.e4m3_to_f64(0x39)    # 1.0 and 1.125
+    assert oracle.f64_to_e4m3((one + nxt) / 2) == 0x38              # tie -> even (0x38)
+    assert oracle.f64_to_e4m3(one + (nxt - one) * 0.51) == 0x39
+    nxt2 = oracle.e4m3_to_f64(0x3A)
+    assert oracle.f64_to_e4m3((nxt + nxt2) / 2) == 0x3A              # tie -> even (0x3A)
+    assert oracle.f64_to_e4m3(1000.0) == 0x7E and oracle.f64_to_e4m3(-1e9) == 0xFE
+
+
+def test_fp8_decode_equals_bf16_decode_of_the_dequantised_cache():
+    """Decoding an E4M3 cache equals decoding the cache its codes stand for."""
+    case = wl.random_decode_case(31, num_seqs=3, num_heads=8, num_kv_heads=2, head_dim=16,
+                                 block_size=4, lengths=[3, 9, 14], spare_blocks=0)
+    rng = np.random.default_rng(4)
+    kc8 = rng.integers(0, 126, size=case.key_cache.shape, dtype=np.uint8) | (rng.integers(0, 2, size=case.key_cache.shape, dtype=np.uint8) << 7)
+    vc8 = rng.integers(0, 126, size=case.key_cache.shape, dtype=np.uint8)
+    ks, vs = 0.5, 0.25          # powers of two: the dequantised values are exact bf16 numbers
+    deq = np.vectorize(oracle.e4m3_to_f64)
+    kf = (deq(kc8) * ks).astype(np.float32)
+    vf = (deq(vc8) * vs).astype(np.float32)
+    got = oracle.paged_decode_fp8(case.query, kc8, vc8, case.block_tables, case.seq_lens, case.scale, ks, vs)
+    ref = oracle.paged_decode(case.query, wl.f32_to_bf16_bits(kf), wl.f32_to_bf16_bits(vf),
+                              case.block_tables, case.seq_lens, case.scale)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_cache_write_quantises_each_element():
+    case = wl.random_decode_case(33, num_seqs=2, num_heads=2, num_kv_heads=2, head_dim=16,
+                                 block_size=4, lengths=[5, 6])
+    kc = np.zeros(case.key_cache.shape, np.uint8)
+    vc = np.zeros(case.key_cache.shape, np.uint8)
+    slots = np.array([3, 17], dtype=np.int64)
+    oracle.reshape_and_cache_fp8(case.new_key, case.new_value, kc, vc, slots, 4, 0.03, 0.07)
+    kinv = np.float32(1.0) / np.float32(0.03)
+    for t, slot in enumerate(slots):
+        for h in range(2):
+            for d in range(16):
+                x = np.float32(oracle.bf16_bits_to_f64(case.new_key[t, h, d:d + 1])[0]) * kinv
+                assert kc[slot // 4, slot % 4, h, d] == oracle.f64_to_e4m3(float(np.float32(x)))
+    assert np.count_nonzero(kc) <= 2 * 2 * 16
