@@ -319,6 +319,8 @@ def test_e4m3_round_to_nearest_even_and_saturate():
     nxt2 = oracle.e4m3_to_f64(0x3A)
     assert oracle.f64_to_e4m3((nxt + nxt2) / 2) == 0x3A              # tie -> even (0x3A)
     assert oracle.f64_to_e4m3(1000.0) == 0x7E and oracle.f64_to_e4m3(-1e9) == 0xFE
+    assert oracle.f64_to_e4m3(float("inf")) == 0x7E and oracle.f64_to_e4m3(float("-inf")) == 0xFE
+    assert oracle.f64_to_e4m3(464.0) == 0x7E    # halfway to the next binade's step: still 448
 
 
 def test_fp8_decode_equals_bf16_decode_of_the_dequantised_cache():
