@@ -75,6 +75,8 @@ def _load():
         lib.oracle_paged_decode_fp8.argtypes = [P, P, P, P, P, P, ctypes.c_double, ctypes.c_double,
                                                 ctypes.c_double, I, I, I, I, I, I, I]
         lib.oracle_paged_decode_fp8.restype = None
+        lib.oracle_paged_prefill.argtypes = [P, P, P, P, P, P, P, ctypes.c_double, I, I, I, I, I, I, I]
+        lib.oracle_paged_prefill.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = I
         _lib = lib
@@ -159,6 +161,33 @@ def paged_decode(query, key_cache, value_cache, block_tables, seq_lens, scale: f
     out = np.empty((B, Hq, D), dtype=np.float64)
     lib.oracle_paged_decode(out.ctypes.data_as(ctypes.c_void_p), qp, kcp, vcp, btp, slp,
                             float(scale), bs, Hkv, B, Hq, D, bt.shape[1], int(threads))
+    return out
+
+
+def paged_prefill(query, key_cache, value_cache, block_tables, seq_lens, q_lens, scale: float,
+                  threads: int = 1) -> np.ndarray:
+    """fp64 [T, Hq, D] causal prefill of each sequence's last q_lens[s] positions.
+
+    query: uint16 bf16 bits [T, Hq, D], T = sum(q_lens), rows of sequence s
+    consecutive and in position order."""
+    lib = _load()
+    q, qp = _c(query, np.uint16)
+    kc, kcp = _c(key_cache, np.uint16)
+    vc, vcp = _c(value_cache, np.uint16)
+    bt, btp = _c(block_tables, np.int32)
+    sl, slp = _c(seq_lens, np.int32)
+    ql = np.asarray(q_lens, dtype=np.int64)
+    B = sl.shape[0]
+    assert ql.shape == (B,) and (ql >= 0).all() and (ql <= sl).all()
+    start = np.zeros(B + 1, dtype=np.int32)
+    start[1:] = np.cumsum(ql)
+    st, stp = _c(start, np.int32)
+    T, Hq, D = q.shape
+    nb, bs, Hkv, D2 = kc.shape
+    assert T == int(start[-1]) and D2 == D and Hq % Hkv == 0 and bt.shape[0] == B
+    out = np.empty((T, Hq, D), dtype=np.float64)
+    lib.oracle_paged_prefill(out.ctypes.data_as(ctypes.c_void_p), qp, kcp, vcp, btp, slp, stp, float(scale),
+                             bs, Hkv, B, Hq, D, bt.shape[1], int(threads))
     return out
 
 

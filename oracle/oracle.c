@@ -411,6 +411,59 @@ void oracle_paged_decode_fp8(double *out, const uint16_t *query, const uint8_t *
     }
 }
 
+/*
+ * Multi-query paged prefill over the block table: the chunked-prefill step
+ * ("vLLM 核心源码深度解析 …", milestone list: v0.5 Chunked Prefill -- a long
+ * prompt is fed in chunks so that it does not hold up the decodes) with the
+ * causal rule of [论文专题] (the query at position i attends to positions up to
+ * and including i).  Sequence s holds seq_lens[s] cached positions; the last
+ * q_lens[s] of them are this chunk's new tokens, whose K/V rows are already in
+ * the cache.  New token i of s sits at position p = seq_lens[s] - q_lens[s] + i
+ * and its query row is q_start[s] + i (q_start: int32 [num_seqs + 1],
+ * q_start[s+1] - q_start[s] = q_lens[s]):
+ *   out[row, h, :] = sum_{j <= p} softmax_j(scale * q[row, h] . k_j) v_j
+ * query / out: [num_tokens, num_heads, head_dim] (out double).  Query head h
+ * reads KV head h / (num_heads / num_kv_heads).  Parallel over (row, head).
+ */
+void oracle_paged_prefill(double *out, const uint16_t *query, const uint16_t *key_cache,
+                          const uint16_t *value_cache, const int32_t *block_tables,
+                          const int32_t *seq_lens, const int32_t *q_start, double scale,
+                          int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                          int head_dim, int max_blocks, int nthreads)
+{
+    int group = num_heads / num_kv_heads;
+    int64_t rows = q_start[num_seqs];
+    int64_t units = rows * num_heads;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int64_t u = 0; u < units; ++u) {
+        int64_t row = u / num_heads;
+        int h = (int)(u % num_heads);
+        int s = 0;
+        while (q_start[s + 1] <= row) ++s;   /* the sequence owning this row */
+        int q_len = q_start[s + 1] - q_start[s];
+        int pos = seq_lens[s] - q_len + (int)(row - q_start[s]);
+        int len = pos + 1;                   /* positions 0..pos */
+        int kv_head = h / group;
+        double *o = out + u * head_dim;
+        double *q = malloc(sizeof(double) * head_dim);
+        double *k = malloc(sizeof(double) * (size_t)len * head_dim);
+        double *v = malloc(sizeof(double) * (size_t)len * head_dim);
+        double *x = malloc(sizeof(double) * (size_t)len);
+        const uint16_t *qrow = query + u * head_dim;
+        for (int d = 0; d < head_dim; ++d) q[d] = widen_bf16(qrow[d]);
+        const int32_t *table = block_tables + (int64_t)s * max_blocks;
+        gather_rows(k, key_cache, table, 0, len, kv_head, num_kv_heads, head_dim, block_size);
+        gather_rows(v, value_cache, table, 0, len, kv_head, num_kv_heads, head_dim, block_size);
+        double m, l;
+        partial_attention(&m, &l, o, q, k, v, len, head_dim, scale, x);
+        for (int d = 0; d < head_dim; ++d) o[d] /= l;
+        free(q); free(k); free(v); free(x);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -354,3 +354,83 @@ def test_fp8_cache_write_quantises_each_element():
                 x = np.float32(oracle.bf16_bits_to_f64(case.new_key[t, h, d:d + 1])[0]) * kinv
                 assert kc[slot // 4, slot % 4, h, d] == oracle.f64_to_e4m3(float(np.float32(x)))
     assert np.count_nonzero(kc) <= 2 * 2 * 16
+
+
+# ---- multi-query paged prefill (causal within the chunk) -----------------------------
+
+def _prefill_case(seed, bs, Hq, Hkv, D, lens, q_lens):
+    case = wl.random_decode_case(seed, num_seqs=len(lens), num_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                                 block_size=bs, lengths=lens)
+    q = wl.bf16_normal(np.random.default_rng(seed + 99), (int(sum(q_lens)), Hq, D))
+    return case, q
+
+
+def _sdpa_prefill(case, q_bits, q_lens):
+    """torch SDPA (fp64) per sequence on the gathered rows, with the causal mask
+    of a chunk that starts at position L - q_len."""
+    Hq, D = q_bits.shape[1:]
+    out = np.zeros(q_bits.shape)
+    row = 0
+    for s, (L, n) in enumerate(zip(case.seq_lens, q_lens)):
+        L, n = int(L), int(n)
+        if n == 0:
+            continue
+        ks, vs = zip(*[_contiguous(case, s, g) for g in range(case.num_kv_heads)])
+        k = torch.from_numpy(np.stack(ks))[None]
+        v = torch.from_numpy(np.stack(vs))[None]
+        q = torch.from_numpy(oracle.bf16_bits_to_f64(q_bits[row:row + n])).permute(1, 0, 2)[None]  # [1, Hq, n, D]
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+        o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=case.scale,
+                                                             enable_gqa=(Hq != case.num_kv_heads))
+        out[row:row + n] = o[0].permute(1, 0, 2).numpy()
+        row += n
+    return out
+
+
+@pytest.mark.parametrize("bs,Hq,Hkv,D", [(4, 4, 4, 16), (16, 8, 2, 64), (8, 16, 1, 32)])
+def test_prefill_matches_torch_sdpa_with_chunk_causal_mask(bs, Hq, Hkv, D):
+    lens = [1, 7, 16, 40, 33, 5]
+    q_lens = [1, 7, 5, 40, 1, 0]      # whole prompts, a mid chunk, single tokens, an idle sequence
+    case, q = _prefill_case(21 + bs + D, bs, Hq, Hkv, D, lens, q_lens)
+    got = oracle.paged_prefill(q, case.key_cache, case.value_cache, case.block_tables, case.seq_lens,
+                               q_lens, case.scale)
+    ref = _sdpa_prefill(case, q, q_lens)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_of_single_tokens_is_decode():
+    case, q = _prefill_case(31, 4, 8, 2, 16, [3, 9, 17], [1, 1, 1])
+    got = oracle.paged_prefill(q, case.key_cache, case.value_cache, case.block_tables, case.seq_lens,
+                               [1, 1, 1], case.scale)
+    dec = oracle.paged_decode(q, case.key_cache, case.value_cache, case.block_tables, case.seq_lens, case.scale)
+    assert np.array_equal(got, dec)
+
+
+def test_prefill_chunks_equal_whole_prompt():
+    """A prompt fed as chunks [0, 9), [9, 20), [20, 37) gives the rows of the
+    whole-prompt prefill: each token's result depends only on its position."""
+    L = 37
+    case, q = _prefill_case(41, 8, 4, 2, 32, [L], [L])
+    whole = oracle.paged_prefill(q, case.key_cache, case.value_cache, case.block_tables, case.seq_lens,
+                                 [L], case.scale)
+    for a, b in ((0, 9), (9, 20), (20, 37)):
+        part = oracle.paged_prefill(q[a:b], case.key_cache, case.value_cache, case.block_tables,
+                                    np.array([b], np.int32), [b - a], case.scale)
+        assert np.array_equal(part, whole[a:b])
+
+
+def test_prefill_first_position_and_permutation():
+    case, q = _prefill_case(51, 4, 4, 4, 16, [6, 11], [6, 11])
+    got = oracle.paged_prefill(q, case.key_cache, case.value_cache, case.block_tables, case.seq_lens,
+                               [6, 11], case.scale)
+    for s, row in ((0, 0), (1, 6)):   # position 0 attends to itself only: out = v_0
+        _, v = zip(*[_contiguous(case, s, g) for g in range(4)])
+        assert np.array_equal(got[row], np.stack([vv[0] for vv in v]))
+    perm = np.random.default_rng(1).permutation(case.num_blocks)
+    kc = np.empty_like(case.key_cache)
+    vc = np.empty_like(case.value_cache)
+    kc[perm] = case.key_cache
+    vc[perm] = case.value_cache
+    tables = np.where(case.block_tables >= 0, perm[np.maximum(case.block_tables, 0)], -1).astype(np.int32)
+    moved = oracle.paged_prefill(q, kc, vc, tables, case.seq_lens, [6, 11], case.scale)
+    assert np.array_equal(got, moved)
