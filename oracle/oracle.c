@@ -318,14 +318,15 @@ double oracle_e4m3_to_f64(uint8_t c)
     return sign ? -v : v;
 }
 
-/* Nearest E4M3 code to x (ties to the even code), magnitudes beyond 448 clamped
+/* Nearest E4M3 code to x (ties to the even code, the sign kept, zero included),
+ * magnitudes beyond 448 clamped
  * to +-448 (infinities included: the format has none, and a saturating
  * conversion keeps the sign and takes the largest finite value), NaN to 0x7F:
  * a linear scan over the 127 non-negative finite codes. */
 uint8_t oracle_f64_to_e4m3(double x)
 {
     if (x != x) return 0x7F;
-    uint8_t sign = x < 0 ? 0x80 : 0;
+    uint8_t sign = signbit(x) ? 0x80 : 0;   /* -0 and negative underflows keep the sign */
     double a = fabs(x);
     if (a > 448.0) return (uint8_t)(sign | 0x7E);
     int best = 0;

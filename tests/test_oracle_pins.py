@@ -312,7 +312,7 @@ def test_e4m3_round_to_nearest_even_and_saturate():
     # every code round-trips; midpoints go to the even code; overflow saturates
     for c in range(127):
         assert oracle.f64_to_e4m3(oracle.e4m3_to_f64(c)) == c
-        assert oracle.f64_to_e4m3(-oracle.e4m3_to_f64(c)) == (c | 0x80 if c else oracle.f64_to_e4m3(-0.0))
+        assert oracle.f64_to_e4m3(-oracle.e4m3_to_f64(c)) == c | 0x80
     one, nxt = oracle.e4m3_to_f64(0x38), oracle.e4m3_to_f64(0x39)    # 1.0 and 1.125
     assert oracle.f64_to_e4m3((one + nxt) / 2) == 0x38              # tie -> even (0x38)
     assert oracle.f64_to_e4m3(one + (nxt - one) * 0.51) == 0x39
@@ -321,6 +321,8 @@ def test_e4m3_round_to_nearest_even_and_saturate():
     assert oracle.f64_to_e4m3(1000.0) == 0x7E and oracle.f64_to_e4m3(-1e9) == 0xFE
     assert oracle.f64_to_e4m3(float("inf")) == 0x7E and oracle.f64_to_e4m3(float("-inf")) == 0xFE
     assert oracle.f64_to_e4m3(464.0) == 0x7E    # halfway to the next binade's step: still 448
+    assert oracle.f64_to_e4m3(-0.0) == 0x80 and oracle.f64_to_e4m3(0.0) == 0x00   # signed zero
+    assert oracle.f64_to_e4m3(-1e-9) == 0x80 and oracle.f64_to_e4m3(1e-9) == 0x00  # underflow keeps the sign
 
 
 def test_fp8_decode_equals_bf16_decode_of_the_dequantised_cache():
