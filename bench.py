@@ -52,10 +52,12 @@ def workload_description(w) -> str:
             f"shuffled pool of {w.num_blocks} blocks (1.2x)")
 
 
-def algorithmic_bytes(seq_lens, block_size, num_heads, num_kv_heads, head_dim) -> int:
-    """KV blocks touched (K and V) + queries + outputs + block-table entries read + seq_lens."""
+def algorithmic_bytes(seq_lens, block_size, num_heads, num_kv_heads, head_dim, kv_elem_bytes: int = 2) -> int:
+    """KV blocks touched (K and V) + queries + outputs + block-table entries read + seq_lens.
+
+    kv_elem_bytes: 2 for a bf16 cache, 1 for an FP8 (E4M3) cache."""
     blocks = -(-np.asarray(seq_lens, dtype=np.int64) // block_size)
-    kv = int(blocks.sum()) * block_size * num_kv_heads * head_dim * 2 * 2
+    kv = int(blocks.sum()) * block_size * num_kv_heads * head_dim * 2 * kv_elem_bytes
     qo = 2 * len(seq_lens) * num_heads * head_dim * 2
     tables = int(blocks.sum()) * 4 + 4 * len(seq_lens)
     return kv + qo + tables

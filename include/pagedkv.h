@@ -226,6 +226,53 @@ int pa_lse_reduce(void *out, const void *workspace, const int32_t *seq_lens, int
                   void *stream);
 
 /* --------------------------------------------------------------------------
+ * FP8 KV cache ([深度解析], milestone list: "FP8 KV Cache" -- one byte per
+ * cached K/V element).  key_cache and value_cache hold OCP FP8 E4M3 codes
+ * (uint8 [num_blocks, block_size, num_kv_heads, head_dim]: sign, 4 exponent
+ * bits with bias 7, 3 mantissa bits; exponent 0 subnormal; S.1111.111 NaN;
+ * largest finite magnitude 448).  A code c stands for e4m3(c) * k_scale in the
+ * key cache and e4m3(c) * v_scale in the value cache: one positive, finite
+ * fp32 scale per cache tensor (otherwise PA_ERR_BAD_SHAPE).
+ *
+ * pa_reshape_and_cache_fp8: pa_reshape_and_cache with quantisation.  key and
+ * value are bf16 [num_tokens, num_kv_heads, head_dim]; each element x becomes
+ * the code nearest to fp32(x * fp32(1 / scale)) (the inverse scale rounded to
+ * fp32 once; ties to the even code; magnitudes beyond 448, infinities
+ * included, saturate to +-448; NaN gives 0x7F).  num_kv_heads * head_dim must
+ * be a multiple of 16 (PA_ERR_UNSUPPORTED otherwise).  Slot rules as in
+ * pa_reshape_and_cache.
+ * ------------------------------------------------------------------------ */
+int pa_reshape_and_cache_fp8(const void *key, const void *value, void *key_cache,
+                             void *value_cache, const int64_t *slot_mapping, int num_tokens,
+                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                             float k_scale, float v_scale, void *stream);
+
+/* pa_decode over an FP8 cache: the same result with K = e4m3(code) * k_scale
+ * and V = e4m3(code) * v_scale.  query and out stay bf16.  Supported: head_dim
+ * 128, block_size 8 or 16, G = num_heads / num_kv_heads in 1..16
+ * (PA_ERR_UNSUPPORTED otherwise).  The logits are formed in fp32 from the
+ * query rounded to fp16 (exact for |q| in [2^-17, 65504] -- bf16 has 8
+ * significant bits) and the codes (every E4M3 value is an fp16 value); the
+ * softmax weights enter the value product as fp16.  Same plan, workspace
+ * contract and workspace size as pa_decode. */
+int pa_decode_fp8(void *out, const void *query, const void *key_cache, const void *value_cache,
+                  const int32_t *block_tables, const int32_t *seq_lens, float scale, float k_scale,
+                  float v_scale, int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                  int head_dim, int max_blocks_per_seq, int num_blocks, int max_seq_len,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* pa_decode_fp8 with an explicit plan: partition_size 0 = one pass (workspace
+ * optional: NULL hands items out round-robin), otherwise the split form of
+ * pa_decode_split with that partition size (workspace required). */
+int pa_decode_fp8_split(void *out, const void *query, const void *key_cache,
+                        const void *value_cache, const int32_t *block_tables,
+                        const int32_t *seq_lens, float scale, float k_scale, float v_scale,
+                        int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                        int head_dim, int max_blocks_per_seq, int num_blocks, int max_seq_len,
+                        int partition_size, void *workspace, size_t workspace_bytes,
+                        void *stream);
+
+/* --------------------------------------------------------------------------
  * Precondition check on the device: counts, into *bad_count (device int32,
  * overwritten), the sequences whose seq_len is negative or above max_seq_len,
  * whose ceil(seq_len/block_size) exceeds max_blocks_per_seq, or whose used

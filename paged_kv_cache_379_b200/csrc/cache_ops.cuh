@@ -64,6 +64,46 @@ __global__ void reshape_and_cache_kernel(const uint4 *__restrict__ key, const ui
     value_cache[dst] = v;
 }
 
+// FP8 cache write: one thread per 16 values of a token's [num_kv_heads, head_dim]
+// row (32 bytes of bf16 in, one 16-byte chunk of E4M3 codes out); each code is
+// e4m3(x * inv_scale) with the product taken in fp32, rounded to nearest even,
+// finite overflow saturating to +-448.
+__device__ __forceinline__ uint4 quantise16(uint4 a, uint4 b, float inv)
+{
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f0 = unpack_bf16x2(w[2 * i]);
+        const float2 f1 = unpack_bf16x2(w[2 * i + 1]);
+        const uint32_t lo = f32x2_to_e4m3x2(__fmul_rn(f0.x, inv), __fmul_rn(f0.y, inv));
+        const uint32_t hi = f32x2_to_e4m3x2(__fmul_rn(f1.x, inv), __fmul_rn(f1.y, inv));
+        out[i] = lo | (hi << 16);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+__global__ void reshape_and_cache_fp8_kernel(const uint4 *__restrict__ key, const uint4 *__restrict__ value,
+                                             uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache,
+                                             const int64_t *__restrict__ slot_mapping, int num_tokens,
+                                             int chunks_per_token, int64_t num_slots, float k_inv_scale,
+                                             float v_inv_scale)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)num_tokens * chunks_per_token) return;
+    const int64_t t = i / chunks_per_token;
+    const int64_t c = i - t * chunks_per_token;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0 || slot >= num_slots) return;
+    const int64_t dst = slot * chunks_per_token + c;
+    const uint4 k0 = key[2 * i], k1 = key[2 * i + 1];
+    const uint4 v0 = value[2 * i], v1 = value[2 * i + 1];
+    key_cache[dst] = quantise16(k0, k1, k_inv_scale);
+    value_cache[dst] = quantise16(v0, v1, v_inv_scale);
+}
+
 // One CTA per (pair, slice): copies `per_cta` 16-byte chunks of the source block
 // into the destination block, in both caches, with 4 loads in flight per thread.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ key_cache,

@@ -61,7 +61,8 @@ struct DecodeParams {
     float *ws_m;                      // [B, Hq, max_parts]      natural-log units
     float *ws_l;                      // [B, Hq, max_parts]
     int *sched;                       // [2] item counter, finished-CTA counter; nullptr = round robin
-    float scale_log2;                 // scale * log2(e)
+    float scale_log2;                 // scale * log2(e) (times the K scale of an FP8 cache)
+    float v_scale;                    // value scale of an FP8 cache (1 for bf16)
     int num_seqs, num_heads, num_kv_heads, group, max_blocks;
     int part_tokens;                  // positions per partition (multiple of 16); 0 = one pass
     int max_parts;                    // partitions per sequence (workspace stride); 1 = one pass
@@ -139,6 +140,35 @@ struct TileGeom {
     }
 };
 
+// Ring tiles of an FP8 (E4M3) cache, head_dim 128: one 128-byte row per token
+// (one swizzle row), TMA box {128 codes, 1, 1 head, bs tokens}, 1024-byte
+// aligned block slots, 128-byte swizzle.  The consumers read the codes with
+// 16-byte loads straight into MMA fragments (no widened copy in shared memory).
+template <int D, int BS>
+struct TileGeom8 {
+    static_assert(D == 128, "FP8 cache: head_dim 128");
+    static_assert(BS == 8 || BS == 16, "FP8 cache: block_size 8 or 16");
+    static constexpr int kHalves = 1;
+    static constexpr int kBlkBytes = BS * D;                      // bytes TMA delivers per block
+    static constexpr int kSlotRows = BS;
+    static constexpr int kBlocksPerTile = kTileTokens / BS;
+    static constexpr int kTileSmem = kBlocksPerTile * kSlotRows * 128;
+    static constexpr int kPlaneSmem = kTileSmem;
+    static constexpr int kStageSmem = 2 * kTileSmem;
+    static constexpr int kStages = 16;                            // a multiple of the consumer warps
+    static_assert(kStages % kConsumerWarps == 0, "ring depth");
+    static constexpr int kPipeSmem = kStages * kStageSmem;
+
+    __device__ static __forceinline__ uint32_t row_offset(int t) { return (uint32_t)(t * 128); }
+    // 16-byte chunk c (codes 16c .. 16c+15) of token t
+    __device__ static __forceinline__ uint32_t chunk_offset(int t, int c)
+    {
+        const uint32_t ro = row_offset(t);
+        return ro + ((((uint32_t)c & 7u) ^ ((ro >> 7) & 7u)) << 4);
+    }
+    __device__ static __forceinline__ uint32_t box_offset(int k, int) { return (uint32_t)(k * kSlotRows * 128); }
+};
+
 // Per-item merge scratch: each consumer warp's running max (log2 units), sum
 // and accumulator of up to ROWS heads.
 template <int D, int ROWS>
@@ -192,19 +222,19 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  : "memory");
 }
 
-template <int D, int BS, int MODE, int GC>
+template <int D, int BS, int MODE, int GC, bool FP8>
 struct DecodeSmem {
     static constexpr int ROWS = MODE == 0 ? GC : (MODE == 1 ? 8 : 16);
-    using Geo = TileGeom<D, BS>;
+    using Ring = std::conditional_t<FP8, TileGeom8<D, BS>, TileGeom<D, BS>>;
     using Merge = MergeScratch<D, ROWS>;
-    static constexpr int kMergeOff = Geo::kPipeSmem;
+    static constexpr int kMergeOff = Ring::kPipeSmem;
     static constexpr int kQOff = (kMergeOff + (int)sizeof(Merge) + 127) & ~127;
     static constexpr int kQBytes = ROWS * D * 2;                  // one item's query rows
     static constexpr int kItemOff = kQOff + kItemSlots * kQBytes;
     static constexpr int kChunkOff = kItemOff + kItemSlots * (int)sizeof(ItemInfo);
     static constexpr int kBarOff = (kChunkOff + kChunkSlots * (int)sizeof(ChunkInfo) + 7) & ~7;
     // barriers: full[kStages], empty[kStages], item_full, item_empty, chunk_full, chunk_empty
-    static constexpr int kNumBars = 2 * Geo::kStages + 2 * kItemSlots + 2 * kChunkSlots;
+    static constexpr int kNumBars = 2 * Ring::kStages + 2 * kItemSlots + 2 * kChunkSlots;
     static constexpr int kFlagOff = kBarOff + kNumBars * 8;
     static constexpr int kPrefixOff = kFlagOff + 16;
     // bytes of dynamic shared memory for a launch over num_seqs sequences
@@ -212,16 +242,17 @@ struct DecodeSmem {
     static constexpr int bytes(int num_seqs) { return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys); }
 };
 
-template <int D, int BS, int MODE, int GC>
+template <int D, int BS, int MODE, int GC, bool FP8>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
     paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v)
 {
+    static_assert(!FP8 || MODE != 0, "FP8 caches use the tensor-core consumers");
     // MODE 0: CUDA cores, GC (1 or 2) query heads per KV head.
     // MODE 1: tensor cores, up to 8 query heads per KV head (one 8-head tile).
     // MODE 2: tensor cores, up to 16 query heads per KV head (two 8-head tiles).
-    using Geo = TileGeom<D, BS>;
-    using Lay = DecodeSmem<D, BS, MODE, GC>;
+    using Lay = DecodeSmem<D, BS, MODE, GC, FP8>;
+    using Geo = typename Lay::Ring;                                         // ring tiles
     using Merge = typename Lay::Merge;
     constexpr int kStages = Geo::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -711,7 +742,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 constexpr int MT = D / 16;               // 16-row d tiles of O^T
                 const int gq = lane >> 2;                // MMA groupID
                 const int tq = lane & 3;                 // MMA thread-in-group
-                // B operand of S^T = K Q^T: b0 = Q[head][d 16kk+2tq..+1], b1 = Q[head][d 16kk+8+2tq..+1]
+                // B operand of S^T = K Q^T: b0 = Q[head][d 16kk+2tq..+1], b1 = Q[head][d 16kk+8+2tq..+1].
+                // FP8 cache: the contraction order is permuted so that a lane's four
+                // k-slots {2tq, 2tq+1, 2tq+8, 2tq+9} of k-step kk = 4S + i are the four
+                // consecutive codes d = 16(4S + tq) + 4i + {0..3} of a key row; Q
+                // follows the same order and is multiplied in fp16.
                 uint32_t qb[NH][KSTEPS][2];
 #pragma unroll
                 for (int nh = 0; nh < NH; ++nh) {
@@ -720,8 +755,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     for (int kk = 0; kk < KSTEPS; ++kk) {
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
-                            const int col = kk * 16 + hh * 8 + tq * 2;
-                            qb[nh][kk][hh] = head < G ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
+                            const int col = FP8 ? 16 * (4 * (kk >> 2) + tq) + 4 * (kk & 3) + 2 * hh
+                                                : kk * 16 + hh * 8 + tq * 2;
+                            uint32_t v = head < G ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
+                            if constexpr (FP8) {
+                                const float2 f = unpack_bf16x2(v);
+                                v = pack_f16x2(f.x, f.y);
+                            }
+                            qb[nh][kk][hh] = v;
                         }
                     }
                 }
@@ -745,10 +786,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 for (int j = warp; j < it.n_tiles; j += kConsumerWarps) {
                     const int ring = it.ring_base + j;
                     if (!wait_full(ring)) break;
+                    const int valid = min(kTileTokens, it.t_end - (it.t_begin + j * kTileTokens));
                     const uint32_t kt = base + (ring % kStages) * Geo::kStageSmem;
                     const uint32_t vt = kt + Geo::kTileSmem;
-                    const int valid = min(kTileTokens, it.t_end - (it.t_begin + j * kTileTokens));
-                    if (valid < kTileTokens) zero_tail(vt, valid);
+                    if constexpr (!FP8) {
+                        if (valid < kTileTokens) zero_tail(vt, valid);
+                    }
 
                     // S^T[token][head] = K Q^T, as two independent MMA chains (even and
                     // odd k-steps) summed at the end: half the dependent latency
@@ -757,13 +800,41 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
                         for (int c = 0; c < 4; ++c) sc[nh][c] = sd[nh][c] = 0.f;
+                    if constexpr (FP8) {
+                        // key rows gq and gq+8, code chunks tq (set 0) and tq + 4 (set 1); the
+                        // lanes of odd gq load set 1 first so that each 8-lane phase of a
+                        // 16-byte load touches 8 distinct swizzled chunks
+                        const bool odd = gq & 1;
+                        uint4 kr[2][2];  // [row gq / gq+8][set]
 #pragma unroll
-                    for (int kk = 0; kk < KSTEPS; ++kk) {
-                        uint32_t a0, a1, a2, a3;
-                        ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
+                        for (int r = 0; r < 2; ++r) {
+                            const int tok = gq + 8 * r;
+                            const uint4 x = lds128(kt + Geo::chunk_offset(tok, tq + (odd ? 4 : 0)));
+                            const uint4 y = lds128(kt + Geo::chunk_offset(tok, tq + (odd ? 0 : 4)));
+                            kr[r][0] = odd ? y : x;
+                            kr[r][1] = odd ? x : y;
+                        }
 #pragma unroll
-                        for (int nh = 0; nh < NH; ++nh)
-                            mma_bf16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                        for (int kk = 0; kk < KSTEPS; ++kk) {
+                            const uint32_t w0 = u4_word(kr[0][kk >> 2], kk & 3);
+                            const uint32_t w1 = u4_word(kr[1][kk >> 2], kk & 3);
+                            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(w0 & 0xFFFFu));
+                            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(w0 >> 16));
+                            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(w1 & 0xFFFFu));
+                            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(w1 >> 16));
+#pragma unroll
+                            for (int nh = 0; nh < NH; ++nh)
+                                mma_f16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < KSTEPS; ++kk) {
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
+#pragma unroll
+                            for (int nh = 0; nh < NH; ++nh)
+                                mma_bf16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                        }
                     }
 #pragma unroll
                     for (int nh = 0; nh < NH; ++nh)
@@ -817,22 +888,54 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         }
 #pragma unroll
                         for (int row = 0; row < 2; ++row) {
-                            const uint32_t hi = pack_bf16x2(pr[0][row], pr[1][row]);
-                            const float2 hf = unpack_bf16x2(hi);
-                            const uint32_t lo = pack_bf16x2(pr[0][row] - hf.x, pr[1][row] - hf.y);
-                            bh[nh][row] = movmatrix_trans(hi);
-                            bl[nh][row] = movmatrix_trans(lo);
+                            if constexpr (FP8) {  // fp16 weights: 11 significant bits, one MMA
+                                bh[nh][row] = movmatrix_trans(pack_f16x2(pr[0][row], pr[1][row]));
+                                bl[nh][row] = 0u;
+                            } else {
+                                const uint32_t hi = pack_bf16x2(pr[0][row], pr[1][row]);
+                                const float2 hf = unpack_bf16x2(hi);
+                                const uint32_t lo = pack_bf16x2(pr[0][row] - hf.x, pr[1][row] - hf.y);
+                                bh[nh][row] = movmatrix_trans(hi);
+                                bl[nh][row] = movmatrix_trans(lo);
+                            }
                         }
                     }
                     // O^T[d][head] += V^T P^T
+                    if constexpr (FP8) {
+                        // FP8 cache: the rows of O^T are permuted so that this lane's rows
+                        // gq and gq+8 of d-tile mt are d = 16gq + 2mt and 16gq + 2mt + 1,
+                        // i.e. code chunk gq of value rows 2tq, 2tq+1, 2tq+8, 2tq+9 (one
+                        // 16-byte load each, 8 distinct swizzled chunks per phase).  Rows
+                        // past the sequence end are zeroed here: stale codes may be NaN.
+                        uint4 vr[4];
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        uint32_t a0, a1, a2, a3;
-                        ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * mt + vpar), a0, a1, a2, a3);
+                        for (int r = 0; r < 4; ++r) {
+                            const int tok = 2 * tq + (r & 1) + 8 * (r >> 1);
+                            vr[r] = tok < valid ? lds128(vt + Geo::chunk_offset(tok, gq)) : make_uint4(0u, 0u, 0u, 0u);
+                        }
 #pragma unroll
-                        for (int nh = 0; nh < NH; ++nh) {
-                            mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
-                            mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
+                        for (int mt = 0; mt < MT; ++mt) {
+                            // bytes 2mt, 2mt+1 of each row, token pairs interleaved
+                            const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+                            const uint32_t lo = prmt(u4_word(vr[0], mt >> 1), u4_word(vr[1], mt >> 1), sel);
+                            const uint32_t hi = prmt(u4_word(vr[2], mt >> 1), u4_word(vr[3], mt >> 1), sel);
+                            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(lo & 0xFFFFu));
+                            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(lo >> 16));
+                            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(hi & 0xFFFFu));
+                            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(hi >> 16));
+#pragma unroll
+                            for (int nh = 0; nh < NH; ++nh) mma_f16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * mt + vpar), a0, a1, a2, a3);
+#pragma unroll
+                            for (int nh = 0; nh < NH; ++nh) {
+                                mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
+                                mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
+                            }
                         }
                     }
                     release(ring, valid);
@@ -854,8 +957,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         if (head < G) {
 #pragma unroll
                             for (int mt = 0; mt < MT; ++mt) {
-                                ms->o[warp][head][mt * 16 + gq] = o[mt][nh][jj];
-                                ms->o[warp][head][mt * 16 + gq + 8] = o[mt][nh][2 + jj];
+                                const int d0 = FP8 ? 16 * gq + 2 * mt : mt * 16 + gq;
+                                const int d1 = FP8 ? d0 + 1 : d0 + 8;
+                                ms->o[warp][head][d0] = o[mt][nh][jj];
+                                ms->o[warp][head][d1] = o[mt][nh][2 + jj];
                             }
                             if (gq == 0) {
                                 ms->m[warp][head] = m[nh][jj];
@@ -906,6 +1011,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 }
                 const int64_t hrow = (int64_t)it.s * p.num_heads + (int64_t)it.g * G + row;
                 const float den = ms->den[row];
+                acc.x *= p.v_scale;
+                acc.y *= p.v_scale;
+                acc.z *= p.v_scale;
+                acc.w *= p.v_scale;
                 if (direct) {
                     const float inv = den > 0.f ? 1.f / den : 0.f;
                     uint2 packed;

@@ -42,15 +42,22 @@ static EncodeTiledFn encode_fn()
 //   {64 elements = 128 B, D/64, Hkv, num_blocks*bs slots}
 // with a box of one 64-wide d-plane of one block of one head: {64, 1, 1, bs},
 // 128-byte swizzle.
-static int make_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int bs, int hkv, int d)
+// An FP8 cache (1-byte codes, head_dim 128) is {128 codes = 128 B, 1, Hkv, slots}
+// with a box {128, 1, 1, bs}: one 128-byte row per token.
+static int make_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int bs, int hkv, int d,
+                          bool fp8 = false)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return check_cuda(cudaErrorNotSupported);
-    const cuuint64_t dims[4] = {64, (cuuint64_t)(d / 64), (cuuint64_t)hkv, (cuuint64_t)(num_blocks * bs)};
-    const cuuint64_t strides[3] = {128, (cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
-    const cuuint32_t box[4] = {64, 1, 1, (cuuint32_t)bs};
+    const int esize = fp8 ? 1 : 2;
+    const int inner = 128 / esize;  // elements per 128-byte row
+    const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)(d / inner), (cuuint64_t)hkv,
+                                (cuuint64_t)(num_blocks * bs)};
+    const cuuint64_t strides[3] = {128, (cuuint64_t)d * esize, (cuuint64_t)hkv * d * esize};
+    const cuuint32_t box[4] = {(cuuint32_t)inner, 1, 1, (cuuint32_t)bs};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(cache), dims, strides, box,
+    const CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                          const_cast<void *>(cache), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -94,12 +101,12 @@ static int sm_count()
 }
 
 // Persistent launch: (resident CTAs per SM) x (SM count) CTAs, at most one per item.
-template <int D, int BS, int MODE, int GC>
+template <int D, int BS, int MODE, int GC, bool FP8 = false>
 static int launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int64_t max_items,
                            cudaStream_t st)
 {
-    using Lay = DecodeSmem<D, BS, MODE, GC>;
-    auto kernel = paged_decode_kernel<D, BS, MODE, GC>;
+    using Lay = DecodeSmem<D, BS, MODE, GC, FP8>;
+    auto kernel = paged_decode_kernel<D, BS, MODE, GC, FP8>;
     const size_t smem = (size_t)Lay::bytes(p.num_seqs);
     if (smem > 227 * 1024) return PA_ERR_BAD_SHAPE;  // too many sequences for the enumeration tables
     int rc = ensure_smem(reinterpret_cast<const void *>(kernel), smem);
@@ -122,6 +129,16 @@ static int launch_decode_bs(const DecodeParams &p, const CUtensorMap &tk, const 
     if (G == 2) return launch_decode_t<D, BS, 0, 2>(p, tk, tv, grid, st);
     if (G <= 8) return launch_decode_t<D, BS, 1, 0>(p, tk, tv, grid, st);
     if (G <= 16) return launch_decode_t<D, BS, 2, 0>(p, tk, tv, grid, st);
+    return PA_ERR_UNSUPPORTED;
+}
+
+// FP8 cache (head_dim 128, bs 8 or 16): always the tensor-core consumers.
+template <int BS>
+static int launch_decode_fp8_bs(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int64_t grid,
+                                cudaStream_t st)
+{
+    if (p.group <= 8) return launch_decode_t<128, BS, 1, 0, true>(p, tk, tv, grid, st);
+    if (p.group <= 16) return launch_decode_t<128, BS, 2, 0, true>(p, tk, tv, grid, st);
     return PA_ERR_UNSUPPORTED;
 }
 
@@ -151,6 +168,8 @@ struct DecodeArgs {
     const int32_t *block_tables, *seq_lens;
     float scale;
     int block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks, num_blocks, max_seq_len;
+    bool fp8 = false;             // caches hold E4M3 codes
+    float k_scale = 1.f, v_scale = 1.f;
 };
 
 static int check_decode_args(const DecodeArgs &a, bool need_out)
@@ -164,6 +183,9 @@ static int check_decode_args(const DecodeArgs &a, bool need_out)
     if (a.head_dim != 64 && a.head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (a.block_size != 4 && a.block_size != 8 && a.block_size != 16) return PA_ERR_UNSUPPORTED;
     if (a.num_heads / a.num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+    if (a.fp8 && (a.head_dim != 128 || a.block_size < 8)) return PA_ERR_UNSUPPORTED;
+    if (a.fp8 && !(a.k_scale > 0.f && a.v_scale > 0.f && a.k_scale < INFINITY && a.v_scale < INFINITY))
+        return PA_ERR_BAD_SHAPE;
     if ((int64_t)a.num_blocks * a.block_size > INT_MAX) return PA_ERR_BAD_SHAPE;
     if ((int64_t)a.max_blocks * a.block_size > INT_MAX) return PA_ERR_BAD_SHAPE;
     if (!aligned16(a.query) || !aligned16(a.key_cache) || !aligned16(a.value_cache) ||
@@ -213,7 +235,8 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
     p.query = static_cast<const __nv_bfloat16 *>(a.query);
     p.block_tables = a.block_tables;
     p.seq_lens = a.seq_lens;
-    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.scale_log2 = a.scale * (a.fp8 ? a.k_scale : 1.f) * 1.4426950408889634f;
+    p.v_scale = a.fp8 ? a.v_scale : 1.f;
     p.num_seqs = a.num_seqs;
     p.num_heads = a.num_heads;
     p.num_kv_heads = a.num_kv_heads;
@@ -240,12 +263,16 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
     const int64_t max_items = (int64_t)p.max_parts * a.num_seqs * a.num_kv_heads;
     if (max_items > INT_MAX) return PA_ERR_BAD_SHAPE;
     CUtensorMap tk, tv;
-    rc = make_cache_map(&tk, a.key_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim);
+    rc = make_cache_map(&tk, a.key_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim, a.fp8);
     if (rc != PA_OK) return rc;
-    rc = make_cache_map(&tv, a.value_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim);
+    rc = make_cache_map(&tv, a.value_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim, a.fp8);
     if (rc != PA_OK) return rc;
-    rc = a.head_dim == 64 ? launch_decode_d<64>(a.block_size, p, tk, tv, max_items, st)
-                          : launch_decode_d<128>(a.block_size, p, tk, tv, max_items, st);
+    if (a.fp8)
+        rc = a.block_size == 8 ? launch_decode_fp8_bs<8>(p, tk, tv, max_items, st)
+                               : launch_decode_fp8_bs<16>(p, tk, tv, max_items, st);
+    else
+        rc = a.head_dim == 64 ? launch_decode_d<64>(a.block_size, p, tk, tv, max_items, st)
+                              : launch_decode_d<128>(a.block_size, p, tk, tv, max_items, st);
     if (rc != PA_OK || mode != 1) return rc;
     ReduceParams r = {};
     r.out = p.out;
@@ -348,6 +375,31 @@ int pa_reshape_and_cache(const void *key, const void *value, void *key_cache, vo
                       static_cast<const uint4 *>(value), static_cast<uint4 *>(key_cache),
                       static_cast<uint4 *>(value_cache), slot_mapping, num_tokens, chunks,
                       (int64_t)num_blocks * block_size);
+}
+
+int pa_reshape_and_cache_fp8(const void *key, const void *value, void *key_cache, void *value_cache,
+                             const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                             int block_size, int num_blocks, float k_scale, float v_scale, void *stream)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PA_ERR_BAD_SHAPE;
+    if (!(k_scale > 0.f && v_scale > 0.f && k_scale < INFINITY && v_scale < INFINITY)) return PA_ERR_BAD_SHAPE;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL_POINTER;
+    if (((int64_t)num_kv_heads * head_dim) % 16 != 0) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return PA_ERR_ALIGNMENT;
+    const int chunks = (int)((int64_t)num_kv_heads * head_dim / 16);
+    const int64_t total = (int64_t)num_tokens * chunks;
+    const int threads = 256;
+    if (cdiv64(total, threads) > INT_MAX) return PA_ERR_BAD_SHAPE;
+    // the inverse scales are rounded to fp32 once, here
+    const float k_inv = 1.0f / k_scale, v_inv = 1.0f / v_scale;
+    return launch_pdl(reshape_and_cache_fp8_kernel, dim3((unsigned)cdiv64(total, threads)), dim3(threads), 0,
+                      static_cast<cudaStream_t>(stream), static_cast<const uint4 *>(key),
+                      static_cast<const uint4 *>(value), static_cast<uint4 *>(key_cache),
+                      static_cast<uint4 *>(value_cache), slot_mapping, num_tokens, chunks,
+                      (int64_t)num_blocks * block_size, k_inv, v_inv);
 }
 
 int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pairs, int num_pairs,
@@ -465,6 +517,42 @@ int pa_decode_split(void *out, const void *query, const void *key_cache, const v
     const DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
                           num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
     return run_decode(a, 1, partition_size, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pa_decode_fp8(void *out, const void *query, const void *key_cache, const void *value_cache,
+                  const int32_t *block_tables, const int32_t *seq_lens, float scale, float k_scale, float v_scale,
+                  int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                  int max_blocks_per_seq, int num_blocks, int max_seq_len, void *workspace, size_t workspace_bytes,
+                  void *stream)
+{
+    DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                    num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    a.fp8 = true;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int part = workspace ? pa_decode_plan(num_seqs, num_heads, num_kv_heads, head_dim, max_seq_len,
+                                                workspace_bytes)
+                               : 0;
+    if (part > 0) return run_decode(a, 1, part, workspace, workspace_bytes, st);
+    const bool counters = workspace && workspace_bytes >= kSchedBytes;
+    return run_decode(a, 0, 0, counters ? workspace : nullptr, counters ? workspace_bytes : 0, st);
+}
+
+int pa_decode_fp8_split(void *out, const void *query, const void *key_cache, const void *value_cache,
+                        const int32_t *block_tables, const int32_t *seq_lens, float scale, float k_scale,
+                        float v_scale, int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                        int max_blocks_per_seq, int num_blocks, int max_seq_len, int partition_size,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                    num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    a.fp8 = true;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (partition_size == 0) return run_decode(a, 0, 0, workspace, workspace ? workspace_bytes : 0, st);
+    return run_decode(a, 1, partition_size, workspace, workspace_bytes, st);
 }
 
 // Scratch of pa_decode_split_noalloc: one fixed array per device, part of the

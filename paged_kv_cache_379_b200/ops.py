@@ -12,6 +12,8 @@ Tensor conventions (see include/pagedkv.h):
   seq_lens               : int32 [num_seqs]
   slot_mapping           : int64 [num_tokens]
   src_dst_pairs          : int64 [num_pairs, 2]
+  FP8 caches             : uint8 E4M3 codes [num_blocks, block_size, num_kv_heads, head_dim]
+                           with one fp32 scale per cache (k_scale, v_scale)
 """
 
 from __future__ import annotations
@@ -27,7 +29,7 @@ __all__ = [
     "slot_mapping", "reshape_and_cache", "copy_blocks", "decode", "decode_one_pass",
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
-    "decode_split_noalloc", "swap_blocks",
+    "decode_split_noalloc", "swap_blocks", "reshape_and_cache_fp8", "decode_fp8", "decode_fp8_split",
 ]
 
 
@@ -53,9 +55,9 @@ def _dev(t: torch.Tensor | None, dtype, name: str, ndim: int | None = None):
     return t.data_ptr()
 
 
-def _cache_dims(key_cache, value_cache):
-    _dev(key_cache, torch.bfloat16, "key_cache", 4)
-    _dev(value_cache, torch.bfloat16, "value_cache", 4)
+def _cache_dims(key_cache, value_cache, dtype=torch.bfloat16):
+    _dev(key_cache, dtype, "key_cache", 4)
+    _dev(value_cache, dtype, "value_cache", 4)
     if key_cache.shape != value_cache.shape:
         raise ValueError("key_cache and value_cache shapes differ")
     nb, bs, hkv, d = key_cache.shape
@@ -94,6 +96,23 @@ def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, stream=N
         _stream(stream)))
 
 
+def reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_scale: float, v_scale: float,
+                          stream=None) -> None:
+    """pa_reshape_and_cache_fp8: bf16 rows quantised to E4M3 codes in uint8 caches."""
+    lib = load()
+    nb, bs, hkv, d = _cache_dims(key_cache, value_cache, torch.uint8)
+    k = _dev(key, torch.bfloat16, "key", 3)
+    v = _dev(value, torch.bfloat16, "value", 3)
+    if tuple(key.shape[1:]) != (hkv, d) or key.shape != value.shape:
+        raise ValueError("key/value must be [num_tokens, num_kv_heads, head_dim] matching the cache")
+    sm = _dev(slot_mapping, torch.int64, "slot_mapping", 1)
+    if slot_mapping.shape[0] != key.shape[0]:
+        raise ValueError("slot_mapping length != num_tokens")
+    check("pa_reshape_and_cache_fp8", lib.pa_reshape_and_cache_fp8(
+        k, v, key_cache.data_ptr(), value_cache.data_ptr(), sm, key.shape[0], hkv, d, bs, nb, float(k_scale),
+        float(v_scale), _stream(stream)))
+
+
 def copy_blocks(key_cache, value_cache, src_dst_pairs, stream=None) -> None:
     lib = load()
     nb, bs, hkv, d = _cache_dims(key_cache, value_cache)
@@ -130,8 +149,8 @@ def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, 
         dst_key_cache.shape[0], _stream(stream)))
 
 
-def _decode_common(query, key_cache, value_cache, block_tables, seq_lens):
-    nb, bs, hkv, d = _cache_dims(key_cache, value_cache)
+def _decode_common(query, key_cache, value_cache, block_tables, seq_lens, cache_dtype=torch.bfloat16):
+    nb, bs, hkv, d = _cache_dims(key_cache, value_cache, cache_dtype)
     q = _dev(query, torch.bfloat16, "query", 3)
     B, hq, dq = query.shape
     if dq != d:
@@ -180,6 +199,35 @@ def decode(query, key_cache, value_cache, block_tables, seq_lens, scale: float, 
     wp, wb = _ws(workspace)
     check("pa_decode", lib.pa_decode(o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale),
                                      bs, hkv, B, hq, d, mb, nb, int(max_seq_len), wp, wb, _stream(stream)))
+    return out
+
+
+def decode_fp8(query, key_cache, value_cache, block_tables, seq_lens, scale: float, k_scale: float,
+               v_scale: float, max_seq_len: int, *, out=None, workspace=None, stream=None):
+    """pa_decode_fp8: pa_decode over uint8 E4M3 caches with per-tensor scales."""
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens,
+                                                          torch.uint8)
+    o, out = _out(out, query)
+    wp, wb = _ws(workspace)
+    check("pa_decode_fp8", lib.pa_decode_fp8(
+        o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), float(k_scale), float(v_scale),
+        bs, hkv, B, hq, d, mb, nb, int(max_seq_len), wp, wb, _stream(stream)))
+    return out
+
+
+def decode_fp8_split(query, key_cache, value_cache, block_tables, seq_lens, scale: float, k_scale: float,
+                     v_scale: float, max_seq_len: int, partition_size: int, workspace=None, *, out=None,
+                     stream=None):
+    """pa_decode_fp8_split: partition_size 0 = one pass, else the split form."""
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens,
+                                                          torch.uint8)
+    o, out = _out(out, query)
+    wp, wb = _ws(workspace)
+    check("pa_decode_fp8_split", lib.pa_decode_fp8_split(
+        o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), float(k_scale), float(v_scale),
+        bs, hkv, B, hq, d, mb, nb, int(max_seq_len), int(partition_size), wp, wb, _stream(stream)))
     return out
 
 

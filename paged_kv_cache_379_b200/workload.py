@@ -92,6 +92,33 @@ def _fill_cache(rng, num_blocks, bs, hkv, d, free):
     return cache
 
 
+E4M3_NAN = np.uint8(0x7F)
+
+
+def fp8_codes(rng: np.random.Generator, shape, zero_exp_frac: float = 0.05) -> np.ndarray:
+    """Random E4M3 codes (uint8): sign uniform, mantissa field uniform in 0..7,
+    exponent field uniform in 3..9 (magnitudes 2^-4 .. 2^2 * 1.875), except a
+    fraction `zero_exp_frac` of codes with exponent field 0 (zero and
+    subnormals).  Never the NaN pattern (exponent 15, mantissa 7)."""
+    n = int(np.prod(shape))
+    sign = rng.integers(0, 2, n, dtype=np.uint8) << 7
+    exp = rng.integers(3, 10, n, dtype=np.uint8)
+    exp[rng.random(n) < zero_exp_frac] = 0
+    man = rng.integers(0, 8, n, dtype=np.uint8)
+    return (sign | (exp << 3) | man).astype(np.uint8).reshape(shape)
+
+
+def fp8_cache(rng: np.random.Generator, num_blocks: int, bs: int, hkv: int, d: int, free) -> np.ndarray:
+    """An E4M3 code cache: random codes in owned blocks, the NaN code in unowned ones."""
+    cache = np.empty((num_blocks, bs, hkv, d), dtype=np.uint8)
+    is_free = np.zeros(num_blocks, dtype=bool)
+    is_free[np.asarray(free, dtype=np.int64)] = True
+    owned = np.flatnonzero(~is_free)
+    cache[is_free] = E4M3_NAN
+    cache[owned] = fp8_codes(rng, (owned.size, bs, hkv, d))
+    return cache
+
+
 @dataclass
 class Workload:
     name: str

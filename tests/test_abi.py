@@ -78,6 +78,35 @@ def test_argument_errors_without_gpu(lib):
     assert lib.pa_reshape_and_cache(fake, fake, fake, fake, fake, 3, 8, 128, 16, 0, None) == -2
 
 
+def test_fp8_argument_errors_without_gpu(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    # (out, q, kc, vc, bt, sl, scale, k_scale, v_scale, bs, Hkv, B, Hq, D, max_blocks, nb, max_len, ws, ws_bytes, st)
+    assert lib.pa_decode_fp8(fake, fake, fake, fake, fake, fake, 1.0, 1.0, 1.0, 16, 8, 4, 64, 64, 8, 100, 128,
+                             None, 0, None) == -3       # head_dim 64 not compiled for FP8
+    assert lib.pa_decode_fp8(fake, fake, fake, fake, fake, fake, 1.0, 1.0, 1.0, 4, 8, 4, 64, 128, 8, 100, 128,
+                             None, 0, None) == -3       # block_size 4 not compiled for FP8
+    assert lib.pa_decode_fp8(fake, fake, fake, fake, fake, fake, 1.0, 0.0, 1.0, 16, 8, 4, 64, 128, 8, 100, 128,
+                             None, 0, None) == -2       # scales must be positive and finite
+    assert lib.pa_decode_fp8(fake, fake, fake, fake, fake, fake, 1.0, 1.0, float("nan"), 16, 8, 4, 64, 128, 8,
+                             100, 128, None, 0, None) == -2
+    assert lib.pa_decode_fp8_split(fake, fake, fake, fake, fake, fake, 1.0, 1.0, 1.0, 16, 8, 4, 64, 128, 8, 100,
+                                   128, 512, None, 0, None) == -4   # split form needs a workspace
+    # (k, v, kc, vc, slots, T, Hkv, D, bs, nb, k_scale, v_scale, st)
+    assert lib.pa_reshape_and_cache_fp8(fake, fake, fake, fake, fake, 3, 8, 128, 16, 10, -1.0, 1.0, None) == -2
+    assert lib.pa_reshape_and_cache_fp8(fake, fake, fake, fake, fake, 3, 1, 8, 16, 10, 1.0, 1.0, None) == -3
+    assert lib.pa_reshape_and_cache_fp8(None, None, None, None, None, 0, 8, 128, 16, 10, 1.0, 1.0, None) == 0
+
+
+def test_fp8_code_generator_never_draws_nan():
+    import numpy as np
+    from paged_kv_cache_379_b200 import workload as wl
+    c = wl.fp8_codes(np.random.default_rng(0), (200000,))
+    assert c.dtype == np.uint8 and not ((c & 0x7F) == 0x7F).any()
+    exps = np.unique((c >> 3) & 15)
+    assert 0 in exps and set(exps) <= {0, 3, 4, 5, 6, 7, 8, 9}
+
+
 def test_workspace_size(lib):
     # 256-byte scheduler header, then for 4 seqs x 8 heads x ceil(1000/512)=2 parts:
     # o = 64*128*4 B, m and l = 64*4 B each (each 256-aligned)
