@@ -273,6 +273,32 @@ int pa_decode_fp8_split(void *out, const void *query, const void *key_cache,
                         void *stream);
 
 /* --------------------------------------------------------------------------
+ * Multi-query paged prefill: the chunked-prefill step ([深度解析], milestone
+ * list: v0.5 "Chunked Prefill" -- a long prompt is fed in chunks so that it
+ * does not hold up decodes) with the causal rule of [论文专题] (the query at
+ * position i attends to positions up to and including i).
+ *   seq_lens  int32 [num_seqs]: cached positions of each sequence, this
+ *             chunk's tokens included (their K/V rows are already in the cache,
+ *             e.g. written by pa_reshape_and_cache);
+ *   q_start   int32 [num_seqs + 1] (device): the chunk of sequence s is query
+ *             rows q_start[s] .. q_start[s+1]-1, in position order, and holds
+ *             its last q_len = q_start[s+1] - q_start[s] positions;
+ *   query, out: bf16 [num_tokens, num_heads, head_dim], num_tokens = q_start[num_seqs].
+ * Row q_start[s] + i (position p = seq_len - q_len + i) gets
+ *     out = sum_{j <= p} softmax_j(scale * q . k_j) v_j,
+ * with K/V read block by block through the table.  Sequences with q_len <= 0
+ * or q_len > seq_len are skipped (their rows are not written).
+ * Supported: head_dim 64 or 128, block_size 8, 16 or 32, G = num_heads /
+ * num_kv_heads in 1..16.  fp32 accumulation on the tensor cores (tcgen05),
+ * softmax weights as a bf16 high part plus a bf16 residual; output rounded to
+ * bf16.  No workspace; one launch.
+ * ------------------------------------------------------------------------ */
+int pa_prefill(void *out, const void *query, const void *key_cache, const void *value_cache,
+               const int32_t *block_tables, const int32_t *seq_lens, const int32_t *q_start,
+               float scale, int block_size, int num_kv_heads, int num_seqs, int num_heads,
+               int head_dim, int max_blocks_per_seq, int num_blocks, int num_tokens, void *stream);
+
+/* --------------------------------------------------------------------------
  * Precondition check on the device: counts, into *bad_count (device int32,
  * overwritten), the sequences whose seq_len is negative or above max_seq_len,
  * whose ceil(seq_len/block_size) exceeds max_blocks_per_seq, or whose used

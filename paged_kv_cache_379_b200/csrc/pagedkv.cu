@@ -11,6 +11,7 @@
 #include "cache_ops.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "prefill.cuh"
 
 namespace pakv {
 
@@ -58,6 +59,26 @@ static int make_cache_map(CUtensorMap *map, const void *cache, int64_t num_block
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                           const_cast<void *>(cache), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_last_cuda_error(cudaErrorInvalidValue);
+        return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
+// The queries [T, Hq, D] as {64 elements, D/64, Hq, T} with a box of one
+// 64-wide d-plane of G heads x q_box tokens: rows token-major, head-minor.
+static int make_query_map(CUtensorMap *map, const void *query, int64_t tokens, int hq, int d, int g, int q_box)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return check_cuda(cudaErrorNotSupported);
+    const cuuint64_t dims[4] = {64, (cuuint64_t)(d / 64), (cuuint64_t)hq, (cuuint64_t)tokens};
+    const cuuint64_t strides[3] = {128, (cuuint64_t)d * 2, (cuuint64_t)hq * d * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)g, (cuuint32_t)q_box};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(query), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -310,6 +331,30 @@ static int choose_plan(int num_seqs, int num_kv_heads, int max_seq_len)
     return part;
 }
 
+template <int D, int BS>
+static int launch_prefill_t(const PrefillParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                            const CUtensorMap &tv, int64_t tiles, cudaStream_t st)
+{
+    auto kernel = paged_prefill_kernel<D, BS>;
+    const size_t smem = (size_t)PfLayout<D>::kAlloc;
+    int rc = ensure_smem(reinterpret_cast<const void *>(kernel), smem);
+    if (rc != PA_OK) return rc;
+    return launch_pdl(kernel, dim3((unsigned)tiles, (unsigned)p.num_kv_heads), dim3(kPfThreads), smem, st, p, tq,
+                      tk, tv);
+}
+
+template <int D>
+static int launch_prefill_d(int bs, const PrefillParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                            const CUtensorMap &tv, int64_t tiles, cudaStream_t st)
+{
+    switch (bs) {
+    case 8: return launch_prefill_t<D, 8>(p, tq, tk, tv, tiles, st);
+    case 16: return launch_prefill_t<D, 16>(p, tq, tk, tv, tiles, st);
+    case 32: return launch_prefill_t<D, 32>(p, tq, tk, tv, tiles, st);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
 }  // namespace pakv
 
 using namespace pakv;
@@ -553,6 +598,54 @@ int pa_decode_fp8_split(void *out, const void *query, const void *key_cache, con
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (partition_size == 0) return run_decode(a, 0, 0, workspace, workspace ? workspace_bytes : 0, st);
     return run_decode(a, 1, partition_size, workspace, workspace_bytes, st);
+}
+
+int pa_prefill(void *out, const void *query, const void *key_cache, const void *value_cache,
+               const int32_t *block_tables, const int32_t *seq_lens, const int32_t *q_start, float scale,
+               int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+               int num_blocks, int num_tokens, void *stream)
+{
+    if (num_seqs < 0 || num_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+        return PA_ERR_BAD_SHAPE;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_BAD_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (block_size != 8 && block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+    const int G = num_heads / num_kv_heads;
+    if (G > 16) return PA_ERR_UNSUPPORTED;
+    if ((int64_t)num_blocks * block_size > INT_MAX || (int64_t)max_blocks_per_seq * block_size > INT_MAX)
+        return PA_ERR_BAD_SHAPE;
+    if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !q_start)
+        return PA_ERR_NULL_POINTER;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+        return PA_ERR_ALIGNMENT;
+    PrefillParams p = {};
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.q_start = q_start;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = G;
+    p.max_blocks = max_blocks_per_seq;
+    p.tq = kPfRows / G;
+    p.q_box = std::min(p.tq, num_tokens);
+    // the tiles of all sequences number at most T / tq + B
+    const int64_t tiles = (int64_t)num_tokens / p.tq + num_seqs;
+    if (tiles > INT_MAX) return PA_ERR_BAD_SHAPE;
+    CUtensorMap tq, tk, tv;
+    int rc = make_query_map(&tq, query, num_tokens, num_heads, head_dim, G, p.q_box);
+    if (rc != PA_OK) return rc;
+    rc = make_cache_map(&tk, key_cache, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc != PA_OK) return rc;
+    rc = make_cache_map(&tv, value_cache, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc != PA_OK) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return head_dim == 64 ? launch_prefill_d<64>(block_size, p, tq, tk, tv, tiles, st)
+                          : launch_prefill_d<128>(block_size, p, tq, tk, tv, tiles, st);
 }
 
 // Scratch of pa_decode_split_noalloc: one fixed array per device, part of the

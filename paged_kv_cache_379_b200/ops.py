@@ -30,6 +30,7 @@ __all__ = [
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
     "decode_split_noalloc", "swap_blocks", "reshape_and_cache_fp8", "decode_fp8", "decode_fp8_split",
+    "prefill",
 ]
 
 
@@ -228,6 +229,29 @@ def decode_fp8_split(query, key_cache, value_cache, block_tables, seq_lens, scal
     check("pa_decode_fp8_split", lib.pa_decode_fp8_split(
         o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), float(k_scale), float(v_scale),
         bs, hkv, B, hq, d, mb, nb, int(max_seq_len), int(partition_size), wp, wb, _stream(stream)))
+    return out
+
+
+def prefill(query, key_cache, value_cache, block_tables, seq_lens, q_start, scale: float, *, out=None,
+            stream=None):
+    """pa_prefill: causal multi-query attention of each sequence's chunk (query rows
+    q_start[s] .. q_start[s+1]-1, the last positions of the sequence) over its paged cache."""
+    lib = load()
+    nb, bs, hkv, d = _cache_dims(key_cache, value_cache)
+    q = _dev(query, torch.bfloat16, "query", 3)
+    T, hq, dq = query.shape
+    if dq != d:
+        raise ValueError("query head_dim != cache head_dim")
+    bt = _dev(block_tables, torch.int32, "block_tables", 2)
+    sl = _dev(seq_lens, torch.int32, "seq_lens", 1)
+    qs = _dev(q_start, torch.int32, "q_start", 1)
+    B = seq_lens.shape[0]
+    if block_tables.shape[0] != B or q_start.shape[0] != B + 1:
+        raise ValueError("block_tables rows / q_start length do not match seq_lens")
+    o, out = _out(out, query)
+    check("pa_prefill", lib.pa_prefill(o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, qs,
+                                       float(scale), bs, hkv, B, hq, d, block_tables.shape[1], nb, T,
+                                       _stream(stream)))
     return out
 
 
