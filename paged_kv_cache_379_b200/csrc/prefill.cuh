@@ -11,17 +11,20 @@
 // 128 MMA rows = tq tokens x G query heads (row r = token r / G, head r % G),
 // so every K/V tile read from the cache feeds all G heads of the KV head.
 //   warps 0-3  softmax: warp w owns TMEM lanes 32w..32w+31, i.e. one row per
-//              thread; reads S from TMEM, online softmax with a lazily moved
-//              reference max, writes P (bf16 high part and bf16 residual) to
-//              shared memory, rescales O in TMEM when a reference moves, and
-//              finally normalises O and stores the output rows;
+//              thread; reads S_j from TMEM, online softmax with a lazily moved
+//              reference max, and writes P_j back over S_j in TMEM as a bf16
+//              high part and a bf16 residual (each truncated); rescales O in
+//              TMEM when a reference moves; finally normalises O and stores the
+//              output rows;
 //   warp 4     producer: TMA loads of the query tile (once) and of 128-key K/V
-//              tiles, block by block through the table, into a 2-stage ring;
-//   warp 5     MMA: allocates TMEM (S double-buffered in columns 0..255, O in
-//              256..256+D) and one thread issues tcgen05.mma:
-//                S_j = Q K_j^T        (M 128, N 128, K D; both operands K-major)
-//                O  += P_hi V_j + P_lo V_j   (M 128, N D, K 128; V MN-major)
-//              with completion tracked by tcgen05.commit on mbarriers.
+//              tiles, block by block through the table, into a 3-stage ring;
+//   warp 5     MMA: allocates TMEM -- three S/P buffers in columns 0..383, O in
+//              384..384+D -- and one thread issues tcgen05.mma:
+//                S_j = Q K_j^T              (SS form: M 128, N 128, K D)
+//                O  += P_hi V_j + P_lo V_j  (TS form, P read from TMEM; V an
+//                                            MN-major shared-memory operand)
+//              with completion tracked by tcgen05.commit on mbarriers.  S_j
+//              reuses buffer j % 3 once P_{j-3} V has completed.
 // Every wait is bounded in time; after a timeout the CTA drains its own TMA
 // loads and MMAs (bounded again), frees TMEM and returns.
 #pragma once
@@ -47,8 +50,9 @@ constexpr int kPfProducerWarp = 4;
 constexpr int kPfMmaWarp = 5;
 constexpr int kPfRows = 128;          // MMA M: query rows per tile
 constexpr int kPfKeys = 128;          // keys per K/V tile
+constexpr int kPfStages = 3;          // K/V ring stages = TMEM S/P buffers
 constexpr uint32_t kPfTmemCols = 512;
-constexpr uint32_t kPfTmemO = 256;    // first TMEM column of O
+constexpr uint32_t kPfTmemO = 384;    // first TMEM column of O
 // A row's softmax reference max moves only when a logit exceeds it by more
 // than this (log2 units), so unnormalised weights stay below 2^8.
 constexpr float kPfRescaleSlack = 8.f;
@@ -61,11 +65,9 @@ struct PfLayout {
     static constexpr int kTile = kPlanes * kPlane;         // Q, K or V tile
     static constexpr int kStage0 = kQ + kTile;
     static constexpr int kStageBytes = 2 * kTile;          // K tile then V tile
-    static constexpr int kPhi = kStage0 + 2 * kStageBytes;
-    static constexpr int kPlo = kPhi + 2 * kPlane;         // P: 128 rows x 128 keys
-    static constexpr int kBar = kPlo + 2 * kPlane;
-    // q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done, drain
-    static constexpr int kNumBars = 12;
+    static constexpr int kBar = kStage0 + kPfStages * kStageBytes;
+    // q_full, then per stage: kv_full, kv_empty, s_full, p_full, o_done; drain
+    static constexpr int kNumBars = 2 + 5 * kPfStages;
     static constexpr int kMisc = kBar + kNumBars * 8;      // TMEM base, abort flag, item
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
@@ -91,13 +93,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
     const uint32_t bar0 = base + Lay::kBar;
     const uint32_t q_full = bar0;
-    const uint32_t p_full = bar0 + 8 * 9;
-    const uint32_t o_done = bar0 + 8 * 10;
-    const uint32_t drain = bar0 + 8 * 11;
-    auto kv_full = [&](int st) { return bar0 + 8u * (1 + st); };
-    auto kv_empty = [&](int st) { return bar0 + 8u * (3 + st); };
-    auto s_full = [&](int b) { return bar0 + 8u * (5 + b); };
-    auto s_free = [&](int b) { return bar0 + 8u * (7 + b); };
+    const uint32_t drain = bar0 + 8;
+    auto kv_full = [&](int st) { return bar0 + 8u * (2 + st); };
+    auto kv_empty = [&](int st) { return bar0 + 8u * (2 + kPfStages + st); };
+    auto s_full = [&](int b) { return bar0 + 8u * (2 + 2 * kPfStages + b); };
+    auto p_full = [&](int b) { return bar0 + 8u * (2 + 3 * kPfStages + b); };
+    auto o_done = [&](int b) { return bar0 + 8u * (2 + 4 * kPfStages + b); };
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(base_ptr + Lay::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Lay::kMisc + 4);
     volatile int *item = reinterpret_cast<volatile int *>(base_ptr + Lay::kMisc + 16);
@@ -141,15 +142,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     if (threadIdx.x == 32) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        mbar_init(drain, 1);
+        for (int i = 0; i < kPfStages; ++i) {
             mbar_init(kv_full(i), 1);
             mbar_init(kv_empty(i), 1);
             mbar_init(s_full(i), 1);
-            mbar_init(s_free(i), 128);
+            mbar_init(p_full(i), 128);
+            mbar_init(o_done(i), 1);
         }
-        mbar_init(p_full, 128);
-        mbar_init(o_done, 1);
-        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -198,13 +198,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 tma_load_4d(base + Lay::kQ + pl * kPlane, &tmap_q, q_full, 0, pl, g * G, q0 + t_begin);
         }
         const int32_t *table = p.block_tables + (int64_t)s * p.max_blocks;
-        int last[2] = {-1, -1};
+        int last[kPfStages] = {-1, -1, -1};
         for (int j = 0; j < nk; ++j) {
-            const int st = j & 1;
+            const int st = j % kPfStages;
             const int key0 = j * kPfKeys;
             const int nblk = min(kPfKeys / BS, (L - key0 + BS - 1) / BS);
             const int phys = lane < nblk ? table[key0 / BS + lane] : 0;
-            if (j >= 2 && !__all_sync(0xffffffffu, wait(kv_empty(st), ((j >> 1) - 1) & 1))) break;
+            if (j >= kPfStages &&
+                !__all_sync(0xffffffffu, wait(kv_empty(st), (j / kPfStages - 1) & 1)))
+                break;
             if (lane == 0) mbar_arrive_expect_tx(kv_full(st), (uint32_t)(nblk * BS * D * 2 * 2));
             const uint32_t kdst = base + Lay::kStage0 + st * Lay::kStageBytes;
             const uint32_t vdst = kdst + Lay::kTile;
@@ -222,8 +224,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         if (lane == 0 && *abort_flag) {  // let the loads this CTA issued land before it exits
             mbar_wait_bounded(q_full, 0);
-            for (int st = 0; st < 2; ++st)
-                if (last[st] >= 0) mbar_wait_bounded(kv_full(st), (last[st] >> 1) & 1);
+            for (int st = 0; st < kPfStages; ++st)
+                if (last[st] >= 0) mbar_wait_bounded(kv_full(st), (last[st] / kPfStages) & 1);
         }
     } else if (warp == kPfMmaWarp) {
         // ------------------------------------------------------------ MMA issue
@@ -232,8 +234,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         bool ok = __all_sync(0xffffffffu, wait(q_full, 0));
         for (int j = 0; ok && j <= nk; ++j) {
             if (j < nk) {
-                const int st = j & 1;
-                ok = __all_sync(0xffffffffu, wait(kv_full(st), (j >> 1) & 1));
+                const int st = j % kPfStages;  // ring stage and TMEM S/P buffer
+                ok = __all_sync(0xffffffffu, wait(kv_full(st), (j / kPfStages) & 1));
                 if (!ok) break;
                 // value rows past the sequence end hold stale or foreign data (maybe
                 // NaN); P is 0 there, but 0 * NaN is NaN in the MMA: zero them
@@ -248,9 +250,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                const int b = j & 1;
-                if (j >= 2) {
-                    ok = __all_sync(0xffffffffu, wait(s_free(b), ((j >> 1) - 1) & 1));
+                if (j >= kPfStages) {  // buffer st is free once P_{j-3} V has completed
+                    ok = __all_sync(0xffffffffu, wait(o_done(st), (j / kPfStages - 1) & 1));
                     if (!ok) break;
                 }
                 tc_fence_after();
@@ -259,32 +260,33 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * kPlane + (kk & 3) * 32;
-                        tc_mma_bf16(tmem + b * kPfKeys, desc_kmajor_sw128(base + Lay::kQ + off),
+                        tc_mma_bf16(tmem + st * kPfKeys, desc_kmajor_sw128(base + Lay::kQ + off),
                                     desc_kmajor_sw128(kt + off), kIdS, kk > 0);
                     }
-                    tc_commit(s_full(b));
+                    tc_commit(s_full(st));
                 }
                 __syncwarp();
             }
             if (j >= 1) {
-                const int jp = j - 1;
-                ok = __all_sync(0xffffffffu, wait(p_full, jp & 1));
+                const int jp = j - 1, bp = jp % kPfStages;
+                ok = __all_sync(0xffffffffu, wait(p_full(bp), (jp / kPfStages) & 1));
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t vt = base + Lay::kStage0 + (jp & 1) * Lay::kStageBytes + Lay::kTile;
+                    const uint32_t vt = base + Lay::kStage0 + bp * Lay::kStageBytes + Lay::kTile;
+                    // P_hi in columns [0, 64) of the buffer, P_lo in [64, 128); a K step
+                    // of 16 keys is 8 columns
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
-                        const uint32_t pb = base + (half ? Lay::kPlo : Lay::kPhi);
 #pragma unroll
                         for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-                            tc_mma_bf16(tmem + kPfTmemO, desc_kmajor_sw128(pb + (kk >> 2) * kPlane + (kk & 3) * 32),
-                                        desc_mnmajor_sw128(vt + kk * 16 * 128, kPlane), kIdO,
-                                        jp > 0 || half > 0 || kk > 0);
+                            tc_mma_bf16_ts(tmem + kPfTmemO, tmem + bp * kPfKeys + half * 64 + kk * 8,
+                                           desc_mnmajor_sw128(vt + kk * 16 * 128, kPlane), kIdO,
+                                           jp > 0 || half > 0 || kk > 0);
                         }
                     }
-                    tc_commit(kv_empty(jp & 1));
-                    tc_commit(o_done);
+                    tc_commit(kv_empty(bp));
+                    tc_commit(o_done(bp));
                 }
                 __syncwarp();
             }
@@ -298,76 +300,79 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const bool row_ok = tok < p.tq && i < t_end;
         const int pos = row_ok ? ctx + i : L - 1;
         const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-        uint8_t *const phi = base_ptr + Lay::kPhi + r * 128;
-        uint8_t *const plo = base_ptr + Lay::kPlo + r * 128;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nk; ++j) {
-            const int b = j & 1;
-            ok = __all_sync(0xffffffffu, wait(s_full(b), (j >> 1) & 1));
+            const int b = j % kPfStages;
+            ok = __all_sync(0xffffffffu, wait(s_full(b), (j / kPfStages) & 1));
             if (!ok) break;
             tc_fence_after();
             float x[kPfKeys];
+            tmem_ld128(lane_addr + b * kPfKeys, x);
+            // causal mask, only in tiles that reach past some row's position
+            const int lim = pos - j * kPfKeys;  // keys c <= lim are visible
+            if (!__all_sync(0xffffffffu, lim >= kPfKeys - 1)) {
 #pragma unroll
-            for (int c = 0; c < kPfKeys / 32; ++c) tmem_ld32(lane_addr + b * kPfKeys + c * 32, x + c * 32);
-            tc_fence_before();
-            mbar_arrive(s_free(b));
-            const int key0 = j * kPfKeys;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < kPfKeys; ++c) {
-                x[c] = key0 + c <= pos ? x[c] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, x[c]);
+                for (int c = 0; c < kPfKeys; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
             }
-            // lazily moved reference max: weights stay <= 2^kPfRescaleSlack
+            // row max as a tree over 8 independent partial maxima
+            float pm[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pm[u] = x[u];
+#pragma unroll
+            for (int c = 8; c < kPfKeys; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
+            const float mx =
+                fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) *
+                p.scale_log2;  // scale > 0: the max commutes with it
+            // lazily moved reference max (log2 units): weights stay <= 2^kPfRescaleSlack
             const bool bump = mx > m + kPfRescaleSlack;
             float corr = 1.f;
             if (bump) {
-                corr = exp2f(m - mx);  // 0 on the first tile (m = -inf)
+                corr = fast_exp2(m - mx);  // 0 on the first tile (m = -inf)
                 m = mx;
             }
-            l *= corr;
-            if (j >= 1) {  // P buffers and O are free once the previous P V is done
-                ok = __all_sync(0xffffffffu, wait(o_done, (j - 1) & 1));
+            // weights, their sum (8 independent partial sums), and P split into a
+            // bf16 high part and a bf16 residual, both by truncation (the pair
+            // keeps 16 significant bits: relative error below 2^-15)
+            float ps[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+            uint32_t hl[kPfKeys];  // [0, 64): high parts, [64, 128): residuals
+#pragma unroll
+            for (int e = 0; e < kPfKeys / 2; ++e) {
+                const float p0 = fast_exp2(fmaf(x[2 * e], p.scale_log2, -m));
+                const float p1 = fast_exp2(fmaf(x[2 * e + 1], p.scale_log2, -m));
+                ps[e & 7] += p0 + p1;
+                const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                hl[e] = prmt(b0, b1, 0x7632u);  // high halves: bf16(p0) | bf16(p1) << 16
+                const float r0 = p0 - __uint_as_float(b0 & 0xFFFF0000u);
+                const float r1 = p1 - __uint_as_float(b1 & 0xFFFF0000u);
+                hl[kPfKeys / 2 + e] = prmt(__float_as_uint(r0), __float_as_uint(r1), 0x7632u);
+            }
+            l = l * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+            if (j >= 1 && __any_sync(0xffffffffu, bump)) {
+                // O holds P_{<j} V: rescale it once P_{j-1} V has completed
+                const int jp = j - 1;
+                ok = __all_sync(0xffffffffu, wait(o_done(jp % kPfStages), (jp / kPfStages) & 1));
                 if (!ok) break;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, bump)) {
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        float o[32];
-                        tmem_ld32(lane_addr + kPfTmemO + c * 32, o);
+                for (int c = 0; c < D / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(lane_addr + kPfTmemO + c * 32, o);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= corr;
-                        tmem_st32(lane_addr + kPfTmemO + c * 32, o);
-                    }
-                    tmem_wait_st();
+                    for (int e = 0; e < 32; ++e) o[e] *= corr;
+                    tmem_st32(lane_addr + kPfTmemO + c * 32, o);
                 }
             }
-            float rs = 0.f;
-#pragma unroll
-            for (int c8 = 0; c8 < kPfKeys / 8; ++c8) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(x[c8 * 8 + 2 * e] - m);
-                    const float p1 = exp2f(x[c8 * 8 + 2 * e + 1] - m);
-                    rs += p0 + p1;
-                    hi[e] = pack_bf16x2(p0, p1);
-                    const float2 h = unpack_bf16x2(hi[e]);
-                    lo[e] = pack_bf16x2(p0 - h.x, p1 - h.y);
-                }
-                // row r of the P tile, keys 8 c8 .. 8 c8 + 7: plane c8 / 8, 16-byte
-                // chunk c8 % 8, swizzled with r % 8
-                const int off = (c8 >> 3) * kPlane + (((c8 & 7) ^ (r & 7)) << 4);
-                *reinterpret_cast<uint4 *>(phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-            l += rs;
-            fence_proxy_async_smem();
+            // P over S in this buffer's columns
+            tmem_st64(lane_addr + b * kPfKeys, hl);
+            tmem_st64(lane_addr + b * kPfKeys + 64, hl + 64);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(p_full(b));
         }
-        if (ok) ok = __all_sync(0xffffffffu, wait(o_done, (nk - 1) & 1));
+        if (ok) ok = __all_sync(0xffffffffu, wait(o_done((nk - 1) % kPfStages), ((nk - 1) / kPfStages) & 1));
         if (ok) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
