@@ -9,6 +9,14 @@ lengths lognormal (median 1024, sigma 0.8) clipped to [16, 4096], shuffled
 block pool 1.2x.  Inputs are seeded synthetic data already resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa|gqa-fp8|prefill]
+
+The default workload is the line above.  Two more rows of the path are
+measured the same way on request: `gqa-fp8` (the same batch with an FP8 E4M3
+cache: slot mapping -> quantising cache write -> decode over codes; KV GB/s of
+1-byte elements) and `prefill` (8 x 2048-token prompts with the same heads:
+slot mapping -> cache write of the prompts' K/V -> causal paged prefill on the
+tensor cores; useful TFLOP/s).
 
 Prints ONE JSON line (rank 0).  `value` = KV GB/s: the decode's algorithmic
 bytes per step (KV blocks touched + queries + block tables + outputs) over the
@@ -43,7 +51,12 @@ SPEC_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_gqa_ncu.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_379_b200", "csrc", f)
-                  for f in ("decode.cuh", "common.cuh", "pagedkv.cu")]
+                  for f in ("decode.cuh", "common.cuh", "pagedkv.cu", "cache_ops.cuh", "prefill.cuh", "tc05.cuh")]
+PROFILE_FP8 = os.path.join(ROOT, "profiles", "paged_decode_fp8_gqa_ncu.md")
+PROFILE_PREFILL = os.path.join(ROOT, "profiles", "paged_prefill_prompt2k_ncu.md")
+METRIC_FP8 = "paged-decode KV GB/s, FP8 E4M3 KV cache (per-tensor scales), GQA 64q/8kv d128 b16"
+METRIC_PREFILL = "paged-prefill useful TFLOP/s (causal), 8 x 2048-token prompts, GQA 64q/8kv d128 b16"
+PREFILL_SHAPE = dict(num_seqs=8, prompt=2048, num_heads=64, num_kv_heads=8, head_dim=128, block_size=16)
 
 
 def workload_description(w) -> str:
@@ -80,18 +93,29 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel sources (else None)."""
+def profiled_traffic(path=PROFILE_SUMMARY, key="dram_bytes_per_decode_call"):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(path).read()
     except OSError:
         return None
     m_hash = re.search(r"kernel_source_sha256_16\s*=\s*([0-9a-f]+)", text)
-    m_bytes = re.search(r"dram_bytes_per_decode_call\s*=\s*([0-9]+)", text)
+    m_bytes = re.search(key + r"\s*=\s*([0-9]+)", text)
     if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
         return None
     return int(m_bytes.group(1))
+
+
+def measured_tensor_peak():
+    """Sustained dense bf16 TFLOP/s (a kernel timed inside a long loop)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured (MEASURED_PEAKS.json bf16_tflops_sustained)"
+    except Exception:
+        return 1400.0, "fallback (sustained bf16 figure of the profiling recipe)"
 
 
 # ------------------------------------------------------------------ clocks
@@ -386,6 +410,199 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     return line
 
 
+# ------------------------------------------------------- the other path rows
+
+def _timed_loop(step, K, W, stream, dev, dist, sampler):
+    """W untimed steps, then K timed steps between barriers; step(i) gets the
+    step index (or None in warm-up).  Returns (total_ms, clocks, remeasured)."""
+    import torch
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(W):
+        step(None)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+
+    def region():
+        barrier()
+        t0 = time.perf_counter()
+        e0.record(stream)
+        for i in range(K):
+            step(i)
+        e1.record(stream)
+        barrier()
+        return t0, time.perf_counter()
+
+    t0, t1 = region()
+    clocks = sampler.window(t0, t1)
+    remeasured = False
+    if set(clocks["reasons"]) & BAD_REASONS:
+        first = clocks
+        t0, t1 = region()
+        clocks = sampler.window(t0, t1)
+        clocks["first_attempt"] = first
+        remeasured = True
+    return e0.elapsed_time(e1), clocks, remeasured
+
+
+def prefill_flops(seq_lens, q_lens, num_heads, head_dim) -> int:
+    """Useful FLOPs of a causal prefill: 4 * D * Hq per (query row, visible key)."""
+    total = 0
+    for L, n in zip(seq_lens, q_lens):
+        L, n = int(L), int(n)
+        ctx = L - n
+        total += n * ctx + n * (n + 1) // 2
+    return 4 * head_dim * num_heads * total
+
+
+def make_prefill_case(seed):
+    """8 prompts of 2048 tokens (chunk = whole prompt), 64/8 heads, d128, bs16,
+    tables drawn from a shuffled pool of 1.2x the blocks needed."""
+    from paged_kv_cache_379_b200 import workload as wlmod
+    sh = PREFILL_SHAPE
+    B, P, bs = sh["num_seqs"], sh["prompt"], sh["block_size"]
+    lens = [P] * B
+    w = wlmod.random_decode_case(seed, num_seqs=B, num_heads=sh["num_heads"], num_kv_heads=sh["num_kv_heads"],
+                                 head_dim=sh["head_dim"], block_size=bs, lengths=lens,
+                                 spare_blocks=int(0.2 * B * P / bs))
+    rng = np.random.Generator(np.random.PCG64(seed + 1))
+    T = B * P
+    query = wlmod.bf16_normal(rng, (T, sh["num_heads"], sh["head_dim"]))
+    new_k = wlmod.bf16_normal(rng, (T, sh["num_kv_heads"], sh["head_dim"]))
+    new_v = wlmod.bf16_normal(rng, (T, sh["num_kv_heads"], sh["head_dim"]))
+    return w, lens, query, new_k, new_v
+
+
+def run_row(args, rank: int, world: int, local_rank: int) -> dict | None:
+    """gqa-fp8 or prefill, timed like the main line (device events, max over ranks)."""
+    import torch
+
+    from paged_kv_cache_379_b200 import ops
+    from paged_kv_cache_379_b200 import workload as wlmod
+    from paged_kv_cache_379_b200.step import bf16_to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    stream = torch.cuda.current_stream(dev)
+    K, W = args.steps, args.warmup
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)  # noqa: E731
+
+    if args.workload == "gqa-fp8":
+        w = wlmod.make("gqa", seed=rank_seed(rank), fill_cache=False)
+        rng = np.random.Generator(np.random.PCG64(rank_seed(rank) + 17))
+        kc_h = wlmod.fp8_cache(rng, w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.free_blocks)
+        vc_h = wlmod.fp8_cache(rng, w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.free_blocks)
+        kc, vc = torch.from_numpy(kc_h).to(dev), torch.from_numpy(vc_h).to(dev)
+        ks, vs = 0.25, 0.25
+        q, nk, nv = (bf16_to_device(a, dev) for a in (w.query, w.new_key, w.new_value))
+        bt, sl = i32(w.block_tables), i32(w.seq_lens)
+        slots = torch.empty(w.num_seqs, dtype=torch.int64, device=dev)
+        out = torch.empty_like(q)
+        ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, device=dev)
+        plan = ops.decode_plan(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, ws.numel())
+        units = algorithmic_bytes(w.seq_lens, w.block_size, w.num_heads, w.num_kv_heads, w.head_dim, 1)
+        launches = 2 + (2 if plan else 1)
+
+        def step(i):
+            ops.slot_mapping(bt, w.block_size, seq_lens=sl, out=slots, stream=stream)
+            ops.reshape_and_cache_fp8(nk, nv, kc, vc, slots, ks, vs, stream=stream)
+            if i is not None:
+                ev0[i].record(stream)
+            ops.decode_fp8(q, kc, vc, bt, sl, w.scale, ks, vs, w.max_seq_len, out=out, workspace=ws,
+                           stream=stream)
+            if i is not None:
+                ev1[i].record(stream)
+    else:
+        w, lens, qh, nkh, nvh = make_prefill_case(rank_seed(rank))
+        B, T = w.num_seqs, qh.shape[0]
+        kc, vc = bf16_to_device(w.key_cache, dev), bf16_to_device(w.value_cache, dev)
+        q, nk, nv = (bf16_to_device(a, dev) for a in (qh, nkh, nvh))
+        bt, sl = i32(w.block_tables), i32(lens)
+        start = np.zeros(B + 1, np.int32)
+        start[1:] = np.cumsum(lens)
+        qs = i32(start)
+        seq_ids = i32(np.repeat(np.arange(B), lens))
+        positions = torch.from_numpy(np.concatenate([np.arange(L) for L in lens]).astype(np.int64)).to(dev)
+        slots = torch.empty(T, dtype=torch.int64, device=dev)
+        out = torch.empty_like(q)
+        units = prefill_flops(lens, lens, w.num_heads, w.head_dim)
+        launches = 3
+
+        def step(i):
+            ops.slot_mapping(bt, w.block_size, positions=positions, seq_ids=seq_ids, out=slots, stream=stream)
+            ops.reshape_and_cache(nk, nv, kc, vc, slots, stream=stream)
+            if i is not None:
+                ev0[i].record(stream)
+            ops.prefill(q, kc, vc, bt, sl, qs, w.scale, out=out, stream=stream)
+            if i is not None:
+                ev1[i].record(stream)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    total_ms, clocks, remeasured = _timed_loop(step, K, W, stream, dev, dist, sampler)
+    sampler.stop()
+    kern_ms = float(np.mean([ev0[i].elapsed_time(ev1[i]) for i in range(K)]))
+    total_ms, _, all_units, all_seqs = aggregate_over_ranks(total_ms, 0.0, units, w.num_seqs, dev, dist)
+    if rank != 0:
+        return None
+    fp8 = args.workload == "gqa-fp8"
+    value = all_units * K / (total_ms * 1e-3) / (1e9 if fp8 else 1e12)
+    achieved = units / (kern_ms * 1e-3) / (1e9 if fp8 else 1e12)
+    if fp8:
+        peak, peak_src = measured_peak()
+        peak_src = f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src
+        traffic = profiled_traffic(PROFILE_FP8)
+    else:
+        peak, peak_src = measured_tensor_peak()
+        traffic = profiled_traffic(PROFILE_PREFILL, "dram_bytes_per_prefill_call")
+    line = {
+        "metric": METRIC_FP8 if fp8 else METRIC_PREFILL,
+        "value": round(value, 2),
+        "unit": "GB/s" if fp8 else "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 KV, bf16 q/out, fp16 MMA" if fp8 else "bf16",
+        "data": "synthetic (seeded)",
+        "config": ({"workload": f"gqa-fp8: {workload_description(w)}; E4M3 codes, k_scale = v_scale = 0.25",
+                    "decode_path": f"split, partition {plan}" if plan else "one pass",
+                    "step": "slot_mapping -> reshape_and_cache_fp8 -> decode_fp8",
+                    "algorithmic_bytes_per_step": units,
+                    "l2": f"inputs larger than L2 ({units / 1e9:.2f} GB read per step); no flush"}
+                   if fp8 else
+                   {"workload": "prefill: 8 prompts x 2048 tokens (whole-prompt chunks), 64 query / 8 KV heads, "
+                                "head_dim 128, block_size 16, shuffled pool 1.2x",
+                    "step": "slot_mapping (16384 tokens) -> reshape_and_cache -> prefill",
+                    "useful_flops_per_step": units,
+                    "l2": "compute bound; K/V (67 MB) re-read from L2 by every query tile; no flush"}),
+        "clocks": clocks,
+        "gpu_launches": launches * K,
+        "roofline": {"bound": "hbm" if fp8 else "tensor",
+                     "kernel": "pa_decode_fp8" if fp8 else "pa_prefill (paged_prefill_kernel)",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s" if fp8 else "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_src, "traffic": traffic,
+                     "avg_launch_ms": round(kern_ms, 5)},
+        "e2e": None,
+        "e2e_note": "end-to-end host-buffer timing is measured on the default workload only",
+    }
+    if remeasured:
+        line["clocks_note"] = "first timed region saw a thermal/hw slowdown reason; re-measured once"
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = (cpu_baseline_fp8(w, kc_h, vc_h, ks, vs, args.cpu_budget) if fp8 else
+                                cpu_baseline_prefill(w, qh, args.cpu_budget))
+    return line
+
+
 # ---------------------------------------------------------------- the oracle
 
 def cpu_baseline(w, budget_s: float = 15.0) -> dict:
@@ -408,6 +625,45 @@ def cpu_baseline(w, budget_s: float = 15.0) -> dict:
             "sample": f"{done_seqs} sequence decodes cycling through the {w.num_seqs}-sequence {WORKLOAD} batch "
                       f"(decode only), {elapsed:.1f} s, fp64, OpenMP over (sequence, head)",
             "seqs_per_s": round(done_seqs / elapsed, 2)}
+
+
+def cpu_baseline_fp8(w, kc, vc, ks, vs, budget_s: float) -> dict:
+    import oracle
+    threads = oracle.num_threads()
+    done, seqs, elapsed, i = 0, 0, 0.0, 0
+    while elapsed < budget_s:
+        idx = (np.arange(8) + i) % w.num_seqs
+        t = time.perf_counter()
+        oracle.paged_decode_fp8(w.query[idx], kc, vc, w.block_tables[idx], w.seq_lens[idx], w.scale, ks, vs,
+                                threads=threads)
+        elapsed += time.perf_counter() - t
+        done += algorithmic_bytes(w.seq_lens[idx], w.block_size, w.num_heads, w.num_kv_heads, w.head_dim, 1)
+        seqs += len(idx)
+        i += 8
+    return {"value": round(done / elapsed / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{seqs} FP8 sequence decodes cycling through the gqa batch, {elapsed:.1f} s, fp64"}
+
+
+def cpu_baseline_prefill(w, q, budget_s: float) -> dict:
+    """The oracle's prefill on windows of 16 query rows at spread positions."""
+    import oracle
+    threads = oracle.num_threads()
+    P = PREFILL_SHAPE["prompt"]
+    flops, rows, elapsed, i = 0, 0, 0.0, 0
+    while elapsed < budget_s:
+        s = i % w.num_seqs
+        end = 16 + (i * 389) % (P - 16)
+        qrows = q[s * P + end - 16: s * P + end]
+        t = time.perf_counter()
+        oracle.paged_prefill(qrows, w.key_cache, w.value_cache, w.block_tables[s:s + 1],
+                             np.array([end], np.int32), [16], w.scale, threads=threads)
+        elapsed += time.perf_counter() - t
+        flops += prefill_flops([end], [16], w.num_heads, w.head_dim)
+        rows += 16
+        i += 1
+    return {"value": round(flops / elapsed / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} query rows (windows of 16 at spread positions of the 2048-token prompts), "
+                      f"{elapsed:.1f} s, fp64"}
 
 
 def run_reference(args, rank: int) -> dict | None:
@@ -465,6 +721,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--workload", choices=["gqa", "gqa-fp8", "prefill"], default="gqa")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -473,6 +730,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
+        if args.workload != "gqa":
+            ap.error("--impl reference is the default workload's reference arm")
         line = run_reference(args, rank)
         if line is not None:
             print(json.dumps(line), flush=True)
@@ -490,7 +749,8 @@ def main():
     if world > 1:
         dist.barrier()
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = run_ours(args, rank, world, local_rank) if args.workload == "gqa" else \
+            run_row(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
