@@ -1,8 +1,8 @@
 #!/usr/bin/env python
 """Benchmark of the paged-KV decode hot path on B200.
 
-One step = slot mapping (new token's position -> cache slot) -> cache write of
-the new K/V -> paged decode attention (one pass, or partition kernel + LSE
+One step = slot mapping (new token's position -> cache slot) and cache write of
+the new K/V (one fused launch) -> paged decode attention (one pass, or partition kernel + LSE
 reduce, as the library chooses), over one batch of the GQA 70B-style layer
 workload: 128 sequences, 64 query / 8 KV heads, head_dim 128, block_size 16,
 lengths lognormal (median 1024, sigma 0.8) clipped to [16, 4096], shuffled
@@ -13,7 +13,7 @@ block pool 1.2x.  Inputs are seeded synthetic data already resident in HBM.
 
 The default workload is the line above.  Two more rows of the path are
 measured the same way on request: `gqa-fp8` (the same batch with an FP8 E4M3
-cache: slot mapping -> quantising cache write -> decode over codes; KV GB/s of
+cache: slot mapping + quantising cache write -> decode over codes; KV GB/s of
 1-byte elements) and `prefill` (8 x 2048-token prompts with the same heads:
 slot mapping -> cache write of the prompts' K/V -> causal paged prefill on the
 tensor cores; useful TFLOP/s).
@@ -232,7 +232,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     stream = torch.cuda.current_stream(dev)
     ws_bytes = 0 if batch.workspace is None else batch.workspace.numel()
     plan = ops.decode_plan(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, batch.max_seq_len, ws_bytes)
-    launches_per_step = 2 + (2 if plan else 1) + (1 if batch.pairs is not None else 0)
+    launches_per_step = 1 + (2 if plan else 1) + (1 if batch.pairs is not None else 0)
     step_bytes = algorithmic_bytes(w.seq_lens, w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
 
     K, W = args.steps, args.warmup
@@ -321,8 +321,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                 S["sl"].copy_(h_sl, non_blocking=True)
                 ev_in[b].record(up)
             stream.wait_event(ev_in[b])
-            ops.slot_mapping(S["bt"], w.block_size, seq_lens=S["sl"], out=S["slots"], stream=stream)
-            ops.reshape_and_cache(S["k"], S["v"], batch.key_cache, batch.value_cache, S["slots"], stream=stream)
+            ops.append_decode_kv(S["k"], S["v"], batch.key_cache, batch.value_cache, S["bt"], S["sl"],
+                                 slot_mapping=S["slots"], stream=stream)
             ops.decode(S["q"], batch.key_cache, batch.value_cache, S["bt"], S["sl"], w.scale, batch.max_seq_len,
                        out=S["out"], workspace=batch.workspace, stream=stream)
             ev_done[b].record(stream)
@@ -376,7 +376,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
             "head_dim": w.head_dim, "block_size": w.block_size, "sum_seq_len": int(w.seq_lens.sum()),
             "max_seq_len": w.max_seq_len, "algorithmic_bytes_per_step": step_bytes,
             "decode_path": f"split, partition {plan} (partition kernel + LSE reduce)" if plan else "one pass",
-            "step": "slot_mapping -> reshape_and_cache -> decode",
+            "step": "append_decode_kv (slot mapping + cache write, one launch) -> decode",
             "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB read per step vs 126 MB L2); no flush",
             "parallelism": f"dp{world}: independent batch per GPU, no collective on the data path",
         },
@@ -511,11 +511,10 @@ def run_row(args, rank: int, world: int, local_rank: int) -> dict | None:
         ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, device=dev)
         plan = ops.decode_plan(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, ws.numel())
         units = algorithmic_bytes(w.seq_lens, w.block_size, w.num_heads, w.num_kv_heads, w.head_dim, 1)
-        launches = 2 + (2 if plan else 1)
+        launches = 1 + (2 if plan else 1)
 
         def step(i):
-            ops.slot_mapping(bt, w.block_size, seq_lens=sl, out=slots, stream=stream)
-            ops.reshape_and_cache_fp8(nk, nv, kc, vc, slots, ks, vs, stream=stream)
+            ops.append_decode_kv_fp8(nk, nv, kc, vc, bt, sl, ks, vs, slot_mapping=slots, stream=stream)
             if i is not None:
                 ev0[i].record(stream)
             ops.decode_fp8(q, kc, vc, bt, sl, w.scale, ks, vs, w.max_seq_len, out=out, workspace=ws,
@@ -576,7 +575,7 @@ def run_row(args, rank: int, world: int, local_rank: int) -> dict | None:
         "data": "synthetic (seeded)",
         "config": ({"workload": f"gqa-fp8: {workload_description(w)}; E4M3 codes, k_scale = v_scale = 0.25",
                     "decode_path": f"split, partition {plan}" if plan else "one pass",
-                    "step": "slot_mapping -> reshape_and_cache_fp8 -> decode_fp8",
+                    "step": "append_decode_kv_fp8 (slot mapping + quantising cache write) -> decode_fp8",
                     "algorithmic_bytes_per_step": units,
                     "l2": f"inputs larger than L2 ({units / 1e9:.2f} GB read per step); no flush"}
                    if fp8 else

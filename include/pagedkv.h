@@ -101,6 +101,21 @@ int pa_reshape_and_cache(const void *key, const void *value, void *key_cache, vo
                          int head_dim, int block_size, int num_blocks, void *stream);
 
 /* --------------------------------------------------------------------------
+ * a1 + a2 in one launch, decode form: for each sequence s, its newest position
+ * pos = seq_lens[s] - 1 is translated to a slot exactly as pa_slot_mapping does
+ * (slot -1 when seq_lens[s] == 0, the position falls past the table row, or
+ * the table entry is negative) and key[s] / value[s] (bf16 [num_seqs,
+ * num_kv_heads, head_dim]) are stored there as pa_reshape_and_cache stores
+ * them.  slot_mapping (int64 [num_seqs], device) receives the slots, or is
+ * NULL.  The same result as pa_slot_mapping followed by pa_reshape_and_cache,
+ * one kernel instead of two.  num_kv_heads * head_dim must be a multiple of 8.
+ * ------------------------------------------------------------------------ */
+int pa_append_decode_kv(const void *key, const void *value, void *key_cache, void *value_cache,
+                        const int32_t *block_tables, const int32_t *seq_lens, int64_t *slot_mapping,
+                        int num_seqs, int max_blocks_per_seq, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, void *stream);
+
+/* --------------------------------------------------------------------------
  * a3. Copy-on-write block copy ([源码解析 §五] allocate_or_get_cow: a new block
  * receives a copy of the shared one; [深度解析 «Copy-on-Write 与 Prefix Caching»]).
  *   src_dst_pairs: int64 [num_pairs, 2] (device), pair i copies the whole
@@ -156,10 +171,10 @@ int pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, const void *src_k
  * pa_device_status() has reported a timeout, zero the workspace again.
  *
  * The decode kernel is persistent: (resident CTAs per SM) x (SMs) CTAs loop
- * over (sequence, partition, KV head) work items.  Sequence count limit of the
- * split form: the per-CTA prefix table of num_seqs+1 ints must fit in shared
- * memory next to the pipeline (num_seqs up to about 35000); beyond that the
- * call returns PA_ERR_BAD_SHAPE.
+ * over (sequence, partition, KV head) work items.  Sequence count limit: the
+ * per-CTA enumeration tables (10 bytes per sequence) must fit in shared memory
+ * next to the pipeline (num_seqs up to about 11000); beyond that the call
+ * returns PA_ERR_BAD_SHAPE.
  * ------------------------------------------------------------------------ */
 int pa_decode(void *out, const void *query, const void *key_cache, const void *value_cache,
               const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
@@ -246,6 +261,15 @@ int pa_reshape_and_cache_fp8(const void *key, const void *value, void *key_cache
                              void *value_cache, const int64_t *slot_mapping, int num_tokens,
                              int num_kv_heads, int head_dim, int block_size, int num_blocks,
                              float k_scale, float v_scale, void *stream);
+
+/* pa_append_decode_kv into FP8 caches: the slot rules of pa_append_decode_kv,
+ * the quantisation of pa_reshape_and_cache_fp8 (num_kv_heads * head_dim a
+ * multiple of 16). */
+int pa_append_decode_kv_fp8(const void *key, const void *value, void *key_cache, void *value_cache,
+                            const int32_t *block_tables, const int32_t *seq_lens,
+                            int64_t *slot_mapping, int num_seqs, int max_blocks_per_seq,
+                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                            float k_scale, float v_scale, void *stream);
 
 /* pa_decode over an FP8 cache: the same result with K = e4m3(code) * k_scale
  * and V = e4m3(code) * v_scale.  query and out stay bf16.  Supported: head_dim

@@ -104,6 +104,45 @@ __global__ void reshape_and_cache_fp8_kernel(const uint4 *__restrict__ key, cons
     value_cache[dst] = quantise16(v0, v1, v_inv_scale);
 }
 
+// The decode step's cache write with its own address translation, in one
+// launch: token s is sequence s's newest position seq_lens[s] - 1; its slot is
+// computed as slot_mapping_kernel does (optionally written to slots_out) and
+// its K/V row stored there -- copied (bf16) or quantised (FP8: one thread per 16
+// codes).  chunks_per_token counts 16-byte chunks of the destination row.
+template <bool FP8>
+__global__ void append_kv_kernel(const uint4 *__restrict__ key, const uint4 *__restrict__ value,
+                                 uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache,
+                                 const int32_t *__restrict__ block_tables, const int32_t *__restrict__ seq_lens,
+                                 int64_t *__restrict__ slots_out, int num_seqs, int max_blocks,
+                                 int chunks_per_token, int block_size, int64_t num_slots, float k_inv, float v_inv)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)num_seqs * chunks_per_token) return;
+    const int s = (int)(i / chunks_per_token);
+    const int c = (int)(i - (int64_t)s * chunks_per_token);
+    const int64_t pos = (int64_t)seq_lens[s] - 1;
+    int64_t slot = -1;
+    if (pos >= 0) {
+        const int64_t block_number = pos / block_size;
+        if (block_number < max_blocks) {
+            const int32_t physical = block_tables[(int64_t)s * max_blocks + block_number];
+            if (physical >= 0) slot = (int64_t)physical * block_size + (pos - block_number * block_size);
+        }
+    }
+    if (c == 0 && slots_out) slots_out[s] = slot;
+    if (slot < 0 || slot >= num_slots) return;
+    const int64_t dst = slot * chunks_per_token + c;
+    if constexpr (FP8) {
+        key_cache[dst] = quantise16(key[2 * i], key[2 * i + 1], k_inv);
+        value_cache[dst] = quantise16(value[2 * i], value[2 * i + 1], v_inv);
+    } else {
+        key_cache[dst] = key[i];
+        value_cache[dst] = value[i];
+    }
+}
+
 // One CTA per (pair, slice): copies `per_cta` 16-byte chunks of the source block
 // into the destination block, in both caches, with 4 loads in flight per thread.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ key_cache,

@@ -238,8 +238,11 @@ struct DecodeSmem {
     static constexpr int kFlagOff = kBarOff + kNumBars * 8;
     static constexpr int kPrefixOff = kFlagOff + 16;
     // bytes of dynamic shared memory for a launch over num_seqs sequences
-    // (enumeration tables: pf[B + 1], rest_order[B], sort keys)
-    static constexpr int bytes(int num_seqs) { return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys); }
+    // (enumeration tables: pf[B + 1], rest_order[B], sort bases, int16 keys[B])
+    static constexpr int bytes(int num_seqs)
+    {
+        return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys) + ((2 * num_seqs + 3) & ~3);
+    }
 };
 
 template <int D, int BS, int MODE, int GC, bool FP8>
@@ -313,6 +316,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     int *const pf = prefix;                    // [B + 1]
     int *const rest_order = prefix + B + 1;    // [B]
     int *const sort_base = rest_order + B;     // [kSortKeys]
+    int16_t *const keys = reinterpret_cast<int16_t *>(sort_base + kSortKeys);  // [B] rest keys
     const int Lcap = p.max_blocks * BS;
     auto full_of = [&](int L) {
         return (split && L > 0) ? min(L / p.part_tokens, p.max_parts) : 0;
@@ -324,13 +328,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         return min((r + kTileTokens - 1) / kTileTokens, kSortKeys - 1);
     };
     __shared__ int warp_tot[kDecodeThreads / 32];
+    __shared__ int rest_count;
+    // one coalesced pass over the lengths: each sequence's rest key, and its
+    // full-partition count parked in pf[s] for the scan below
+    if (threadIdx.x == 0) rest_count = 0;
+    __syncthreads();
+    {
+        int nrest = 0;
+        for (int s = threadIdx.x; s < B; s += kDecodeThreads) {
+            const int L = min(p.seq_lens[s], Lcap);
+            const int key = rest_key(L);
+            keys[s] = (int16_t)key;
+            nrest += key >= 0;
+            pf[s] = full_of(L);
+        }
+        if (nrest) atomicAdd(&rest_count, nrest);
+    }
+    __syncthreads();
     if (split) {
+        // block-wide exclusive scan of the full-partition counts
         const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
         const int s0 = min(B, (int)threadIdx.x * per);
         const int s1 = min(B, s0 + per);
         int local = 0;
-        for (int s = s0; s < s1; ++s) local += full_of(min(p.seq_lens[s], Lcap));
-        // block-wide exclusive scan of `local`
+        for (int s = s0; s < s1; ++s) local += pf[s];
         int incl = local;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -342,61 +363,71 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         int run = incl - local;
         for (int w = 0; w < warp; ++w) run += warp_tot[w];
         for (int s = s0; s < s1; ++s) {
+            const int f = pf[s];
             pf[s] = run;
-            run += full_of(min(p.seq_lens[s], Lcap));
+            run += f;
         }
         if (threadIdx.x == kDecodeThreads - 1) pf[B] = run;
     }
     __syncthreads();
     const int total_full = split ? pf[B] : 0;
+    const int total_rest = rest_count;
 
     if (warp == kSchedulerWarp) {
         // ------------------------------------------------------------ scheduler
         // rest pairs sorted by size, largest first: counting sort over kSortKeys
-        // tile-count keys, stable in sequence order (match_any ranks lanes)
-        for (int k = lane; k < kSortKeys; k += 32) sort_base[k] = 0;
-        __syncwarp();
-        for (int c = 0; c < B; c += 32) {
-            const int key = c + lane < B ? rest_key(min(p.seq_lens[c + lane], Lcap)) : -1;
-            if (key >= 0) atomicAdd(&sort_base[key], 1);
-        }
-        __syncwarp();
-        int total_rest;
-        {
-            // exclusive scan in descending key order; lane owns kSortKeys/32 keys
-            constexpr int KPL = kSortKeys / 32;
-            int cnt[KPL], sum = 0;
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                cnt[i] = sort_base[kSortKeys - 1 - (lane * KPL + i)];
-                sum += cnt[i];
-            }
-            int incl = sum;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
-            }
-            total_rest = __shfl_sync(0xffffffffu, incl, 31);
-            int run = incl - sum;
+        // tile-count keys, stable in sequence order (match_any ranks lanes).  When
+        // this CTA's first item is a full partition the sort runs after that item
+        // has been handed to the producer, so the first loads start sooner.
+        auto sort_rest = [&]() {
+            for (int k = lane; k < kSortKeys; k += 32) sort_base[k] = 0;
             __syncwarp();
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                sort_base[kSortKeys - 1 - (lane * KPL + i)] = run;
-                run += cnt[i];
+            for (int c = 0; c < B; c += 32) {
+                const int key = c + lane < B ? keys[c + lane] : -1;
+                if (key >= 0) atomicAdd(&sort_base[key], 1);
             }
-        }
-        __syncwarp();
-        for (int c = 0; c < B; c += 32) {
-            const int key = c + lane < B ? rest_key(min(p.seq_lens[c + lane], Lcap)) : -1;
-            const unsigned peers = __match_any_sync(0xffffffffu, key);
-            const int rank = __popc(peers & ((1u << lane) - 1u));
-            if (key >= 0) rest_order[sort_base[key] + rank] = c + lane;
             __syncwarp();
-            if (key >= 0 && rank == 0) sort_base[key] += __popc(peers);
+            {
+                // exclusive scan in descending key order; lane owns kSortKeys/32 keys
+                constexpr int KPL = kSortKeys / 32;
+                int cnt[KPL], sum = 0;
+#pragma unroll
+                for (int i = 0; i < KPL; ++i) {
+                    cnt[i] = sort_base[kSortKeys - 1 - (lane * KPL + i)];
+                    sum += cnt[i];
+                }
+                int incl = sum;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                int run = incl - sum;
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < KPL; ++i) {
+                    sort_base[kSortKeys - 1 - (lane * KPL + i)] = run;
+                    run += cnt[i];
+                }
+            }
             __syncwarp();
-        }
+            for (int c = 0; c < B; c += 32) {
+                const int key = c + lane < B ? keys[c + lane] : -1;
+                const unsigned peers = __match_any_sync(0xffffffffu, key);
+                const int rank = __popc(peers & ((1u << lane) - 1u));
+                if (key >= 0) rest_order[sort_base[key] + rank] = c + lane;
+                __syncwarp();
+                if (key >= 0 && rank == 0) sort_base[key] += __popc(peers);
+                __syncwarp();
+            }
+            __syncwarp();
+        };
         const int total_items = (total_full + total_rest) * Hkv;
+        bool sorted = false;
+        if ((int)blockIdx.x >= total_full * Hkv) {
+            sort_rest();
+            sorted = true;
+        }
 
         // Each CTA starts on item blockIdx.x; later items come from the atomic
         // counter (offset by the grid size) or round-robin without a workspace.
@@ -415,11 +446,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             first_grab = false;
             return __shfl_sync(0xffffffffu, v, 0);
         };
-        int idx = grab();
+        // An item is taken only once its slot is free, i.e. when the item two
+        // before it has been consumed: one item ahead of the consumers (so the
+        // producer runs on across items) and no earlier, so the largest-first
+        // order still decides what runs at the tail of the launch.
+        int idx = 0;
         int item_seq = 0, chunk_seq = 0, ring_base = 0;
         while (true) {
-            const bool have = idx < total_items;
-            const int next_idx = have ? grab() : idx;  // one item ahead
             // item slot
             const int islot = item_seq % kItemSlots;
             bool ok = true;
@@ -432,6 +465,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
+            idx = grab();
+            const bool have = idx < total_items;
             ItemInfo it = {};
             int first_blk = 0, end_blk = 0;
             if (have) {
@@ -510,9 +545,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 if (it.stop) break;
             }
             if (!ok || it.stop) break;
+            if (!sorted) {  // before the next item can be a rest pair
+                sort_rest();
+                sorted = true;
+            }
             ring_base += it.n_tiles;
             ++item_seq;
-            idx = next_idx;
         }
     } else if (warp == kProducerWarp) {
         // ------------------------------------------------------------- producer

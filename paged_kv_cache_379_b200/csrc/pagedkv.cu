@@ -447,6 +447,58 @@ int pa_reshape_and_cache_fp8(const void *key, const void *value, void *key_cache
                       (int64_t)num_blocks * block_size, k_inv, v_inv);
 }
 
+static int append_kv(bool fp8, const void *key, const void *value, void *key_cache, void *value_cache,
+                     const int32_t *block_tables, const int32_t *seq_lens, int64_t *slot_mapping, int num_seqs,
+                     int max_blocks_per_seq, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                     float k_scale, float v_scale, void *stream)
+{
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0)
+        return PA_ERR_BAD_SHAPE;
+    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && k_scale < INFINITY && v_scale < INFINITY))
+        return PA_ERR_BAD_SHAPE;
+    if (num_seqs == 0) return PA_OK;
+    if (!key || !value || !key_cache || !value_cache || !block_tables || !seq_lens) return PA_ERR_NULL_POINTER;
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    if (row % (fp8 ? 16 : 8) != 0) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return PA_ERR_ALIGNMENT;
+    const int chunks = (int)(row / (fp8 ? 16 : 8));
+    const int64_t total = (int64_t)num_seqs * chunks;
+    const int threads = 256;
+    if (cdiv64(total, threads) > INT_MAX) return PA_ERR_BAD_SHAPE;
+    const dim3 grid((unsigned)cdiv64(total, threads));
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t slots = (int64_t)num_blocks * block_size;
+    if (fp8)
+        return launch_pdl(append_kv_kernel<true>, grid, dim3(threads), 0, st, static_cast<const uint4 *>(key),
+                          static_cast<const uint4 *>(value), static_cast<uint4 *>(key_cache),
+                          static_cast<uint4 *>(value_cache), block_tables, seq_lens, slot_mapping, num_seqs,
+                          max_blocks_per_seq, chunks, block_size, slots, 1.0f / k_scale, 1.0f / v_scale);
+    return launch_pdl(append_kv_kernel<false>, grid, dim3(threads), 0, st, static_cast<const uint4 *>(key),
+                      static_cast<const uint4 *>(value), static_cast<uint4 *>(key_cache),
+                      static_cast<uint4 *>(value_cache), block_tables, seq_lens, slot_mapping, num_seqs,
+                      max_blocks_per_seq, chunks, block_size, slots, 1.f, 1.f);
+}
+
+int pa_append_decode_kv(const void *key, const void *value, void *key_cache, void *value_cache,
+                        const int32_t *block_tables, const int32_t *seq_lens, int64_t *slot_mapping, int num_seqs,
+                        int max_blocks_per_seq, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        void *stream)
+{
+    return append_kv(false, key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping, num_seqs,
+                     max_blocks_per_seq, num_kv_heads, head_dim, block_size, num_blocks, 1.f, 1.f, stream);
+}
+
+int pa_append_decode_kv_fp8(const void *key, const void *value, void *key_cache, void *value_cache,
+                            const int32_t *block_tables, const int32_t *seq_lens, int64_t *slot_mapping,
+                            int num_seqs, int max_blocks_per_seq, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, float k_scale, float v_scale, void *stream)
+{
+    return append_kv(true, key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping, num_seqs,
+                     max_blocks_per_seq, num_kv_heads, head_dim, block_size, num_blocks, k_scale, v_scale, stream);
+}
+
 int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, void *stream)
 {

@@ -30,7 +30,7 @@ __all__ = [
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
     "decode_split_noalloc", "swap_blocks", "reshape_and_cache_fp8", "decode_fp8", "decode_fp8_split",
-    "prefill",
+    "prefill", "append_decode_kv", "append_decode_kv_fp8",
 ]
 
 
@@ -112,6 +112,36 @@ def reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_sc
     check("pa_reshape_and_cache_fp8", lib.pa_reshape_and_cache_fp8(
         k, v, key_cache.data_ptr(), value_cache.data_ptr(), sm, key.shape[0], hkv, d, bs, nb, float(k_scale),
         float(v_scale), _stream(stream)))
+
+
+def _append_args(key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping, cache_dtype):
+    nb, bs, hkv, d = _cache_dims(key_cache, value_cache, cache_dtype)
+    k = _dev(key, torch.bfloat16, "key", 3)
+    v = _dev(value, torch.bfloat16, "value", 3)
+    B = seq_lens.shape[0]
+    if tuple(key.shape) != (B, hkv, d) or key.shape != value.shape:
+        raise ValueError("key/value must be [num_seqs, num_kv_heads, head_dim] matching the cache")
+    bt = _dev(block_tables, torch.int32, "block_tables", 2)
+    if block_tables.shape[0] != B:
+        raise ValueError("block_tables rows != num_seqs")
+    sm = _dev(slot_mapping, torch.int64, "slot_mapping", 1)
+    return (k, v, key_cache.data_ptr(), value_cache.data_ptr(), bt, _dev(seq_lens, torch.int32, "seq_lens", 1), sm,
+            B, block_tables.shape[1], hkv, d, bs, nb)
+
+
+def append_decode_kv(key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping=None,
+                     stream=None) -> None:
+    """pa_append_decode_kv: slot of each sequence's newest position + cache write, one launch."""
+    a = _append_args(key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping, torch.bfloat16)
+    check("pa_append_decode_kv", load().pa_append_decode_kv(*a, _stream(stream)))
+
+
+def append_decode_kv_fp8(key, value, key_cache, value_cache, block_tables, seq_lens, k_scale: float,
+                         v_scale: float, slot_mapping=None, stream=None) -> None:
+    """pa_append_decode_kv_fp8: as append_decode_kv into E4M3 code caches."""
+    a = _append_args(key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping, torch.uint8)
+    check("pa_append_decode_kv_fp8", load().pa_append_decode_kv_fp8(*a, float(k_scale), float(v_scale),
+                                                                    _stream(stream)))
 
 
 def copy_blocks(key_cache, value_cache, src_dst_pairs, stream=None) -> None:

@@ -81,12 +81,13 @@ class DecodeBatch:
                                                device=self.device)
 
     def run_step(self, stream=None, decode_fn=None):
+        """Copy-on-write copies (if any), then the newest token's slot and cache
+        write in one launch, then the decode."""
         wl = self.wl
-        ops.slot_mapping(self.block_tables, wl.block_size, seq_lens=self.seq_lens, out=self.slots, stream=stream)
         if self.pairs is not None:
             ops.copy_blocks(self.key_cache, self.value_cache, self.pairs, stream=stream)
-        ops.reshape_and_cache(self.new_key, self.new_value, self.key_cache, self.value_cache, self.slots,
-                              stream=stream)
+        ops.append_decode_kv(self.new_key, self.new_value, self.key_cache, self.value_cache, self.block_tables,
+                             self.seq_lens, slot_mapping=self.slots, stream=stream)
         if decode_fn is None:
             ops.decode(self.query, self.key_cache, self.value_cache, self.block_tables, self.seq_lens,
                        wl.scale, self.max_seq_len, out=self.out, workspace=self.workspace, stream=stream)

@@ -106,3 +106,62 @@ def test_copy_blocks_small_block_shapes():
         oracle.copy_blocks(kc0, vc0, pairs)
         assert np.array_equal(bf16_to_host_bits(kc), kc0)
         assert np.array_equal(bf16_to_host_bits(vc), vc0)
+
+
+# ---- slot mapping + cache write fused (decode form) ---------------------------------
+
+S_EMPTY, S_NEG = 1, 2
+
+
+def _append_case(name):
+    """Sequence S_EMPTY has length 0 and sequence S_NEG a negative table entry
+    at its newest position: both get slot -1 (the documented rule of the slot
+    mapping) and write nothing.  Returns the workload, lengths, table and the
+    expected slots."""
+    w = wl.make(name)
+    sl = w.seq_lens.copy()
+    sl[S_EMPTY] = 0
+    pos = sl.astype(np.int64) - 1
+    ref = oracle.slot_mapping(w.block_tables, np.arange(w.num_seqs, dtype=np.int32), pos, w.block_size)
+    tb = w.block_tables.copy()
+    tb[S_NEG, (int(sl[S_NEG]) - 1) // w.block_size] = -1
+    ref[S_NEG] = -1
+    return w, sl, tb, ref
+
+
+@pytest.mark.parametrize("name", ["tiny", "gqa"])
+def test_append_decode_kv_equals_slot_mapping_then_cache_write(name):
+    w, sl, tb, slots_ref = _append_case(name)
+    ref_k, ref_v = w.key_cache.copy(), w.value_cache.copy()
+    oracle.reshape_and_cache(w.new_key, w.new_value, ref_k, ref_v, slots_ref, w.block_size)
+    kc, vc = bf16_to_device(w.key_cache, DEV), bf16_to_device(w.value_cache, DEV)
+    slots = torch.full((w.num_seqs,), 12345, dtype=torch.int64, device=DEV)
+    ops.append_decode_kv(bf16_to_device(w.new_key, DEV), bf16_to_device(w.new_value, DEV), kc, vc, _i32(tb),
+                         _i32(sl), slot_mapping=slots)
+    torch.cuda.synchronize()
+    assert np.array_equal(slots.cpu().numpy(), slots_ref)
+    assert slots_ref[S_EMPTY] == -1 and slots_ref[S_NEG] == -1
+    assert np.array_equal(bf16_to_host_bits(kc), ref_k)
+    assert np.array_equal(bf16_to_host_bits(vc), ref_v)
+    # without the slot output
+    kc2, vc2 = bf16_to_device(w.key_cache, DEV), bf16_to_device(w.value_cache, DEV)
+    ops.append_decode_kv(bf16_to_device(w.new_key, DEV), bf16_to_device(w.new_value, DEV), kc2, vc2, _i32(tb),
+                         _i32(sl))
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_to_host_bits(kc2), ref_k)
+
+
+def test_append_decode_kv_fp8_equals_oracle():
+    w, sl, tb, slots_ref = _append_case("gqa")
+    rng = np.random.default_rng(3)
+    kc8 = wl.fp8_codes(rng, w.key_cache.shape)
+    vc8 = wl.fp8_codes(rng, w.value_cache.shape)
+    ref_k, ref_v = kc8.copy(), vc8.copy()
+    oracle.reshape_and_cache_fp8(w.new_key, w.new_value, ref_k, ref_v, slots_ref, w.block_size, 0.05, 0.3)
+    dk = torch.from_numpy(kc8).to(DEV)
+    dv = torch.from_numpy(vc8).to(DEV)
+    ops.append_decode_kv_fp8(bf16_to_device(w.new_key, DEV), bf16_to_device(w.new_value, DEV), dk, dv, _i32(tb),
+                             _i32(sl), 0.05, 0.3)
+    torch.cuda.synchronize()
+    assert np.array_equal(dk.cpu().numpy(), ref_k)
+    assert np.array_equal(dv.cpu().numpy(), ref_v)
