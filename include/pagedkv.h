@@ -274,11 +274,13 @@ int pa_append_decode_kv_fp8(const void *key, const void *value, void *key_cache,
 /* pa_decode over an FP8 cache: the same result with K = e4m3(code) * k_scale
  * and V = e4m3(code) * v_scale.  query and out stay bf16.  Supported: head_dim
  * 128, block_size 8 or 16, G = num_heads / num_kv_heads in 1..16
- * (PA_ERR_UNSUPPORTED otherwise).  The logits are formed in fp32 from the
- * query rounded to fp16 (exact for |q| in [2^-17, 65504] -- bf16 has 8
- * significant bits) and the codes (every E4M3 value is an fp16 value); the
- * softmax weights enter the value product as fp16.  Same plan, workspace
- * contract and workspace size as pa_decode. */
+ * (PA_ERR_UNSUPPORTED otherwise).  The logits are E4M3 x E4M3 tensor-core
+ * products accumulated in fp32: each query head is scaled by a power of two
+ * (its largest |q| into [128, 256)) and split into two E4M3 terms whose sum is
+ * the bf16 query exactly for every element within 2^9 of the head's largest
+ * (smaller elements are off by less than 2^-17 of the largest).  The value
+ * product widens the codes to fp16 (exact) and takes the softmax weights as
+ * fp16.  Same plan, workspace contract and workspace size as pa_decode. */
 int pa_decode_fp8(void *out, const void *query, const void *key_cache, const void *value_cache,
                   const int32_t *block_tables, const int32_t *seq_lens, float scale, float k_scale,
                   float v_scale, int block_size, int num_kv_heads, int num_seqs, int num_heads,

@@ -169,6 +169,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes)
     return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
+// D = A(16x32, row) * B(32x8, col) + D, E4M3 inputs (four codes per register,
+// the lowest k in the low byte), fp32 accumulate.
+__device__ __forceinline__ void mma_e4m3_16832(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // 16-byte shared-memory load (shared-window address)
 __device__ __forceinline__ uint4 lds128(uint32_t addr)
 {
@@ -189,6 +201,15 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
+}
+
+// Two packed fp16 values (low half first) -> two floats.
+__device__ __forceinline__ float2 f16x2_to_float2(uint32_t v)
+{
+    __half2_raw r;
+    r.x = (unsigned short)(v & 0xFFFFu);
+    r.y = (unsigned short)(v >> 16);
+    return __half22float2(__half2(r));
 }
 
 // Two floats -> two E4M3 codes (round to nearest even, finite overflow saturates

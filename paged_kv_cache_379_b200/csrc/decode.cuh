@@ -781,27 +781,88 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 const int gq = lane >> 2;                // MMA groupID
                 const int tq = lane & 3;                 // MMA thread-in-group
                 // B operand of S^T = K Q^T: b0 = Q[head][d 16kk+2tq..+1], b1 = Q[head][d 16kk+8+2tq..+1].
-                // FP8 cache: the contraction order is permuted so that a lane's four
-                // k-slots {2tq, 2tq+1, 2tq+8, 2tq+9} of k-step kk = 4S + i are the four
-                // consecutive codes d = 16(4S + tq) + 4i + {0..3} of a key row; Q
-                // follows the same order and is multiplied in fp16.
-                uint32_t qb[NH][KSTEPS][2];
+                uint32_t qb[NH][FP8 ? 1 : KSTEPS][2];
+                // FP8 cache: S^T = K Q^T runs on E4M3 MMAs (m16n8k32) straight from the
+                // codes.  Q is scaled by a power of two per head (max |q| into
+                // [128, 256)) and split into two E4M3 terms, q1 = e4m3(q) and
+                // q2 = e4m3(q - q1), whose sum is the bf16 value exactly for every
+                // element within 2^9 of the head's largest (smaller ones are off by
+                // less than 2^-17 of the largest); the logit scale divides the power
+                // of two out again.  The contraction order over head_dim is
+                // permuted so that a lane's k-slots 4tq..4tq+3 and 16+4tq..16+4tq+3
+                // of k-step kk are words 2(kk&1) and 2(kk&1)+1 of code chunk
+                // tq + 4(kk>>1) of its key row.
+                uint32_t q8[NH][FP8 ? 4 : 1][2][2];  // [head tile][k-step][term][b0/b1]
+                float qscale[NH][2];       // logit scale of accumulator columns 2tq, 2tq+1
+                if constexpr (FP8) {
 #pragma unroll
-                for (int nh = 0; nh < NH; ++nh) {
-                    const int head = nh * 8 + gq;
+                    for (int nh = 0; nh < NH; ++nh) {
+                        const int head = nh * 8 + gq;
+                        float v[4][2][4];
+                        float amax = 0.f;
 #pragma unroll
-                    for (int kk = 0; kk < KSTEPS; ++kk) {
+                        for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int col = FP8 ? 16 * (4 * (kk >> 2) + tq) + 4 * (kk & 3) + 2 * hh
-                                                : kk * 16 + hh * 8 + tq * 2;
-                            uint32_t v = head < G ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
-                            if constexpr (FP8) {
-                                const float2 f = unpack_bf16x2(v);
-                                v = pack_f16x2(f.x, f.y);
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const int col = 16 * (tq + 4 * (kk >> 1)) + 8 * (kk & 1) + 4 * hh;
+                                uint2 w = make_uint2(0u, 0u);
+                                if (head < G) w = *reinterpret_cast<const uint2 *>(qsm + (head * D + col) * 2);
+                                const float2 f0 = unpack_bf16x2(w.x), f1 = unpack_bf16x2(w.y);
+                                v[kk][hh][0] = f0.x;
+                                v[kk][hh][1] = f0.y;
+                                v[kk][hh][2] = f1.x;
+                                v[kk][hh][3] = f1.y;
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[kk][hh][e]));
                             }
-                            qb[nh][kk][hh] = v;
+                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                        // sigma = 2^(8 - e) for amax = m 2^e, m in [0.5, 1): sigma amax in [128, 256)
+                        int e2 = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 126;
+                        int se = 8 - e2;
+                        se = amax > 0.f ? min(max(se, -126), 127) : 0;
+                        const float sigma = __uint_as_float((uint32_t)(se + 127) << 23);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                float a[4], r[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) a[e] = v[kk][hh][e] * sigma;
+                                const uint16_t c01 = f32x2_to_e4m3x2(a[0], a[1]);
+                                const uint16_t c23 = f32x2_to_e4m3x2(a[2], a[3]);
+                                const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2(c01));
+                                const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2(c23));
+                                r[0] = a[0] - d01.x;
+                                r[1] = a[1] - d01.y;
+                                r[2] = a[2] - d23.x;
+                                r[3] = a[3] - d23.y;
+                                q8[nh][kk][0][hh] = (uint32_t)c01 | ((uint32_t)c23 << 16);
+                                q8[nh][kk][1][hh] = (uint32_t)f32x2_to_e4m3x2(r[0], r[1]) |
+                                                    ((uint32_t)f32x2_to_e4m3x2(r[2], r[3]) << 16);
+                            }
+                        // accumulator column 2tq + jj of this head tile is head nh*8 + 2tq + jj,
+                        // whose sigma the lanes of group 2tq + jj computed
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const float sg = __shfl_sync(0xffffffffu, sigma, (2 * tq + jj) * 4);
+                            qscale[nh][jj] = p.scale_log2 / sg;
                         }
+                    }
+                } else {
+#pragma unroll
+                    for (int nh = 0; nh < NH; ++nh) {
+                        const int head = nh * 8 + gq;
+#pragma unroll
+                        for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const int col = kk * 16 + hh * 8 + tq * 2;
+                                qb[nh][kk][hh] =
+                                    head < G ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
+                            }
+                        }
+                        qscale[nh][0] = qscale[nh][1] = p.scale_log2;
                     }
                 }
                 float o[MT][NH][4];
@@ -853,16 +914,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             kr[r][1] = odd ? x : y;
                         }
 #pragma unroll
-                        for (int kk = 0; kk < KSTEPS; ++kk) {
-                            const uint32_t w0 = u4_word(kr[0][kk >> 2], kk & 3);
-                            const uint32_t w1 = u4_word(kr[1][kk >> 2], kk & 3);
-                            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(w0 & 0xFFFFu));
-                            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(w0 >> 16));
-                            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(w1 & 0xFFFFu));
-                            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(w1 >> 16));
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t a0 = u4_word(kr[0][kk >> 1], 2 * (kk & 1));
+                            const uint32_t a2 = u4_word(kr[0][kk >> 1], 2 * (kk & 1) + 1);
+                            const uint32_t a1 = u4_word(kr[1][kk >> 1], 2 * (kk & 1));
+                            const uint32_t a3 = u4_word(kr[1][kk >> 1], 2 * (kk & 1) + 1);
 #pragma unroll
-                            for (int nh = 0; nh < NH; ++nh)
-                                mma_f16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                            for (int nh = 0; nh < NH; ++nh) {
+                                mma_e4m3_16832(sc[nh], a0, a1, a2, a3, q8[nh][kk][0][0], q8[nh][kk][0][1]);
+                                mma_e4m3_16832(sd[nh], a0, a1, a2, a3, q8[nh][kk][1][0], q8[nh][kk][1][1]);
+                            }
                         }
                     } else {
 #pragma unroll
@@ -893,8 +954,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         bool bump = false;
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
-                            x[jj][0] = in0 ? sc[nh][jj] * p.scale_log2 : -INFINITY;
-                            x[jj][1] = in1 ? sc[nh][2 + jj] * p.scale_log2 : -INFINITY;
+                            x[jj][0] = in0 ? sc[nh][jj] * qscale[nh][jj] : -INFINITY;
+                            x[jj][1] = in1 ? sc[nh][2 + jj] * qscale[nh][jj] : -INFINITY;
                             float v = fmaxf(x[jj][0], x[jj][1]);
                             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
                             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
