@@ -222,6 +222,11 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  : "memory");
 }
 
+// Whether the decode loads a block with one TMA box covering its 64-wide
+// d-planes (planes as the box's outer dimension) instead of one box per plane:
+// only where a tile is one block, so the box lands plane-major.
+__host__ __device__ constexpr bool decode_block_box(int D, int BS, bool FP8) { return !FP8 && D == 128 && BS == 16; }
+
 template <int D, int BS, int MODE, int GC, bool FP8>
 struct DecodeSmem {
     static constexpr int ROWS = MODE == 0 ? GC : (MODE == 1 ? 8 : 16);
@@ -258,6 +263,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     using Geo = typename Lay::Ring;                                         // ring tiles
     using Merge = typename Lay::Merge;
     constexpr int kStages = Geo::kStages;
+    // bf16, head_dim 128, bs 16: a block's two planes are one tile's two planes,
+    // so one TMA box (planes as its outer dimension) loads the whole block
+    constexpr bool kBlockBox = decode_block_box(D, BS, FP8);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -587,10 +595,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     for (int k = 0; k < Geo::kBlocksPerTile; ++k) {
                         if (k < valid) {
                             const int row = c->phys[j + k] * BS;
+                            if constexpr (kBlockBox) {
+                                // one box per block: both 64-wide planes, plane-major
+                                tma_load_4d(kdst + Geo::box_offset(k, 0), &tmap_k, bar, 0, row, 0, g);
+                                tma_load_4d(vdst + Geo::box_offset(k, 0), &tmap_v, bar, 0, row, 0, g);
+                            } else {
 #pragma unroll
-                            for (int h = 0; h < Geo::kHalves; ++h) {
-                                tma_load_4d(kdst + Geo::box_offset(k, h), &tmap_k, bar, 0, h, g, row);
-                                tma_load_4d(vdst + Geo::box_offset(k, h), &tmap_v, bar, 0, h, g, row);
+                                for (int h = 0; h < Geo::kHalves; ++h) {
+                                    tma_load_4d(kdst + Geo::box_offset(k, h), &tmap_k, bar, 0, h, g, row);
+                                    tma_load_4d(vdst + Geo::box_offset(k, h), &tmap_v, bar, 0, h, g, row);
+                                }
                             }
                         }
                     }

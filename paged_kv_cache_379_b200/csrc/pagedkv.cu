@@ -45,17 +45,31 @@ static EncodeTiledFn encode_fn()
 // 128-byte swizzle.
 // An FP8 cache (1-byte codes, head_dim 128) is {128 codes = 128 B, 1, Hkv, slots}
 // with a box {128, 1, 1, bs}: one 128-byte row per token.
+// With block_box the dimensions are ordered {64 elements, slots, D/64 planes,
+// Hkv} (strides Hkv*D*2, 128, D*2 bytes) and the box is {64, bs, D/64, 1}: one
+// block of one head, both planes, landing plane-major.
 static int make_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int bs, int hkv, int d,
-                          bool fp8 = false)
+                          bool fp8 = false, bool block_box = false)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return check_cuda(cudaErrorNotSupported);
     const int esize = fp8 ? 1 : 2;
     const int inner = 128 / esize;  // elements per 128-byte row
-    const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)(d / inner), (cuuint64_t)hkv,
-                                (cuuint64_t)(num_blocks * bs)};
-    const cuuint64_t strides[3] = {128, (cuuint64_t)d * esize, (cuuint64_t)hkv * d * esize};
-    const cuuint32_t box[4] = {(cuuint32_t)inner, 1, 1, (cuuint32_t)bs};
+    cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)(d / inner), (cuuint64_t)hkv,
+                          (cuuint64_t)(num_blocks * bs)};
+    cuuint64_t strides[3] = {128, (cuuint64_t)d * esize, (cuuint64_t)hkv * d * esize};
+    cuuint32_t box[4] = {(cuuint32_t)inner, 1, 1, (cuuint32_t)bs};
+    if (block_box) {
+        dims[1] = (cuuint64_t)(num_blocks * bs);
+        dims[2] = (cuuint64_t)(d / inner);
+        dims[3] = (cuuint64_t)hkv;
+        strides[0] = (cuuint64_t)hkv * d * esize;
+        strides[1] = 128;
+        strides[2] = (cuuint64_t)d * esize;
+        box[1] = (cuuint32_t)bs;
+        box[2] = (cuuint32_t)(d / inner);
+        box[3] = 1;
+    }
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                           const_cast<void *>(cache), dims, strides, box,
@@ -284,9 +298,10 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
     const int64_t max_items = (int64_t)p.max_parts * a.num_seqs * a.num_kv_heads;
     if (max_items > INT_MAX) return PA_ERR_BAD_SHAPE;
     CUtensorMap tk, tv;
-    rc = make_cache_map(&tk, a.key_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim, a.fp8);
+    const bool bb = decode_block_box(a.head_dim, a.block_size, a.fp8);
+    rc = make_cache_map(&tk, a.key_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim, a.fp8, bb);
     if (rc != PA_OK) return rc;
-    rc = make_cache_map(&tv, a.value_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim, a.fp8);
+    rc = make_cache_map(&tv, a.value_cache, a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim, a.fp8, bb);
     if (rc != PA_OK) return rc;
     if (a.fp8)
         rc = a.block_size == 8 ? launch_decode_fp8_bs<8>(p, tk, tv, max_items, st)
