@@ -31,6 +31,12 @@
  *   launched.  A launch failure returns PA_ERR_CUDA (pa_last_cuda_error() gives
  *   the cudaError_t).  The library never aborts the process and never traps on
  *   the device.
+ * - Every kernel is launched with programmatic dependent launch and lets the
+ *   next kernel of the stream start early.  The decode kernels read seq_lens,
+ *   block_tables and query before waiting for the previous kernel of the
+ *   stream to finish (everything else after it); no kernel of this library
+ *   writes those, and a kernel launched without that attribute (or one that
+ *   never triggers its dependents early) is waited for as usual.
  * - Preconditions NOT checked in the launch path (pa_validate_tables checks
  *   them on the device): table entries below num_blocks for the blocks a
  *   sequence uses; ceil(seq_len/block_size) <= max_blocks_per_seq;
@@ -184,7 +190,7 @@ int pa_decode(void *out, const void *query, const void *key_cache, const void *v
 
 /* The plan pa_decode follows for these sizes: 0 = one pass (one launch),
  * otherwise the partition size of the split form (partition kernel + reduce
- * kernel, two launches).  One pass when max_seq_len <= 2048 and the
+ * kernel, two launches).  One pass when max_seq_len <= 4096 and the
  * (sequence, KV head) units give every SM several items; else partitions of
  * 1024 positions (2048 beyond 16384), halved while the batch is too small to
  * give every SM several items.  A workspace smaller than the split form needs

@@ -309,7 +309,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         prefetch_tensormap(&tmap_k);
         prefetch_tensormap(&tmap_v);
     }
-    pdl_wait();
+    // Programmatic dependent launch: this grid may start while the previous
+    // kernel of the stream still runs.  The enumeration below reads only the
+    // lengths (and the scheduler the tables and queries), which no kernel of
+    // this library writes, so it runs before griddepcontrol.wait; every
+    // access to the caches, the outputs, the workspace and its counters comes
+    // after it (producer before its first load, scheduler before its first
+    // counter access, all threads before the partitions-only fill and the
+    // counter reset).
     pdl_launch_dependents();
 
     // ---- enumeration of the work items, largest first.  Per sequence (length L
@@ -473,6 +480,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
+            if (item_seq == 1) pdl_wait();  // the counters belong to the previous grid until here
             idx = grab();
             const bool have = idx < total_items;
             ItemInfo it = {};
@@ -562,6 +570,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         }
     } else if (warp == kProducerWarp) {
         // ------------------------------------------------------------- producer
+        pdl_wait();  // the caches may still be written by the previous grid until here
         int chunk_seq = 0, ring = 0;
         while (true) {
             const int cslot = chunk_seq % kChunkSlots;
@@ -626,6 +635,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         }
     } else {
         // ------------------------------------------------------------ consumers
+        pdl_wait();  // outputs and partials may still be touched by the previous grid until here
         // Zero the V rows of tokens [valid, 16) so masked positions contribute
         // exactly 0 (stale or NaN data is never multiplied).
         auto zero_tail = [&](uint32_t vt, int valid) {
@@ -1153,6 +1163,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     // Partitions-only form: partitions that hold no position (past the end of
     // their sequence) report m = -inf, l = 0, o = 0.  Grid-strided over all
     // (sequence, head, partition) triples, after the CTA's items.
+    pdl_wait();
     if (split && !p.direct_single) {
         const int64_t triples = (int64_t)B * p.num_heads * p.max_parts;
         for (int64_t t = (int64_t)blockIdx.x * kDecodeThreads + threadIdx.x; t < triples;

@@ -327,14 +327,16 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
 
 // pa_decode's plan: 0 = one pass, else the partition size of the split form.
 // Chosen from measurements on B200 (head_dim 128, bs 16, largest-first item
-// order): one pass wins when every sequence is short and the (sequence, KV
-// head) units alone give every SM several items (MHA batch, max 2048: 209 us
-// one pass vs 212 us at 512; shared-prefix batch, max 1280: 192 vs 206 us);
-// otherwise 1024-token partitions (GQA batch, max 4096: 115 us vs 118 us at 512
-// and 126 us one pass) up to 16K positions and 2048-token ones beyond (128K
-// context: 439 us vs 458 us at 1024); partitions shrink until a small batch
-// still yields several items per resident CTA.
-static constexpr int kOnePassMaxLen = 2048;
+// order, items taken when their slot frees): one pass wins when no sequence is
+// longer than 4096 and the (sequence, KV head) units alone give every SM
+// several items -- GQA batch, max 4096: 101.7 us one pass vs 103.9 us at 1024
+// and 107.1 us at 512; MHA batch, max 2048: 183.3 vs 185.4 us; shared-prefix
+// batch, max 1280: 159.4 vs 161.9 us at 2048 -- as the one pass needs no
+// partials and no reduce.  Otherwise 1024-token partitions up to 16K positions
+// and 2048-token ones beyond (128K context: 421.4 us vs 438.9 us at 1024);
+// partitions shrink until a small batch still yields several items per
+// resident CTA.
+static constexpr int kOnePassMaxLen = 4096;
 
 static int choose_plan(int num_seqs, int num_kv_heads, int max_seq_len)
 {
@@ -700,8 +702,9 @@ int pa_prefill(void *out, const void *query, const void *key_cache, const void *
     p.max_blocks = max_blocks_per_seq;
     p.tq = kPfRows / G;
     p.q_box = std::min(p.tq, num_tokens);
-    // the tiles of all sequences number at most T / tq + B
-    const int64_t tiles = (int64_t)num_tokens / p.tq + num_seqs;
+    // the query tiles of all sequences number at most T / tq + B, their pairs
+    // (one CTA each) at most T / (2 tq) + B
+    const int64_t tiles = (int64_t)num_tokens / (2 * p.tq) + num_seqs + 1;
     if (tiles > INT_MAX) return PA_ERR_BAD_SHAPE;
     CUtensorMap tq, tk, tv;
     int rc = make_query_map(&tq, query, num_tokens, num_heads, head_dim, G, p.q_box);
