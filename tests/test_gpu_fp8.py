@@ -192,3 +192,30 @@ def test_decode_fp8_rejects_unsupported_shapes():
                        w64.scale, 1.0, 1.0, 20)
     torch.cuda.synchronize()
     assert ops.device_status() == 0
+
+
+def test_fp8_bench_workload_full_batch():
+    """The bench's FP8 row in its launch configuration: the gqa batch (128
+    sequences, 64 query / 8 KV heads) over E4M3 caches, one decode step through
+    the fused slot mapping + quantising cache write, then the planned decode;
+    caches bit-exact and every output element against the oracle."""
+    import bench
+    w = wl.make("gqa", seed=bench.rank_seed(0), fill_cache=False)
+    rng = np.random.Generator(np.random.PCG64(bench.rank_seed(0) + 17))
+    kc = wl.fp8_cache(rng, w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.free_blocks)
+    vc = wl.fp8_cache(rng, w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.free_blocks)
+    ks, vs = 0.25, 0.25
+    slots = oracle.slot_mapping(w.block_tables, np.arange(w.num_seqs, dtype=np.int32),
+                                w.seq_lens.astype(np.int64) - 1, w.block_size)
+    ref_k, ref_v = kc.copy(), vc.copy()
+    oracle.reshape_and_cache_fp8(w.new_key, w.new_value, ref_k, ref_v, slots, w.block_size, ks, vs)
+    ref = oracle.paged_decode_fp8(w.query, ref_k, ref_v, w.block_tables, w.seq_lens, w.scale, ks, vs, threads=0)
+    dk, dv = _u8(kc), _u8(vc)
+    bt, sl = _i32(w.block_tables), _i32(w.seq_lens)
+    ops.append_decode_kv_fp8(bf16_to_device(w.new_key, DEV), bf16_to_device(w.new_value, DEV), dk, dv, bt, sl, ks, vs)
+    ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, device=DEV)
+    out = ops.decode_fp8(bf16_to_device(w.query, DEV), dk, dv, bt, sl, w.scale, ks, vs, w.max_seq_len, workspace=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(dk.cpu().numpy(), ref_k) and np.array_equal(dv.cpu().numpy(), ref_v)
+    assert_close(bf16_to_host_bits(out), ref, "gqa FP8 batch")
+    assert ops.device_status() == 0

@@ -111,3 +111,34 @@ def test_prefill_rejects_unsupported_shapes():
         _run(w, q, [8])
     torch.cuda.synchronize()
     assert ops.device_status() == 0
+
+
+def test_prefill_bench_workload_sampled_rows():
+    """The bench's prefill workload (8 x 2048-token prompts, 64 query / 8 KV heads,
+    head_dim 128, block size 16) in its launch configuration, checked on sampled
+    rows: windows of 16 query rows at spread positions, each against the oracle's
+    prefill of that window (a chunk ending at the window's last position)."""
+    import bench
+    w, lens, q, nk, nv = bench.make_prefill_case(bench.rank_seed(0))
+    B, P = w.num_seqs, lens[0]
+    T = q.shape[0]
+    # the step's cache write: the prompts' K/V rows at their slots
+    seq_ids = np.repeat(np.arange(B), lens).astype(np.int32)
+    pos = np.concatenate([np.arange(L) for L in lens]).astype(np.int64)
+    slots = oracle.slot_mapping(w.block_tables, seq_ids, pos, w.block_size)
+    kc, vc = w.key_cache.copy(), w.value_cache.copy()
+    oracle.reshape_and_cache(nk, nv, kc, vc, slots, w.block_size)
+    start = np.zeros(B + 1, np.int32)
+    start[1:] = np.cumsum(lens)
+    out = ops.prefill(bf16_to_device(q, DEV), bf16_to_device(kc, DEV), bf16_to_device(vc, DEV),
+                      _i32(w.block_tables), _i32(np.asarray(lens)), _i32(start), w.scale)
+    torch.cuda.synchronize()
+    got = bf16_to_host_bits(out)
+    rng = np.random.default_rng(11)
+    for s in range(B):
+        for end in (16, int(rng.integers(17, P)), P):
+            rows = slice(s * P + end - 16, s * P + end)
+            ref = oracle.paged_prefill(q[rows], kc, vc, w.block_tables[s:s + 1], np.array([end], np.int32), [16],
+                                       w.scale, threads=16)
+            assert_close(got[rows], ref, f"seq {s} rows {end - 16}..{end - 1}")
+    assert ops.device_status() == 0
