@@ -65,6 +65,7 @@ extern "C" {
 #define PA_ERR_DEVICE_TIMEOUT (-9) /* a bounded on-device wait gave up (see below)   */
 #define PA_ERR_SCRATCH_TOO_SMALL (-10) /* the built-in scratch of the no-allocation call is too small */
 #define PA_ERR_NOT_DEVICE_ACCESSIBLE (-11) /* a pointer the kernel would read is not device-accessible */
+#define PA_ERR_VALUE_RANGE (-12)   /* a kernel met a value outside its operand range (see pa_prefill) */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *pa_status_string(int status);
@@ -321,8 +322,12 @@ int pa_decode_fp8_split(void *out, const void *query, const void *key_cache,
  * with K/V read block by block through the table.  Sequences with q_len <= 0
  * or q_len > seq_len are skipped (their rows are not written).
  * Supported: head_dim 64 or 128, block_size 8, 16 or 32, G = num_heads /
- * num_kv_heads in 1..16.  fp32 accumulation on the tensor cores (tcgen05),
- * softmax weights as a bf16 high part plus a bf16 residual; output rounded to
+ * num_kv_heads in 1..16.  fp32 accumulation on the tensor cores (tcgen05):
+ * q . k in bf16; P V in fp16 -- the softmax weights rounded to fp16 and the
+ * value rows converted to fp16 in shared memory, exact for 2^-17 <= |v| <=
+ * 65504.  A value entry of larger magnitude that a row reads saturates to
+ * +-65504 and sets PA_ERR_VALUE_RANGE in the device status (pa_device_status);
+ * the output rows that attend to it are then not exact.  Output rounded to
  * bf16.  No workspace; one launch.
  * ------------------------------------------------------------------------ */
 int pa_prefill(void *out, const void *query, const void *key_cache, const void *value_cache,
@@ -380,7 +385,9 @@ int pa_decode_split_noalloc(void *out, const void *query, const void *key_cache,
  * pipeline stage being released) gives up after about one second, records a
  * nonzero code in a device word and lets the kernel return.  This call reads
  * and clears that word for the current device (synchronising the device);
- * 0 means no wait ever gave up, otherwise PA_ERR_DEVICE_TIMEOUT. */
+ * 0 means no wait ever gave up and no kernel met an out-of-range value;
+ * otherwise PA_ERR_DEVICE_TIMEOUT, or PA_ERR_VALUE_RANGE when pa_prefill read
+ * a value-cache entry of magnitude above 65504 (its P.V operand is fp16). */
 int pa_device_status(void);
 
 /* --------------------------------------------------------------------------

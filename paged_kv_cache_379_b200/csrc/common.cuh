@@ -25,6 +25,9 @@ namespace pakv {
 constexpr int kTimeoutFullBarrier = 1;
 constexpr int kTimeoutEmptyBarrier = 2;
 constexpr int kTimeoutDrain = 3;
+// Code written when a kernel met an input value outside the range of the
+// arithmetic it uses (the prefill's fp16 P.V operand: |v| > 65504).
+constexpr int kStatusValueRange = 4;
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
@@ -241,6 +244,7 @@ __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepc
 __device__ int g_pa_device_status = 0;
 
 __device__ __forceinline__ void record_timeout(int code) { atomicCAS(&g_pa_device_status, 0, code); }
+__device__ __forceinline__ void record_status(int code) { atomicCAS(&g_pa_device_status, 0, code); }
 
 // ------------------------------------------------------------------ host side
 

@@ -391,6 +391,7 @@ const char *pa_status_string(int status)
     case PA_ERR_BAD_BLOCK: return "bad block id";
     case PA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case PA_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
+    case PA_ERR_VALUE_RANGE: return "an input value outside the range a kernel's arithmetic represents";
     case PA_ERR_NOT_DEVICE_ACCESSIBLE: return "memory not accessible from the device (pageable host memory?)";
     case PA_ERR_SCRATCH_TOO_SMALL:
         return "split workspace exceeds the built-in scratch of pa_decode_split_noalloc (use a larger "
@@ -827,7 +828,7 @@ int pa_device_status(void)
         const int zero = 0;
         rc = check_cuda(cudaMemcpyToSymbol(g_pa_device_status, &zero, sizeof(int)));
         if (rc != PA_OK) return rc;
-        return PA_ERR_DEVICE_TIMEOUT;
+        return v == pakv::kStatusValueRange ? PA_ERR_VALUE_RANGE : PA_ERR_DEVICE_TIMEOUT;
     }
     return PA_OK;
 }

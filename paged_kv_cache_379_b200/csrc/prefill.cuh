@@ -11,11 +11,11 @@
 // tile is 128 MMA rows = tq tokens x G query heads (row r = token r / G, head
 // r % G), so every K/V tile read from the cache feeds all G heads of the KV
 // head -- and, as the CTA holds two consecutive query tiles A and B, both of
-// them.  Keys are processed in tiles of 64.  Eleven warps:
+// them.  Keys are processed in tiles of 64.  Fifteen warps:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: warp w owns TMEM
 //              lanes 32(w % 4) .. +31, one row per thread; it reads S from
 //              TMEM, keeps a lazily moved reference max, writes P back over S
-//              as bf16 high parts and bf16 residuals (each truncated),
+//              as fp16 (rounded to nearest: 11 significant bits),
 //              rescales O in TMEM when a reference moves, and finally
 //              normalises O and stores the output rows;
 //   warp 8     producer: TMA loads of the two query tiles (once) and of 64-key
@@ -25,12 +25,21 @@
 //              query tile (A: columns 0..127, B: 128..255), O of A from 256, O
 //              of B from 256 + D; one thread of warp 9 issues tile A's
 //              tcgen05.mma, one of warp 10 tile B's:
-//                S_X = Q_X K_j^T              (SS form: M 128, N 64, K D)
-//                O_X += P_hi V_j + P_lo V_j   (TS form, P read from TMEM; V an
-//                                              MN-major shared-memory operand)
+//                S_X = Q_X K_j^T    (SS form, bf16: M 128, N 64, K D)
+//                O_X += P V_j       (TS form, fp16: P read from TMEM; V an
+//                                    MN-major shared-memory operand)
 //              S_X(j) goes to buffer j % 2, so it overlaps the softmax of
 //              S_X(j-1); completion is tracked by tcgen05.commit on mbarriers,
-//              one per buffer.  The two tiles' chains run independently.
+//              one per buffer.  The two tiles' chains run independently;
+//   warps 11-14 convert every V tile in shared memory from bf16 to fp16 in
+//              place as soon as it lands (16 keys each), zeroing rows past the
+//              sequence end; the four quarters meet on a per-stage mbarrier
+//              that both tiles' P V wait for.
+// P V runs on fp16 operands: a bf16 P (8 significant bits) is too coarse for
+// the attention tolerance, and a bf16 high part + residual pair costs a second
+// P V product.  A bf16 value converts to fp16 exactly for 2^-17 <= |v| <= 65504
+// (smaller magnitudes round by at most 2^-25; larger ones saturate and record
+// kStatusValueRange in the device status word).
 // Every wait is bounded in time; after a timeout the CTA drains its own TMA
 // loads and MMAs (bounded again), frees TMEM and returns.
 #pragma once
@@ -53,7 +62,8 @@ struct PrefillParams {
 
 constexpr int kPfProducerWarp = 8;
 constexpr int kPfMmaWarp = 9;         // tile A's MMAs; warp 10 issues tile B's
-constexpr int kPfThreads = 352;
+constexpr int kPfConvWarp = 11;        // first of the 4 V-conversion warps
+constexpr int kPfThreads = 480;
 constexpr int kPfRows = 128;          // MMA M: query rows per tile
 constexpr int kPfKeys = 64;           // keys per K/V tile
 constexpr int kPfStages = 4;          // K/V ring stages
@@ -61,6 +71,22 @@ constexpr uint32_t kPfTmemCols = 512;
 // A row's softmax reference max moves only when a logit exceeds it by more
 // than this (log2 units), so unnormalised weights stay below 2^8.
 constexpr float kPfRescaleSlack = 8.f;
+// Weights are computed as 2^(logit - reference + kPfP16Shift), i.e. in
+// (0, 2^15]: inside the fp16 range, and 2^7 further from fp16's subnormals.
+// The factor cancels between O and the row sum.
+constexpr float kPfP16Shift = 7.f;
+
+// bf16x2 -> f16x2 (round to nearest), tracking the largest magnitude seen.
+// Magnitudes beyond the fp16 range saturate to +-65504 rather than becoming
+// infinite, so a zero weight times such an entry stays 0 for the other rows.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float &amax)
+{
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+    amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+    uint32_t d;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
 
 template <int D>
 struct PfLayout {
@@ -74,8 +100,9 @@ struct PfLayout {
     static constexpr int kStageBytes = 2 * kKTile;
     static constexpr int kBar = kStage0 + kPfStages * kStageBytes;
     // q_full, drain[2], kv_full[4], kv_empty[4], then per query tile and
-    // S/P buffer: s_full[2][2], p_full[2][2], o_done[2][2]
-    static constexpr int kNumBars = 3 + 2 * kPfStages + 12;
+    // S/P buffer: s_full[2][2], p_full[2][2], o_done[2][2]; then v16[4] (the V
+    // tile of a stage converted to fp16)
+    static constexpr int kNumBars = 3 + 3 * kPfStages + 12;
     static constexpr int kMisc = kBar + kNumBars * 8;      // TMEM base, abort flag, item
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
@@ -109,6 +136,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     auto s_full = [&](int x, int b) { return bar0 + 8u * (3 + 2 * kPfStages + 2 * x + b); };
     auto p_full = [&](int x, int b) { return bar0 + 8u * (7 + 2 * kPfStages + 2 * x + b); };
     auto o_done = [&](int x, int b) { return bar0 + 8u * (11 + 2 * kPfStages + 2 * x + b); };
+    auto v16 = [&](int st) { return bar0 + 8u * (15 + 2 * kPfStages + st); };
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(base_ptr + Lay::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Lay::kMisc + 4);
     volatile int *item = reinterpret_cast<volatile int *>(base_ptr + Lay::kMisc + 16);
@@ -164,6 +192,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 mbar_init(p_full(x, b), 128);
                 mbar_init(o_done(x, b), 1);
             }
+        for (int st = 0; st < kPfStages; ++st) mbar_init(v16(st), 4);  // one arrival per conversion warp
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -242,17 +271,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int st = 0; st < kPfStages; ++st)
                 if (last[st] >= 0) mbar_wait_bounded(kv_full(st), (last[st] / kPfStages) & 1);
         }
-    } else if (warp >= kPfMmaWarp) {
+    } else if (warp >= kPfMmaWarp && warp < kPfConvWarp) {
         // ------------------------------------------------------------ MMA issue
         // Warp 9 issues tile A's products, warp 10 tile B's.  Per key tile j:
-        // S_X(j) into buffer j % 2 (after P_X(j-2) V has read that buffer), then
-        // P_X(j) V once the softmax has written P.  Each warp releases the K/V
-        // stage with its own commit, also for key tiles its query tile skips.
+        // S_X(j+1) into buffer (j+1) % 2 (after P_X(j-1) V has read it), then
+        // P_X(j) V once the softmax has written P and V(j) is fp16.  Each warp
+        // releases the K/V stage with its own commit, also for key tiles its
+        // query tile skips.
         const int x = warp - kPfMmaWarp;
         const bool act = x == 0 || hasB;
         const int nkx = x == 0 ? nkA : nk;
         constexpr uint32_t kIdS = idesc_bf16_f32(kPfRows, kPfKeys, false, false);
-        constexpr uint32_t kIdO = idesc_bf16_f32(kPfRows, D, false, true);
+        constexpr uint32_t kIdO = idesc_f16_f32(kPfRows, D, false, true);
         bool ok = __all_sync(0xffffffffu, wait(q_full, 0));
         const uint32_t qt = base + Lay::kQ + x * Lay::kQTile;
         // S_X(j) for key tile j into buffer j % 2 (after P_X(j-2) V has read it)
@@ -276,7 +306,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
         // The S product of the next key tile is issued before waiting for this
         // tile's P, so the softmax always finds its next S ready.
-        if (act && nkx > 0) ok = issue_s(0);
+        if (ok && act && nkx > 0) ok = issue_s(0);
         for (int j = 0; ok && j < nk; ++j) {
             const int st = j % kPfStages;
             const int b = j & 1;
@@ -286,36 +316,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     ok = issue_s(j + 1);
                     if (!ok) break;
                 }
-                // value rows past the sequence end hold stale or foreign data (maybe
-                // NaN); P is 0 there, but 0 * NaN is NaN in the MMA: zero them (both
-                // MMA warps may do it: they write the same zeros)
-                const int kv_valid = min(kPfKeys, L - j * kPfKeys);
-                if (kv_valid < kPfKeys) {
-                    uint8_t *vt = base_ptr + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
-                    const int chunks = (kPfKeys - kv_valid) * 8;
-                    for (int i = lane; i < kPlanes * chunks; i += 32) {
-                        const int pl = i / chunks, c = i - pl * chunks;
-                        *reinterpret_cast<uint4 *>(vt + pl * kKPlane + kv_valid * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
                 ok = __all_sync(0xffffffffu, wait(p_full(x, b), (j >> 1) & 1));
+                if (ok) ok = __all_sync(0xffffffffu, wait(v16(st), (j / kPfStages) & 1));
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t vt = base + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
-                    // P of the tile's 64 keys in the buffer: high parts in columns
-                    // [0, 32), residuals in [32, 64); a K step of 16 keys is 8 columns
+                    // P of the tile's 64 keys: fp16 pairs in columns [0, 32); a K
+                    // step of 16 keys is 8 columns
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-                            tc_mma_bf16_ts(tmem + Lay::kTmemO + x * D,
-                                           tmem + x * 2 * kPfKeys + b * kPfKeys + half * 32 + kk * 8,
-                                           desc_mnmajor_sw128(vt + kk * 16 * 128, kKPlane), kIdO,
-                                           j > 0 || half > 0 || kk > 0);
-                        }
+                    for (int kk = 0; kk < kPfKeys / 16; ++kk) {
+                        tc_mma_bf16_ts(tmem + Lay::kTmemO + x * D, tmem + x * 2 * kPfKeys + b * kPfKeys + kk * 8,
+                                       desc_mnmajor_sw128(vt + kk * 16 * 128, kKPlane), kIdO, j > 0 || kk > 0);
                     }
                     tc_commit(o_done(x, b));
                 }
@@ -329,6 +341,45 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (lane == 0) tc_commit(kv_empty(st));
             __syncwarp();
         }
+    } else if (warp >= kPfConvWarp) {
+        // ------------------------------------------------------------ V to fp16
+        // Warp 11 + c converts keys 16c .. 16c + 15 of every V tile (every
+        // plane) in place as soon as the tile lands; rows past the sequence end
+        // become 0 (they may hold stale or foreign data, even NaN, and P = 0
+        // there would still give 0 * NaN = NaN).  The stage cannot be reloaded
+        // before the P V that waits for this conversion has completed.
+        const int c = warp - kPfConvWarp;
+        float amax = 0.f;
+        for (int t = 0; t < nk; ++t) {
+            const int st = t % kPfStages;
+            if (!__all_sync(0xffffffffu, wait(kv_full(st), (t / kPfStages) & 1))) break;
+            const int kv_valid = min(kPfKeys, L - t * kPfKeys);
+            uint8_t *vt = base_ptr + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
+            uint4 v[kPlanes][4];
+#pragma unroll
+            for (int pl = 0; pl < kPlanes; ++pl)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    v[pl][k] = reinterpret_cast<const uint4 *>(vt + pl * kKPlane + c * 16 * 128)[lane + 32 * k];
+#pragma unroll
+            for (int pl = 0; pl < kPlanes; ++pl)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int key = 16 * c + 4 * k + (lane >> 3);  // 8 chunks of 16 bytes per 128-byte row
+                    uint4 o = make_uint4(0, 0, 0, 0);
+                    if (key < kv_valid) {
+                        o.x = bf16x2_to_f16x2(v[pl][k].x, amax);
+                        o.y = bf16x2_to_f16x2(v[pl][k].y, amax);
+                        o.z = bf16x2_to_f16x2(v[pl][k].z, amax);
+                        o.w = bf16x2_to_f16x2(v[pl][k].w, amax);
+                    }
+                    reinterpret_cast<uint4 *>(vt + pl * kKPlane + c * 16 * 128)[lane + 32 * k] = o;
+                }
+            fence_proxy_async_smem();  // the tensor cores read it through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(v16(st));
+        }
+        if (amax > 65504.f) record_status(kStatusValueRange);
     } else {
         // ------------------------------------------------------------ softmax
         const int x = warp >> 2;                 // query tile: 0 = A, 1 = B
@@ -375,22 +426,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 corr = fast_exp2(m - mx);  // 0 on the first tile (m = -inf)
                 m = mx;
             }
-            // weights and their sum (8 partial sums); P split into a bf16 high
-            // part and a bf16 residual, both truncated (16 significant bits)
+            // weights (scaled by 2^kPfP16Shift) and their sum (8 partial sums);
+            // P as fp16 pairs, the lower key in the low half
+            const float mneg = kPfP16Shift - m;
             float ps[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-            uint32_t hl[kPfKeys];  // [0, 32): high parts, [32, 64): residuals
+            float pw[kPfKeys / 2];
 #pragma unroll
             for (int e = 0; e < kPfKeys / 2; ++e) {
-                const float p0 = fast_exp2(fmaf(xs[2 * e], p.scale_log2, -m));
-                const float p1 = fast_exp2(fmaf(xs[2 * e + 1], p.scale_log2, -m));
+                const float p0 = fast_exp2(fmaf(xs[2 * e], p.scale_log2, mneg));
+                const float p1 = fast_exp2(fmaf(xs[2 * e + 1], p.scale_log2, mneg));
                 ps[e & 7] += p0 + p1;
-                const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                hl[e] = prmt(b0, b1, 0x7632u);  // high halves: bf16(p0) | bf16(p1) << 16
-                const float r0 = p0 - __uint_as_float(b0 & 0xFFFF0000u);
-                const float r1 = p1 - __uint_as_float(b1 & 0xFFFF0000u);
-                hl[kPfKeys / 2 + e] = prmt(__float_as_uint(r0), __float_as_uint(r1), 0x7632u);
+                pw[e] = __uint_as_float(pack_f16x2(p0, p1));
             }
             l = l * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
             if (j >= 1 && __any_sync(0xffffffffu, bump)) {
@@ -409,7 +457,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
             }
             // P over S in this buffer (all of S is in registers)
-            tmem_st64(s_addr, hl);
+            tmem_st32(s_addr, pw);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full(x, b));
@@ -445,7 +493,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ---- teardown: every role has left its loop (done or aborted)
     tc_fence_before();
     __syncthreads();
-    if (warp >= kPfMmaWarp) {
+    if (warp >= kPfMmaWarp && warp < kPfConvWarp) {
         tc_fence_after();
         // all MMAs this CTA issued (by either MMA warp) have completed before
         // TMEM is released

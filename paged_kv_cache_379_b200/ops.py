@@ -385,5 +385,7 @@ def validate_tables(block_tables, seq_lens, block_size: int, num_blocks: int, ma
 
 
 def device_status() -> int:
-    """0, or the negative status PA_ERR_DEVICE_TIMEOUT if a bounded device wait gave up."""
+    """0, or a negative status: PA_ERR_DEVICE_TIMEOUT (-9) if a bounded device wait
+    gave up, PA_ERR_VALUE_RANGE (-12) if the prefill read a value entry beyond the
+    fp16 range of its P.V operand.  Reading clears it."""
     return int(load().pa_device_status())

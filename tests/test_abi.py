@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings(lib):
     assert _lib.status_string(0) == "ok"
-    for code in range(-1, -11, -1):
+    for code in range(-1, -13, -1):
         assert _lib.status_string(code) != "unknown status"
     assert lib.pa_version() >= 10000
 

@@ -142,3 +142,22 @@ def test_prefill_bench_workload_sampled_rows():
                                        w.scale, threads=16)
             assert_close(got[rows], ref, f"seq {s} rows {end - 16}..{end - 1}")
     assert ops.device_status() == 0
+
+
+def test_prefill_value_beyond_fp16_range_sets_status():
+    """P V runs on fp16 operands: a value-cache entry of magnitude above 65504
+    read by the prefill saturates and sets PA_ERR_VALUE_RANGE in the device
+    status; rows that do not attend to it still match the oracle.  65280 (the
+    largest bf16 value inside the fp16 range) does not set it."""
+    lens, q_lens = [200], [200]
+    w, q = _case(7500, 16, 8, 2, 128, lens, q_lens)
+    last = int(w.block_tables[0, (200 - 1) // 16])
+    off = (200 - 1) % 16
+    w.value_cache[last, off, 1, 5] = np.uint16(0x47C3)  # 99840: beyond fp16, only the last row attends to it
+    got = _run(w, q, q_lens)
+    assert ops.device_status() == -12
+    ref = oracle.paged_prefill(q, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, q_lens, w.scale,
+                               threads=16)
+    assert_close(got[:199], ref[:199], "rows before the out-of-range entry")
+    w.value_cache[last, off, 1, 5] = np.uint16(0x477F)  # 65280: inside the fp16 range
+    _check(w, q, q_lens, "largest in-range value")
