@@ -974,25 +974,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     uint32_t bh[NH][2], bl[NH][2];
 #pragma unroll
                     for (int nh = 0; nh < NH; ++nh) {
-                        float x[2][2], mx[2];  // [head j][token row]
+                        // Each lane tests its own two logits per column against the
+                        // column's reference; the column max (3 shuffles) is formed
+                        // only when some lane's logit passes it by the slack.  The
+                        // true max is kept per lane and reduced once per item.
+                        float x[2][2], lv[2];  // [head j][token row]
                         bool bump = false;
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
                             x[jj][0] = in0 ? sc[nh][jj] * qscale[nh][jj] : -INFINITY;
                             x[jj][1] = in1 ? sc[nh][2 + jj] * qscale[nh][jj] : -INFINITY;
-                            float v = fmaxf(x[jj][0], x[jj][1]);
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                            mx[jj] = v;
-                            mtrue[nh][jj] = fmaxf(mtrue[nh][jj], v);
-                            bump |= v > m[nh][jj] + kRescaleSlack;
+                            lv[jj] = fmaxf(x[jj][0], x[jj][1]);
+                            mtrue[nh][jj] = fmaxf(mtrue[nh][jj], lv[jj]);
+                            bump |= lv[jj] > m[nh][jj] + kRescaleSlack;
                         }
                         if (__any_sync(0xffffffffu, bump)) {
 #pragma unroll
                             for (int jj = 0; jj < 2; ++jj) {
-                                const float m_new = mx[jj] > m[nh][jj] + kRescaleSlack ? mx[jj] : m[nh][jj];
-                                const float corr = exp2f(m[nh][jj] - m_new);  // 1 for an unmoved column
+                                float v = lv[jj];
+                                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                                const float m_new = v > m[nh][jj] + kRescaleSlack ? v : m[nh][jj];
+                                const float corr = fast_exp2(m[nh][jj] - m_new);  // 1 for an unmoved column
                                 m[nh][jj] = m_new;
                                 l[nh][jj] *= corr;
 #pragma unroll
@@ -1005,8 +1009,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         float pr[2][2];
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
-                            pr[jj][0] = exp2f(x[jj][0] - m[nh][jj]);
-                            pr[jj][1] = exp2f(x[jj][1] - m[nh][jj]);
+                            pr[jj][0] = fast_exp2(x[jj][0] - m[nh][jj]);
+                            pr[jj][1] = fast_exp2(x[jj][1] - m[nh][jj]);
                             l[nh][jj] += pr[jj][0] + pr[jj][1];
                         }
 #pragma unroll
@@ -1070,6 +1074,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         l[nh][jj] += __shfl_xor_sync(0xffffffffu, l[nh][jj], 4);
                         l[nh][jj] += __shfl_xor_sync(0xffffffffu, l[nh][jj], 8);
                         l[nh][jj] += __shfl_xor_sync(0xffffffffu, l[nh][jj], 16);
+                        mtrue[nh][jj] = fmaxf(mtrue[nh][jj], __shfl_xor_sync(0xffffffffu, mtrue[nh][jj], 4));
+                        mtrue[nh][jj] = fmaxf(mtrue[nh][jj], __shfl_xor_sync(0xffffffffu, mtrue[nh][jj], 8));
+                        mtrue[nh][jj] = fmaxf(mtrue[nh][jj], __shfl_xor_sync(0xffffffffu, mtrue[nh][jj], 16));
                     }
                 }
 #pragma unroll

@@ -152,15 +152,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
         : "memory");
 }
 
-// 2^x by the special-function unit (ex2.approx, flush-to-zero): relative
-// error about 2^-22; results below 2^-126 flush to 0, -inf gives 0.
-__device__ __forceinline__ float fast_exp2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // 64 consecutive 32-bit columns of this lane from registers (no wait).
 __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t *v)
 {
