@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                 q0 + tA + x * p.tq);
         }
         const int32_t *table = p.block_tables + (int64_t)s * p.max_blocks;
-        int last[kPfStages] = {-1, -1, -1, -1};
+        int issued = 0;  // key tiles whose loads were issued
         for (int t = 0; t < nk; ++t) {
             const int st = t % kPfStages;
             const int key0 = t * kPfKeys;
@@ -264,12 +264,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                 }
             }
-            last[st] = t;
+            issued = t + 1;
         }
         if (lane == 0 && *abort_flag) {  // let the loads this CTA issued land before it exits
             mbar_wait_bounded(q_full, 0);
             for (int st = 0; st < kPfStages; ++st)
-                if (last[st] >= 0) mbar_wait_bounded(kv_full(st), (last[st] / kPfStages) & 1);
+                if (st < issued) {  // the stage's last tile: the largest t < issued with t % kPfStages == st
+                    const int last = issued - 1 - (issued - 1 - st) % kPfStages;
+                    mbar_wait_bounded(kv_full(st), (last / kPfStages) & 1);
+                }
         }
     } else if (warp >= kPfMmaWarp && warp < kPfConvWarp) {
         // ------------------------------------------------------------ MMA issue
