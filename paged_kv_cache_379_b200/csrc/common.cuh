@@ -181,6 +181,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes)
     return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
+// Four E4M3 codes (one 32-bit register) widened exactly to two f16x2 words:
+// codes 0, 1 (the low half) into lo, codes 2, 3 into hi.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t &lo, uint32_t &hi)
+{
+    asm("{\n\t.reg .b16 c01, c23;\n\t"
+        "mov.b32 {c01, c23}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c01;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, c23;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(codes));
+}
+
 // D = A(16x32, row) * B(32x8, col) + D, E4M3 inputs (four codes per register,
 // the lowest k in the low byte), fp32 accumulate.
 __device__ __forceinline__ void mma_e4m3_16832(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

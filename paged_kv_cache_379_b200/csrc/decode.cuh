@@ -1046,10 +1046,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
                             const uint32_t lo = prmt(u4_word(vr[0], mt >> 1), u4_word(vr[1], mt >> 1), sel);
                             const uint32_t hi = prmt(u4_word(vr[2], mt >> 1), u4_word(vr[3], mt >> 1), sel);
-                            const uint32_t a0 = e4m3x2_to_f16x2((uint16_t)(lo & 0xFFFFu));
-                            const uint32_t a1 = e4m3x2_to_f16x2((uint16_t)(lo >> 16));
-                            const uint32_t a2 = e4m3x2_to_f16x2((uint16_t)(hi & 0xFFFFu));
-                            const uint32_t a3 = e4m3x2_to_f16x2((uint16_t)(hi >> 16));
+                            uint32_t a0, a1, a2, a3;
+                            e4m3x4_to_f16x2x2(lo, a0, a1);
+                            e4m3x4_to_f16x2x2(hi, a2, a3);
 #pragma unroll
                             for (int nh = 0; nh < NH; ++nh) mma_f16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
                         }
