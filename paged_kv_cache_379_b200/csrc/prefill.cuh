@@ -76,13 +76,46 @@ constexpr float kPfRescaleSlack = 8.f;
 // The factor cancels between O and the row sum.
 constexpr float kPfP16Shift = 7.f;
 
+// Packed fp32 pairs (one 64-bit register pair, two lanes of one instruction).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f32x2_split(uint64_t v)
+{
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+// a * b + c on both lanes
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // bf16x2 -> f16x2 (round to nearest), tracking the largest magnitude seen.
 // Magnitudes beyond the fp16 range saturate to +-65504 rather than becoming
 // infinite, so a zero weight times such an entry stays 0 for the other rows.
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float &amax)
 {
     const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
-    amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+    amax = max3f(amax, fabsf(lo), fabsf(hi));
     uint32_t d;
     asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
@@ -414,14 +447,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kPfKeys; ++c) xs[c] = c <= lim ? xs[c] : -INFINITY;
             }
-            float pm[8];
+            // row max: four chains of three-input maxima
+            float pm[4] = {xs[0], xs[1], xs[2], xs[3]};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) pm[u] = xs[u];
-#pragma unroll
-            for (int c = 8; c < kPfKeys; ++c) pm[c & 7] = fmaxf(pm[c & 7], xs[c]);
-            const float mx =
-                fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) *
-                p.scale_log2;  // scale > 0: the max commutes with it
+            for (int c = 4; c < kPfKeys; c += 8) {
+                pm[0] = max3f(pm[0], xs[c], xs[c + 1]);
+                pm[1] = max3f(pm[1], xs[c + 2], xs[c + 3]);
+                pm[2] = max3f(pm[2], xs[c + 4], xs[c + 5]);
+                pm[3] = max3f(pm[3], xs[c + 6], xs[c + 7]);
+            }
+            const float mx = fmaxf(max3f(pm[0], pm[1], pm[2]), pm[3]) * p.scale_log2;  // scale > 0: the max commutes with it
             // lazily moved reference max (log2 units): weights stay <= 2^kPfRescaleSlack
             const bool bump = mx > m + kPfRescaleSlack;
             float corr = 1.f;
@@ -431,19 +466,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
             // weights (scaled by 2^kPfP16Shift) and their sum (8 partial sums);
             // P as fp16 pairs, the lower key in the low half
+            // (logit scale, shift) on key pairs by packed fp32 FMAs; the row sum
+            // in four packed fp32 accumulators
             const float mneg = kPfP16Shift - m;
-            float ps[8];
+            const uint64_t scale2 = f32x2(p.scale_log2, p.scale_log2), shift2 = f32x2(mneg, mneg);
+            uint64_t ps[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+            for (int u = 0; u < 4; ++u) ps[u] = 0ull;
             float pw[kPfKeys / 2];
 #pragma unroll
             for (int e = 0; e < kPfKeys / 2; ++e) {
-                const float p0 = fast_exp2(fmaf(xs[2 * e], p.scale_log2, mneg));
-                const float p1 = fast_exp2(fmaf(xs[2 * e + 1], p.scale_log2, mneg));
-                ps[e & 7] += p0 + p1;
+                const float2 y = f32x2_split(fma_f32x2(f32x2(xs[2 * e], xs[2 * e + 1]), scale2, shift2));
+                const float p0 = fast_exp2(y.x);
+                const float p1 = fast_exp2(y.y);
+                ps[e & 3] = add_f32x2(ps[e & 3], f32x2(p0, p1));
                 pw[e] = __uint_as_float(pack_f16x2(p0, p1));
             }
-            l = l * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+            const float2 q01 = f32x2_split(add_f32x2(ps[0], ps[1])), q23 = f32x2_split(add_f32x2(ps[2], ps[3]));
+            l = l * corr + ((q01.x + q01.y) + (q23.x + q23.y));
             if (j >= 1 && __any_sync(0xffffffffu, bump)) {
                 // O holds P_{<j} V: rescale it once P_{j-1} V has completed
                 const int jp = j - 1;
