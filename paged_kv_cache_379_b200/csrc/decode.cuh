@@ -86,6 +86,7 @@ constexpr int kTileTokens = 16;
 constexpr int kItemSlots = 2;
 constexpr int kChunkSlots = 4;
 constexpr int kChunkBlocks = 32;
+constexpr int kProducerLanes = 4;  // producer lanes issuing consecutive tiles together
 constexpr int kSortKeys = 256;  // size classes (16-token tiles) of the largest-first item order
 constexpr float kLn2 = 0.693147180559945309f;
 // A column's softmax reference max moves only when a logit exceeds it by more
@@ -584,42 +585,57 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             if (!ok) break;
             const ChunkInfo *c = chunks + cslot;
             if (c->stop) break;
-            if (lane == 0) {
+            {
+                // kProducerLanes lanes take consecutive tiles of the chunk at once:
+                // their ring waits, transaction counts and TMA issues go out as
+                // one instruction each, so the per-tile handoff latency is shared.
                 const int n = c->n_blocks;
                 const int g = c->g;
-                for (int j = 0; j < n; j += Geo::kBlocksPerTile) {
-                    const int valid = min(Geo::kBlocksPerTile, n - j);
-                    const int stage = ring % kStages;
-                    if (*abort_flag || !mbar_wait_bounded(empty_bar + 8 * stage, ((ring / kStages) & 1) ^ 1)) {
-                        if (!*abort_flag) record_timeout(kTimeoutEmptyBarrier);
-                        *abort_flag = 1;
+                const int ntiles = (n + Geo::kBlocksPerTile - 1) / Geo::kBlocksPerTile;
+                for (int t0 = 0; t0 < ntiles; t0 += kProducerLanes) {
+                    const int t = t0 + lane;
+                    const bool mine = lane < kProducerLanes && t < ntiles;
+                    const int r = ring + lane;  // ring position of tile t
+                    const int stage = r % kStages;
+                    bool w_ok = true;
+                    if (mine) w_ok = !*abort_flag && mbar_wait_bounded(empty_bar + 8 * stage, ((r / kStages) & 1) ^ 1);
+                    if (!__all_sync(0xffffffffu, w_ok)) {
+                        if (lane == 0) {
+                            if (!*abort_flag) record_timeout(kTimeoutEmptyBarrier);
+                            *abort_flag = 1;
+                        }
                         ok = false;
                         break;
                     }
-                    const uint32_t kdst = base + stage * Geo::kStageSmem;
-                    const uint32_t vdst = kdst + Geo::kTileSmem;
-                    const uint32_t bar = full_bar + 8 * stage;
-                    mbar_arrive_expect_tx(bar, (uint32_t)(valid * Geo::kBlkBytes * 2));
+                    if (mine) {
+                        const int j = t * Geo::kBlocksPerTile;
+                        const int valid = min(Geo::kBlocksPerTile, n - j);
+                        const uint32_t kdst = base + stage * Geo::kStageSmem;
+                        const uint32_t vdst = kdst + Geo::kTileSmem;
+                        const uint32_t bar = full_bar + 8 * stage;
+                        mbar_arrive_expect_tx(bar, (uint32_t)(valid * Geo::kBlkBytes * 2));
 #pragma unroll
-                    for (int k = 0; k < Geo::kBlocksPerTile; ++k) {
-                        if (k < valid) {
-                            const int row = c->phys[j + k] * BS;
-                            if constexpr (kBlockBox) {
-                                // one box per block: both 64-wide planes, plane-major
-                                tma_load_4d(kdst + Geo::box_offset(k, 0), &tmap_k, bar, 0, row, 0, g);
-                                tma_load_4d(vdst + Geo::box_offset(k, 0), &tmap_v, bar, 0, row, 0, g);
-                            } else {
+                        for (int k = 0; k < Geo::kBlocksPerTile; ++k) {
+                            if (k < valid) {
+                                const int row = c->phys[j + k] * BS;
+                                if constexpr (kBlockBox) {
+                                    // one box per block: both 64-wide planes, plane-major
+                                    tma_load_4d(kdst + Geo::box_offset(k, 0), &tmap_k, bar, 0, row, 0, g);
+                                    tma_load_4d(vdst + Geo::box_offset(k, 0), &tmap_v, bar, 0, row, 0, g);
+                                } else {
 #pragma unroll
-                                for (int h = 0; h < Geo::kHalves; ++h) {
-                                    tma_load_4d(kdst + Geo::box_offset(k, h), &tmap_k, bar, 0, h, g, row);
-                                    tma_load_4d(vdst + Geo::box_offset(k, h), &tmap_v, bar, 0, h, g, row);
+                                    for (int h = 0; h < Geo::kHalves; ++h) {
+                                        tma_load_4d(kdst + Geo::box_offset(k, h), &tmap_k, bar, 0, h, g, row);
+                                        tma_load_4d(vdst + Geo::box_offset(k, h), &tmap_v, bar, 0, h, g, row);
+                                    }
                                 }
                             }
                         }
                     }
-                    ++ring;
+                    ring += min(kProducerLanes, ntiles - t0);
                 }
-                if (ok) mbar_arrive(cempty_bar + 8 * cslot);
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(cempty_bar + 8 * cslot);
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             ring = __shfl_sync(0xffffffffu, ring, 0);
