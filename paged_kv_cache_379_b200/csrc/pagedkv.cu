@@ -329,12 +329,14 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
 // Chosen from measurements on B200 (head_dim 128, bs 16, largest-first item
 // order, items taken when their slot frees): one pass wins when no sequence is
 // longer than 4096 and the (sequence, KV head) units alone give every SM
-// several items -- GQA batch, max 4096: 101.7 us one pass vs 103.9 us at 1024
-// and 107.1 us at 512; MHA batch, max 2048: 183.3 vs 185.4 us; shared-prefix
-// batch, max 1280: 159.4 vs 161.9 us at 2048 -- as the one pass needs no
-// partials and no reduce.  Otherwise 1024-token partitions up to 16K positions
-// and 2048-token ones beyond (128K context: 421.4 us vs 438.9 us at 1024);
-// partitions shrink until a small batch still yields several items per
+// several items -- GQA batch, max 4096: 99.4 us one pass vs 101.4 us at 1024
+// and 100.3 us at 2048 (FP8 cache: 60.9 vs 66.0 and 63.2 us); MHA batch, max
+// 2048: 182.2 vs 185.4 us -- as the one pass needs no partials and no reduce.
+// (A batch whose sequences share 1024-token prompts runs faster split at 1024,
+// 123.1 vs 134.2 us, because the shared parts are then read together; lengths
+// alone do not show sharing.)  Otherwise 1024-token partitions up to 16K
+// positions and 2048-token ones beyond (128K context: 412.8 us vs 430.3 us at
+// 1024); partitions shrink until a small batch still yields several items per
 // resident CTA.
 static constexpr int kOnePassMaxLen = 4096;
 
