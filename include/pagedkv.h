@@ -390,6 +390,13 @@ int pa_decode_split_noalloc(void *out, const void *query, const void *key_cache,
  * a value-cache entry of magnitude above 65504 (its P.V operand is fp16). */
 int pa_device_status(void);
 
+/* Self-test of the bounded-wait path: launches one thread that waits on an
+ * mbarrier nothing ever arrives on.  The wait gives up after its limit (about
+ * one second), records the timeout in the device status word and the kernel
+ * returns; pa_device_status() then reports PA_ERR_DEVICE_TIMEOUT (and clears
+ * it), and the context stays usable.  Returns PA_OK or PA_ERR_CUDA (launch). */
+int pa_selftest_bounded_wait(void *stream);
+
 /* --------------------------------------------------------------------------
  * a7. Host block pool (host memory only; it generates block tables, slots and
  * copy pairs, it never touches the GPU):

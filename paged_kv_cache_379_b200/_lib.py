@@ -44,6 +44,7 @@ SIGNATURES = {
     "pa_lse_reduce": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_validate_tables": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "pa_device_status": (_I, []),
+    "pa_selftest_bounded_wait": (_I, [_P]),
     "pa_pool_create": (_P, [_I, _I, _P]),
     "pa_pool_destroy": (None, [_P]),
     "pa_pool_num_free": (_I, [_P]),

@@ -374,6 +374,19 @@ static int launch_prefill_d(int bs, const PrefillParams &p, const CUtensorMap &t
     }
 }
 
+// A wait that nothing satisfies, for testing the bounded-wait path: one
+// thread waits on an mbarrier that no one arrives on; at the wait limit it
+// records kTimeoutFullBarrier in the device status word and the kernel returns.
+__global__ void bounded_wait_selftest_kernel()
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_mbarrier_init();
+    if (!mbar_wait_bounded(b, 0)) record_timeout(kTimeoutFullBarrier);
+}
+
 }  // namespace pakv
 
 using namespace pakv;
@@ -405,6 +418,11 @@ const char *pa_status_string(int status)
 int pa_last_cuda_error(void) { return t_last_cuda_error; }
 
 int pa_version(void) { return 10000; }
+
+int pa_selftest_bounded_wait(void *stream)
+{
+    return launch_pdl(bounded_wait_selftest_kernel, dim3(1), dim3(32), 0, static_cast<cudaStream_t>(stream));
+}
 
 int pa_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables, int num_seqs, int max_blocks_per_seq,
                     const int32_t *seq_ids, const int64_t *positions, const int32_t *seq_lens, int num_tokens,

@@ -62,7 +62,7 @@ struct PrefillParams {
 
 constexpr int kPfProducerWarp = 8;
 constexpr int kPfMmaWarp = 9;         // tile A's MMAs; warp 10 issues tile B's
-constexpr int kPfConvWarp = 11;        // first of the 4 V-conversion warps
+constexpr int kPfConvWarp = 11;       // first of the 4 V-conversion warps
 constexpr int kPfThreads = 480;
 constexpr int kPfRows = 128;          // MMA M: query rows per tile
 constexpr int kPfKeys = 64;           // keys per K/V tile

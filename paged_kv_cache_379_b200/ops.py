@@ -30,7 +30,7 @@ __all__ = [
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
     "decode_split_noalloc", "swap_blocks", "reshape_and_cache_fp8", "decode_fp8", "decode_fp8_split",
-    "prefill", "append_decode_kv", "append_decode_kv_fp8",
+    "prefill", "append_decode_kv", "append_decode_kv_fp8", "selftest_bounded_wait",
 ]
 
 
@@ -382,6 +382,12 @@ def validate_tables(block_tables, seq_lens, block_size: int, num_blocks: int, ma
         block_tables.shape[0], block_tables.shape[1], int(block_size), int(num_blocks), int(max_seq_len),
         bad.data_ptr(), _stream(stream)))
     return int(bad.item())
+
+
+def selftest_bounded_wait(stream=None) -> None:
+    """Launch one device wait that nothing satisfies; it gives up after about a
+    second and leaves PA_ERR_DEVICE_TIMEOUT for device_status() to report."""
+    check("pa_selftest_bounded_wait", load().pa_selftest_bounded_wait(_stream(stream)))
 
 
 def device_status() -> int:

@@ -195,3 +195,20 @@ def test_validate_tables():
     assert ops.validate_tables(bt, d["seq_lens"], w.block_size, w.num_blocks, w.max_seq_len) == 1
     assert ops.validate_tables(d["block_tables"], d["seq_lens"], w.block_size, w.num_blocks, 40) == 1
     assert ops.device_status() == 0
+
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    """A device wait that nothing satisfies gives up after its limit, leaves
+    PA_ERR_DEVICE_TIMEOUT in the device status (read once, then cleared), and the
+    context stays usable: a decode right after it matches the oracle."""
+    assert ops.device_status() == 0
+    ops.selftest_bounded_wait()
+    assert ops.device_status() == -9
+    assert ops.device_status() == 0
+    w = wl.make("tiny")
+    b = DecodeBatch(w, DEV)
+    out = b.run_step()
+    torch.cuda.synchronize()
+    _, _, _, ref = oracle_step(w)
+    assert_close(bf16_to_host_bits(out), ref, "decode after a timed-out wait")
+    assert ops.device_status() == 0
