@@ -23,10 +23,12 @@
 //    query rows into an item slot, and loads the item's block-table entries in
 //    chunks of 32 into a chunk queue -- running ahead of the other warps, so
 //    their latency is hidden.
-//  * Producer warp: for each chunk, one elected lane issues TMA tile loads of the
-//    K and V blocks (one box {64 d, 1 head, bs tokens} per 64-wide d-plane,
-//    128B-swizzled) into an 8-stage shared-memory ring guarded by mbarriers.  The
-//    ring runs continuously across items.
+//  * Producer warp: for each chunk, four lanes take four consecutive tiles at
+//    once (their ring waits, transaction counts and copies share each warp
+//    instruction) and issue TMA tile loads of the K and V blocks (one box
+//    {64 d, 1 head, bs tokens} per 64-wide d-plane, or one box per block with
+//    both planes, 128B-swizzled) into a shared-memory ring guarded by
+//    mbarriers.  The ring runs continuously across items.
 //  * 4 consumer warps: 16-token tile i of an item goes to warp i % 4.  Every warp
 //    keeps its own running max m, sum l and fp32 accumulator; the four states
 //    are merged through shared memory at the end of the item (consumer-only
@@ -35,7 +37,8 @@
 //      bf16 mma.sync m16n8k16 in transposed form, S^T = K Q^T with the K tile as
 //      the A operand (rows = tokens, via ldmatrix) and Q^T in registers, then
 //      O^T += V^T P^T with V^T through ldmatrix.trans and P^T moved out of the
-//      S^T accumulators by movmatrix.trans; P goes in as bf16 hi + residual.
+//      S^T accumulators by movmatrix.trans; P goes in as bf16 hi + residual
+//      (an FP8 cache: E4M3 key products and fp16 P, see below).
 //    - G <= 2 (MHA-like, a matrix-vector product): CUDA cores, 16-byte shared
 //      loads, warp-shuffle reductions for the dot products, max and sum.
 //  * Masking selects (-inf logits, zeroed V rows) instead of multiplying by 0,
