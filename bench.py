@@ -295,23 +295,37 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     # e2e: the same step through the C ABI with host buffers.  Every step's
     # inputs (query, new K/V, block tables, lengths) come from pinned host memory
     # and its output goes back to pinned host memory inside the timed region.
-    # As a serving loop would, the copies run on their own streams, double
-    # buffered: step i+1's inputs go up and step i's output comes back while
-    # step i computes.  The KV cache stays resident.
+    # As a serving loop would, the inputs sit in one pinned staging buffer
+    # (16-byte aligned sections, one copy per step), and the copies run on their
+    # own streams, double buffered: step i+1's inputs go up and step i's output
+    # comes back while step i computes.  The KV cache stays resident.
     e2e = None
     if not args.no_e2e:
-        h_q = torch.from_numpy(w.query.view(np.int16)).pin_memory()
-        h_k = torch.from_numpy(w.new_key.view(np.int16)).pin_memory()
-        h_v = torch.from_numpy(w.new_value.view(np.int16)).pin_memory()
-        h_bt = torch.from_numpy(np.ascontiguousarray(w.block_tables, np.int32)).pin_memory()
-        h_sl = torch.from_numpy(w.seq_lens.astype(np.int32)).pin_memory()
+        parts = [("q", w.query.view(np.int16), torch.bfloat16, batch.query.shape),
+                 ("k", w.new_key.view(np.int16), torch.bfloat16, batch.new_key.shape),
+                 ("v", w.new_value.view(np.int16), torch.bfloat16, batch.new_value.shape),
+                 ("bt", np.ascontiguousarray(w.block_tables, np.int32), torch.int32, batch.block_tables.shape),
+                 ("sl", w.seq_lens.astype(np.int32), torch.int32, batch.seq_lens.shape)]
+        offs, nbytes_in = {}, 0
+        for name, a, _, _ in parts:
+            offs[name] = (nbytes_in, a.nbytes)
+            nbytes_in += -(-a.nbytes // 16) * 16
+        h_in = torch.zeros(nbytes_in, dtype=torch.uint8).pin_memory()
+        h_np = h_in.numpy()
+        for name, a, _, _ in parts:
+            o, n = offs[name]
+            h_np[o:o + n] = np.frombuffer(np.ascontiguousarray(a).tobytes(), np.uint8)
         h_out = [torch.empty(batch.out.shape, dtype=torch.int16).pin_memory() for _ in range(2)]
-        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_bt, h_sl))
+        h2d = nbytes_in
         d2h = h_out[0].numel() * h_out[0].element_size()
-        sets = [dict(q=torch.empty_like(batch.query), k=torch.empty_like(batch.new_key),
-                     v=torch.empty_like(batch.new_value), bt=torch.empty_like(batch.block_tables),
-                     sl=torch.empty_like(batch.seq_lens), slots=torch.empty_like(batch.slots),
-                     out=torch.empty_like(batch.out)) for _ in range(2)]
+
+        def input_set():
+            buf = torch.empty(nbytes_in, dtype=torch.uint8, device=dev)
+            S = {name: buf[offs[name][0]:offs[name][0] + offs[name][1]].view(dt).view(shape)
+                 for name, _, dt, shape in parts}
+            S.update(buf=buf, slots=torch.empty_like(batch.slots), out=torch.empty_like(batch.out))
+            return S
+        sets = [input_set() for _ in range(2)]
         up = torch.cuda.Stream(dev)
         down = torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
@@ -323,11 +337,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
             S = sets[b]
             up.wait_event(ev_free[b])            # this buffer set's previous output is back on the host
             with torch.cuda.stream(up):
-                S["q"].view(torch.int16).copy_(h_q, non_blocking=True)
-                S["k"].view(torch.int16).copy_(h_k, non_blocking=True)
-                S["v"].view(torch.int16).copy_(h_v, non_blocking=True)
-                S["bt"].copy_(h_bt, non_blocking=True)
-                S["sl"].copy_(h_sl, non_blocking=True)
+                S["buf"].copy_(h_in, non_blocking=True)
                 ev_in[b].record(up)
             stream.wait_event(ev_in[b])
             ops.append_decode_kv(S["k"], S["v"], batch.key_cache, batch.value_cache, S["bt"], S["sl"],
