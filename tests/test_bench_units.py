@@ -1,0 +1,45 @@
+"""The units bench.py reports: algorithmic bytes of a decode call, useful FLOPs
+of a causal prefill, and the code-only hash that keys recorded ncu counters."""
+
+import numpy as np
+
+import bench
+
+
+def test_algorithmic_bytes_hand_case():
+    # 2 sequences of 5 and 17 positions, block size 4: 2 + 5 blocks touched;
+    # 4 query / 2 KV heads, head_dim 8, bf16
+    got = bench.algorithmic_bytes([5, 17], 4, 4, 2, 8)
+    kv = 7 * 4 * 2 * 8 * 2 * 2          # blocks x bs x Hkv x D x (K, V) x 2 bytes
+    q_and_out = 2 * 2 * 4 * 8 * 2        # (query, output) x B x Hq x D x 2 bytes
+    tables_and_lens = 7 * 4 + 2 * 4      # one int32 per block touched, one length per sequence
+    assert got == kv + q_and_out + tables_and_lens
+    # an FP8 cache halves the KV term only
+    assert bench.algorithmic_bytes([5, 17], 4, 4, 2, 8, 1) == kv // 2 + q_and_out + tables_and_lens
+    # an empty sequence touches no block
+    assert bench.algorithmic_bytes([0], 16, 8, 8, 128) == 2 * 8 * 128 * 2 + 4
+
+
+def test_prefill_flops_matches_brute_force():
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        B = int(rng.integers(1, 5))
+        lens = rng.integers(1, 200, B)
+        q_lens = [int(rng.integers(1, L + 1)) for L in lens]
+        pairs = 0
+        for L, n in zip(lens, q_lens):
+            for i in range(n):               # new token i sits at position L - n + i
+                pairs += (L - n + i) + 1     # and sees positions 0 .. L - n + i
+        assert bench.prefill_flops(lens, q_lens, 8, 64) == 4 * 64 * 8 * pairs
+    # the bench's workload: 8 whole 2048-token prompts, 64 heads, d128
+    n = 2048
+    assert bench.prefill_flops([n] * 8, [n] * 8, 64, 128) == 4 * 128 * 64 * 8 * n * (n + 1) // 2
+
+
+def test_code_hash_ignores_comments_and_layout_only():
+    a = "int f(int x) {\n  // twice\n  return 2 * x; /* doubled */\n}\n"
+    b = "int f(int x)   {   return 2 * x;\n\n}  // changed comment\n"
+    c = "int f(int x) { return 3 * x; }"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert len(bench.kernel_source_hash()) == 16
