@@ -9,7 +9,7 @@ lengths lognormal (median 1024, sigma 0.8) clipped to [16, 4096], shuffled
 block pool 1.2x.  Inputs are seeded synthetic data already resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|gqa-fp8|prefill]
+                    [--workload gqa|gqa-fp8|prefill|cow]
 
 The default workload is the line above.  Two more rows of the path are
 measured the same way on request: `gqa-fp8` (the same batch with an FP8 E4M3
@@ -621,6 +621,77 @@ def run_row(args, rank: int, world: int, local_rank: int) -> dict | None:
     return line
 
 
+def run_cow(args, rank: int, world: int, local_rank: int) -> dict | None:
+    """The copy-on-write block copies of the shared-prefix step (256 sequences
+    forked from 32 prompts, each writing into a shared block), L2 flushed
+    before every launch; per-launch device time by events (max over ranks)."""
+    import torch
+
+    from paged_kv_cache_379_b200 import ops
+    from paged_kv_cache_379_b200 import workload as wlmod
+    from paged_kv_cache_379_b200.step import DecodeBatch, host_step
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    stream = torch.cuda.current_stream(dev)
+    K, W = args.steps, args.warmup
+    w = wlmod.make("shared", seed=wlmod.SEED_BASE + wlmod.NAMES.index("shared") + 1000 * rank)
+    _, tables, _, _, pairs = host_step(w, fork_all=True)
+    batch = DecodeBatch(w, dev, tables=tables, pairs=pairs)
+    n_pairs = int(pairs.shape[0])
+    blk_bytes = w.block_size * w.num_kv_heads * w.head_dim * 2
+    units = n_pairs * blk_bytes * 2 * 2  # K and V blocks, each read and written
+    flush = torch.empty(L2_BYTES * 2, dtype=torch.uint8, device=dev)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def step(i):
+        flush.fill_((i or 0) & 255)  # evicts the copies' blocks from L2
+        if i is not None:
+            ev0[i].record(stream)
+        ops.copy_blocks(batch.key_cache, batch.value_cache, batch.pairs, stream=stream)
+        if i is not None:
+            ev1[i].record(stream)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    total_ms, clocks, remeasured = _timed_loop(step, K, W, stream, dev, dist, sampler)
+    sampler.stop()
+    kern_ms = float(np.mean([ev0[i].elapsed_time(ev1[i]) for i in range(K)]))
+    if dist is not None:
+        t = torch.tensor([kern_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        kern_ms = float(t.item())
+    if rank != 0:
+        return None
+    achieved = units / (kern_ms * 1e-3) / 1e9
+    peak, peak_src = measured_peak()
+    line = {
+        "metric": "copy-on-write block copy GB/s (read + written), shared-prefix step",
+        "value": round(achieved * world, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(kern_ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (bit copy)", "data": "synthetic (seeded)",
+        "config": {"workload": f"shared: {w.num_seqs} sequences forked from 32 prompts of 1024 tokens, "
+                               f"{n_pairs} (src, dst) block pairs of {blk_bytes} bytes per cache",
+                   "step": "copy_blocks of the step's pairs (K and V caches)",
+                   "l2": f"flushed before every launch ({2 * L2_BYTES >> 20} MiB written, outside the events)",
+                   "value_from": "per-launch device time (events around the copy only)"},
+        "clocks": clocks,
+        "gpu_launches": K,
+        "roofline": {"bound": "hbm", "kernel": "pa_copy_blocks (copy_blocks_kernel)", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_source": peak_src, "traffic": None, "avg_launch_ms": round(kern_ms, 5)},
+        "e2e": None,
+        "e2e_note": "end-to-end host-buffer timing is measured on the default workload only",
+    }
+    if remeasured:
+        line["clocks_note"] = "first timed region saw a thermal/hw slowdown reason; re-measured once"
+    return line
+
+
 # ---------------------------------------------------------------- the oracle
 
 def cpu_baseline(w, budget_s: float = 15.0) -> dict:
@@ -739,7 +810,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--workload", choices=["gqa", "gqa-fp8", "prefill"], default="gqa")
+    ap.add_argument("--workload", choices=["gqa", "gqa-fp8", "prefill", "cow"], default="gqa")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -767,8 +838,12 @@ def main():
     if world > 1:
         dist.barrier()
     try:
-        line = run_ours(args, rank, world, local_rank) if args.workload == "gqa" else \
-            run_row(args, rank, world, local_rank)
+        if args.workload == "gqa":
+            line = run_ours(args, rank, world, local_rank)
+        elif args.workload == "cow":
+            line = run_cow(args, rank, world, local_rank)
+        else:
+            line = run_row(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
