@@ -322,7 +322,8 @@ int pa_decode_fp8_split(void *out, const void *query, const void *key_cache,
  * with K/V read block by block through the table.  Sequences with q_len <= 0
  * or q_len > seq_len are skipped (their rows are not written).
  * Supported: head_dim 64 or 128, block_size 8, 16 or 32, G = num_heads /
- * num_kv_heads in 1..16.  fp32 accumulation on the tensor cores (tcgen05):
+ * num_kv_heads in 1..16; scale > 0 (the kernel takes a row's max logit before
+ * scaling it, so a non-positive scale is outside the contract).  fp32 accumulation on the tensor cores (tcgen05):
  * q . k in bf16; P V in fp16 -- the softmax weights rounded to fp16 and the
  * value rows converted to fp16 in shared memory, exact for 2^-17 <= |v| <=
  * 65504.  A value entry of larger magnitude that a row reads saturates to

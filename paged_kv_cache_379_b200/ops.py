@@ -266,6 +266,8 @@ def prefill(query, key_cache, value_cache, block_tables, seq_lens, q_start, scal
             stream=None):
     """pa_prefill: causal multi-query attention of each sequence's chunk (query rows
     q_start[s] .. q_start[s+1]-1, the last positions of the sequence) over its paged cache."""
+    if not (float(scale) > 0.0 and float(scale) < float("inf")):
+        raise ValueError("scale must be positive and finite")
     lib = load()
     nb, bs, hkv, d = _cache_dims(key_cache, value_cache)
     q = _dev(query, torch.bfloat16, "query", 3)

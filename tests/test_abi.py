@@ -113,3 +113,27 @@ def test_workspace_size(lib):
     assert lib.pa_decode_workspace_size(4, 8, 2, 128, 1000, 512) == 256 + 64 * 128 * 4 + 2 * 256
     assert lib.pa_decode_workspace_size(4, 8, 2, 128, 0, 512) == 256 + 32 * 128 * 4 + 2 * 256
     assert lib.pa_decode_workspace_size(0, 8, 2, 128, 10, 512) == 0
+
+
+def test_prefill_argument_errors_without_gpu(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    # (out, q, kc, vc, bt, sl, q_start, scale, bs, Hkv, B, Hq, D, max_blocks, nb, T, stream)
+    ok_args = (fake, fake, fake, fake, fake, fake, fake, 0.1, 16, 8, 4, 64, 128, 8, 100, 64, None)
+
+    def call(**kw):
+        names = ["out", "q", "kc", "vc", "bt", "sl", "qs", "scale", "bs", "hkv", "b", "hq", "d", "mb", "nb", "t",
+                 "st"]
+        args = dict(zip(names, ok_args))
+        args.update(kw)
+        return lib.pa_prefill(*[args[n] for n in names])
+
+    assert call(d=96) == -3            # head_dim not compiled
+    assert call(bs=4) == -3            # block_size not compiled
+    assert call(hq=136, hkv=8) == -3   # G = 17 > 16
+    assert call(hq=63) == -2           # num_heads not a multiple of num_kv_heads
+    assert call(nb=0) == -2
+    assert call(t=0) == 0              # no query rows: nothing to do
+    assert call(b=0) == 0
+    assert call(out=None) == -1
+    assert call(q=P(4100)) == -8       # misaligned query
