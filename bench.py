@@ -9,14 +9,21 @@ lengths lognormal (median 1024, sigma 0.8) clipped to [16, 4096], shuffled
 block pool 1.2x.  Inputs are seeded synthetic data already resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|gqa-fp8|prefill|cow]
+                    [--workload tiny|mha|gqa|long|shared|gqa-fp8|prefill|cow]
+                    [--partition P] [--l2-flush]
 
-The default workload is the line above.  Two more rows of the path are
-measured the same way on request: `gqa-fp8` (the same batch with an FP8 E4M3
+The default workload is the line above.  The other decode workloads run the
+same step: `tiny` (4 sequences, block size 4), `mha` (64 sequences, 32/32
+heads), `long` (8 sequences of 32K..128K positions; --partition 512 is the
+workload's stated split), `shared` (256 sequences forked from 32 shared
+1024-token prompts: the step starts with the copy-on-write block copies; its
+roofline counts every shared block once).  --l2-flush empties L2 before every
+step.  Three more rows of the path: `gqa-fp8` (the gqa batch with an FP8 E4M3
 cache: slot mapping + quantising cache write -> decode over codes; KV GB/s of
-1-byte elements) and `prefill` (8 x 2048-token prompts with the same heads:
-slot mapping -> cache write of the prompts' K/V -> causal paged prefill on the
-tensor cores; useful TFLOP/s).
+1-byte elements), `prefill` (8 x 2048-token prompts with the gqa heads: slot
+mapping -> cache write of the prompts' K/V -> causal paged prefill on the
+tensor cores; useful TFLOP/s) and `cow` (the shared step's block copies
+alone).
 
 Prints ONE JSON line (rank 0).  `value` = KV GB/s: the decode's algorithmic
 bytes per step (KV blocks touched + queries + block tables + outputs) over the
@@ -59,10 +66,59 @@ METRIC_PREFILL = "paged-prefill useful TFLOP/s (causal), 8 x 2048-token prompts,
 PREFILL_SHAPE = dict(num_seqs=8, prompt=2048, num_heads=64, num_kv_heads=8, head_dim=128, block_size=16)
 
 
+DECODE_ROWS = ("tiny", "mha", "gqa", "long", "shared")
+ROW_METRICS = {
+    "tiny": "paged-decode KV GB/s and seqs/s, tiny 4 seqs 4q/4kv d64 bs4",
+    "mha": "paged-decode KV GB/s (% of B200 HBM peak) and seqs/s, MHA 32q/32kv d128 b64",
+    "gqa": METRIC,
+    "long": "paged-decode KV GB/s (% of B200 HBM peak) and seqs/s, long-context 32q/8kv d128 b8 L 32K-128K, split-K",
+    "shared": "shared-prefix CoW decode step: KV GB/s (unique and logical) and seqs/s, 256 seqs 32q/8kv d128",
+}
+
+
 def workload_description(w) -> str:
-    return (f"{w.num_seqs} seqs, {w.num_heads} query / {w.num_kv_heads} KV heads, head_dim {w.head_dim}, "
-            f"block_size {w.block_size}, lengths lognormal(median 1024, sigma 0.8) clipped [16, 4096], "
+    heads = (f"{w.num_heads} query / {w.num_kv_heads} KV heads, head_dim {w.head_dim}, "
+             f"block_size {w.block_size}")
+    if w.name == "tiny":
+        return (f"{w.num_seqs} seqs of lengths {{7, 16, 33, 50}}, {heads}, pool of {w.num_blocks} blocks, "
+                "tables drawn without replacement")
+    if w.name == "mha":
+        return f"{w.num_seqs} seqs, {heads}, lengths uniform in [128, 2048], shuffled pool of {w.num_blocks} blocks (1.25x)"
+    if w.name == "long":
+        return (f"{w.num_seqs} seqs, {heads}, lengths uniform in [32768, 131072], shuffled pool of "
+                f"{w.num_blocks} blocks (1.2x)")
+    if w.name == "shared":
+        return (f"{w.num_seqs} seqs = 32 prompts of 1024 tokens x 8 samples (prompt blocks shared), private tails "
+                f"uniform in [1, 256], {heads}, shuffled pool of {w.num_blocks} blocks (1.2x); every sequence "
+                "forked before the step, so its token's write copies the block it lands in")
+    return (f"{w.num_seqs} seqs, {heads}, lengths lognormal(median 1024, sigma 0.8) clipped [16, 4096], "
             f"shuffled pool of {w.num_blocks} blocks (1.2x)")
+
+
+def decode_config(w, world: int, l2_flush: bool) -> dict:
+    """The workload's description: the same dict in both arms."""
+    return {
+        "workload": f"{w.name}: {workload_description(w)}",
+        "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+        "head_dim": w.head_dim, "block_size": w.block_size, "sum_seq_len": int(w.seq_lens.sum()),
+        "max_seq_len": w.max_seq_len,
+        "l2": "flushed before every step (2x L2 written outside the step's events)" if l2_flush else
+              "no flush: each step reads more than L2 (126 MB)" if w.name in ("mha", "gqa", "long", "shared") else
+              "no flush: the tiny working set stays in L2 across steps",
+        "parallelism": f"dp{world}: independent batch per GPU, no collective on the data path",
+    }
+
+
+def unique_bytes(tables, seq_lens, block_size, num_heads, num_kv_heads, head_dim, kv_elem_bytes: int = 2) -> int:
+    """algorithmic_bytes with every physical block counted once, however many
+    sequences' tables point at it (what HBM must supply at least when
+    sequences share blocks)."""
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    blocks = -(-lens // block_size)
+    ids = np.concatenate([np.asarray(tables[s, :blocks[s]]) for s in range(len(lens))]) if len(lens) else []
+    kv = int(np.unique(ids).size) * block_size * num_kv_heads * head_dim * 2 * kv_elem_bytes
+    qo = 2 * len(lens) * num_heads * head_dim * 2
+    return kv + qo + int(blocks.sum()) * 4 + 4 * len(lens)
 
 
 def algorithmic_bytes(seq_lens, block_size, num_heads, num_kv_heads, head_dim, kv_elem_bytes: int = 2) -> int:
@@ -139,7 +195,8 @@ BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 
 class ClockSampler:
     """Samples the SM clock and the clock-event reasons through NVML (the data
-    nvidia-smi reports) every 10 ms on a background thread."""
+    nvidia-smi reports) every 5 ms on a background thread, and on request
+    from the timing thread (sample_now)."""
 
     def __init__(self, cuda_index: int):
         import torch
@@ -178,7 +235,18 @@ class ClockSampler:
                     self.h, self.nv.NVML_CLOCK_SM)), self._reasons()))
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.005)
+
+    def sample_now(self):
+        """One sample from the calling thread: taken inside the timed region
+        right after the steps are enqueued, while the GPU still runs them, so
+        that a timed region shorter than the background period has samples."""
+        if self.ok:
+            try:
+                self.samples.append((time.perf_counter(), float(self.nv.nvmlDeviceGetClockInfo(
+                    self.h, self.nv.NVML_CLOCK_SM)), self._reasons()))
+            except Exception:
+                pass
 
     def start(self):
         if self.ok:
@@ -218,102 +286,131 @@ def aggregate_over_ranks(total_ms, e2e_ms, step_bytes, num_seqs, device, dist=No
     return t, e, b, n
 
 
-def rank_seed(rank: int) -> int:
+def rank_seed(rank: int, name: str = WORKLOAD) -> int:
     """Each rank decodes its own independent batch of the same shape (weak scaling)."""
     from paged_kv_cache_379_b200 import workload as wlmod
-    return wlmod.SEED_BASE + wlmod.NAMES.index(WORKLOAD) + 1000 * rank
+    return wlmod.SEED_BASE + wlmod.NAMES.index(name) + 1000 * rank
 
 
-def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
+def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
+    """One decode row: tiny, mha, gqa (the default line), long or shared.
+
+    Step = [copy-on-write block copies (shared)] -> slot mapping + cache write
+    of each sequence's new token (one launch) -> decode (the library's plan, or
+    the split form at --partition).  Device events around every stage of every
+    timed step; the whole K-step window between barriers gives the step time
+    (with --l2-flush: the sum of the per-step event intervals, the flush
+    writes sitting between them)."""
     import torch
 
     from paged_kv_cache_379_b200 import ops
     from paged_kv_cache_379_b200 import workload as wlmod
-    from paged_kv_cache_379_b200.step import DecodeBatch, bf16_to_device
+    from paged_kv_cache_379_b200.step import DecodeBatch, host_step
 
+    name = args.workload
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     dist = None
     if world > 1:
         import torch.distributed as dist
-    w = wlmod.make(WORKLOAD, seed=rank_seed(rank))
-    batch = DecodeBatch(w, dev)
+    w = wlmod.make(name, seed=rank_seed(rank, name), num_seqs=args.num_seqs or None)
+    tables, pairs_h, cow_h = w.block_tables, None, None
+    if name == "shared":
+        # the host pool's step: every sequence forked, so each token's write into
+        # an existing block takes a copy (the pool's (src, dst) pairs); fused, the
+        # copies run in the cache write's launch from per-sequence sources
+        _, tables, _, slots_h, pairs_h = host_step(w, fork_all=True)
+        if not args.unfused_cow:
+            cow_h = ops.cow_sources(slots_h, w.block_size, pairs_h)
+    batch = DecodeBatch(w, dev, tables=tables, pairs=pairs_h, workspace=False, cow_src=cow_h)
     stream = torch.cuda.current_stream(dev)
-    ws_bytes = 0 if batch.workspace is None else batch.workspace.numel()
-    plan = ops.decode_plan(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, batch.max_seq_len, ws_bytes)
-    launches_per_step = 1 + (2 if plan else 1) + (1 if batch.pairs is not None else 0)
+    part = int(args.partition)
+    if part:
+        ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, part,
+                               device=dev)
+        plan = part
+    else:
+        ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, device=dev)
+        plan = ops.decode_plan(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, ws.numel())
+    n_pairs = 0 if batch.pairs is None else int(batch.pairs.shape[0])
+    fused = batch.cow_src is not None
+    launches_per_step = (1 if n_pairs and not fused else 0) + 1 + (2 if plan else 1)
     step_bytes = algorithmic_bytes(w.seq_lens, w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
+    uniq = unique_bytes(tables, w.seq_lens, w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
+    roof_bytes = uniq if name == "shared" else step_bytes
+    blk_bytes = w.block_size * w.num_kv_heads * w.head_dim * 2
+    copy_bytes = n_pairs * blk_bytes * 2 * 2     # K and V blocks, each read and written
 
+    def device_step(S, ev=None):
+        """One step on input set S (tensors on the device); ev: per-stage events."""
+        if ev is not None:
+            ev[0].record(stream)
+        if S["pairs"] is not None and S["cow"] is None:
+            ops.copy_blocks(batch.key_cache, batch.value_cache, S["pairs"], stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if S["cow"] is not None:
+            ops.append_decode_kv_cow(S["k"], S["v"], batch.key_cache, batch.value_cache, S["bt"], S["sl"],
+                                     S["cow"], slot_mapping=S["slots"], stream=stream)
+        else:
+            ops.append_decode_kv(S["k"], S["v"], batch.key_cache, batch.value_cache, S["bt"], S["sl"],
+                                 slot_mapping=S["slots"], stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        if part:
+            ops.decode_split(S["q"], batch.key_cache, batch.value_cache, S["bt"], S["sl"], w.scale,
+                             batch.max_seq_len, part, ws, out=S["out"], stream=stream)
+        else:
+            ops.decode(S["q"], batch.key_cache, batch.value_cache, S["bt"], S["sl"], w.scale, batch.max_seq_len,
+                       out=S["out"], workspace=ws, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    resident = dict(q=batch.query, k=batch.new_key, v=batch.new_value, bt=batch.block_tables, sl=batch.seq_lens,
+                    pairs=batch.pairs, cow=batch.cow_src, slots=batch.slots, out=batch.out)
     K, W = args.steps, args.warmup
-    ev_d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if args.l2_flush else None
 
-    def decode_timed(i):
-        def fn(b):
-            ev_d0[i].record(stream)
-            ops.decode(b.query, b.key_cache, b.value_cache, b.block_tables, b.seq_lens, w.scale, b.max_seq_len,
-                       out=b.out, workspace=b.workspace, stream=stream)
-            ev_d1[i].record(stream)
-        return fn
-
-    def barrier():
-        torch.cuda.synchronize(dev)
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
+    def step(i):
+        if flush is not None:
+            flush.fill_((0 if i is None else i) & 255)   # evicts the previous step's lines from L2
+        device_step(resident, None if i is None else evs[i])
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    for _ in range(W):
-        batch.run_step(stream=stream)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-
-    def timed_region():
-        barrier()
-        t0 = time.perf_counter()
-        e0.record(stream)
-        for i in range(K):
-            batch.run_step(stream=stream, decode_fn=decode_timed(i))
-        e1.record(stream)
-        barrier()
-        t1 = time.perf_counter()
-        return t0, t1
-
-    t0, t1 = timed_region()
-    clocks = sampler.window(t0, t1)
-    remeasured = False
-    if set(clocks["reasons"]) & BAD_REASONS:
-        first = clocks
-        t0, t1 = timed_region()
-        clocks = sampler.window(t0, t1)
-        clocks["first_attempt"] = first
-        remeasured = True
-    total_ms = e0.elapsed_time(e1)
-    dec_ms = [ev_d0[i].elapsed_time(ev_d1[i]) for i in range(K)]
+    total_ms, clocks, remeasured = _timed_loop(step, K, W, stream, dev, dist, sampler)
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(K)])
+    copy_ms, append_ms, dec_ms = (float(x) for x in stage.mean(axis=0))
+    if flush is not None:
+        total_ms = float(stage.sum())
 
     # e2e: the same step through the C ABI with host buffers.  Every step's
-    # inputs (query, new K/V, block tables, lengths) come from pinned host memory
-    # and its output goes back to pinned host memory inside the timed region.
-    # As a serving loop would, the inputs sit in one pinned staging buffer
-    # (16-byte aligned sections, one copy per step), and the copies run on their
-    # own streams, double buffered: step i+1's inputs go up and step i's output
-    # comes back while step i computes.  The KV cache stays resident.
+    # inputs (query, new K/V, block tables, lengths, copy pairs) come from pinned
+    # host memory and its output goes back to pinned host memory inside the timed
+    # region.  As a serving loop would, the inputs sit in one pinned staging
+    # buffer (16-byte aligned sections, one copy per step), and the copies run on
+    # their own streams, double buffered: step i+1's inputs go up and step i's
+    # output comes back while step i computes.  The KV cache stays resident.
     e2e = None
     if not args.no_e2e:
         parts = [("q", w.query.view(np.int16), torch.bfloat16, batch.query.shape),
                  ("k", w.new_key.view(np.int16), torch.bfloat16, batch.new_key.shape),
                  ("v", w.new_value.view(np.int16), torch.bfloat16, batch.new_value.shape),
-                 ("bt", np.ascontiguousarray(w.block_tables, np.int32), torch.int32, batch.block_tables.shape),
+                 ("bt", np.ascontiguousarray(tables, np.int32), torch.int32, batch.block_tables.shape),
                  ("sl", w.seq_lens.astype(np.int32), torch.int32, batch.seq_lens.shape)]
+        if fused:
+            parts.append(("cow", np.ascontiguousarray(cow_h, np.int32), torch.int32, batch.cow_src.shape))
+        elif n_pairs:
+            parts.append(("pairs", np.ascontiguousarray(pairs_h, np.int64), torch.int64, batch.pairs.shape))
         offs, nbytes_in = {}, 0
-        for name, a, _, _ in parts:
-            offs[name] = (nbytes_in, a.nbytes)
+        for pname, a, _, _ in parts:
+            offs[pname] = (nbytes_in, a.nbytes)
             nbytes_in += -(-a.nbytes // 16) * 16
         h_in = torch.zeros(nbytes_in, dtype=torch.uint8).pin_memory()
         h_np = h_in.numpy()
-        for name, a, _, _ in parts:
-            o, n = offs[name]
+        for pname, a, _, _ in parts:
+            o, n = offs[pname]
             h_np[o:o + n] = np.frombuffer(np.ascontiguousarray(a).tobytes(), np.uint8)
         h_out = [torch.empty(batch.out.shape, dtype=torch.int16).pin_memory() for _ in range(2)]
         h2d = nbytes_in
@@ -321,8 +418,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
 
         def input_set():
             buf = torch.empty(nbytes_in, dtype=torch.uint8, device=dev)
-            S = {name: buf[offs[name][0]:offs[name][0] + offs[name][1]].view(dt).view(shape)
-                 for name, _, dt, shape in parts}
+            S = {pname: buf[offs[pname][0]:offs[pname][0] + offs[pname][1]].view(dt).view(shape)
+                 for pname, _, dt, shape in parts}
+            S.setdefault("pairs", None)
+            S.setdefault("cow", None)
             S.update(buf=buf, slots=torch.empty_like(batch.slots), out=torch.empty_like(batch.out))
             return S
         sets = [input_set() for _ in range(2)]
@@ -340,15 +439,18 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                 S["buf"].copy_(h_in, non_blocking=True)
                 ev_in[b].record(up)
             stream.wait_event(ev_in[b])
-            ops.append_decode_kv(S["k"], S["v"], batch.key_cache, batch.value_cache, S["bt"], S["sl"],
-                                 slot_mapping=S["slots"], stream=stream)
-            ops.decode(S["q"], batch.key_cache, batch.value_cache, S["bt"], S["sl"], w.scale, batch.max_seq_len,
-                       out=S["out"], workspace=batch.workspace, stream=stream)
+            device_step(S)
             ev_done[b].record(stream)
             down.wait_event(ev_done[b])
             with torch.cuda.stream(down):
                 h_out[b].copy_(S["out"].view(torch.int16), non_blocking=True)
                 ev_free[b].record(down)
+
+        def barrier():
+            torch.cuda.synchronize(dev)
+            if dist is not None:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
 
         for i in range(W):
             e2e_step(i)
@@ -361,8 +463,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         down.wait_event(ev_free[(K - 1) % 2])
         f1.record(down)
         barrier()
-        e2e_ms = f0.elapsed_time(f1)
-        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+        e2e = {"ms": f0.elapsed_time(f1), "h2d": h2d, "d2h": d2h}
     sampler.stop()
 
     total_ms, e2e_max_ms, all_bytes, all_seqs = aggregate_over_ranks(
@@ -372,12 +473,17 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
 
     ms_per_step = total_ms / K
     gbs = all_bytes * K / (total_ms * 1e-3) / 1e9
-    dec_avg_ms = float(np.mean(dec_ms))
-    achieved = step_bytes / (dec_avg_ms * 1e-3) / 1e9
+    achieved = roof_bytes / (dec_ms * 1e-3) / 1e9
     peak, peak_src = measured_peak()
-    traffic = profiled_traffic()
+    traffic = profiled_traffic() if (name == "gqa" and not part) else None
+    path = f"split, partition {plan} (partition kernel + LSE reduce)" if plan else "one pass"
+    if fused:
+        step_desc = "append_decode_kv_cow (copy-on-write copies + slot mapping + cache write, one launch) -> decode"
+    else:
+        step_desc = ("copy_blocks (CoW pairs) -> " if n_pairs else "") + \
+            "append_decode_kv (slot mapping + cache write, one launch) -> decode"
     line = {
-        "metric": METRIC,
+        "metric": ROW_METRICS[name] + (f" {part}" if name == "long" and part else ""),
         "value": round(gbs, 2),
         "unit": "GB/s",
         "n_gpus": world,
@@ -388,19 +494,18 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16 values, lognormal lengths, shuffled block pool)",
-        "config": {
-            "workload": f"{WORKLOAD}: {workload_description(w)}",
-            "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
-            "head_dim": w.head_dim, "block_size": w.block_size, "sum_seq_len": int(w.seq_lens.sum()),
-            "max_seq_len": w.max_seq_len, "algorithmic_bytes_per_step": step_bytes,
-            "decode_path": f"split, partition {plan} (partition kernel + LSE reduce)" if plan else "one pass",
-            "step": "append_decode_kv (slot mapping + cache write, one launch) -> decode",
-            "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB read per step vs 126 MB L2); no flush",
-            "parallelism": f"dp{world}: independent batch per GPU, no collective on the data path",
-        },
+        "data": "synthetic (seeded N(0,1) bf16 values, the workload's lengths, shuffled block pool)",
+        "config": decode_config(w, world, bool(args.l2_flush)),
+        "reduced_batch": (f"first {w.num_seqs} sequences only (--num-seqs): a profiling case, not the workload"
+                          if args.num_seqs else None),
+        "decode_path": path + (" (forced by --partition)" if part else " (the library's plan)"),
+        "step": step_desc,
+        "algorithmic_bytes_per_step": step_bytes,
         "seqs_per_s": round(all_seqs * K / (total_ms * 1e-3), 1),
         "frac_of_spec_hbm": round(gbs / world / SPEC_HBM_GBS, 4),
+        "stage_ms": ({"append_decode_kv_cow": round(append_ms, 5), "decode": round(dec_ms, 5)} if fused else
+                     {"copy_blocks": round(copy_ms, 5) if n_pairs else None, "append_decode_kv": round(append_ms, 5),
+                      "decode": round(dec_ms, 5)}),
         "clocks": clocks,
         "gpu_launches": launches_per_step * K,
         "roofline": {
@@ -412,10 +517,21 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
             "frac": round(achieved / peak, 4),
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
             "traffic": traffic,
-            "algorithmic_bytes": step_bytes,
-            "avg_launch_ms": round(dec_avg_ms, 5),
+            "algorithmic_bytes": roof_bytes,
+            "avg_launch_ms": round(dec_ms, 5),
         },
     }
+    if name == "shared":
+        line["roofline"]["bytes_basis"] = ("unique physical bytes: every shared block counted once "
+                                           f"({uniq} of {step_bytes} logical bytes)")
+        line["logical_kv_gbs_decode"] = round(step_bytes / (dec_ms * 1e-3) / 1e9, 2)
+        line["unique_gbs_step"] = round(uniq * world * K / (total_ms * 1e-3) / 1e9, 2)
+        cow_ms = append_ms if fused else copy_ms      # fused: the copies and the 256-row cache write
+        line["copy_on_write"] = {"pairs": n_pairs, "bytes_read_and_written": copy_bytes,
+                                 "fused_with_cache_write": fused,
+                                 "ms": round(cow_ms, 5),
+                                 "gbs": round(copy_bytes / (cow_ms * 1e-3) / 1e9, 2) if cow_ms > 0 else None,
+                                 "share_of_step": round(cow_ms / (copy_ms + append_ms + dec_ms), 4)}
     if remeasured:
         line["clocks_note"] = "first timed region saw a thermal/hw slowdown reason; re-measured once"
     if e2e:
@@ -423,9 +539,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": round(e2e_max_ms / K, 5),
                        "how": "pa_* C-ABI calls on pinned host inputs; host-to-device and device-to-host copies "
-                              "on their own streams, double buffered across steps"}
+                              "on their own streams, double buffered across steps" +
+                              ("; no L2 flush between these steps" if flush is not None else "")}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(w, tables, budget_s=args.cpu_budget)
     return line
 
 
@@ -454,6 +571,7 @@ def _timed_loop(step, K, W, stream, dev, dist, sampler):
         for i in range(K):
             step(i)
         e1.record(stream)
+        sampler.sample_now()           # all steps enqueued; the GPU is still running them
         barrier()
         return t0, time.perf_counter()
 
@@ -694,26 +812,39 @@ def run_cow(args, rank: int, world: int, local_rank: int) -> dict | None:
 
 # ---------------------------------------------------------------- the oracle
 
-def cpu_baseline(w, budget_s: float = 15.0) -> dict:
-    """The oracle (fp64 CPU, as it stands) on a bounded sample of the same workload."""
+def _oracle_decode_rate(w, tables, threads: int, budget_s: float):
+    """The oracle's decode over chunks of the batch's sequences, cycling, until
+    budget_s seconds of oracle time: (bytes/s, seqs/s, sequences, seconds)."""
     import oracle
-    threads = oracle.num_threads()
-    done_bytes, done_seqs, elapsed = 0, 0, 0.0
-    i = 0
-    chunk = 8
+    chunk = max(1, min(8, int(2e5 // max(float(w.seq_lens.mean()), 1.0))))
+    done_bytes, done_seqs, elapsed, i = 0, 0, 0.0, 0
     while elapsed < budget_s:
         idx = (np.arange(chunk) + i) % w.num_seqs
         t = time.perf_counter()
-        oracle.paged_decode(w.query[idx], w.key_cache, w.value_cache, w.block_tables[idx], w.seq_lens[idx],
+        oracle.paged_decode(w.query[idx], w.key_cache, w.value_cache, tables[idx], w.seq_lens[idx],
                             w.scale, threads=threads)
         elapsed += time.perf_counter() - t
         done_bytes += algorithmic_bytes(w.seq_lens[idx], w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
         done_seqs += len(idx)
         i += chunk
-    return {"value": round(done_bytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done_seqs} sequence decodes cycling through the {w.num_seqs}-sequence {WORKLOAD} batch "
-                      f"(decode only), {elapsed:.1f} s, fp64, OpenMP over (sequence, head)",
-            "seqs_per_s": round(done_seqs / elapsed, 2)}
+    return done_bytes / elapsed, done_seqs / elapsed, done_seqs, elapsed
+
+
+def cpu_baseline(w, tables, budget_s: float = 15.0) -> dict:
+    """The oracle (fp64 CPU, as it stands) on a bounded sample of the same
+    workload (tables: the step's block tables): once with OpenMP over
+    (sequence, head) on all host cores, once single-threaded."""
+    import oracle
+    threads = oracle.num_threads()
+    bps, sps, n, el = _oracle_decode_rate(w, tables, threads, budget_s)
+    bps1, sps1, n1, el1 = _oracle_decode_rate(w, tables, 1, max(2.0, budget_s / 3))
+    return {"value": round(bps / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} sequence decodes cycling through the {w.num_seqs}-sequence {w.name} batch "
+                      f"(decode only), {el:.1f} s, fp64, OpenMP over (sequence, head)",
+            "seqs_per_s": round(sps, 2),
+            "single_thread": {"value": round(bps1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "seqs_per_s": round(sps1, 3),
+                              "sample": f"{n1} sequence decodes, {el1:.1f} s, fp64, one thread"}}
 
 
 def cpu_baseline_fp8(w, kc, vc, ks, vs, budget_s: float) -> dict:
@@ -755,20 +886,26 @@ def cpu_baseline_prefill(w, q, budget_s: float) -> dict:
                       f"{elapsed:.1f} s, fp64"}
 
 
-def run_reference(args, rank: int) -> dict | None:
-    """Reference arm: the oracle timed as it stands, each step a bounded sample."""
+def run_reference(args, rank: int, world: int) -> dict | None:
+    """Reference arm: the oracle timed as it stands, each step a bounded sample
+    of the same workload; rank 0 alone runs it."""
     if rank != 0:
         return None
     import oracle
     from paged_kv_cache_379_b200 import workload as wlmod
 
     oracle.build()
-    w = wlmod.make(WORKLOAD)
+    name = args.workload
+    w = wlmod.make(name, seed=rank_seed(0, name), num_seqs=args.num_seqs or None)
+    tables = w.block_tables
+    if name == "shared":   # the step's tables: each token's block exists (fresh or copied)
+        from paged_kv_cache_379_b200.step import host_step
+        _, tables, _, _, _ = host_step(w, fork_all=True)
     threads = oracle.num_threads()
     # sample size per step: one sequence, or more while a step stays short
     per_step_budget = max(0.02, 120.0 / max(args.steps + args.warmup, 1))
     t = time.perf_counter()
-    oracle.paged_decode(w.query[:1], w.key_cache, w.value_cache, w.block_tables[:1], w.seq_lens[:1], w.scale,
+    oracle.paged_decode(w.query[:1], w.key_cache, w.value_cache, tables[:1], w.seq_lens[:1], w.scale,
                         threads=threads)
     one = time.perf_counter() - t
     mean_len = float(w.seq_lens.mean())
@@ -777,7 +914,7 @@ def run_reference(args, rank: int) -> dict | None:
 
     def step(j):
         idx = (np.arange(S) + j * S) % w.num_seqs
-        oracle.paged_decode(w.query[idx], w.key_cache, w.value_cache, w.block_tables[idx], w.seq_lens[idx],
+        oracle.paged_decode(w.query[idx], w.key_cache, w.value_cache, tables[idx], w.seq_lens[idx],
                             w.scale, threads=threads)
         return algorithmic_bytes(w.seq_lens[idx], w.block_size, w.num_heads, w.num_kv_heads, w.head_dim)
 
@@ -789,12 +926,14 @@ def run_reference(args, rank: int) -> dict | None:
         nbytes += step(args.warmup + j)
     dt = time.perf_counter() - t0
     value = nbytes / dt / 1e9
-    sample = f"{S} sequence(s) of the {WORKLOAD} batch per step, cycling; fp64 oracle decode"
+    sample = f"{S} sequence(s) of the {name} batch per step, cycling; fp64 oracle decode"
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "impl": "reference", "metric": ROW_METRICS[name] + (f" {args.partition}" if name == "long" and args.partition
+                                                            else ""), "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": f"{WORKLOAD}: {workload_description(w)}"},
+        "data": "synthetic (seeded N(0,1) bf16 values, the workload's lengths, shuffled block pool)",
+        "config": decode_config(w, world, bool(args.l2_flush)),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -810,18 +949,32 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--workload", choices=["gqa", "gqa-fp8", "prefill", "cow"], default="gqa")
+    ap.add_argument("--workload", choices=list(DECODE_ROWS) + ["gqa-fp8", "prefill", "cow"], default="gqa")
+    ap.add_argument("--partition", type=int, default=0,
+                    help="decode rows: force the split form with this many positions per partition "
+                         "(0 = the library's plan)")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="decode rows: only the first N sequences of the workload (a smaller case for "
+                         "profiler captures; the line then says so)")
+    ap.add_argument("--unfused-cow", action="store_true",
+                    help="shared: the copy-on-write copies as their own launch (pa_copy_blocks) before the "
+                         "cache write, instead of fused into it")
+    ap.add_argument("--l2-flush", action="store_true",
+                    help="decode rows: flush L2 before every step; the step time is then the sum of the "
+                         "per-step event intervals")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.partition and (args.partition < 16 or args.partition % 16):
+        ap.error("--partition must be a positive multiple of 16")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        if args.workload != "gqa":
-            ap.error("--impl reference is the default workload's reference arm")
-        line = run_reference(args, rank)
+        if args.workload not in DECODE_ROWS:
+            ap.error("--impl reference times the oracle's decode: use a decode workload")
+        line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -838,8 +991,8 @@ def main():
     if world > 1:
         dist.barrier()
     try:
-        if args.workload == "gqa":
-            line = run_ours(args, rank, world, local_rank)
+        if args.workload in DECODE_ROWS:
+            line = run_decode(args, rank, world, local_rank)
         elif args.workload == "cow":
             line = run_cow(args, rank, world, local_rank)
         else:

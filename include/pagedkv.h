@@ -123,6 +123,29 @@ int pa_append_decode_kv(const void *key, const void *value, void *key_cache, voi
                         int block_size, int num_blocks, void *stream);
 
 /* --------------------------------------------------------------------------
+ * a3 + a1 + a2 in one launch: the decode step's copy-on-write copies and cache
+ * write ([源码解析 §五] allocate_or_get_cow: a write into a shared block goes to
+ * a new block that first receives the old block's contents; [论文专题
+ * «共享前缀和 copy-on-write»]).  As pa_append_decode_kv, sequence s stores
+ * key[s] / value[s] at its newest position pos = seq_lens[s] - 1, in block
+ * dst = block_tables[s][pos / block_size] (the table already names the new
+ * block), row pos % block_size.  cow_src (int32 [num_seqs], device, or NULL =
+ * no copies): when cow_src[s] >= 0, dst first receives a copy of block
+ * cow_src[s] -- every row but the new token's, which gets the new K/V.  The
+ * caches end up byte for byte as after pa_copy_blocks of the pairs
+ * (cow_src[s], dst) followed by pa_append_decode_kv, in one kernel instead of
+ * two.  cow_src entries outside [0, num_blocks) or equal to dst copy nothing;
+ * a sequence whose slot is -1 (see pa_append_decode_kv) writes nothing.
+ * Precondition: the destinations of sequences with a copy are distinct and are
+ * not copy sources.  pa_cow_sources turns the pool's (src, dst) pairs and the
+ * step's slots into cow_src.  num_seqs <= 65535.
+ * ------------------------------------------------------------------------ */
+int pa_append_decode_kv_cow(const void *key, const void *value, void *key_cache, void *value_cache,
+                            const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cow_src,
+                            int64_t *slot_mapping, int num_seqs, int max_blocks_per_seq, int num_kv_heads,
+                            int head_dim, int block_size, int num_blocks, void *stream);
+
+/* --------------------------------------------------------------------------
  * a3. Copy-on-write block copy ([源码解析 §五] allocate_or_get_cow: a new block
  * receives a copy of the shared one; [深度解析 «Copy-on-Write 与 Prefix Caching»]).
  *   src_dst_pairs: int64 [num_pairs, 2] (device), pair i copies the whole
@@ -369,7 +392,10 @@ int pa_validate_tables(const int32_t *block_tables, const int32_t *seq_lens, int
  * The call allocates no device memory and calls no allocating routine.
  * The first call on each device looks up the array's device address on that
  * device (with the device current); make that first call before any stream
- * capture.  Each call clears the scheduler counters (an asynchronous memset on
+ * capture.  The address is kept per CUDA context (by the context's
+ * process-unique id): after cudaDeviceReset, or any other end of the context
+ * the array was found in, the next call looks it up again in the new context
+ * -- again a set-up call, to be made outside stream capture.  Each call clears the scheduler counters (an asynchronous memset on
  * `stream`) and leaves its partial results in the array.  All calls share the
  * one array: calls that may overlap on the GPU (different streams, or other
  * host threads) race on it and must be serialised by the caller.
@@ -451,6 +477,14 @@ int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, i
                            int64_t *slot_mapping, int64_t *src_dst_pairs, int *num_pairs);
 /* Release every block of the first n entries of a table row. */
 int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n);
+/* Per-sequence copy sources for pa_append_decode_kv_cow (host arrays):
+ * cow_src[s] = the src of the pair (src, dst) of src_dst_pairs (int64
+ * [num_pairs, 2]) whose dst is the block of slot_mapping[s] (slot / block_size),
+ * or -1 when no pair writes that block or the slot is negative.  Returns
+ * PA_ERR_BAD_SHAPE if two pairs share a destination. */
+int pa_cow_sources(const int64_t *slot_mapping, int num_seqs, int block_size, const int64_t *src_dst_pairs,
+                   int num_pairs, int32_t *cow_src);
+
 
 /* Swap planning between two pools (GPU pool and host pool): every distinct
  * block of table[0..n) gets a block in `dst` (reference count = its number of

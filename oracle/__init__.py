@@ -146,6 +146,19 @@ def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, 
                            dst_value_cache.ctypes.data_as(ctypes.c_void_p), skp, svp, prp, pr.shape[0], H, D, bs)
 
 
+def _check_tables(block_tables, seq_lens, block_size: int, num_blocks: int) -> None:
+    """The decode's precondition, checked before the C loop reads a block:
+    every table entry a sequence uses lies in [0, num_blocks)."""
+    bt = np.asarray(block_tables)
+    for s, L in enumerate(np.asarray(seq_lens)):
+        n = -(-int(L) // block_size) if L > 0 else 0
+        if n > bt.shape[1]:
+            raise ValueError(f"sequence {s}: {n} blocks needed, table width {bt.shape[1]}")
+        used = bt[s, :n]
+        if n and (used.min() < 0 or used.max() >= num_blocks):
+            raise ValueError(f"sequence {s}: a table entry outside [0, {num_blocks})")
+
+
 def paged_decode(query, key_cache, value_cache, block_tables, seq_lens, scale: float,
                  threads: int = 1) -> np.ndarray:
     """fp64 [B, Hq, D] output.  query: uint16 bf16 bits [B, Hq, D]."""
@@ -158,6 +171,7 @@ def paged_decode(query, key_cache, value_cache, block_tables, seq_lens, scale: f
     B, Hq, D = q.shape
     nb, bs, Hkv, D2 = kc.shape
     assert D2 == D and Hq % Hkv == 0 and bt.shape[0] == B and sl.shape[0] == B
+    _check_tables(bt, sl, bs, nb)
     out = np.empty((B, Hq, D), dtype=np.float64)
     lib.oracle_paged_decode(out.ctypes.data_as(ctypes.c_void_p), qp, kcp, vcp, btp, slp,
                             float(scale), bs, Hkv, B, Hq, D, bt.shape[1], int(threads))

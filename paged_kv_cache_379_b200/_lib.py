@@ -31,6 +31,7 @@ SIGNATURES = {
                                  _P]),
     "pa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "pa_append_decode_kv": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "pa_append_decode_kv_cow": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "pa_append_decode_kv_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "pa_swap_blocks": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
@@ -56,6 +57,7 @@ SIGNATURES = {
     "pa_pool_cow": (_I, [_P, _I, _P, _P]),
     "pa_pool_import": (_I, [_P, _P, _I, _I, _P]),
     "pa_pool_prepare_decode": (_I, [_P, _I, _P, _I, _P, _P, _P, _P, _P]),
+    "pa_cow_sources": (_I, [_P, _I, _I, _P, _I, _P]),
     "pa_pool_free_table": (_I, [_P, _P, _I]),
     "pa_block_hash": (ctypes.c_uint64, [ctypes.c_uint64, _P, _I]),
     "pa_pool_allocate_prompt_cached": (_I, [_P, _P, _I, _P, _I, _P, _P]),

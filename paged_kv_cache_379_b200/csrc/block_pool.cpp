@@ -236,6 +236,25 @@ int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, i
     return PA_OK;
 }
 
+int pa_cow_sources(const int64_t *slot_mapping, int num_seqs, int block_size, const int64_t *src_dst_pairs,
+                   int num_pairs, int32_t *cow_src)
+{
+    if (num_seqs < 0 || num_pairs < 0 || block_size <= 0) return PA_ERR_BAD_SHAPE;
+    if ((num_seqs > 0 && (!slot_mapping || !cow_src)) || (num_pairs > 0 && !src_dst_pairs))
+        return PA_ERR_NULL_POINTER;
+    std::unordered_map<int64_t, int64_t> src_of;  // dst block -> src block
+    src_of.reserve((size_t)num_pairs * 2);
+    for (int p = 0; p < num_pairs; ++p)
+        if (!src_of.emplace(src_dst_pairs[2 * p + 1], src_dst_pairs[2 * p]).second) return PA_ERR_BAD_SHAPE;
+    for (int s = 0; s < num_seqs; ++s) {
+        cow_src[s] = -1;
+        if (slot_mapping[s] < 0) continue;
+        const auto it = src_of.find(slot_mapping[s] / block_size);
+        if (it != src_of.end()) cow_src[s] = (int32_t)it->second;
+    }
+    return PA_OK;
+}
+
 int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n)
 {
     if (!pool || (n > 0 && !table)) return PA_ERR_NULL_POINTER;

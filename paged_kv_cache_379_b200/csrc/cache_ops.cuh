@@ -143,6 +143,87 @@ __global__ void append_kv_kernel(const uint4 *__restrict__ key, const uint4 *__r
     }
 }
 
+// The decode step's copy-on-write and cache write in one launch
+// ("vLLM 源码解析 …", §五: a write into a shared block goes to a new block that
+// first receives a copy of the old one; "论文专题讲解 …", «共享前缀和
+// copy-on-write»).  Sequence s writes its newest position pos = seq_lens[s] - 1
+// into block dst = block_tables[s][pos / bs] at row o = pos % bs.  When
+// cow_src[s] >= 0, dst is a fresh block that must first hold a copy of block
+// cow_src[s]: every row of cow_src[s] but row o is copied into dst, and row o
+// receives the new K/V -- the bytes that a block copy followed by the cache
+// write leave, with no ordering between the two needed, as no byte is written
+// twice.  Grid: (row slices of the block, sequence); a CTA covers rows
+// [r0, r0 + rows_per_cta) of both caches, one thread per 16-byte chunk with two
+// chunks per cache in flight.  Sequences without a copy only run the CTA that
+// holds row o.
+__global__ void __launch_bounds__(256) append_kv_cow_kernel(
+    const uint4 *__restrict__ key, const uint4 *__restrict__ value, uint4 *__restrict__ key_cache,
+    uint4 *__restrict__ value_cache, const int32_t *__restrict__ block_tables, const int32_t *__restrict__ seq_lens,
+    const int32_t *__restrict__ cow_src, int64_t *__restrict__ slots_out, int max_blocks, int chunks_per_token,
+    int block_size, int rows_per_cta, int64_t num_blocks)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int s = blockIdx.y;
+    const int r0 = blockIdx.x * rows_per_cta;
+    const int r1 = min(block_size, r0 + rows_per_cta);
+    const int64_t pos = (int64_t)seq_lens[s] - 1;
+    int64_t dst = -1, slot = -1;
+    int o = -1;
+    if (pos >= 0) {
+        const int64_t block_number = pos / block_size;
+        if (block_number < max_blocks) {
+            const int32_t physical = block_tables[(int64_t)s * max_blocks + block_number];
+            if (physical >= 0 && physical < num_blocks) {
+                dst = physical;
+                o = (int)(pos - block_number * block_size);
+                slot = dst * block_size + o;
+            }
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0 && slots_out) slots_out[s] = slot;
+    if (dst < 0) return;
+    const int32_t src = cow_src ? cow_src[s] : -1;
+    const bool copy = src >= 0 && src < num_blocks && src != dst;
+    const bool has_row = o >= r0 && o < r1;
+    if (!copy && !has_row) return;
+    const int64_t chunks_per_block = (int64_t)block_size * chunks_per_token;
+    uint4 *kd = key_cache + dst * chunks_per_block;
+    uint4 *vd = value_cache + dst * chunks_per_block;
+    const int64_t c_begin = (int64_t)(copy ? r0 : o) * chunks_per_token;
+    const int64_t c_end = (int64_t)(copy ? r1 : o + 1) * chunks_per_token;
+    const int64_t row_begin = (int64_t)o * chunks_per_token;
+    // copy source (only read when copying) and the new row
+    const uint4 *ks = copy ? key_cache + (int64_t)src * chunks_per_block : kd;
+    const uint4 *vs = copy ? value_cache + (int64_t)src * chunks_per_block : vd;
+    const uint4 *kn = key + (int64_t)s * chunks_per_token;
+    const uint4 *vn = value + (int64_t)s * chunks_per_token;
+    constexpr int U = 2;
+    int64_t c = c_begin + threadIdx.x;
+    for (; c + (U - 1) * blockDim.x < c_end; c += U * blockDim.x) {
+        uint4 k[U], v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t cc = c + u * blockDim.x;
+            const int64_t rc = cc - row_begin;  // chunk within the new row, if it is in it
+            const bool nr = rc >= 0 && rc < chunks_per_token;
+            k[u] = nr ? kn[rc] : ks[cc];
+            v[u] = nr ? vn[rc] : vs[cc];
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            kd[c + u * blockDim.x] = k[u];
+            vd[c + u * blockDim.x] = v[u];
+        }
+    }
+    for (; c < c_end; c += blockDim.x) {
+        const int64_t rc = c - row_begin;
+        const bool nr = rc >= 0 && rc < chunks_per_token;
+        kd[c] = nr ? kn[rc] : ks[c];
+        vd[c] = nr ? vn[rc] : vs[c];
+    }
+}
+
 // One CTA per (pair, slice): copies `per_cta` 16-byte chunks of the source block
 // into the destination block, in both caches, with 4 loads in flight per thread.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ key_cache,

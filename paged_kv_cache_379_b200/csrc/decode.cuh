@@ -91,6 +91,7 @@ constexpr int kChunkSlots = 4;
 constexpr int kChunkBlocks = 32;
 constexpr int kProducerLanes = 4;  // producer lanes issuing consecutive tiles together
 constexpr int kSortKeys = 256;  // size classes (16-token tiles) of the largest-first item order
+constexpr int kLateGrabTiles = 128;  // items of this many tiles or more take their successor late (see below)
 constexpr float kLn2 = 0.693147180559945309f;
 // A column's softmax reference max moves only when a logit exceeds it by more
 // than this (log2 units), so unnormalised weights stay below 2^8.
@@ -351,13 +352,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     // one coalesced pass over the lengths: each sequence's rest key, and its
     // full-partition count parked in pf[s] for the scan below
     if (threadIdx.x == 0) rest_count = 0;
+    for (int k = threadIdx.x; k < kSortKeys; k += kDecodeThreads) sort_base[k] = 0;
     __syncthreads();
     {
+        // ... and the histogram of the rest keys, for the largest-first order
         int nrest = 0;
         for (int s = threadIdx.x; s < B; s += kDecodeThreads) {
             const int L = min(p.seq_lens[s], Lcap);
             const int key = rest_key(L);
             keys[s] = (int16_t)key;
+            if (key >= 0) atomicAdd(&sort_base[key], 1);
             nrest += key >= 0;
             pf[s] = full_of(L);
         }
@@ -394,42 +398,66 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 
     if (warp == kSchedulerWarp) {
         // ------------------------------------------------------------ scheduler
-        // rest pairs sorted by size, largest first: counting sort over kSortKeys
-        // tile-count keys, stable in sequence order (match_any ranks lanes).  When
-        // this CTA's first item is a full partition the sort runs after that item
-        // has been handed to the producer, so the first loads start sooner.
-        auto sort_rest = [&]() {
-            for (int k = lane; k < kSortKeys; k += 32) sort_base[k] = 0;
+        // Rest pairs sorted by size, largest first: a counting sort over
+        // kSortKeys tile-count keys (histogram taken in the pass over the
+        // lengths), stable in sequence order.  The CTA's first item needs only
+        // its own rank, so it is selected from the scanned histogram right away
+        // (its key's bin, then the n-th sequence of that key by ballots) and the
+        // full order is scattered after that item has been handed to the
+        // producer, off the path to the first loads.
+        const int total_items = (total_full + total_rest) * Hkv;
+        int first_rest = -1;   // sequence of this CTA's first item, if that is a rest pair
+        {
+            // exclusive scan in descending key order; lane owns kSortKeys/32 keys
+            constexpr int KPL = kSortKeys / 32;
+            int cnt[KPL], sum = 0;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                cnt[i] = sort_base[kSortKeys - 1 - (lane * KPL + i)];
+                sum += cnt[i];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            int run = incl - sum;
+            const int r = (int)blockIdx.x / Hkv - total_full;   // rest rank of the first item
+            int sel_key = -1, sel_off = 0;
             __syncwarp();
-            for (int c = 0; c < B; c += 32) {
-                const int key = c + lane < B ? keys[c + lane] : -1;
-                if (key >= 0) atomicAdd(&sort_base[key], 1);
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                const int k = kSortKeys - 1 - (lane * KPL + i);
+                if (r >= run && r < run + cnt[i]) {
+                    sel_key = k;
+                    sel_off = r - run;
+                }
+                sort_base[k] = run;
+                run += cnt[i];
             }
             __syncwarp();
-            {
-                // exclusive scan in descending key order; lane owns kSortKeys/32 keys
-                constexpr int KPL = kSortKeys / 32;
-                int cnt[KPL], sum = 0;
-#pragma unroll
-                for (int i = 0; i < KPL; ++i) {
-                    cnt[i] = sort_base[kSortKeys - 1 - (lane * KPL + i)];
-                    sum += cnt[i];
-                }
-                int incl = sum;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += v;
-                }
-                int run = incl - sum;
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < KPL; ++i) {
-                    sort_base[kSortKeys - 1 - (lane * KPL + i)] = run;
-                    run += cnt[i];
+            const unsigned who = __ballot_sync(0xffffffffu, sel_key >= 0);
+            if (who) {
+                const int src = __ffs(who) - 1;
+                sel_key = __shfl_sync(0xffffffffu, sel_key, src);
+                sel_off = __shfl_sync(0xffffffffu, sel_off, src);
+                for (int c = 0; c < B; c += 32) {
+                    const int key = c + lane < B ? keys[c + lane] : -1;
+                    const unsigned m = __ballot_sync(0xffffffffu, key == sel_key);
+                    const int n = __popc(m);
+                    if (sel_off < n) {
+                        const int pre = __popc(m & ((1u << lane) - 1u));
+                        const unsigned hit = __ballot_sync(0xffffffffu, key == sel_key && pre == sel_off);
+                        first_rest = c + __ffs(hit) - 1;
+                        break;
+                    }
+                    sel_off -= n;
                 }
             }
-            __syncwarp();
+        }
+        // stable scatter of the rest pairs into rest_order (match_any ranks lanes)
+        auto scatter_rest = [&]() {
             for (int c = 0; c < B; c += 32) {
                 const int key = c + lane < B ? keys[c + lane] : -1;
                 const unsigned peers = __match_any_sync(0xffffffffu, key);
@@ -441,12 +469,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             }
             __syncwarp();
         };
-        const int total_items = (total_full + total_rest) * Hkv;
         bool sorted = false;
-        if ((int)blockIdx.x >= total_full * Hkv) {
-            sort_rest();
-            sorted = true;
-        }
 
         // Each CTA starts on item blockIdx.x; later items come from the atomic
         // counter (offset by the grid size) or round-robin without a workspace.
@@ -501,7 +524,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     it.s = lo;
                     it.part = sp - pf[lo];
                 } else {
-                    it.s = rest_order[sp - total_full];
+                    // before the scatter, the only rest pair taken is the CTA's first item
+                    it.s = sorted ? rest_order[sp - total_full] : first_rest;
                     it.part = -1;  // the rest pair: after the full partitions
                 }
                 const int L = min(p.seq_lens[it.s], Lcap);
@@ -566,8 +590,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             }
             if (!ok || it.stop) break;
             if (!sorted) {  // before the next item can be a rest pair
-                sort_rest();
+                scatter_rest();
                 sorted = true;
+            }
+            // After an item of kLateGrabTiles tiles or more, the next item is
+            // taken only once the producer has taken this item's last chunk,
+            // i.e. when at most a ring's depth of its tiles is left to consume:
+            // taken at the item's start, it would be reserved long before it
+            // runs, and a CTA that starts on one of the largest items would end
+            // the launch with a medium one; the largest-first order then decides
+            // what runs last.  The next item's queries and table entries still
+            // arrive while the ring drains.  Shorter items keep their successor
+            // one item ahead, which hides its set-up behind the current item.
+            if (it.n_tiles >= kLateGrabTiles && chunk_seq > 0) {
+                const int last = chunk_seq - 1;
+                bool lok = true;
+                if (lane == 0 && (*abort_flag ||
+                                  !mbar_wait_bounded(cempty_bar + 8 * (last % kChunkSlots), (last / kChunkSlots) & 1))) {
+                    if (!*abort_flag) record_timeout(kTimeoutEmptyBarrier);
+                    *abort_flag = 1;
+                    lok = false;
+                }
+                if (!__shfl_sync(0xffffffffu, lok, 0)) break;
             }
             ring_base += it.n_tiles;
             ++item_seq;
@@ -1214,74 +1258,121 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     }
 }
 
-// Log-sum-exp merge of the partitions of one (sequence, head) per warp:
+// Log-sum-exp merge of the partitions of one (sequence, head) row:
 //   M = max_p m_p,  out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p.
 // The partials were just written and sit in L2; the kernel is bound by load
-// latency, so it keeps many loads in flight: lane p reads m_p and l_p (one
-// round), then the o rows of 8 partitions at a time are read together, each as
-// one coalesced 16-byte (D = 128) or 8-byte (D = 64) vector per lane.
+// latency, so it keeps many loads in flight.  WPR warps share a row (a CTA of
+// kReduceWarps warps serves kReduceWarps / WPR rows): warp w of a row takes
+// partitions w, w + WPR, ...; lane i reads m and l of every 32nd of them (one
+// round), then the o rows of 8 of its partitions are read together, each as one
+// coalesced 16-byte (D = 128) or 8-byte (D = 64) vector per lane.  Each warp
+// merges its partitions against its own maximum; the WPR warp states of a row
+// are then merged through shared memory the same way.  WPR = 1 for rows of a
+// few partitions, 8 for rows of many (a 128K-position sequence in 512-token
+// partitions has 256: 4 rounds of 8 loads per warp instead of 32).
 constexpr int kReduceWarps = 8;
 
-template <int D>
+template <int D, int WPR>
 __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const ReduceParams r)
 {
+    static_assert(kReduceWarps % WPR == 0, "warps per row");
     constexpr int VEC = D / 32;
-    constexpr int U = 8;  // partitions whose o rows are in flight together
+    constexpr int U = 8;  // partitions whose o rows are in flight together, per warp
+    __shared__ float sh_acc[kReduceWarps][D];
+    __shared__ float sh_m[kReduceWarps], sh_den[kReduceWarps];
     pdl_wait();
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
-    if (row >= (int64_t)r.num_seqs * r.num_heads) return;
-    const int s = (int)(row / r.num_heads);
-    const int L = r.seq_lens[s];
-    int nparts = L > 0 ? (L + r.part_tokens - 1) / r.part_tokens : 1;
-    nparts = min(nparts, r.max_parts);
-    if (r.skip_single && nparts == 1) return;
-    const float *m = r.ws_m + row * r.max_parts;
-    const float *l = r.ws_l + row * r.max_parts;
-    const float *o = r.ws_o + row * r.max_parts * D + lane * VEC;
-
-    float M = -INFINITY;
-    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, m[i]);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const int warp = threadIdx.x >> 5;
+    const int wr = warp % WPR;  // this warp's share of its row
+    const int64_t row = (int64_t)blockIdx.x * (kReduceWarps / WPR) + warp / WPR;
+    const bool live = row < (int64_t)r.num_seqs * r.num_heads;
+    int nparts = 0;
+    if (live) {
+        const int L = r.seq_lens[row / r.num_heads];
+        nparts = L > 0 ? (L + r.part_tokens - 1) / r.part_tokens : 1;
+        nparts = min(nparts, r.max_parts);
+    }
+    const bool skip = !live || (r.skip_single && nparts == 1);
+    float Mw = -INFINITY, den = 0.f;
     float acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-    float den = 0.f;
-    if (M != -INFINITY) {
-        for (int i = lane; i < nparts; i += 32) {
-            const float mi = m[i];
-            if (mi != -INFINITY) den = fmaf(expf(mi - M), l[i], den);  // an empty partition weighs 0
-        }
+    if (!skip) {
+        const float *m = r.ws_m + row * r.max_parts;
+        const float *l = r.ws_l + row * r.max_parts;
+        const float *o = r.ws_o + row * r.max_parts * D + lane * VEC;
+        // this warp's partitions: j = wr + WPR * k, k = 0 .. mine - 1
+        const int mine = nparts > wr ? (nparts - wr + WPR - 1) / WPR : 0;
+        for (int k = lane; k < mine; k += 32) Mw = fmaxf(Mw, m[wr + WPR * k]);
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-        for (int j0 = 0; j0 < nparts; j0 += U) {
-            float v[U][VEC], w[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int j = j0 + u;
-                w[u] = 0.f;
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
-                if (j < nparts) {
-                    const float mj = m[j];
-                    w[u] = mj != -INFINITY ? expf(mj - M) : 0.f;
-                    const float *src = o + (int64_t)j * D;
-                    if constexpr (VEC == 4) {
-                        const float4 f = *reinterpret_cast<const float4 *>(src);
-                        v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
-                    } else {
-                        const float2 f = *reinterpret_cast<const float2 *>(src);
-                        v[u][0] = f.x; v[u][1] = f.y;
-                    }
-                }
+        for (int off = 16; off >= 1; off >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(0xffffffffu, Mw, off));
+        if (Mw != -INFINITY) {
+            for (int k = lane; k < mine; k += 32) {
+                const int j = wr + WPR * k;
+                const float mj = m[j];
+                if (mj != -INFINITY) den = fmaf(expf(mj - Mw), l[j], den);  // an empty partition weighs 0
             }
 #pragma unroll
-            for (int u = 0; u < U; ++u)
+            for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+            for (int k0 = 0; k0 < mine; k0 += U) {
+                float v[U][VEC], w[U];
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[e] = fmaf(w[u], v[u][e], acc[e]);
+                for (int u = 0; u < U; ++u) {
+                    const int k = k0 + u;
+                    w[u] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
+                    if (k < mine) {
+                        const int j = wr + WPR * k;
+                        const float mj = m[j];
+                        w[u] = mj != -INFINITY ? expf(mj - Mw) : 0.f;
+                        const float *src = o + (int64_t)j * D;
+                        if constexpr (VEC == 4) {
+                            const float4 f = *reinterpret_cast<const float4 *>(src);
+                            v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+                        } else {
+                            const float2 f = *reinterpret_cast<const float2 *>(src);
+                            v[u][0] = f.x; v[u][1] = f.y;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[e] = fmaf(w[u], v[u][e], acc[e]);
+            }
         }
+    }
+    if constexpr (WPR > 1) {
+        // merge the row's warp states: M = max_w M_w, weights e^{M_w - M}
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sh_acc[warp][lane * VEC + e] = acc[e];
+        if (lane == 0) {
+            sh_m[warp] = Mw;
+            sh_den[warp] = den;
+        }
+        __syncthreads();
+        if (skip || wr != 0) return;
+        const int w0 = warp;  // first warp of this row
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < WPR; ++w) M = fmaxf(M, sh_m[w0 + w]);
+        den = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < WPR; ++w) {
+                const float mw = sh_m[w0 + w];
+                const float c = mw != -INFINITY ? expf(mw - M) : 0.f;
+                den = fmaf(c, sh_den[w0 + w], den);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[e] = fmaf(c, sh_acc[w0 + w][lane * VEC + e], acc[e]);
+            }
+        }
+    } else if (skip) {
+        return;
     }
     __nv_bfloat16 *dst = r.out + row * D + lane * VEC;
 #pragma unroll

@@ -189,12 +189,20 @@ static int launch_decode_d(int bs, const DecodeParams &p, const CUtensorMap &tk,
     }
 }
 
+// Rows of more than 32 partitions are merged by a whole CTA (8 warps) each,
+// the others by one warp each.
 static int launch_reduce(const ReduceParams &r, cudaStream_t st)
 {
     const int64_t rows = (int64_t)r.num_seqs * r.num_heads;
-    const dim3 grid((unsigned)cdiv64(rows, kReduceWarps));
-    if (r.head_dim == 64) return launch_pdl(lse_reduce_kernel<64>, grid, dim3(kReduceWarps * 32), 0, st, r);
-    return launch_pdl(lse_reduce_kernel<128>, grid, dim3(kReduceWarps * 32), 0, st, r);
+    const bool wide = r.max_parts > 32;
+    const int rows_per_cta = wide ? 1 : kReduceWarps;
+    if (cdiv64(rows, rows_per_cta) > INT_MAX) return PA_ERR_BAD_SHAPE;
+    const dim3 grid((unsigned)cdiv64(rows, rows_per_cta)), block(kReduceWarps * 32);
+    if (r.head_dim == 64)
+        return wide ? launch_pdl(lse_reduce_kernel<64, kReduceWarps>, grid, block, 0, st, r)
+                    : launch_pdl(lse_reduce_kernel<64, 1>, grid, block, 0, st, r);
+    return wide ? launch_pdl(lse_reduce_kernel<128, kReduceWarps>, grid, block, 0, st, r)
+                : launch_pdl(lse_reduce_kernel<128, 1>, grid, block, 0, st, r);
 }
 
 struct DecodeArgs {
@@ -537,6 +545,32 @@ int pa_append_decode_kv_fp8(const void *key, const void *value, void *key_cache,
                      max_blocks_per_seq, num_kv_heads, head_dim, block_size, num_blocks, k_scale, v_scale, stream);
 }
 
+int pa_append_decode_kv_cow(const void *key, const void *value, void *key_cache, void *value_cache,
+                            const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cow_src,
+                            int64_t *slot_mapping, int num_seqs, int max_blocks_per_seq, int num_kv_heads,
+                            int head_dim, int block_size, int num_blocks, void *stream)
+{
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0)
+        return PA_ERR_BAD_SHAPE;
+    if (num_seqs == 0) return PA_OK;
+    if (!key || !value || !key_cache || !value_cache || !block_tables || !seq_lens) return PA_ERR_NULL_POINTER;
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    if (row % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (num_seqs > 65535) return PA_ERR_BAD_SHAPE;  // one grid row per sequence
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return PA_ERR_ALIGNMENT;
+    const int cpt = (int)(row / 8);
+    // about 1024 chunks (16 KB) of each cache per CTA, whole rows
+    const int rows_per_cta = std::max(1, std::min(block_size, 1024 / std::max(cpt, 1)));
+    const dim3 grid((unsigned)((block_size + rows_per_cta - 1) / rows_per_cta), (unsigned)num_seqs);
+    return launch_pdl(append_kv_cow_kernel, grid, dim3(256), 0, static_cast<cudaStream_t>(stream),
+                      static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
+                      static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), block_tables, seq_lens,
+                      cow_src, slot_mapping, max_blocks_per_seq, cpt, block_size, rows_per_cta,
+                      (int64_t)num_blocks);
+}
+
 int pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *src_dst_pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, void *stream)
 {
@@ -699,6 +733,9 @@ int pa_prefill(void *out, const void *query, const void *key_cache, const void *
         block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
         return PA_ERR_BAD_SHAPE;
     if (num_heads % num_kv_heads != 0) return PA_ERR_BAD_SHAPE;
+    // the softmax takes the row max of the unscaled logits: only a finite,
+    // positive scale keeps that max the max of the scaled ones
+    if (!(scale > 0.f && scale < INFINITY)) return PA_ERR_BAD_SHAPE;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (block_size != 8 && block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
     const int G = num_heads / num_kv_heads;
@@ -743,22 +780,61 @@ int pa_prefill(void *out, const void *query, const void *key_cache, const void *
 // library image, so that the call needs no allocation by anyone.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch on the current device, looked up on the
-// first call per device (host code may not use the symbol itself as a pointer).
+// Device address of g_noalloc_scratch in the current context.  The address is
+// looked up once per context (with the context's device current) and cached
+// under the context's process-unique id: after a device reset the runtime
+// loads the library's module again in a new primary context, where the array
+// may sit elsewhere, and a new id makes the next call look it up again.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+static int current_context_id(unsigned long long *id)
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &a, 12000, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPointByVersion("cuCtxGetId", &b, 12000, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+            get_id = reinterpret_cast<CtxGetIdFn>(b);
+        }
+    });
+    if (!get_current || !get_id) return check_cuda(cudaErrorNotSupported);
+    CUcontext ctx = nullptr;
+    *id = 0;  // 0: no context is current yet
+    if (get_current(&ctx) != CUDA_SUCCESS) return check_cuda(cudaErrorDeviceUninitialized);
+    if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return check_cuda(cudaErrorDeviceUninitialized);
+    return PA_OK;
+}
+
 static int noalloc_scratch(void **ptr)
 {
     static std::mutex mu;
+    static unsigned long long ctx_of[64] = {};
     static void *addr[64] = {};
     int dev = 0;
     int rc = check_cuda(cudaGetDevice(&dev));
     if (rc != PA_OK) return rc;
     if (dev < 0 || dev >= 64) return check_cuda(cudaErrorInvalidDevice);
+    unsigned long long ctx = 0;
+    rc = current_context_id(&ctx);
+    if (rc != PA_OK) return rc;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || ctx == 0 || ctx_of[dev] != ctx) {
+        // the lookup makes the device's primary context current if none was
         void *p = nullptr;
         rc = check_cuda(cudaGetSymbolAddress(&p, g_noalloc_scratch));
         if (rc != PA_OK) return rc;
+        rc = current_context_id(&ctx);
+        if (rc != PA_OK) return rc;
+        if (ctx == 0) return check_cuda(cudaErrorDeviceUninitialized);
         addr[dev] = p;
+        ctx_of[dev] = ctx;
     }
     *ptr = addr[dev];
     return PA_OK;

@@ -18,6 +18,9 @@ Tensor conventions (see include/pagedkv.h):
 
 from __future__ import annotations
 
+import ctypes
+
+import numpy as np
 import torch
 
 from ._lib import PagedKVError, check, load  # noqa: F401
@@ -30,7 +33,8 @@ __all__ = [
     "decode_split", "decode_partitions", "lse_reduce", "decode_workspace_size", "decode_plan",
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
     "decode_split_noalloc", "swap_blocks", "reshape_and_cache_fp8", "decode_fp8", "decode_fp8_split",
-    "prefill", "append_decode_kv", "append_decode_kv_fp8", "selftest_bounded_wait",
+    "prefill", "append_decode_kv", "append_decode_kv_fp8", "selftest_bounded_wait", "append_decode_kv_cow",
+    "cow_sources",
 ]
 
 
@@ -134,6 +138,30 @@ def append_decode_kv(key, value, key_cache, value_cache, block_tables, seq_lens,
     """pa_append_decode_kv: slot of each sequence's newest position + cache write, one launch."""
     a = _append_args(key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping, torch.bfloat16)
     check("pa_append_decode_kv", load().pa_append_decode_kv(*a, _stream(stream)))
+
+
+def append_decode_kv_cow(key, value, key_cache, value_cache, block_tables, seq_lens, cow_src, slot_mapping=None,
+                         stream=None) -> None:
+    """pa_append_decode_kv_cow: the step's copy-on-write copies and cache write,
+    one launch; cow_src int32 [num_seqs] (device): the block each sequence's
+    write block is a copy of, or -1 (see cow_sources)."""
+    a = _append_args(key, value, key_cache, value_cache, block_tables, seq_lens, slot_mapping, torch.bfloat16)
+    cs = _dev(cow_src, torch.int32, "cow_src", 1)
+    if cow_src is not None and cow_src.shape[0] != seq_lens.shape[0]:
+        raise ValueError("cow_src length != num_seqs")
+    check("pa_append_decode_kv_cow", load().pa_append_decode_kv_cow(*a[:6], cs, *a[6:], _stream(stream)))
+
+
+def cow_sources(slot_mapping, block_size: int, src_dst_pairs) -> np.ndarray:
+    """pa_cow_sources (host): per-sequence copy source of the block each slot
+    lies in, from the pool's (src, dst) pairs; -1 where none."""
+    slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    pairs = np.ascontiguousarray(src_dst_pairs, dtype=np.int64).reshape(-1, 2)
+    out = np.empty(slots.shape[0], dtype=np.int32)
+    check("pa_cow_sources", load().pa_cow_sources(
+        slots.ctypes.data_as(ctypes.c_void_p), int(slots.shape[0]), int(block_size),
+        pairs.ctypes.data_as(ctypes.c_void_p), int(pairs.shape[0]), out.ctypes.data_as(ctypes.c_void_p)))
+    return out
 
 
 def append_decode_kv_fp8(key, value, key_cache, value_cache, block_tables, seq_lens, k_scale: float,

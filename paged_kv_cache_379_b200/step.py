@@ -2,7 +2,8 @@
 
 A step is:  slot mapping (a1)  ->  copy-on-write block copies (a3, if any)
             ->  cache write of the new tokens (a2)  ->  decode attention (a4, or
-            the partition kernel a5 + log-sum-exp reduce a6).
+            the partition kernel a5 + log-sum-exp reduce a6); a1-a3 run as one
+            launch (a1 + a2, or a1 + a2 + a3 given per-sequence copy sources).
 Every stage is one call of the C ABI; this module only moves arrays to the
 device and sequences the calls on one stream.  The host-side block-pool work
 of a step (a7: growth and copy-on-write decisions) is `host_step`.
@@ -58,7 +59,7 @@ class DecodeBatch:
     """Device copies of a workload plus the buffers a step writes."""
 
     def __init__(self, wl: Workload, device="cuda", tables: np.ndarray | None = None,
-                 pairs: np.ndarray | None = None, workspace: bool = True):
+                 pairs: np.ndarray | None = None, workspace: bool = True, cow_src: np.ndarray | None = None):
         self.wl = wl
         self.device = torch.device(device)
         self.key_cache = bf16_to_device(wl.key_cache, self.device)
@@ -74,6 +75,10 @@ class DecodeBatch:
         self.pairs = None
         if pairs is not None and len(pairs):
             self.pairs = torch.from_numpy(np.ascontiguousarray(pairs, dtype=np.int64)).to(self.device)
+        # per-sequence copy sources: the step's copies run fused with its cache write
+        self.cow_src = None
+        if cow_src is not None:
+            self.cow_src = torch.from_numpy(np.ascontiguousarray(cow_src, dtype=np.int32)).to(self.device)
         self.max_seq_len = wl.max_seq_len
         self.workspace = None
         if workspace:
@@ -82,12 +87,18 @@ class DecodeBatch:
 
     def run_step(self, stream=None, decode_fn=None):
         """Copy-on-write copies (if any), then the newest token's slot and cache
-        write in one launch, then the decode."""
+        write in one launch, then the decode.  With per-sequence copy sources
+        the copies and the cache write are one launch."""
         wl = self.wl
-        if self.pairs is not None:
-            ops.copy_blocks(self.key_cache, self.value_cache, self.pairs, stream=stream)
-        ops.append_decode_kv(self.new_key, self.new_value, self.key_cache, self.value_cache, self.block_tables,
-                             self.seq_lens, slot_mapping=self.slots, stream=stream)
+        if self.cow_src is not None:
+            ops.append_decode_kv_cow(self.new_key, self.new_value, self.key_cache, self.value_cache,
+                                     self.block_tables, self.seq_lens, self.cow_src, slot_mapping=self.slots,
+                                     stream=stream)
+        else:
+            if self.pairs is not None:
+                ops.copy_blocks(self.key_cache, self.value_cache, self.pairs, stream=stream)
+            ops.append_decode_kv(self.new_key, self.new_value, self.key_cache, self.value_cache, self.block_tables,
+                                 self.seq_lens, slot_mapping=self.slots, stream=stream)
         if decode_fn is None:
             ops.decode(self.query, self.key_cache, self.value_cache, self.block_tables, self.seq_lens,
                        wl.scale, self.max_seq_len, out=self.out, workspace=self.workspace, stream=stream)

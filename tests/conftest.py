@@ -31,3 +31,20 @@ def read_golden(name: str) -> dict:
 @pytest.fixture
 def golden():
     return read_golden
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Observed attention error per comparison: max-abs and max-rel beside the
+    allclose bound |gpu - ref| <= 2e-3 + 1e-2 |ref| the tests apply."""
+    try:
+        from _helpers import ERROR_LOG
+    except ImportError:
+        return
+    if not ERROR_LOG:
+        return
+    tr = terminalreporter
+    tr.section("attention error vs the fp64 oracle (bound: 2e-3 + 1e-2*|ref| per element)")
+    tr.write_line(f"{'comparison':<56} {'elements':>9} {'max_abs':>9} {'max_rel':>9} {'rel|>=.2':>9} "
+                  f"{'err/bound':>9}")
+    for what, n, a, r, rb, q in ERROR_LOG:
+        tr.write_line(f"{what[:56]:<56} {n:>9} {a:>9.3g} {r:>9.3g} {rb:>9.3g} {q:>9.3f}")

@@ -132,6 +132,8 @@ def test_prefill_argument_errors_without_gpu(lib):
     assert call(bs=4) == -3            # block_size not compiled
     assert call(hq=136, hkv=8) == -3   # G = 17 > 16
     assert call(hq=63) == -2           # num_heads not a multiple of num_kv_heads
+    for bad in (0.0, -0.125, float("nan"), float("inf")):
+        assert call(scale=bad) == -2   # the scale must be finite and > 0
     assert call(nb=0) == -2
     assert call(t=0) == 0              # no query rows: nothing to do
     assert call(b=0) == 0

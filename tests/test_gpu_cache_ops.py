@@ -165,3 +165,67 @@ def test_append_decode_kv_fp8_equals_oracle():
     torch.cuda.synchronize()
     assert np.array_equal(dk.cpu().numpy(), ref_k)
     assert np.array_equal(dv.cpu().numpy(), ref_v)
+
+
+# ---- copy-on-write copies + slot mapping + cache write fused (decode form) -----------
+
+def _fused_cow_matches(w, tables, seq_lens, cow_src, slots_ref, pairs_ref):
+    """pa_append_decode_kv_cow against the oracle's block copies of pairs_ref
+    followed by its cache write at slots_ref: caches and slots bit for bit."""
+    ref_k, ref_v = w.key_cache.copy(), w.value_cache.copy()
+    if len(pairs_ref):
+        oracle.copy_blocks(ref_k, ref_v, np.asarray(pairs_ref, np.int64))
+    oracle.reshape_and_cache(w.new_key, w.new_value, ref_k, ref_v, np.asarray(slots_ref, np.int64), w.block_size)
+    kc, vc = bf16_to_device(w.key_cache, DEV), bf16_to_device(w.value_cache, DEV)
+    slots = torch.full((w.num_seqs,), 777, dtype=torch.int64, device=DEV)
+    ops.append_decode_kv_cow(bf16_to_device(w.new_key, DEV), bf16_to_device(w.new_value, DEV), kc, vc,
+                             _i32(tables), _i32(seq_lens), _i32(cow_src), slot_mapping=slots)
+    torch.cuda.synchronize()
+    assert np.array_equal(slots.cpu().numpy(), np.asarray(slots_ref, np.int64))
+    assert np.array_equal(bf16_to_host_bits(kc), ref_k)
+    assert np.array_equal(bf16_to_host_bits(vc), ref_v)
+    assert ops.device_status() == 0
+
+
+@pytest.mark.parametrize("kw,fork_all", [({}, True),
+                                         ({"num_seqs": 8, "shared_prompt_len": 1020, "lengths": [1] * 8}, False)])
+def test_append_decode_kv_cow_equals_copies_then_cache_write(kw, fork_all):
+    """The shared-prefix step through the host pool: every sequence forked (one
+    copy per sequence whose token lands in an existing block), and 8 samples
+    writing into their shared partial prompt block (7 copies, the last owner
+    writes in place)."""
+    w = wl.make("shared", **kw)
+    _, tables, _, slots, pairs = host_step(w, fork_all=fork_all)
+    cow_src = ops.cow_sources(slots, w.block_size, pairs)
+    assert int((cow_src >= 0).sum()) == len(pairs)
+    _fused_cow_matches(w, tables, w.seq_lens, cow_src, slots, pairs)
+
+
+@pytest.mark.parametrize("bs,H,D", [(4, 4, 64), (8, 2, 128), (16, 8, 128), (16, 32, 128)])
+def test_append_decode_kv_cow_edges(bs, H, D):
+    """Random copy sources on small block shapes, with the edge cases: a
+    sequence of length 0 and one with a negative table entry (slot -1: nothing
+    written, nothing copied), a copy source outside the pool and one equal to
+    its destination (no copy), and sequences without a copy."""
+    lens = [1, 5, 0, bs, bs + 1, 3 * bs - 1, 2 * bs, 7, 40, 33]
+    w = wl.random_decode_case(310 + bs + H, num_seqs=len(lens), num_heads=H, num_kv_heads=H, head_dim=D,
+                              block_size=bs, lengths=lens, spare_blocks=12)
+    sl = w.seq_lens.copy()
+    pos = sl.astype(np.int64) - 1
+    slots_ref = oracle.slot_mapping(w.block_tables, np.arange(w.num_seqs, dtype=np.int32), pos, bs)
+    tb = w.block_tables.copy()
+    tb[1, (int(sl[1]) - 1) // bs] = -1                      # slot -1: negative table entry
+    slots_ref[1] = -1
+    assert slots_ref[2] == -1
+    free = list(int(b) for b in w.free_blocks)
+    cow = np.full(w.num_seqs, -1, np.int32)
+    pairs = []
+    # sequences 3..6 copy from distinct spare blocks into their write block; sequence 1
+    # (slot -1) has a source too, which must be ignored
+    for s in (1, 3, 4, 5, 6):
+        cow[s] = free.pop()
+        if slots_ref[s] >= 0:
+            pairs.append((int(cow[s]), int(slots_ref[s] // bs)))
+    cow[7] = w.num_blocks + 5                                 # outside the pool: no copy
+    cow[8] = int(slots_ref[8] // bs)                          # its own destination: no copy
+    _fused_cow_matches(w, tb, sl, cow, slots_ref, pairs)

@@ -44,15 +44,20 @@ def _run(w, kind, partition=512):
 
 # ---- the five workloads, whole step, in the benchmark's launch configuration --------
 
-@pytest.mark.parametrize("name", ["tiny", "mha", "gqa", "long", "shared"])
+@pytest.mark.parametrize("name", ["tiny", "mha", "gqa", "long", "shared", "shared-fused"])
 def test_workload_step_matches_oracle(name):
-    w = wl.make(name)
-    tables, pairs = w.block_tables, None
-    if name == "shared":
+    """The whole step of each workload as the bench runs it (shared: every
+    sequence forked, copy-on-write copies as their own launch, or fused into
+    the cache write's launch)."""
+    w = wl.make(name.split("-")[0])
+    tables, pairs, cow = w.block_tables, None, None
+    if name.startswith("shared"):
         from paged_kv_cache_379_b200.step import host_step
-        _, tables, _, _, pairs = host_step(w, fork_all=True)
+        _, tables, _, slots, pairs = host_step(w, fork_all=True)
+        if name == "shared-fused":
+            cow = ops.cow_sources(slots, w.block_size, pairs)
     poison_tail_slots(w, tables)
-    batch = DecodeBatch(w, DEV, tables=tables, pairs=pairs)
+    batch = DecodeBatch(w, DEV, tables=tables, pairs=pairs, cow_src=cow)
     out = batch.run_step()
     torch.cuda.synchronize()
     ref_k, ref_v, ref_slots, ref_out = oracle_step(w, tables, pairs)
@@ -84,7 +89,25 @@ def test_variants_match_oracle(D, bs, Hq, Hkv):
     ref = oracle.paged_decode(w.query, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, w.scale,
                               threads=0)
     for kind, part in (("one_pass", 0), ("split", 16), ("split", 64), ("split", 512), ("auto", 0)):
-        assert_close(_run(w, kind, part), ref, f"{kind}/{part}")
+        assert_close(_run(w, kind, part), ref, f"D{D} bs{bs} {Hq}/{Hkv} {kind}/{part}")
+
+
+@pytest.mark.parametrize("B", [256, 257, 600])
+def test_batch_sizes_around_the_rank_sort_limit(B):
+    """The work items of a launch are ordered largest first by a block-wide rank
+    sort for batches of up to 256 sequences and by the scheduler warp's
+    counting sort above that: both orders (and the items' split into
+    partitions) against the oracle, ragged lengths with empty sequences."""
+    rng = np.random.default_rng(900 + B)
+    lens = rng.integers(0, 700, B)
+    lens[::37] = 0
+    w = wl.random_decode_case(910 + B, num_seqs=B, num_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                              lengths=lens.tolist(), spare_blocks=4)
+    ref = oracle.paged_decode(w.query, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, w.scale,
+                              threads=0)
+    for kind, part in (("one_pass", 0), ("split", 128), ("auto", 0)):
+        assert_close(_run(w, kind, part), ref, f"B={B} {kind}/{part}")
+    assert ops.device_status() == 0
 
 
 def test_zero_length_and_single_token():
@@ -176,13 +199,39 @@ def test_one_pass_full_gqa_batch_matches_oracle(sched):
     assert ops.device_status() == 0
 
 
-def test_split_and_one_pass_agree_on_long_sequences():
-    w = wl.make("gqa", num_seqs=16)
-    one = _run(w, "one_pass")
-    for part in (256, 512, 1024):
-        split = _run(w, "split", part)
-        a, b = oracle.bf16_bits_to_f64(one), oracle.bf16_bits_to_f64(split)
-        assert np.max(np.abs(a - b)) <= 4e-3
+@pytest.fixture(scope="module")
+def long_case():
+    """The long-context workload (8 sequences of 32K..128K positions, 32 query /
+    8 KV heads) after one step's cache write, and the oracle's output for it."""
+    w = wl.make("long")
+    poison_tail_slots(w)
+    ref_k, ref_v, ref_slots, ref_out = oracle_step(w)
+    return w, ref_k, ref_v, ref_slots, ref_out
+
+
+@pytest.mark.parametrize("partition", [512, 2048])
+def test_long_context_split_matches_oracle(long_case, partition):
+    """The long-context step in the split form at the workload's stated
+    512-token partitions (64..256 partitions per (sequence, head), all merged by
+    the log-sum-exp reduce) and at the 2048 the library's plan picks: the fused
+    slot mapping + cache write, then partition kernel + reduce, against the
+    oracle element by element."""
+    w, ref_k, ref_v, ref_slots, ref_out = long_case
+    batch = DecodeBatch(w, DEV, workspace=False)
+    ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, partition,
+                           device=DEV)
+    ops.append_decode_kv(batch.new_key, batch.new_value, batch.key_cache, batch.value_cache, batch.block_tables,
+                         batch.seq_lens, slot_mapping=batch.slots)
+    out = ops.decode_split(batch.query, batch.key_cache, batch.value_cache, batch.block_tables, batch.seq_lens,
+                           w.scale, w.max_seq_len, partition, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(batch.slots.cpu().numpy(), ref_slots)
+    assert np.array_equal(bf16_to_host_bits(batch.key_cache), ref_k)
+    assert np.array_equal(bf16_to_host_bits(batch.value_cache), ref_v)
+    if partition == 512:  # the reduce merges well over 128 partitions per (sequence, head)
+        assert int(w.seq_lens.max()) > 128 * 512
+    assert_close(bf16_to_host_bits(out), ref_out, f"long, split {partition}")
+    assert ops.device_status() == 0
 
 
 def test_validate_tables():

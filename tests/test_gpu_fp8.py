@@ -148,6 +148,54 @@ def test_decode_fp8_subnormal_and_extreme_codes():
         assert_close(_decode(w, kc, vc, ks, vs, partition), ref, f"extreme codes, partition={partition}")
 
 
+def _wide_range_queries(rng, num_seqs, num_heads, head_dim):
+    """bf16 queries whose heads reach the edges of the FP8 decode's query split
+    (each head is scaled by a power of two so that its largest |q| lies in
+    [128, 256) and split into two E4M3 terms: exact within 2^9 of the largest
+    element, an error below 2^-17 of it further down).  Head kinds, by h % 5:
+      0: one element of magnitude in [2^7, 2^8], the rest log-uniform in
+         [2^-10, 2^7] (a range of up to 2^18);
+      1: one element in [2^7, 2^8], the rest log-uniform in [2^-2, 2^7]
+         (inside 2^9 of the largest: the split is exact);
+      2: every element log-uniform in [2^-14, 2^-8] (scaled up by 2^15..2^22);
+      3: N(0, 1);
+      4: all zeros but one element of 2^-10."""
+    q = np.empty((num_seqs, num_heads, head_dim), np.float32)
+    sign = lambda *shape: rng.choice(np.array([-1.0, 1.0], np.float32), shape)  # noqa: E731
+    for s in range(num_seqs):
+        for h in range(num_heads):
+            kind = h % 5
+            if kind in (0, 1):
+                lo = -10.0 if kind == 0 else -2.0
+                row = sign(head_dim) * np.exp2(rng.uniform(lo, 7.0, head_dim))
+                row[rng.integers(head_dim)] = sign(1)[0] * rng.uniform(128.0, 256.0)
+            elif kind == 2:
+                row = sign(head_dim) * np.exp2(rng.uniform(-14.0, -8.0, head_dim))
+            elif kind == 3:
+                row = rng.standard_normal(head_dim)
+            else:
+                row = np.zeros(head_dim)
+                row[rng.integers(head_dim)] = 2.0 ** -10
+            q[s, h] = row
+    return wl.f32_to_bf16_bits(q)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 1), (16, 2), (5, 5)])
+@pytest.mark.parametrize("partition", [0, 64])
+def test_decode_fp8_wide_range_queries(Hq, Hkv, partition):
+    """Queries with one large element and many small ones, heads of tiny
+    magnitude, and near-zero heads, through the FP8 decode against the
+    oracle, which keeps the exact bf16 query."""
+    lens = [1, 16, 33, 200, 513, 1000]
+    w, kc, vc = _fp8_case(6100 + Hq + Hkv, Hq, Hkv, 16, lens)
+    w.query = _wide_range_queries(np.random.default_rng(6200 + Hq), w.num_seqs, Hq, 128)
+    ks, vs = 0.045, 0.3
+    ref = oracle.paged_decode_fp8(w.query, kc, vc, w.block_tables, w.seq_lens, w.scale, ks, vs, threads=8)
+    got = _decode(w, kc, vc, ks, vs, partition)
+    assert_close(got, ref, f"fp8 wide-range q, G={Hq // Hkv} partition={partition}")
+    assert ops.device_status() == 0
+
+
 def test_write_then_decode_fp8():
     """One decode step on an FP8 cache: the new token is quantised into its slot,
     then read back by the decode."""

@@ -155,3 +155,28 @@ def test_swap_plan_matches_oracle_and_keeps_bookkeeping():
     new3, p3 = swap_plan(g, c, t3 + t3)
     onew3, op3 = o_swap_plan(og, oc, list(t3 + t3))
     assert new3 == onew3 and len(p3) == 1 and c.refcount(new3[0]) == 2
+
+
+def test_cow_sources_matches_brute_force():
+    """pa_cow_sources: each sequence's copy source is the src of the pair whose
+    dst holds its slot; -1 without one or for slot -1; duplicate destinations
+    are rejected."""
+    from paged_kv_cache_379_b200 import ops
+    from paged_kv_cache_379_b200._lib import PagedKVError
+    for kw, fork_all in (({}, True), ({"num_seqs": 8, "shared_prompt_len": 1020, "lengths": [1] * 8}, False)):
+        w = wl.make("shared", fill_cache=False, **kw)
+        _, tables, nblk, slots, pairs = host_step(w, fork_all=fork_all)
+        slots = slots.copy()
+        slots[0] = -1
+        got = ops.cow_sources(slots, w.block_size, pairs)
+        want = []
+        for s in range(w.num_seqs):
+            src = -1
+            for a, b in pairs.tolist():
+                if slots[s] >= 0 and b == slots[s] // w.block_size:
+                    src = a
+            want.append(src)
+        assert got.tolist() == want
+    assert ops.cow_sources(np.array([5, 9], np.int64), 4, np.zeros((0, 2), np.int64)).tolist() == [-1, -1]
+    with pytest.raises(PagedKVError):
+        ops.cow_sources(np.array([5], np.int64), 4, np.array([[1, 2], [3, 2]], np.int64))
