@@ -325,6 +325,13 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
     batch = DecodeBatch(w, dev, tables=tables, pairs=pairs_h, workspace=False, cow_src=cow_h)
     stream = torch.cuda.current_stream(dev)
     part = int(args.partition)
+    groups = None
+    if name == "shared" and not args.no_groups:
+        # the shared prompts are read once per group of sequences (pa_decode_shared),
+        # the host pool's groups at the prompt's length unless --partition says otherwise
+        part = part or 1024
+        gs_h, gp_h = ops.prefix_groups(tables, w.seq_lens, w.block_size, part)
+        groups = (torch.from_numpy(gs_h).to(dev), torch.from_numpy(gp_h).to(dev))
     if part:
         ws = ops.new_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_seq_len, part,
                                device=dev)
@@ -357,7 +364,10 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
                                  slot_mapping=S["slots"], stream=stream)
         if ev is not None:
             ev[2].record(stream)
-        if part:
+        if groups is not None:
+            ops.decode_shared(S["q"], batch.key_cache, batch.value_cache, S["bt"], S["sl"], w.scale,
+                              batch.max_seq_len, part, S["gs"], S["gp"], ws, out=S["out"], stream=stream)
+        elif part:
             ops.decode_split(S["q"], batch.key_cache, batch.value_cache, S["bt"], S["sl"], w.scale,
                              batch.max_seq_len, part, ws, out=S["out"], stream=stream)
         else:
@@ -367,7 +377,8 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
             ev[3].record(stream)
 
     resident = dict(q=batch.query, k=batch.new_key, v=batch.new_value, bt=batch.block_tables, sl=batch.seq_lens,
-                    pairs=batch.pairs, cow=batch.cow_src, slots=batch.slots, out=batch.out)
+                    pairs=batch.pairs, cow=batch.cow_src, slots=batch.slots, out=batch.out,
+                    gs=None if groups is None else groups[0], gp=None if groups is None else groups[1])
     K, W = args.steps, args.warmup
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if args.l2_flush else None
@@ -401,6 +412,9 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
                  ("sl", w.seq_lens.astype(np.int32), torch.int32, batch.seq_lens.shape)]
         if fused:
             parts.append(("cow", np.ascontiguousarray(cow_h, np.int32), torch.int32, batch.cow_src.shape))
+        if groups is not None:
+            parts.append(("gs", gs_h, torch.int32, groups[0].shape))
+            parts.append(("gp", gp_h, torch.int32, groups[1].shape))
         elif n_pairs:
             parts.append(("pairs", np.ascontiguousarray(pairs_h, np.int64), torch.int64, batch.pairs.shape))
         offs, nbytes_in = {}, 0
@@ -422,6 +436,8 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
                  for pname, _, dt, shape in parts}
             S.setdefault("pairs", None)
             S.setdefault("cow", None)
+            S.setdefault("gs", None)
+            S.setdefault("gp", None)
             S.update(buf=buf, slots=torch.empty_like(batch.slots), out=torch.empty_like(batch.out))
             return S
         sets = [input_set() for _ in range(2)]
@@ -477,6 +493,9 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
     peak, peak_src = measured_peak()
     traffic = profiled_traffic() if (name == "gqa" and not part) else None
     path = f"split, partition {plan} (partition kernel + LSE reduce)" if plan else "one pass"
+    if groups is not None:
+        path = (f"shared-prefix groups ({len(gp_h)} groups; the shared {int(gp_h.max())} x {part}-token "
+                f"partitions computed once per KV head for 16 / G sequences at a time) + split, partition {part}")
     if fused:
         step_desc = "append_decode_kv_cow (copy-on-write copies + slot mapping + cache write, one launch) -> decode"
     else:
@@ -498,7 +517,8 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
         "config": decode_config(w, world, bool(args.l2_flush)),
         "reduced_batch": (f"first {w.num_seqs} sequences only (--num-seqs): a profiling case, not the workload"
                           if args.num_seqs else None),
-        "decode_path": path + (" (forced by --partition)" if part else " (the library's plan)"),
+        "decode_path": path + ("" if groups is not None else
+                               " (forced by --partition)" if args.partition else " (the library's plan)"),
         "step": step_desc,
         "algorithmic_bytes_per_step": step_bytes,
         "seqs_per_s": round(all_seqs * K / (total_ms * 1e-3), 1),
@@ -510,7 +530,8 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
         "gpu_launches": launches_per_step * K,
         "roofline": {
             "bound": "hbm",
-            "kernel": "pa_decode (partition kernel + LSE reduce)" if plan else "pa_decode (one-pass kernel)",
+            "kernel": ("pa_decode_shared (partition kernel with shared-prefix items + LSE reduce)" if groups is not None
+                       else "pa_decode (partition kernel + LSE reduce)" if plan else "pa_decode (one-pass kernel)"),
             "achieved": round(achieved, 2),
             "peak": peak,
             "unit": "GB/s",
@@ -956,6 +977,8 @@ def main():
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="decode rows: only the first N sequences of the workload (a smaller case for "
                          "profiler captures; the line then says so)")
+    ap.add_argument("--no-groups", action="store_true",
+                    help="shared: decode without the shared-prefix groups (pa_decode / pa_decode_split)")
     ap.add_argument("--unfused-cow", action="store_true",
                     help="shared: the copy-on-write copies as their own launch (pa_copy_blocks) before the "
                          "cache write, instead of fused into it")

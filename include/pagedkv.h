@@ -247,6 +247,30 @@ int pa_decode_split(void *out, const void *query, const void *key_cache, const v
                     int max_blocks_per_seq, int num_blocks, int max_seq_len, int partition_size,
                     void *workspace, size_t workspace_bytes, void *stream);
 
+/* a5 + a6 with shared prefixes read once per group of sequences.  When
+ * several sequences' tables start with the same blocks -- the prompt blocks
+ * that parallel sampling or a fork leaves shared ([论文专题 «共享前缀和
+ * copy-on-write»]: the samples reference the prompt's blocks; [深度解析
+ * «Copy-on-Write 与 Prefix Caching»]) -- the decode reads those blocks once per
+ * KV head for several sequences at a time instead of once per sequence.
+ * Groups (device arrays, e.g. from pa_prefix_groups): group g is sequences
+ * group_start[g] .. group_start[g+1]-1 (int32 [num_groups + 1]); its first
+ * group_parts[g] partitions (int32 [num_groups]) are computed once for up to
+ * 16 / G of its sequences per work item (G = num_heads / num_kv_heads) and
+ * every later partition per sequence.  The result is that of pa_decode_split
+ * with the same partition_size (same workspace size).  Preconditions: groups
+ * cover sequences 0 .. num_seqs-1 in order; within group g every sequence's
+ * table entries for the first group_parts[g] * partition_size positions equal
+ * those of the group's first sequence, and every sequence's length is at
+ * least group_parts[g] * partition_size (pa_prefix_groups builds such groups).
+ * bf16 caches only (G <= 16). */
+int pa_decode_shared(void *out, const void *query, const void *key_cache, const void *value_cache,
+                     const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
+                     int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                     int num_blocks, int max_seq_len, int partition_size, const int32_t *group_start,
+                     const int32_t *group_parts, int num_groups, void *workspace, size_t workspace_bytes,
+                     void *stream);
+
 /* a5 alone, for inspection: every partition p < ceil(max_seq_len/partition_size)
  * of every (s, h) writes its local result into the workspace, laid out as
  *   the 256-byte scheduler header,
@@ -477,6 +501,20 @@ int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, i
                            int64_t *slot_mapping, int64_t *src_dst_pairs, int *num_pairs);
 /* Release every block of the first n entries of a table row. */
 int pa_pool_free_table(pa_pool *pool, const int32_t *table, int n);
+/* Shared-prefix groups for pa_decode_shared (host arrays): runs of
+ * consecutive sequences whose tables start with the same blocks.  A run starts
+ * at sequence s and takes s+1, s+2, ... while each one shares at least one
+ * whole partition (partition_size positions, a multiple of block_size) with
+ * the run's first sequence: identical table entries over it, and both lengths
+ * covering it.  group_parts[g] = the partitions every member of group g shares
+ * with the first (the minimum over the members; 0 for a sequence shared with
+ * no neighbour).  Outputs group_start (int32 [num_seqs + 1]: group g is
+ * sequences group_start[g] .. group_start[g+1]-1), group_parts (int32
+ * [num_seqs]) and *num_groups; block_tables int32 [num_seqs, max_blocks],
+ * seq_lens int32 [num_seqs]. */
+int pa_prefix_groups(const int32_t *block_tables, int num_seqs, int max_blocks, const int32_t *seq_lens,
+                     int block_size, int partition_size, int32_t *group_start, int32_t *group_parts,
+                     int *num_groups);
 /* Per-sequence copy sources for pa_append_decode_kv_cow (host arrays):
  * cow_src[s] = the src of the pair (src, dst) of src_dst_pairs (int64
  * [num_pairs, 2]) whose dst is the block of slot_mapping[s] (slot / block_size),

@@ -58,6 +58,9 @@ SIGNATURES = {
     "pa_pool_import": (_I, [_P, _P, _I, _I, _P]),
     "pa_pool_prepare_decode": (_I, [_P, _I, _P, _I, _P, _P, _P, _P, _P]),
     "pa_cow_sources": (_I, [_P, _I, _I, _P, _I, _P]),
+    "pa_prefix_groups": (_I, [_P, _I, _I, _P, _I, _I, _P, _P, _P]),
+    "pa_decode_shared": (_I, [_P, _P, _P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _SZ,
+                              _P]),
     "pa_pool_free_table": (_I, [_P, _P, _I]),
     "pa_block_hash": (ctypes.c_uint64, [ctypes.c_uint64, _P, _I]),
     "pa_pool_allocate_prompt_cached": (_I, [_P, _P, _I, _P, _I, _P, _P]),

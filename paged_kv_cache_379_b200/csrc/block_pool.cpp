@@ -19,6 +19,8 @@
 // The free list is a vector used as a stack: the last entry is handed out first,
 // freed blocks are pushed on the end.  Both are O(1).
 
+#include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -233,6 +235,46 @@ int pa_pool_prepare_decode(pa_pool *pool, int num_seqs, int32_t *block_tables, i
         }
         slot_mapping[s] = (int64_t)row[logical] * bs + offset;
     }
+    return PA_OK;
+}
+
+int pa_prefix_groups(const int32_t *block_tables, int num_seqs, int max_blocks, const int32_t *seq_lens,
+                     int block_size, int partition_size, int32_t *group_start, int32_t *group_parts,
+                     int *num_groups)
+{
+    if (num_seqs < 0 || max_blocks <= 0 || block_size <= 0 || partition_size <= 0 ||
+        partition_size % block_size != 0)
+        return PA_ERR_BAD_SHAPE;
+    if (!num_groups || (num_seqs > 0 && (!block_tables || !seq_lens || !group_start || !group_parts)))
+        return PA_ERR_NULL_POINTER;
+    const int bpp = partition_size / block_size;  // blocks per partition
+    // whole partitions that sequences a and b share: equal leading table
+    // entries, within both lengths and both table rows
+    auto shared_parts = [&](int a, int b) -> int {
+        const int64_t la = std::max(seq_lens[a], 0), lb = std::max(seq_lens[b], 0);
+        const int64_t parts = std::min(std::min(la, lb) / partition_size, (int64_t)max_blocks / bpp);
+        const int32_t *ra = block_tables + (int64_t)a * max_blocks;
+        const int32_t *rb = block_tables + (int64_t)b * max_blocks;
+        int64_t blk = 0;
+        while (blk < parts * bpp && ra[blk] == rb[blk] && ra[blk] >= 0) ++blk;
+        return (int)(blk / bpp);
+    };
+    int g = 0, s = 0;
+    while (s < num_seqs) {
+        int parts = INT32_MAX, e = s + 1;
+        while (e < num_seqs) {
+            const int k = shared_parts(s, e);
+            if (k < 1) break;
+            parts = std::min(parts, k);
+            ++e;
+        }
+        group_start[g] = s;
+        group_parts[g] = e > s + 1 ? parts : 0;
+        ++g;
+        s = e;
+    }
+    group_start[g] = num_seqs;
+    *num_groups = g;
     return PA_OK;
 }
 

@@ -70,6 +70,13 @@ struct DecodeParams {
     int part_tokens;                  // positions per partition (multiple of 16); 0 = one pass
     int max_parts;                    // partitions per sequence (workspace stride); 1 = one pass
     int direct_single;                // a sequence with one partition writes `out`
+    // Shared-prefix groups (split form, tensor-core consumers): group g is
+    // sequences grp_start[g] .. grp_start[g+1]-1, whose first grp_parts[g]
+    // partitions are the same blocks; those partitions are computed once per
+    // KV head for up to ROWS / G sequences of the group at a time.
+    const int32_t *grp_start;         // [num_groups + 1] or nullptr
+    const int32_t *grp_parts;         // [num_groups]
+    int num_groups;                   // 0: no groups
 };
 
 struct ReduceParams {
@@ -91,7 +98,6 @@ constexpr int kChunkSlots = 4;
 constexpr int kChunkBlocks = 32;
 constexpr int kProducerLanes = 4;  // producer lanes issuing consecutive tiles together
 constexpr int kSortKeys = 256;  // size classes (16-token tiles) of the largest-first item order
-constexpr int kLateGrabTiles = 128;  // items of this many tiles or more take their successor late (see below)
 constexpr float kLn2 = 0.693147180559945309f;
 // A column's softmax reference max moves only when a logit exceeds it by more
 // than this (log2 units), so unnormalised weights stay below 2^8.
@@ -193,6 +199,9 @@ struct ItemInfo {
     int t_begin, t_end, n_tiles;
     int ring_base;                    // ring position of the item's first tile
     int stop;                         // 1: no more items
+    int nseq;                         // sequences s .. s+nseq-1 of a shared-prefix item; 0 otherwise
+    int ncols;                        // query rows (MMA columns) of the item: nseq * G, or G
+    int single_mask;                  // shared-prefix item: bit i = sequence s+i has this one partition only
 };
 
 // A run of up to 32 blocks of one item for the producer.
@@ -247,11 +256,14 @@ struct DecodeSmem {
     static constexpr int kNumBars = 2 * Ring::kStages + 2 * kItemSlots + 2 * kChunkSlots;
     static constexpr int kFlagOff = kBarOff + kNumBars * 8;
     static constexpr int kPrefixOff = kFlagOff + 16;
-    // bytes of dynamic shared memory for a launch over num_seqs sequences
-    // (enumeration tables: pf[B + 1], rest_order[B], sort bases, int16 keys[B])
-    static constexpr int bytes(int num_seqs)
+    // bytes of dynamic shared memory for a launch over num_seqs sequences and
+    // num_groups shared-prefix groups (enumeration tables: pf[B + 1],
+    // rest_order[B], sort bases, gf[num_groups + 1], int16 keys[B], int16
+    // kshared[B])
+    static constexpr int bytes(int num_seqs, int num_groups = 0)
     {
-        return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys) + ((2 * num_seqs + 3) & ~3);
+        return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys + num_groups + 1) +
+               2 * ((2 * num_seqs + 3) & ~3);
     }
 };
 
@@ -285,6 +297,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     const uint32_t cfull_bar = iempty_bar + kItemSlots * 8;
     const uint32_t cempty_bar = cfull_bar + kChunkSlots * 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Lay::kFlagOff);
+    // ring position up to which the producer has issued tile loads (a hint for
+    // the scheduler's timing only; written by producer lane 0)
+    volatile int *prod_ring = reinterpret_cast<volatile int *>(base_ptr + Lay::kFlagOff + 4);
     int *const prefix = reinterpret_cast<int *>(base_ptr + Lay::kPrefixOff);
 
     const int warp = threadIdx.x >> 5;
@@ -308,6 +323,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             mbar_init(cempty_bar + 8 * i, 1);
         }
         *abort_flag = 0;
+        *prod_ring = 0;
         fence_mbarrier_init();
     }
     if (threadIdx.x == kProducerWarp * 32) {
@@ -333,10 +349,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     // tail of the launch is made of the smallest items).  One pass: no full
     // partitions, every sequence is a rest pair, so sequences go longest first.
     // Item = pair * Hkv + KV head.  pf[s] = full partitions before sequence s.
+    const int NG = p.num_groups;
     int *const pf = prefix;                    // [B + 1]
     int *const rest_order = prefix + B + 1;    // [B]
     int *const sort_base = rest_order + B;     // [kSortKeys]
-    int16_t *const keys = reinterpret_cast<int16_t *>(sort_base + kSortKeys);  // [B] rest keys
+    int *const gf = sort_base + kSortKeys;     // [NG + 1] shared-prefix pairs before group g
+    int16_t *const keys = reinterpret_cast<int16_t *>(gf + NG + 1);  // [B] rest keys
+    int16_t *const kshared = keys + ((B + 1) & ~1);                 // [B] partitions computed by groups
+    constexpr int kColsMax = Lay::ROWS;        // query rows one item holds
+    const int spi = MODE == 0 ? 1 : max(1, kColsMax / max(G, 1));  // sequences per shared-prefix item
     const int Lcap = p.max_blocks * BS;
     auto full_of = [&](int L) {
         return (split && L > 0) ? min(L / p.part_tokens, p.max_parts) : 0;
@@ -349,32 +370,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     };
     __shared__ int warp_tot[kDecodeThreads / 32];
     __shared__ int rest_count;
-    // one coalesced pass over the lengths: each sequence's rest key, and its
-    // full-partition count parked in pf[s] for the scan below
-    if (threadIdx.x == 0) rest_count = 0;
-    for (int k = threadIdx.x; k < kSortKeys; k += kDecodeThreads) sort_base[k] = 0;
-    __syncthreads();
-    {
-        // ... and the histogram of the rest keys, for the largest-first order
-        int nrest = 0;
-        for (int s = threadIdx.x; s < B; s += kDecodeThreads) {
-            const int L = min(p.seq_lens[s], Lcap);
-            const int key = rest_key(L);
-            keys[s] = (int16_t)key;
-            if (key >= 0) atomicAdd(&sort_base[key], 1);
-            nrest += key >= 0;
-            pf[s] = full_of(L);
-        }
-        if (nrest) atomicAdd(&rest_count, nrest);
-    }
-    __syncthreads();
-    if (split) {
-        // block-wide exclusive scan of the full-partition counts
-        const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
-        const int s0 = min(B, (int)threadIdx.x * per);
-        const int s1 = min(B, s0 + per);
+    // block-wide exclusive scan of arr[0..n) in place; arr[n] = the total
+    auto block_scan = [&](int *arr, int n) {
+        const int per = (n + kDecodeThreads - 1) / kDecodeThreads;
+        const int i0 = min(n, (int)threadIdx.x * per);
+        const int i1 = min(n, i0 + per);
         int local = 0;
-        for (int s = s0; s < s1; ++s) local += pf[s];
+        for (int i = i0; i < i1; ++i) local += arr[i];
         int incl = local;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -385,15 +387,50 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         __syncthreads();
         int run = incl - local;
         for (int w = 0; w < warp; ++w) run += warp_tot[w];
-        for (int s = s0; s < s1; ++s) {
-            const int f = pf[s];
-            pf[s] = run;
+        for (int i = i0; i < i1; ++i) {
+            const int f = arr[i];
+            arr[i] = run;
             run += f;
         }
-        if (threadIdx.x == kDecodeThreads - 1) pf[B] = run;
+        if (threadIdx.x == kDecodeThreads - 1) arr[n] = run;
+        __syncthreads();
+    };
+    // one coalesced pass over the lengths: each sequence's rest key, and its
+    // full-partition count parked in pf[s] for the scan below
+    if (threadIdx.x == 0) rest_count = 0;
+    for (int k = threadIdx.x; k < kSortKeys; k += kDecodeThreads) sort_base[k] = 0;
+    // shared-prefix groups: the partitions each sequence's group computes
+    // (kshared), and each group's item pairs (partitions x column blocks)
+    for (int s = threadIdx.x; s < B; s += kDecodeThreads) kshared[s] = 0;
+    __syncthreads();
+    if (split && NG > 0) {
+        for (int gi = threadIdx.x; gi < NG; gi += kDecodeThreads) {
+            const int s0 = p.grp_start[gi], s1 = p.grp_start[gi + 1];
+            const int k = p.grp_parts[gi];
+            for (int s = s0; s < s1; ++s) kshared[s] = (int16_t)k;
+            gf[gi] = k * ((s1 - s0 + spi - 1) / spi);
+        }
     }
     __syncthreads();
+    {
+        // ... and the histogram of the rest keys, for the largest-first order
+        int nrest = 0;
+        for (int s = threadIdx.x; s < B; s += kDecodeThreads) {
+            const int L = min(p.seq_lens[s], Lcap);
+            const int key = rest_key(L);
+            keys[s] = (int16_t)key;
+            if (key >= 0) atomicAdd(&sort_base[key], 1);
+            nrest += key >= 0;
+            pf[s] = max(0, full_of(L) - kshared[s]);
+        }
+        if (nrest) atomicAdd(&rest_count, nrest);
+    }
+    __syncthreads();
+    if (split) block_scan(pf, B);                 // full partitions before sequence s
+    if (split && NG > 0) block_scan(gf, NG);      // shared-prefix pairs before group g
+    __syncthreads();
     const int total_full = split ? pf[B] : 0;
+    const int total_group = (split && NG > 0) ? gf[NG] : 0;   // shared-prefix pairs come first
     const int total_rest = rest_count;
 
     if (warp == kSchedulerWarp) {
@@ -405,7 +442,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         // (its key's bin, then the n-th sequence of that key by ballots) and the
         // full order is scattered after that item has been handed to the
         // producer, off the path to the first loads.
-        const int total_items = (total_full + total_rest) * Hkv;
+        const int total_items = (total_group + total_full + total_rest) * Hkv;
         int first_rest = -1;   // sequence of this CTA's first item, if that is a rest pair
         {
             // exclusive scan in descending key order; lane owns kSortKeys/32 keys
@@ -423,7 +460,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 if (lane >= off) incl += v;
             }
             int run = incl - sum;
-            const int r = (int)blockIdx.x / Hkv - total_full;   // rest rank of the first item
+            const int r = (int)blockIdx.x / Hkv - total_group - total_full;   // rest rank of the first item
             int sel_key = -1, sel_off = 0;
             __syncwarp();
 #pragma unroll
@@ -512,9 +549,41 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             const bool have = idx < total_items;
             ItemInfo it = {};
             int first_blk = 0, end_blk = 0;
-            if (have) {
-                const int sp = idx / Hkv;
-                it.g = idx - sp * Hkv;
+            if (have && idx / Hkv < total_group) {
+                // a shared-prefix pair: partition `part` of group gi for the
+                // sequences of one column block (pairs of a group: partition-major,
+                // so the column blocks of a partition run together)
+                const int gp = idx / Hkv;
+                it.g = idx - gp * Hkv;
+                int lo = 0, hi = NG;  // largest group with gf[g] <= gp
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (gf[mid] <= gp) lo = mid; else hi = mid;
+                }
+                const int s0 = p.grp_start[lo], n = p.grp_start[lo + 1] - s0;
+                const int nblk = (n + spi - 1) / spi;
+                const int local = gp - gf[lo];
+                const int cbk = local % nblk;
+                it.part = local / nblk;
+                it.s = s0 + cbk * spi;
+                it.nseq = min(spi, n - cbk * spi);
+                it.ncols = it.nseq * G;
+                it.nparts = 0;
+                it.single_mask = 0;  // members whose only partition this is write `out` directly
+                for (int i = 0; i < it.nseq; ++i) {
+                    const int Li = min(p.seq_lens[it.s + i], Lcap);
+                    if (full_of(Li) + (rest_key(Li) >= 0 ? 1 : 0) == 1) it.single_mask |= 1 << i;
+                }
+                it.t_begin = it.part * p.part_tokens;
+                it.t_end = it.t_begin + p.part_tokens;   // every member covers the group's partitions
+                it.n_tiles = p.part_tokens / kTileTokens;
+                it.ring_base = ring_base;
+                it.stop = 0;
+                first_blk = it.t_begin / BS;
+                end_blk = (it.t_end + BS - 1) / BS;
+            } else if (have) {
+                const int sp = idx / Hkv - total_group;
+                it.g = idx - (sp + total_group) * Hkv;
                 if (sp < total_full) {
                     int lo = 0, hi = B;  // largest s with pf[s] <= sp
                     while (hi - lo > 1) {
@@ -522,12 +591,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         if (pf[mid] <= sp) lo = mid; else hi = mid;
                     }
                     it.s = lo;
-                    it.part = sp - pf[lo];
+                    it.part = kshared[lo] + sp - pf[lo];   // after the partitions its group computes
                 } else {
                     // before the scatter, the only rest pair taken is the CTA's first item
                     it.s = sorted ? rest_order[sp - total_full] : first_rest;
                     it.part = -1;  // the rest pair: after the full partitions
                 }
+                it.nseq = 0;
+                it.ncols = G;
+                it.single_mask = 0;
                 const int L = min(p.seq_lens[it.s], Lcap);
                 const int f = full_of(L);
                 it.nparts = f + (rest_key(L) >= 0 ? 1 : 0);
@@ -546,10 +618,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 items[islot] = it;
                 const uint32_t bar = ifull_bar + 8 * islot;
                 if (!it.stop) {
+                    // the G query rows of each of the item's sequences, one after another
                     const uint32_t qbytes = (uint32_t)(G * D * 2);
-                    mbar_arrive_expect_tx(bar, qbytes);
-                    bulk_load(base + Lay::kQOff + islot * Lay::kQBytes,
-                              p.query + ((int64_t)it.s * p.num_heads + (int64_t)it.g * G) * D, qbytes, bar);
+                    const int nq = it.nseq > 0 ? it.nseq : 1;
+                    mbar_arrive_expect_tx(bar, qbytes * (uint32_t)nq);
+                    for (int i = 0; i < nq; ++i)
+                        bulk_load(base + Lay::kQOff + islot * Lay::kQBytes + (uint32_t)i * qbytes,
+                                  p.query + ((int64_t)(it.s + i) * p.num_heads + (int64_t)it.g * G) * D, qbytes, bar);
                 } else {
                     mbar_arrive(bar);
                 }
@@ -593,25 +668,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 scatter_rest();
                 sorted = true;
             }
-            // After an item of kLateGrabTiles tiles or more, the next item is
-            // taken only once the producer has taken this item's last chunk,
-            // i.e. when at most a ring's depth of its tiles is left to consume:
-            // taken at the item's start, it would be reserved long before it
-            // runs, and a CTA that starts on one of the largest items would end
-            // the launch with a medium one; the largest-first order then decides
-            // what runs last.  The next item's queries and table entries still
-            // arrive while the ring drains.  Shorter items keep their successor
-            // one item ahead, which hides its set-up behind the current item.
-            if (it.n_tiles >= kLateGrabTiles && chunk_seq > 0) {
-                const int last = chunk_seq - 1;
-                bool lok = true;
-                if (lane == 0 && (*abort_flag ||
-                                  !mbar_wait_bounded(cempty_bar + 8 * (last % kChunkSlots), (last / kChunkSlots) & 1))) {
-                    if (!*abort_flag) record_timeout(kTimeoutEmptyBarrier);
-                    *abort_flag = 1;
-                    lok = false;
+            // The next item is taken only when the producer is within a ring's
+            // depth (kStages tiles) of this item's end -- with the ring full, about
+            // two rings' worth of tiles before the consumers finish it: late
+            // enough that an item is not reserved long before it runs (a CTA that
+            // starts on one of the largest items would otherwise end the launch
+            // with the medium item it took at the start), so the largest-first
+            // order decides what runs last; early enough that the next item's
+            // queries and table entries arrive before the ring drains.  Items
+            // shorter than the lookahead keep their successor one item ahead.
+            {
+                const int target = ring_base + it.n_tiles - kStages;
+                bool gok = true;
+                if (lane == 0 && *prod_ring < target) {
+                    const unsigned long long t0 = global_timer_ns();
+                    while (*prod_ring < target) {
+                        if (*abort_flag) {
+                            gok = false;
+                            break;
+                        }
+                        if (global_timer_ns() - t0 > kWaitLimitNs) {
+                            record_timeout(kTimeoutEmptyBarrier);
+                            *abort_flag = 1;
+                            gok = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
                 }
-                if (!__shfl_sync(0xffffffffu, lok, 0)) break;
+                if (!__shfl_sync(0xffffffffu, gok, 0)) break;
             }
             ring_base += it.n_tiles;
             ++item_seq;
@@ -680,6 +765,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         }
                     }
                     ring += min(kProducerLanes, ntiles - t0);
+                    if (lane == 0) *prod_ring = ring;
                 }
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(cempty_bar + 8 * cslot);
@@ -893,7 +979,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             for (int hh = 0; hh < 2; ++hh) {
                                 const int col = 16 * (tq + 4 * (kk >> 1)) + 8 * (kk & 1) + 4 * hh;
                                 uint2 w = make_uint2(0u, 0u);
-                                if (head < G) w = *reinterpret_cast<const uint2 *>(qsm + (head * D + col) * 2);
+                                if (head < it.ncols) w = *reinterpret_cast<const uint2 *>(qsm + (head * D + col) * 2);
                                 const float2 f0 = unpack_bf16x2(w.x), f1 = unpack_bf16x2(w.y);
                                 v[kk][hh][0] = f0.x;
                                 v[kk][hh][1] = f0.y;
@@ -946,7 +1032,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             for (int hh = 0; hh < 2; ++hh) {
                                 const int col = kk * 16 + hh * 8 + tq * 2;
                                 qb[nh][kk][hh] =
-                                    head < G ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
+                                    head < it.ncols ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
                             }
                         }
                         qscale[nh][0] = qscale[nh][1] = p.scale_log2;
@@ -968,6 +1054,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 const int kpar = lane >> 4;
                 const int vtok = (lane & 7) + ((lane >> 4) << 3);
                 const int vpar = (lane >> 3) & 1;
+                // 8-column tiles with a query row (two only for items of more than 8)
+                const int nh_used = NH == 1 ? 1 : (it.ncols + 7) / 8;
 
                 for (int j = warp; j < it.n_tiles; j += kConsumerWarps) {
                     const int ring = it.ring_base + j;
@@ -1019,7 +1107,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
 #pragma unroll
                             for (int nh = 0; nh < NH; ++nh)
-                                mma_bf16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                                if (nh < nh_used)
+                                    mma_bf16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
                         }
                     }
 #pragma unroll
@@ -1122,8 +1211,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * mt + vpar), a0, a1, a2, a3);
 #pragma unroll
                             for (int nh = 0; nh < NH; ++nh) {
-                                mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
-                                mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
+                                if (nh < nh_used) {
+                                    mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
+                                    mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
+                                }
                             }
                         }
                     }
@@ -1146,7 +1237,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         const int head = nh * 8 + 2 * tq + jj;
-                        if (head < G) {
+                        if (head < it.ncols) {
 #pragma unroll
                             for (int mt = 0; mt < MT; ++mt) {
                                 const int d0 = FP8 ? 16 * gq + 2 * mt : mt * 16 + gq;
@@ -1169,7 +1260,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             const bool direct = p.direct_single && it.nparts == 1;
             // per head row: the combined true max is the common reference (every
             // warp's own reference is <= it, so the weights are <= 1)
-            if (threadIdx.x < G) {
+            const int ncols = MODE == 0 ? G : it.ncols;
+            if (threadIdx.x < ncols) {
                 const int row = threadIdx.x;
                 float M = -INFINITY;
 #pragma unroll
@@ -1188,7 +1280,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             consumer_bar();
             // weighted sum of the four accumulators, 4 columns per thread
             constexpr int D4 = D / 4;
-            for (int idx = threadIdx.x; idx < G * D4; idx += kConsumerWarps * 32) {
+            for (int idx = threadIdx.x; idx < ncols * D4; idx += kConsumerWarps * 32) {
                 const int row = idx / D4;
                 const int d = (idx - row * D4) * 4;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1201,13 +1293,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     acc.z = fmaf(c, v.z, acc.z);
                     acc.w = fmaf(c, v.w, acc.w);
                 }
-                const int64_t hrow = (int64_t)it.s * p.num_heads + (int64_t)it.g * G + row;
+                // query row: column `row` of a shared-prefix item is head row % G of
+                // its sequence row / G
+                const int64_t hrow = (int64_t)(it.s + row / G) * p.num_heads + (int64_t)it.g * G + row % G;
+                const bool direct_row = direct || (p.direct_single && ((it.single_mask >> (row / G)) & 1));
                 const float den = ms->den[row];
                 acc.x *= p.v_scale;
                 acc.y *= p.v_scale;
                 acc.z *= p.v_scale;
                 acc.w *= p.v_scale;
-                if (direct) {
+                if (direct_row) {
                     const float inv = den > 0.f ? 1.f / den : 0.f;
                     uint2 packed;
                     packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);

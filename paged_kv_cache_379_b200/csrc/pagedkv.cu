@@ -142,7 +142,7 @@ static int launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const C
 {
     using Lay = DecodeSmem<D, BS, MODE, GC, FP8>;
     auto kernel = paged_decode_kernel<D, BS, MODE, GC, FP8>;
-    const size_t smem = (size_t)Lay::bytes(p.num_seqs);
+    const size_t smem = (size_t)Lay::bytes(p.num_seqs, p.num_groups);
     if (smem > 227 * 1024) return PA_ERR_BAD_SHAPE;  // too many sequences for the enumeration tables
     int rc = ensure_smem(reinterpret_cast<const void *>(kernel), smem);
     if (rc != PA_OK) return rc;
@@ -160,6 +160,8 @@ static int launch_decode_bs(const DecodeParams &p, const CUtensorMap &tk, const 
                             cudaStream_t st)
 {
     const int G = p.group;
+    // shared-prefix groups: 16-column tensor-core items, ROWS / G sequences each
+    if (p.num_groups > 0) return G <= 16 ? launch_decode_t<D, BS, 2, 0>(p, tk, tv, grid, st) : PA_ERR_UNSUPPORTED;
     if (G == 1) return launch_decode_t<D, BS, 0, 1>(p, tk, tv, grid, st);
     if (G == 2) return launch_decode_t<D, BS, 0, 2>(p, tk, tv, grid, st);
     if (G <= 8) return launch_decode_t<D, BS, 1, 0>(p, tk, tv, grid, st);
@@ -213,6 +215,8 @@ struct DecodeArgs {
     int block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks, num_blocks, max_seq_len;
     bool fp8 = false;             // caches hold E4M3 codes
     float k_scale = 1.f, v_scale = 1.f;
+    const int32_t *grp_start = nullptr, *grp_parts = nullptr;  // shared-prefix groups (device)
+    int num_groups = 0;
 };
 
 static int check_decode_args(const DecodeArgs &a, bool need_out)
@@ -302,6 +306,9 @@ static int run_decode(const DecodeArgs &a, int mode, int part, void *ws, size_t 
         p.ws_o = L.o;
         p.ws_m = L.m;
         p.ws_l = L.l;
+        p.grp_start = a.grp_start;
+        p.grp_parts = a.grp_parts;
+        p.num_groups = a.num_groups;
     }
     const int64_t max_items = (int64_t)p.max_parts * a.num_seqs * a.num_kv_heads;
     if (max_items > INT_MAX) return PA_ERR_BAD_SHAPE;
@@ -685,6 +692,23 @@ int pa_decode_split(void *out, const void *query, const void *key_cache, const v
 {
     const DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
                           num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    return run_decode(a, 1, partition_size, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pa_decode_shared(void *out, const void *query, const void *key_cache, const void *value_cache,
+                     const int32_t *block_tables, const int32_t *seq_lens, float scale, int block_size,
+                     int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                     int num_blocks, int max_seq_len, int partition_size, const int32_t *group_start,
+                     const int32_t *group_parts, int num_groups, void *workspace, size_t workspace_bytes,
+                     void *stream)
+{
+    DecodeArgs a = {out, query, key_cache, value_cache, block_tables, seq_lens, scale, block_size,
+                    num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len};
+    if (num_groups < 0 || num_groups > num_seqs) return PA_ERR_BAD_SHAPE;
+    if (num_groups > 0 && (!group_start || !group_parts)) return PA_ERR_NULL_POINTER;
+    a.grp_start = group_start;
+    a.grp_parts = group_parts;
+    a.num_groups = num_groups;
     return run_decode(a, 1, partition_size, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 

@@ -34,7 +34,7 @@ __all__ = [
     "validate_tables", "device_status", "PagedKVError", "new_workspace", "workspace_views",
     "decode_split_noalloc", "swap_blocks", "reshape_and_cache_fp8", "decode_fp8", "decode_fp8_split",
     "prefill", "append_decode_kv", "append_decode_kv_fp8", "selftest_bounded_wait", "append_decode_kv_cow",
-    "cow_sources",
+    "cow_sources", "prefix_groups", "decode_shared",
 ]
 
 
@@ -162,6 +162,22 @@ def cow_sources(slot_mapping, block_size: int, src_dst_pairs) -> np.ndarray:
         slots.ctypes.data_as(ctypes.c_void_p), int(slots.shape[0]), int(block_size),
         pairs.ctypes.data_as(ctypes.c_void_p), int(pairs.shape[0]), out.ctypes.data_as(ctypes.c_void_p)))
     return out
+
+
+def prefix_groups(block_tables, seq_lens, block_size: int, partition_size: int):
+    """pa_prefix_groups (host): runs of consecutive sequences sharing leading
+    partitions.  Returns (group_start int32 [G+1], group_parts int32 [G])."""
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B = int(sl.shape[0])
+    start = np.empty(B + 1, dtype=np.int32)
+    parts = np.empty(max(B, 1), dtype=np.int32)
+    n = ctypes.c_int(0)
+    check("pa_prefix_groups", load().pa_prefix_groups(
+        bt.ctypes.data_as(ctypes.c_void_p), B, int(bt.shape[1]) if bt.ndim == 2 else 1,
+        sl.ctypes.data_as(ctypes.c_void_p), int(block_size), int(partition_size),
+        start.ctypes.data_as(ctypes.c_void_p), parts.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)))
+    return start[:n.value + 1].copy(), parts[:n.value].copy()
 
 
 def append_decode_kv_fp8(key, value, key_cache, value_cache, block_tables, seq_lens, k_scale: float,
@@ -335,6 +351,25 @@ def decode_split(query, key_cache, value_cache, block_tables, seq_lens, scale: f
     check("pa_decode_split", lib.pa_decode_split(
         o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), bs, hkv, B, hq, d, mb, nb,
         int(max_seq_len), int(partition_size), wp, wb, _stream(stream)))
+    return out
+
+
+def decode_shared(query, key_cache, value_cache, block_tables, seq_lens, scale: float, max_seq_len: int,
+                  partition_size: int, group_start, group_parts, workspace, *, out=None, stream=None):
+    """pa_decode_shared: the split decode with shared-prefix groups (int32 device
+    tensors group_start [G+1], group_parts [G]; see prefix_groups)."""
+    lib = load()
+    q, bt, sl, B, hq, hkv, d, bs, nb, mb = _decode_common(query, key_cache, value_cache, block_tables, seq_lens)
+    o, out = _out(out, query)
+    wp, wb = _ws(workspace)
+    gs = _dev(group_start, torch.int32, "group_start", 1)
+    gp = _dev(group_parts, torch.int32, "group_parts", 1)
+    ng = int(group_parts.shape[0])
+    if group_start.shape[0] != ng + 1:
+        raise ValueError("group_start must have num_groups + 1 entries")
+    check("pa_decode_shared", lib.pa_decode_shared(
+        o, q, key_cache.data_ptr(), value_cache.data_ptr(), bt, sl, float(scale), bs, hkv, B, hq, d, mb, nb,
+        int(max_seq_len), int(partition_size), gs, gp, ng, wp, wb, _stream(stream)))
     return out
 
 

@@ -20,6 +20,20 @@ def test_algorithmic_bytes_hand_case():
     assert bench.algorithmic_bytes([0], 16, 8, 8, 128) == 2 * 8 * 128 * 2 + 4
 
 
+def test_unique_bytes_counts_shared_blocks_once():
+    # two sequences of 5 and 7 positions, block size 4, sharing their first block
+    # (id 3): blocks touched 2 + 2, distinct 3; 2 query / 2 KV heads, head_dim 8
+    tables = np.array([[3, 5], [3, 6]], np.int32)
+    got = bench.unique_bytes(tables, [5, 7], 4, 2, 2, 8)
+    kv = 3 * 4 * 2 * 8 * 2 * 2
+    q_and_out = 2 * 2 * 2 * 8 * 2
+    tables_and_lens = 4 * 4 + 2 * 4
+    assert got == kv + q_and_out + tables_and_lens
+    # without sharing it equals the algorithmic bytes
+    assert bench.unique_bytes(np.array([[1, 2], [3, 4]], np.int32), [5, 7], 4, 2, 2, 8) == \
+        bench.algorithmic_bytes([5, 7], 4, 2, 2, 8)
+
+
 def test_prefill_flops_matches_brute_force():
     rng = np.random.default_rng(3)
     for _ in range(20):
@@ -48,12 +62,29 @@ def test_code_hash_ignores_comments_and_layout_only():
 def test_reference_arm_prints_one_contract_line():
     """`bench.py --impl reference` times the oracle on the host and prints one
     JSON line with the contract's keys (no GPU needed)."""
-    import json
     import subprocess
     import sys
 
     r = subprocess.run([sys.executable, bench.__file__, "--impl", "reference", "--steps", "3", "--warmup", "3"],
                        capture_output=True, text=True, timeout=600)
+    _check_reference_line(r)
+
+
+def test_reference_arm_on_the_shared_prefix_step():
+    """The reference arm decodes the shared-prefix step with the step's tables
+    (each token's block present: fresh or copied), on a small batch."""
+    import subprocess
+    import sys
+
+    r = subprocess.run([sys.executable, bench.__file__, "--impl", "reference", "--workload", "shared",
+                        "--num-seqs", "16", "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600)
+    d = _check_reference_line(r)
+    assert d["config"]["num_seqs_per_gpu"] == 16
+
+
+def _check_reference_line(r):
+    import json
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -64,3 +95,4 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["steps"] == 3 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    return d

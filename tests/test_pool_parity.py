@@ -180,3 +180,51 @@ def test_cow_sources_matches_brute_force():
     assert ops.cow_sources(np.array([5, 9], np.int64), 4, np.zeros((0, 2), np.int64)).tolist() == [-1, -1]
     with pytest.raises(PagedKVError):
         ops.cow_sources(np.array([5], np.int64), 4, np.array([[1, 2], [3, 2]], np.int64))
+
+
+def _groups_brute_force(tables, lens, bs, part):
+    """The grouping rule written out: a run takes the next sequence while it
+    shares at least one whole partition with the run's first sequence; the
+    group's partitions are the minimum shared by its members (0 alone)."""
+    bpp = part // bs
+
+    def shared(a, b):
+        n = min(lens[a], lens[b]) // part
+        k = 0
+        while k < n and all(tables[a][k * bpp + j] == tables[b][k * bpp + j] >= 0 for j in range(bpp)):
+            k += 1
+        return k
+    start, parts, s = [], [], 0
+    while s < len(lens):
+        e, k = s + 1, None
+        while e < len(lens) and shared(s, e) >= 1:
+            k = shared(s, e) if k is None else min(k, shared(s, e))
+            e += 1
+        start.append(s)
+        parts.append(k or 0)
+        s = e
+    return start + [len(lens)], parts
+
+
+def test_prefix_groups_matches_brute_force():
+    from paged_kv_cache_379_b200 import ops
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        bs = int(rng.choice([4, 8, 16]))
+        part = bs * int(rng.integers(1, 4))
+        B = int(rng.integers(1, 12))
+        width = 12
+        tables = rng.integers(0, 50, (B, width)).astype(np.int32)
+        for s in range(1, B):             # copy a random prefix of the previous row now and then
+            if rng.random() < 0.6:
+                n = int(rng.integers(0, width + 1))
+                tables[s, :n] = tables[s - 1, :n]
+        lens = rng.integers(0, width * bs + 1, B).astype(np.int32)
+        gs, gp = ops.prefix_groups(tables, lens, bs, part)
+        ws, wp = _groups_brute_force(tables.tolist(), lens.tolist(), bs, part)
+        assert gs.tolist() == ws and gp.tolist() == wp, trial
+    # the shared-prefix workload after the fork and the step's copies: 32 groups of 8
+    w = wl.make("shared", fill_cache=False)
+    _, tables, _, _, _ = host_step(w, fork_all=True)
+    gs, gp = ops.prefix_groups(tables, w.seq_lens, w.block_size, 512)
+    assert gs.tolist() == list(range(0, 257, 8)) and gp.tolist() == [2] * 32
