@@ -262,7 +262,7 @@ struct DecodeSmem {
     // kshared[B])
     static constexpr int bytes(int num_seqs, int num_groups = 0)
     {
-        return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys + num_groups + 1) +
+        return 1024 + kPrefixOff + 4 * (2 * num_seqs + 1 + kSortKeys + 2 * (num_groups + 1)) +
                2 * ((2 * num_seqs + 3) & ~3);
     }
 };
@@ -354,7 +354,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     int *const rest_order = prefix + B + 1;    // [B]
     int *const sort_base = rest_order + B;     // [kSortKeys]
     int *const gf = sort_base + kSortKeys;     // [NG + 1] shared-prefix pairs before group g
-    int16_t *const keys = reinterpret_cast<int16_t *>(gf + NG + 1);  // [B] rest keys
+    int *const gstart = gf + NG + 1;           // [NG + 1] first sequence of group g
+    int16_t *const keys = reinterpret_cast<int16_t *>(gstart + NG + 1);  // [B] rest keys
     int16_t *const kshared = keys + ((B + 1) & ~1);                 // [B] partitions computed by groups
     constexpr int kColsMax = Lay::ROWS;        // query rows one item holds
     const int spi = MODE == 0 ? 1 : max(1, kColsMax / max(G, 1));  // sequences per shared-prefix item
@@ -400,18 +401,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     if (threadIdx.x == 0) rest_count = 0;
     for (int k = threadIdx.x; k < kSortKeys; k += kDecodeThreads) sort_base[k] = 0;
     // shared-prefix groups: the partitions each sequence's group computes
-    // (kshared), and each group's item pairs (partitions x column blocks)
+    // (kshared), each group's item pairs (partitions x column blocks) and first
+    // sequence -- read together with the lengths below, one round of loads
+    const bool groups = split && NG > 0;
     for (int s = threadIdx.x; s < B; s += kDecodeThreads) kshared[s] = 0;
     __syncthreads();
-    if (split && NG > 0) {
-        for (int gi = threadIdx.x; gi < NG; gi += kDecodeThreads) {
-            const int s0 = p.grp_start[gi], s1 = p.grp_start[gi + 1];
+    if (groups) {
+        for (int gi = threadIdx.x; gi <= NG; gi += kDecodeThreads) {
+            const int s0 = p.grp_start[gi];
+            gstart[gi] = s0;
+            if (gi == NG) continue;
+            const int s1 = p.grp_start[gi + 1];
             const int k = p.grp_parts[gi];
             for (int s = s0; s < s1; ++s) kshared[s] = (int16_t)k;
             gf[gi] = k * ((s1 - s0 + spi - 1) / spi);
         }
     }
-    __syncthreads();
     {
         // ... and the histogram of the rest keys, for the largest-first order
         int nrest = 0;
@@ -421,10 +426,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             keys[s] = (int16_t)key;
             if (key >= 0) atomicAdd(&sort_base[key], 1);
             nrest += key >= 0;
-            pf[s] = max(0, full_of(L) - kshared[s]);
+            pf[s] = full_of(L);
         }
         if (nrest) atomicAdd(&rest_count, nrest);
     }
+    __syncthreads();
+    if (groups)  // the partitions a sequence's group computes are not its own
+        for (int s = threadIdx.x; s < B; s += kDecodeThreads) pf[s] = max(0, pf[s] - kshared[s]);
     __syncthreads();
     if (split) block_scan(pf, B);                 // full partitions before sequence s
     if (split && NG > 0) block_scan(gf, NG);      // shared-prefix pairs before group g
@@ -560,7 +568,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     const int mid = (lo + hi) >> 1;
                     if (gf[mid] <= gp) lo = mid; else hi = mid;
                 }
-                const int s0 = p.grp_start[lo], n = p.grp_start[lo + 1] - s0;
+                const int s0 = gstart[lo], n = gstart[lo + 1] - s0;
                 const int nblk = (n + spi - 1) / spi;
                 const int local = gp - gf[lo];
                 const int cbk = local % nblk;
@@ -571,8 +579,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 it.nparts = 0;
                 it.single_mask = 0;  // members whose only partition this is write `out` directly
                 for (int i = 0; i < it.nseq; ++i) {
-                    const int Li = min(p.seq_lens[it.s + i], Lcap);
-                    if (full_of(Li) + (rest_key(Li) >= 0 ? 1 : 0) == 1) it.single_mask |= 1 << i;
+                    const int si = it.s + i;   // partitions: the group's, its own full ones, its rest
+                    if (kshared[si] + (pf[si + 1] - pf[si]) + (keys[si] >= 0 ? 1 : 0) == 1) it.single_mask |= 1 << i;
                 }
                 it.t_begin = it.part * p.part_tokens;
                 it.t_end = it.t_begin + p.part_tokens;   // every member covers the group's partitions

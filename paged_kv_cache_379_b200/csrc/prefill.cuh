@@ -132,14 +132,18 @@ struct PfLayout {
     static constexpr int kStage0 = 2 * kQTile;             // stage st: K tile, then V tile
     static constexpr int kStageBytes = 2 * kKTile;
     static constexpr int kBar = kStage0 + kPfStages * kStageBytes;
-    // q_full, drain[2], kv_full[4], kv_empty[4], then per query tile and
-    // S/P buffer: s_full[2][2], p_full[2][2], o_done[2][2]; then v16[4] (the V
-    // tile of a stage converted to fp16)
+    // q_full, drain[2], kv_full[4], kv_empty[4], then per query tile:
+    // s_full[2], s_free[2], and per query tile and P buffer p_full[2][2],
+    // o_done[2][2]; then v16[4] (the V tile of a stage converted to fp16)
     static constexpr int kNumBars = 3 + 3 * kPfStages + 12;
     static constexpr int kMisc = kBar + kNumBars * 8;      // TMEM base, abort flag, item
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
-    static constexpr uint32_t kTmemO = 4 * kPfKeys;        // first TMEM column of O_A; O_B at + D
+    // TMEM columns of query tile x: S at x * kTmemTile (kPfKeys columns), its
+    // two fp16 P buffers after it (kPfKeys / 2 columns each); O_A at kTmemO,
+    // O_B at kTmemO + D
+    static constexpr uint32_t kTmemTile = 2 * kPfKeys;
+    static constexpr uint32_t kTmemO = 2 * kTmemTile;
 };
 
 template <int D, int BS>
@@ -166,7 +170,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     auto drain = [&](int x) { return bar0 + 8u * (1 + x); };
     auto kv_full = [&](int st) { return bar0 + 8u * (3 + st); };
     auto kv_empty = [&](int st) { return bar0 + 8u * (3 + kPfStages + st); };
-    auto s_full = [&](int x, int b) { return bar0 + 8u * (3 + 2 * kPfStages + 2 * x + b); };
+    auto s_full = [&](int x) { return bar0 + 8u * (3 + 2 * kPfStages + x); };
+    auto s_free = [&](int x) { return bar0 + 8u * (5 + 2 * kPfStages + x); };
     auto p_full = [&](int x, int b) { return bar0 + 8u * (7 + 2 * kPfStages + 2 * x + b); };
     auto o_done = [&](int x, int b) { return bar0 + 8u * (11 + 2 * kPfStages + 2 * x + b); };
     auto v16 = [&](int st) { return bar0 + 8u * (15 + 2 * kPfStages + st); };
@@ -219,12 +224,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(kv_full(i), 1);
             mbar_init(kv_empty(i), 2);  // one commit from each MMA warp
         }
-        for (int x = 0; x < 2; ++x)
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(s_full(x), 1);
+            mbar_init(s_free(x), 128);  // every softmax thread of the tile has read S
             for (int b = 0; b < 2; ++b) {
-                mbar_init(s_full(x, b), 1);
                 mbar_init(p_full(x, b), 128);
                 mbar_init(o_done(x, b), 1);
             }
+        }
         for (int st = 0; st < kPfStages; ++st) mbar_init(v16(st), 4);  // one arrival per conversion warp
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -321,21 +328,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         constexpr uint32_t kIdO = idesc_f16_f32(kPfRows, D, false, true);
         bool ok = __all_sync(0xffffffffu, wait(q_full, 0));
         const uint32_t qt = base + Lay::kQ + x * Lay::kQTile;
-        // S_X(j) for key tile j into buffer j % 2 (after P_X(j-2) V has read it)
+        // S_X(j) for key tile j into the tile's S buffer, as soon as the softmax
+        // has read S_X(j-1) out of it (P goes to separate buffers, so S does not
+        // wait for any P V product)
         auto issue_s = [&](int j) -> bool {
-            const int st = j % kPfStages, b = j & 1;
+            const int st = j % kPfStages;
             if (!__all_sync(0xffffffffu, wait(kv_full(st), (j / kPfStages) & 1))) return false;
-            if (j >= 2 && !__all_sync(0xffffffffu, wait(o_done(x, b), ((j >> 1) - 1) & 1))) return false;
+            if (j >= 1 && !__all_sync(0xffffffffu, wait(s_free(x), (j - 1) & 1))) return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t kt = base + Lay::kStage0 + st * Lay::kStageBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    tc_mma_bf16(tmem + x * 2 * kPfKeys + b * kPfKeys,
+                    tc_mma_bf16(tmem + x * Lay::kTmemTile,
                                 desc_kmajor_sw128(qt + (kk >> 2) * kQPlane + (kk & 3) * 32),
                                 desc_kmajor_sw128(kt + (kk >> 2) * kKPlane + (kk & 3) * 32), kIdS, kk > 0);
                 }
-                tc_commit(s_full(x, b));
+                tc_commit(s_full(x));
             }
             __syncwarp();
             return true;
@@ -362,7 +371,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     // step of 16 keys is 8 columns
 #pragma unroll
                     for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-                        tc_mma_bf16_ts(tmem + Lay::kTmemO + x * D, tmem + x * 2 * kPfKeys + b * kPfKeys + kk * 8,
+                        tc_mma_bf16_ts(tmem + Lay::kTmemO + x * D,
+                                       tmem + x * Lay::kTmemTile + kPfKeys + b * (kPfKeys / 2) + kk * 8,
                                        desc_mnmajor_sw128(vt + kk * 16 * 128, kKPlane), kIdO, j > 0 || kk > 0);
                     }
                     tc_commit(o_done(x, b));
@@ -434,13 +444,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         bool ok = true;
         for (int j = 0; active && j < nkx; ++j) {
             const int b = j & 1;
-            const uint32_t s_addr = lane_addr + x * 2 * kPfKeys + b * kPfKeys;
-            ok = __all_sync(0xffffffffu, wait(s_full(x, b), (j >> 1) & 1));
+            const uint32_t s_addr = lane_addr + x * Lay::kTmemTile;
+            const uint32_t p_addr = s_addr + kPfKeys + b * (kPfKeys / 2);
+            ok = __all_sync(0xffffffffu, wait(s_full(x), j & 1));
             if (!ok) break;
             tc_fence_after();
             float xs[kPfKeys];
             tmem_ld32(s_addr, xs);
             tmem_ld32(s_addr + 32, xs + 32);
+            // S is in registers: the next S product may overwrite the buffer
+            tc_fence_before();
+            mbar_arrive(s_free(x));
             // causal mask, only in tiles that reach past some row's position
             const int lim = pos - j * kPfKeys;  // keys c <= lim are visible
             if (!__all_sync(0xffffffffu, lim >= kPfKeys - 1)) {
@@ -499,8 +513,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     tmem_st32(o_addr + c * 32, o);
                 }
             }
-            // P over S in this buffer (all of S is in registers)
-            tmem_st32(s_addr, pw);
+            // P into buffer b, once P_{j-2} V has read it
+            if (j >= 2) {
+                ok = __all_sync(0xffffffffu, wait(o_done(x, b), ((j >> 1) - 1) & 1));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            tmem_st32(p_addr, pw);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full(x, b));
