@@ -373,8 +373,7 @@ static int launch_prefill_t(const PrefillParams &p, const CUtensorMap &tq, const
     const size_t smem = (size_t)PfLayout<D>::kAlloc;
     int rc = ensure_smem(reinterpret_cast<const void *>(kernel), smem);
     if (rc != PA_OK) return rc;
-    return launch_pdl(kernel, dim3((unsigned)tiles, (unsigned)p.num_kv_heads), dim3(kPfThreads), smem, st, p, tq,
-                      tk, tv);
+    return launch_pdl(kernel, dim3((unsigned)tiles), dim3(kPfThreads), smem, st, p, tq, tk, tv);
 }
 
 template <int D>
@@ -784,10 +783,11 @@ int pa_prefill(void *out, const void *query, const void *key_cache, const void *
     p.max_blocks = max_blocks_per_seq;
     p.tq = kPfRows / G;
     p.q_box = std::min(p.tq, num_tokens);
-    // the query tiles of all sequences number at most T / tq + B, their pairs
-    // (one CTA each) at most T / (2 tq) + B
-    const int64_t tiles = (int64_t)num_tokens / (2 * p.tq) + num_seqs + 1;
-    if (tiles > INT_MAX) return PA_ERR_BAD_SHAPE;
+    // persistent: one CTA per SM (shared memory and TMEM hold one), at most one
+    // per work item; the items are (pair of query tiles, KV head), at most
+    // (T / (2 tq) + B) * num_kv_heads of them
+    const int64_t items = ((int64_t)num_tokens / (2 * p.tq) + num_seqs + 1) * num_kv_heads;
+    const int64_t tiles = std::min<int64_t>(items, std::max(1, sm_count()));
     CUtensorMap tq, tk, tv;
     int rc = make_query_map(&tq, query, num_tokens, num_heads, head_dim, G, p.q_box);
     if (rc != PA_OK) return rc;

@@ -66,7 +66,7 @@ constexpr int kPfConvWarp = 11;       // first of the 4 V-conversion warps
 constexpr int kPfThreads = 480;
 constexpr int kPfRows = 128;          // MMA M: query rows per tile
 constexpr int kPfKeys = 64;           // keys per K/V tile
-constexpr int kPfStages = 4;          // K/V ring stages
+constexpr int kPfStages = 3;          // K/V ring stages (two query buffers take the rest)
 constexpr uint32_t kPfTmemCols = 512;
 // A row's softmax reference max moves only when a logit exceeds it by more
 // than this (log2 units), so unnormalised weights stay below 2^8.
@@ -128,15 +128,16 @@ struct PfLayout {
     static constexpr int kPlanes = D / 64;
     static constexpr int kQTile = kPlanes * kQPlane;
     static constexpr int kKTile = kPlanes * kKPlane;       // K or V tile
-    static constexpr int kQ = 0;                           // Q_A, then Q_B
-    static constexpr int kStage0 = 2 * kQTile;             // stage st: K tile, then V tile
+    static constexpr int kQ = 0;                           // Q buffer qb: tile A, then tile B
+    static constexpr int kQBuf = 2 * kQTile;
+    static constexpr int kStage0 = 2 * kQBuf;              // stage st: K tile, then V tile
     static constexpr int kStageBytes = 2 * kKTile;
     static constexpr int kBar = kStage0 + kPfStages * kStageBytes;
-    // q_full, drain[2], kv_full[4], kv_empty[4], then per query tile:
-    // s_full[2], s_free[2], and per query tile and P buffer p_full[2][2],
-    // o_done[2][2]; then v16[4] (the V tile of a stage converted to fp16)
-    static constexpr int kNumBars = 3 + 3 * kPfStages + 12;
-    static constexpr int kMisc = kBar + kNumBars * 8;      // TMEM base, abort flag, item
+    // q_full[2], q_free[2], drain[2], kv_full[S], kv_empty[S], then per query
+    // tile s_full[2], s_free[2], o_free[2], and per query tile and P buffer
+    // p_full[2][2], o_done[2][2]; then v16[S] (the V tile of a stage in fp16)
+    static constexpr int kNumBars = 6 + 3 * kPfStages + 6 + 8;
+    static constexpr int kMisc = kBar + kNumBars * 8;      // TMEM base, abort flag, item count
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
     // TMEM columns of query tile x: S at x * kTmemTile (kPfKeys columns), its
@@ -146,6 +147,21 @@ struct PfLayout {
     static constexpr uint32_t kTmemO = 2 * kTmemTile;
 };
 
+// One work item: a pair of consecutive query tiles (A and B) of one sequence
+// and one KV head.
+struct PfItem {
+    int s, g, q0, q_len, L, ctx, tA;
+    bool hasB;
+    int endA, endB, nkA, nk;  // causal: key tiles of tile A, of the pair (>= nkA)
+};
+
+// Persistent: each CTA walks the work items w = blockIdx.x, + gridDim.x, ...
+// Item w = (r, s, g) with the KV head fastest, then the sequence, then r:
+// the r-th pair of sequence s counted from its end (its longest), so every
+// sequence's longest pairs come first and the CTAs share each length class.
+// Consecutive items of a CTA overlap: the next item's queries load into the
+// other query buffer, and its first S is issued as soon as the softmax has
+// read the last S of the previous item, under that item's epilogue.
 template <int D, int BS>
 __global__ void __launch_bounds__(kPfThreads, 1)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
@@ -157,6 +173,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     constexpr int kQPlane = Lay::kQPlane;
     constexpr int kKPlane = Lay::kKPlane;
     constexpr int kPlanes = Lay::kPlanes;
+    constexpr int S = kPfStages;
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -166,80 +183,63 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int lane = threadIdx.x & 31;
 
     const uint32_t bar0 = base + Lay::kBar;
-    const uint32_t q_full = bar0;
-    auto drain = [&](int x) { return bar0 + 8u * (1 + x); };
-    auto kv_full = [&](int st) { return bar0 + 8u * (3 + st); };
-    auto kv_empty = [&](int st) { return bar0 + 8u * (3 + kPfStages + st); };
-    auto s_full = [&](int x) { return bar0 + 8u * (3 + 2 * kPfStages + x); };
-    auto s_free = [&](int x) { return bar0 + 8u * (5 + 2 * kPfStages + x); };
-    auto p_full = [&](int x, int b) { return bar0 + 8u * (7 + 2 * kPfStages + 2 * x + b); };
-    auto o_done = [&](int x, int b) { return bar0 + 8u * (11 + 2 * kPfStages + 2 * x + b); };
-    auto v16 = [&](int st) { return bar0 + 8u * (15 + 2 * kPfStages + st); };
+    auto q_full = [&](int qb) { return bar0 + 8u * qb; };
+    auto q_free = [&](int qb) { return bar0 + 8u * (2 + qb); };
+    auto drain = [&](int x) { return bar0 + 8u * (4 + x); };
+    auto kv_full = [&](int st) { return bar0 + 8u * (6 + st); };
+    auto kv_empty = [&](int st) { return bar0 + 8u * (6 + S + st); };
+    auto s_full = [&](int x) { return bar0 + 8u * (6 + 2 * S + x); };
+    auto s_free = [&](int x) { return bar0 + 8u * (8 + 2 * S + x); };
+    auto o_free = [&](int x) { return bar0 + 8u * (10 + 2 * S + x); };
+    auto p_full = [&](int x, int b) { return bar0 + 8u * (12 + 2 * S + 2 * x + b); };
+    auto o_done = [&](int x, int b) { return bar0 + 8u * (16 + 2 * S + 2 * x + b); };
+    auto v16 = [&](int st) { return bar0 + 8u * (20 + 2 * S + st); };
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(base_ptr + Lay::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base_ptr + Lay::kMisc + 4);
-    volatile int *item = reinterpret_cast<volatile int *>(base_ptr + Lay::kMisc + 16);
+    volatile int *rmax = reinterpret_cast<volatile int *>(base_ptr + Lay::kMisc + 8);
 
     pdl_wait();
     pdl_launch_dependents();
 
-    // ---- which (sequence, pair of query tiles) this CTA takes: blockIdx.x
-    // enumerates the tile pairs of all sequences, each sequence's last (longest)
-    // pair first.
+    const int G = p.group;
+    const int B = p.num_seqs;
+    const int Hkv = p.num_kv_heads;
+    // pairs of query tiles of sequence s (0: nothing to do)
+    auto pairs_of = [&](int q_len, int L) { return (q_len > 0 && q_len <= L) ? ((q_len + p.tq - 1) / p.tq + 1) / 2 : 0; };
+    // ---- the most pairs any sequence has: the items are w < rmax * B * Hkv
     if (warp == 0) {
-        const int x = blockIdx.x;
-        int found_s = -1, found_qp = 0, running = 0;
-        for (int s0 = 0; s0 < p.num_seqs && found_s < 0; s0 += 32) {
-            const int s = s0 + lane;
-            int pairs = 0;
-            if (s < p.num_seqs) {
-                const int ql = p.q_start[s + 1] - p.q_start[s];
-                if (ql > 0 && ql <= p.seq_lens[s]) pairs = ((ql + p.tq - 1) / p.tq + 1) / 2;
-            }
-            int incl = pairs;
+        int r = 0;
+        for (int s = lane; s < B; s += 32) r = max(r, pairs_of(p.q_start[s + 1] - p.q_start[s], p.seq_lens[s]));
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += t;
-            }
-            const int excl = running + incl - pairs;
-            const unsigned hit = __ballot_sync(0xffffffffu, pairs > 0 && x >= excl && x < excl + pairs);
-            if (hit) {
-                const int src = __ffs(hit) - 1;
-                const int e = __shfl_sync(0xffffffffu, excl, src);
-                const int np = __shfl_sync(0xffffffffu, pairs, src);
-                found_s = s0 + src;
-                found_qp = np - 1 - (x - e);
-            }
-            running += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) {
-            item[0] = found_s;
-            item[1] = found_qp;
-        }
+        for (int o = 16; o >= 1; o >>= 1) r = max(r, __shfl_xor_sync(0xffffffffu, r, o));
+        if (lane == 0) *rmax = r;
     }
     if (threadIdx.x == 32) {
-        mbar_init(q_full, 1);
-        for (int x = 0; x < 2; ++x) mbar_init(drain(x), 1);
-        for (int i = 0; i < kPfStages; ++i) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(q_full(b), 1);
+            mbar_init(q_free(b), 2);  // one commit from each MMA warp after its last S of the item
+            mbar_init(drain(b), 1);
+        }
+        for (int i = 0; i < S; ++i) {
             mbar_init(kv_full(i), 1);
             mbar_init(kv_empty(i), 2);  // one commit from each MMA warp
+            mbar_init(v16(i), 4);       // one arrival per conversion warp
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full(x), 1);
             mbar_init(s_free(x), 128);  // every softmax thread of the tile has read S
+            mbar_init(o_free(x), 128);  // every softmax thread of the tile has read O (epilogue)
             for (int b = 0; b < 2; ++b) {
                 mbar_init(p_full(x, b), 128);
                 mbar_init(o_done(x, b), 1);
             }
         }
-        for (int st = 0; st < kPfStages; ++st) mbar_init(v16(st), 4);  // one arrival per conversion warp
         *abort_flag = 0;
         fence_mbarrier_init();
     }
     __syncthreads();
-    const int s = item[0];
-    if (s < 0) return;  // past the last pair: the whole CTA leaves before any TMEM use
-    const int qp = item[1];
+    const int64_t W = (int64_t)(*rmax) * B * Hkv;
+    if (W == 0 || (int64_t)blockIdx.x >= W) return;  // no work: the whole CTA leaves before any TMEM use
 
     if (warp == kPfMmaWarp) {
         tmem_alloc(base + Lay::kMisc, kPfTmemCols);
@@ -250,18 +250,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const int G = p.group;
-    const int g = blockIdx.y;
-    const int q0 = p.q_start[s];
-    const int q_len = p.q_start[s + 1] - q0;
-    const int L = p.seq_lens[s];
-    const int ctx = L - q_len;
-    const int tA = 2 * qp * p.tq;                     // first token of tile A (tile B follows)
-    const bool hasB = tA + p.tq < q_len;
-    const int endA = min(q_len, tA + p.tq);
-    const int endB = hasB ? min(q_len, tA + 2 * p.tq) : endA;
-    const int nkA = (ctx + endA + kPfKeys - 1) / kPfKeys;  // causal: keys below ctx + end
-    const int nk = (ctx + endB + kPfKeys - 1) / kPfKeys;   // key tiles of the pair (>= nkA)
+    // item w, or false if it holds no pair
+    auto decode = [&](int64_t w, PfItem &it) -> bool {
+        const int64_t per_r = (int64_t)B * Hkv;
+        const int r = (int)(w / per_r);
+        const int rem = (int)(w - (int64_t)r * per_r);
+        it.s = rem / Hkv;
+        it.g = rem - it.s * Hkv;
+        it.q0 = p.q_start[it.s];
+        it.q_len = p.q_start[it.s + 1] - it.q0;
+        it.L = p.seq_lens[it.s];
+        const int qp = pairs_of(it.q_len, it.L) - 1 - r;
+        if (qp < 0) return false;
+        it.ctx = it.L - it.q_len;
+        it.tA = 2 * qp * p.tq;                             // first token of tile A (tile B follows)
+        it.hasB = it.tA + p.tq < it.q_len;
+        it.endA = min(it.q_len, it.tA + p.tq);
+        it.endB = it.hasB ? min(it.q_len, it.tA + 2 * p.tq) : it.endA;
+        it.nkA = (it.ctx + it.endA + kPfKeys - 1) / kPfKeys;
+        it.nk = (it.ctx + it.endB + kPfKeys - 1) / kPfKeys;
+        return true;
+    };
 
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
         if (*abort_flag) return false;
@@ -277,115 +286,151 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             prefetch_tensormap(&tmap_q);
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
-            mbar_arrive_expect_tx(q_full, (uint32_t)(2 * kPlanes * G * p.q_box * 128));
-            for (int x = 0; x < 2; ++x)
-                for (int pl = 0; pl < kPlanes; ++pl)
-                    tma_load_4d(base + Lay::kQ + x * Lay::kQTile + pl * kQPlane, &tmap_q, q_full, 0, pl, g * G,
-                                q0 + tA + x * p.tq);
         }
-        const int32_t *table = p.block_tables + (int64_t)s * p.max_blocks;
-        int issued = 0;  // key tiles whose loads were issued
-        for (int t = 0; t < nk; ++t) {
-            const int st = t % kPfStages;
-            const int key0 = t * kPfKeys;
-            const int nblk = min(kPfKeys / BS, (L - key0 + BS - 1) / BS);
-            const int phys = lane < nblk ? table[key0 / BS + lane] : 0;
-            if (t >= kPfStages && !__all_sync(0xffffffffu, wait(kv_empty(st), (t / kPfStages - 1) & 1))) break;
-            if (lane == 0) mbar_arrive_expect_tx(kv_full(st), (uint32_t)(nblk * BS * D * 2 * 2));
-            const uint32_t kdst = base + Lay::kStage0 + st * Lay::kStageBytes;
-            const uint32_t vdst = kdst + Lay::kKTile;
-            for (int k = 0; k < nblk; ++k) {
-                const int row = __shfl_sync(0xffffffffu, phys, k) * BS;
-                if (lane == 0) {
+        int k = 0;         // items taken
+        int64_t T = 0;     // ring tiles issued
+        bool ok = true;
+        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+            PfItem it;
+            if (!decode(w, it)) continue;
+            const int qb = k & 1;
+            // the query buffer is free once both MMA warps' last S of item k-2 completed
+            if (k >= 2 && !__all_sync(0xffffffffu, wait(q_free(qb), ((k >> 1) - 1) & 1))) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(q_full(qb), (uint32_t)(2 * kPlanes * G * p.q_box * 128));
+                for (int x = 0; x < 2; ++x)
+                    for (int pl = 0; pl < kPlanes; ++pl)
+                        tma_load_4d(base + Lay::kQ + qb * Lay::kQBuf + x * Lay::kQTile + pl * kQPlane, &tmap_q,
+                                    q_full(qb), 0, pl, it.g * G, it.q0 + it.tA + x * p.tq);
+            }
+            ++k;
+            const int32_t *table = p.block_tables + (int64_t)it.s * p.max_blocks;
+            for (int t = 0; t < it.nk; ++t, ++T) {
+                const int st = (int)(T % S);
+                const int key0 = t * kPfKeys;
+                const int nblk = min(kPfKeys / BS, (it.L - key0 + BS - 1) / BS);
+                const int phys = lane < nblk ? table[key0 / BS + lane] : 0;
+                if (T >= S && !__all_sync(0xffffffffu, wait(kv_empty(st), ((T / S) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) mbar_arrive_expect_tx(kv_full(st), (uint32_t)(nblk * BS * D * 2 * 2));
+                const uint32_t kdst = base + Lay::kStage0 + st * Lay::kStageBytes;
+                const uint32_t vdst = kdst + Lay::kKTile;
+                for (int kb = 0; kb < nblk; ++kb) {
+                    const int row = __shfl_sync(0xffffffffu, phys, kb) * BS;
+                    if (lane == 0) {
 #pragma unroll
-                    for (int pl = 0; pl < kPlanes; ++pl) {
-                        tma_load_4d(kdst + pl * kKPlane + k * BS * 128, &tmap_k, kv_full(st), 0, pl, g, row);
-                        tma_load_4d(vdst + pl * kKPlane + k * BS * 128, &tmap_v, kv_full(st), 0, pl, g, row);
+                        for (int pl = 0; pl < kPlanes; ++pl) {
+                            tma_load_4d(kdst + pl * kKPlane + kb * BS * 128, &tmap_k, kv_full(st), 0, pl, it.g, row);
+                            tma_load_4d(vdst + pl * kKPlane + kb * BS * 128, &tmap_v, kv_full(st), 0, pl, it.g, row);
+                        }
                     }
                 }
             }
-            issued = t + 1;
         }
-        if (lane == 0 && *abort_flag) {  // let the loads this CTA issued land before it exits
-            mbar_wait_bounded(q_full, 0);
-            for (int st = 0; st < kPfStages; ++st)
-                if (st < issued) {  // the stage's last tile: the largest t < issued with t % kPfStages == st
-                    const int last = issued - 1 - (issued - 1 - st) % kPfStages;
-                    mbar_wait_bounded(kv_full(st), (last / kPfStages) & 1);
+        if (lane == 0 && *abort_flag) {
+            // let the loads this CTA issued land before it exits: the last two
+            // query loads and each stage's last tile
+            for (int kq = max(0, k - 2); kq < k; ++kq) mbar_wait_bounded(q_full(kq & 1), (kq >> 1) & 1);
+            for (int st = 0; st < S; ++st)
+                if (st < T) {
+                    const int64_t last = T - 1 - (T - 1 - st) % S;
+                    mbar_wait_bounded(kv_full(st), (uint32_t)((last / S) & 1));
                 }
         }
     } else if (warp >= kPfMmaWarp && warp < kPfConvWarp) {
         // ------------------------------------------------------------ MMA issue
-        // Warp 9 issues tile A's products, warp 10 tile B's.  Per key tile j:
-        // S_X(j+1) into buffer (j+1) % 2 (after P_X(j-1) V has read it), then
-        // P_X(j) V once the softmax has written P and V(j) is fp16.  Each warp
-        // releases the K/V stage with its own commit, also for key tiles its
-        // query tile skips.
+        // Warp 9 issues tile A's products, warp 10 tile B's.  Per key tile j of
+        // an item: S_X(j+1) (once the softmax has read S_X(j)) before waiting for
+        // P_X(j), then P_X(j) V once the softmax has written P and V(j) is fp16.
+        // Each warp releases every K/V stage with its own commit, also for key
+        // tiles its query tile skips, and the item's query buffer after its last S.
         const int x = warp - kPfMmaWarp;
-        const bool act = x == 0 || hasB;
-        const int nkx = x == 0 ? nkA : nk;
         constexpr uint32_t kIdS = idesc_bf16_f32(kPfRows, kPfKeys, false, false);
         constexpr uint32_t kIdO = idesc_f16_f32(kPfRows, D, false, true);
-        bool ok = __all_sync(0xffffffffu, wait(q_full, 0));
-        const uint32_t qt = base + Lay::kQ + x * Lay::kQTile;
-        // S_X(j) for key tile j into the tile's S buffer, as soon as the softmax
-        // has read S_X(j-1) out of it (P goes to separate buffers, so S does not
-        // wait for any P V product)
-        auto issue_s = [&](int j) -> bool {
-            const int st = j % kPfStages;
-            if (!__all_sync(0xffffffffu, wait(kv_full(st), (j / kPfStages) & 1))) return false;
-            if (j >= 1 && !__all_sync(0xffffffffu, wait(s_free(x), (j - 1) & 1))) return false;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t kt = base + Lay::kStage0 + st * Lay::kStageBytes;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    tc_mma_bf16(tmem + x * Lay::kTmemTile,
-                                desc_kmajor_sw128(qt + (kk >> 2) * kQPlane + (kk & 3) * 32),
-                                desc_kmajor_sw128(kt + (kk >> 2) * kKPlane + (kk & 3) * 32), kIdS, kk > 0);
-                }
-                tc_commit(s_full(x));
-            }
-            __syncwarp();
-            return true;
-        };
-        // The S product of the next key tile is issued before waiting for this
-        // tile's P, so the softmax always finds its next S ready.
-        if (ok && act && nkx > 0) ok = issue_s(0);
-        for (int j = 0; ok && j < nk; ++j) {
-            const int st = j % kPfStages;
-            const int b = j & 1;
-            const bool work = act && j < nkx;
-            if (work) {
-                if (j + 1 < nkx) {
-                    ok = issue_s(j + 1);
-                    if (!ok) break;
-                }
-                ok = __all_sync(0xffffffffu, wait(p_full(x, b), (j >> 1) & 1));
-                if (ok) ok = __all_sync(0xffffffffu, wait(v16(st), (j / kPfStages) & 1));
-                if (!ok) break;
+        int k = 0;          // items taken
+        int kx = 0;         // items with this query tile active
+        int64_t T = 0;      // ring tiles consumed
+        int64_t n = 0;      // S products of this query tile issued (= its P products)
+        bool ok = true;
+        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+            PfItem it;
+            if (!decode(w, it)) continue;
+            const int qb = k & 1;
+            const bool act = x == 0 || it.hasB;
+            const int nkx = x == 0 ? it.nkA : it.nk;
+            const uint32_t qt = base + Lay::kQ + qb * Lay::kQBuf + x * Lay::kQTile;
+            if (act) ok = __all_sync(0xffffffffu, wait(q_full(qb), (k >> 1) & 1));
+            // S product number nn (tile j of the item, ring tile T0 + j)
+            auto issue_s = [&](int64_t nn, int64_t tr) -> bool {
+                const int st = (int)(tr % S);
+                if (!__all_sync(0xffffffffu, wait(kv_full(st), (uint32_t)((tr / S) & 1)))) return false;
+                if (nn >= 1 && !__all_sync(0xffffffffu, wait(s_free(x), (uint32_t)((nn - 1) & 1)))) return false;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t vt = base + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
-                    // P of the tile's 64 keys: fp16 pairs in columns [0, 32); a K
-                    // step of 16 keys is 8 columns
+                    const uint32_t kt = base + Lay::kStage0 + st * Lay::kStageBytes;
 #pragma unroll
-                    for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-                        tc_mma_bf16_ts(tmem + Lay::kTmemO + x * D,
-                                       tmem + x * Lay::kTmemTile + kPfKeys + b * (kPfKeys / 2) + kk * 8,
-                                       desc_mnmajor_sw128(vt + kk * 16 * 128, kKPlane), kIdO, j > 0 || kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        tc_mma_bf16(tmem + x * Lay::kTmemTile,
+                                    desc_kmajor_sw128(qt + (kk >> 2) * kQPlane + (kk & 3) * 32),
+                                    desc_kmajor_sw128(kt + (kk >> 2) * kKPlane + (kk & 3) * 32), kIdS, kk > 0);
                     }
-                    tc_commit(o_done(x, b));
+                    tc_commit(s_full(x));
                 }
                 __syncwarp();
-            } else {
-                // a key tile this query tile does not need: wait for it to land so the
-                // release below cannot run ahead of the load
-                ok = __all_sync(0xffffffffu, wait(kv_full(st), (j / kPfStages) & 1));
-                if (!ok) break;
+                return true;
+            };
+            if (ok && act && nkx > 0) ok = issue_s(n, T);
+            for (int j = 0; ok && j < it.nk; ++j) {
+                const int64_t tr = T + j;
+                const int st = (int)(tr % S);
+                if (act && j < nkx) {
+                    const int64_t nj = n + j;
+                    const int b = (int)(nj & 1);
+                    if (j + 1 < nkx) {
+                        ok = issue_s(nj + 1, tr + 1);
+                        if (!ok) break;
+                    }
+                    ok = __all_sync(0xffffffffu, wait(p_full(x, b), (uint32_t)((nj >> 1) & 1)));
+                    if (ok) ok = __all_sync(0xffffffffu, wait(v16(st), (uint32_t)((tr / S) & 1)));
+                    // O of the previous item must have been read by its epilogue
+                    if (ok && j == 0 && kx >= 1) ok = __all_sync(0xffffffffu, wait(o_free(x), (uint32_t)((kx - 1) & 1)));
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t vt = base + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
+                        // P of the tile's 64 keys: fp16 pairs in kPfKeys / 2 columns; a K
+                        // step of 16 keys is 8 columns
+#pragma unroll
+                        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
+                            tc_mma_bf16_ts(tmem + Lay::kTmemO + x * D,
+                                           tmem + x * Lay::kTmemTile + kPfKeys + b * (kPfKeys / 2) + kk * 8,
+                                           desc_mnmajor_sw128(vt + kk * 16 * 128, kKPlane), kIdO, j > 0 || kk > 0);
+                        }
+                        tc_commit(o_done(x, b));
+                    }
+                    __syncwarp();
+                } else {
+                    // a key tile this query tile does not need: wait for it to land so the
+                    // release below cannot run ahead of the load
+                    ok = __all_sync(0xffffffffu, wait(kv_full(st), (uint32_t)((tr / S) & 1)));
+                    if (!ok) break;
+                }
+                if (lane == 0) tc_commit(kv_empty(st));
+                __syncwarp();
             }
-            if (lane == 0) tc_commit(kv_empty(st));
+            if (!ok) break;
+            // every S of the item was issued before this commit: the query buffer
+            // frees when they complete
+            if (lane == 0) tc_commit(q_free(qb));
             __syncwarp();
+            T += it.nk;
+            if (act) {
+                n += nkx;
+                ++kx;
+            }
+            ++k;
         }
     } else if (warp >= kPfConvWarp) {
         // ------------------------------------------------------------ V to fp16
@@ -396,143 +441,157 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // before the P V that waits for this conversion has completed.
         const int c = warp - kPfConvWarp;
         float amax = 0.f;
-        for (int t = 0; t < nk; ++t) {
-            const int st = t % kPfStages;
-            if (!__all_sync(0xffffffffu, wait(kv_full(st), (t / kPfStages) & 1))) break;
-            const int kv_valid = min(kPfKeys, L - t * kPfKeys);
-            uint8_t *vt = base_ptr + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
-            uint4 v[kPlanes][4];
-#pragma unroll
-            for (int pl = 0; pl < kPlanes; ++pl)
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    v[pl][k] = reinterpret_cast<const uint4 *>(vt + pl * kKPlane + c * 16 * 128)[lane + 32 * k];
-#pragma unroll
-            for (int pl = 0; pl < kPlanes; ++pl)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int key = 16 * c + 4 * k + (lane >> 3);  // 8 chunks of 16 bytes per 128-byte row
-                    uint4 o = make_uint4(0, 0, 0, 0);
-                    if (key < kv_valid) {
-                        o.x = bf16x2_to_f16x2(v[pl][k].x, amax);
-                        o.y = bf16x2_to_f16x2(v[pl][k].y, amax);
-                        o.z = bf16x2_to_f16x2(v[pl][k].z, amax);
-                        o.w = bf16x2_to_f16x2(v[pl][k].w, amax);
-                    }
-                    reinterpret_cast<uint4 *>(vt + pl * kKPlane + c * 16 * 128)[lane + 32 * k] = o;
+        int64_t T = 0;
+        bool ok = true;
+        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+            PfItem it;
+            if (!decode(w, it)) continue;
+            for (int t = 0; t < it.nk; ++t, ++T) {
+                const int st = (int)(T % S);
+                if (!__all_sync(0xffffffffu, wait(kv_full(st), (uint32_t)((T / S) & 1)))) {
+                    ok = false;
+                    break;
                 }
-            fence_proxy_async_smem();  // the tensor cores read it through the async proxy
-            __syncwarp();
-            if (lane == 0) mbar_arrive(v16(st));
+                const int kv_valid = min(kPfKeys, it.L - t * kPfKeys);
+                uint8_t *vt = base_ptr + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
+                uint4 v[kPlanes][4];
+#pragma unroll
+                for (int pl = 0; pl < kPlanes; ++pl)
+#pragma unroll
+                    for (int kq = 0; kq < 4; ++kq)
+                        v[pl][kq] = reinterpret_cast<const uint4 *>(vt + pl * kKPlane + c * 16 * 128)[lane + 32 * kq];
+#pragma unroll
+                for (int pl = 0; pl < kPlanes; ++pl)
+#pragma unroll
+                    for (int kq = 0; kq < 4; ++kq) {
+                        const int key = 16 * c + 4 * kq + (lane >> 3);  // 8 chunks of 16 bytes per 128-byte row
+                        uint4 o = make_uint4(0, 0, 0, 0);
+                        if (key < kv_valid) {
+                            o.x = bf16x2_to_f16x2(v[pl][kq].x, amax);
+                            o.y = bf16x2_to_f16x2(v[pl][kq].y, amax);
+                            o.z = bf16x2_to_f16x2(v[pl][kq].z, amax);
+                            o.w = bf16x2_to_f16x2(v[pl][kq].w, amax);
+                        }
+                        reinterpret_cast<uint4 *>(vt + pl * kKPlane + c * 16 * 128)[lane + 32 * kq] = o;
+                    }
+                fence_proxy_async_smem();  // the tensor cores read it through the async proxy
+                __syncwarp();
+                if (lane == 0) mbar_arrive(v16(st));
+            }
         }
         if (amax > 65504.f) record_status(kStatusValueRange);
     } else {
         // ------------------------------------------------------------ softmax
         const int x = warp >> 2;                 // query tile: 0 = A, 1 = B
         const int r = threadIdx.x & 127;         // MMA row = TMEM lane
-        const bool active = x == 0 || hasB;
-        const int nkx = x == 0 ? nkA : nk;
         const int tok = r / G;
         const int gi = r - tok * G;
-        const int i = tA + x * p.tq + tok;
-        const int endx = x == 0 ? endA : endB;
-        const bool row_ok = active && tok < p.tq && i < endx;
-        const int pos = row_ok ? ctx + i : L - 1;
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const uint32_t o_addr = lane_addr + Lay::kTmemO + x * D;
-        float m = -INFINITY, l = 0.f;
+        const uint32_t s_addr = lane_addr + x * Lay::kTmemTile;
+        int64_t n = 0;      // S tiles of this query tile consumed (= P tiles written)
         bool ok = true;
-        for (int j = 0; active && j < nkx; ++j) {
-            const int b = j & 1;
-            const uint32_t s_addr = lane_addr + x * Lay::kTmemTile;
-            const uint32_t p_addr = s_addr + kPfKeys + b * (kPfKeys / 2);
-            ok = __all_sync(0xffffffffu, wait(s_full(x), j & 1));
-            if (!ok) break;
-            tc_fence_after();
-            float xs[kPfKeys];
-            tmem_ld32(s_addr, xs);
-            tmem_ld32(s_addr + 32, xs + 32);
-            // S is in registers: the next S product may overwrite the buffer
-            tc_fence_before();
-            mbar_arrive(s_free(x));
-            // causal mask, only in tiles that reach past some row's position
-            const int lim = pos - j * kPfKeys;  // keys c <= lim are visible
-            if (!__all_sync(0xffffffffu, lim >= kPfKeys - 1)) {
-#pragma unroll
-                for (int c = 0; c < kPfKeys; ++c) xs[c] = c <= lim ? xs[c] : -INFINITY;
-            }
-            // row max: four chains of three-input maxima
-            float pm[4] = {xs[0], xs[1], xs[2], xs[3]};
-#pragma unroll
-            for (int c = 4; c < kPfKeys; c += 8) {
-                pm[0] = max3f(pm[0], xs[c], xs[c + 1]);
-                pm[1] = max3f(pm[1], xs[c + 2], xs[c + 3]);
-                pm[2] = max3f(pm[2], xs[c + 4], xs[c + 5]);
-                pm[3] = max3f(pm[3], xs[c + 6], xs[c + 7]);
-            }
-            const float mx = fmaxf(max3f(pm[0], pm[1], pm[2]), pm[3]) * p.scale_log2;  // scale > 0: the max commutes with it
-            // lazily moved reference max (log2 units): weights stay <= 2^kPfRescaleSlack
-            const bool bump = mx > m + kPfRescaleSlack;
-            float corr = 1.f;
-            if (bump) {
-                corr = fast_exp2(m - mx);  // 0 on the first tile (m = -inf)
-                m = mx;
-            }
-            // weights (scaled by 2^kPfP16Shift) and their sum (8 partial sums);
-            // P as fp16 pairs, the lower key in the low half
-            // (logit scale, shift) on key pairs by packed fp32 FMAs; the row sum
-            // in four packed fp32 accumulators
-            const float mneg = kPfP16Shift - m;
-            const uint64_t scale2 = f32x2(p.scale_log2, p.scale_log2), shift2 = f32x2(mneg, mneg);
-            uint64_t ps[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) ps[u] = 0ull;
-            float pw[kPfKeys / 2];
-#pragma unroll
-            for (int e = 0; e < kPfKeys / 2; ++e) {
-                const float2 y = f32x2_split(fma_f32x2(f32x2(xs[2 * e], xs[2 * e + 1]), scale2, shift2));
-                const float p0 = fast_exp2(y.x);
-                const float p1 = fast_exp2(y.y);
-                ps[e & 3] = add_f32x2(ps[e & 3], f32x2(p0, p1));
-                pw[e] = __uint_as_float(pack_f16x2(p0, p1));
-            }
-            const float2 q01 = f32x2_split(add_f32x2(ps[0], ps[1])), q23 = f32x2_split(add_f32x2(ps[2], ps[3]));
-            l = l * corr + ((q01.x + q01.y) + (q23.x + q23.y));
-            if (j >= 1 && __any_sync(0xffffffffu, bump)) {
-                // O holds P_{<j} V: rescale it once P_{j-1} V has completed
-                const int jp = j - 1;
-                ok = __all_sync(0xffffffffu, wait(o_done(x, jp & 1), (jp >> 1) & 1));
+        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+            PfItem it;
+            if (!decode(w, it)) continue;
+            const bool active = x == 0 || it.hasB;
+            if (!active) continue;
+            const int nkx = x == 0 ? it.nkA : it.nk;
+            const int i = it.tA + x * p.tq + tok;
+            const int endx = x == 0 ? it.endA : it.endB;
+            const bool row_ok = tok < p.tq && i < endx;
+            const int pos = row_ok ? it.ctx + i : it.L - 1;
+            float m = -INFINITY, l = 0.f;
+            for (int j = 0; j < nkx; ++j) {
+                const int64_t nj = n + j;
+                const int b = (int)(nj & 1);
+                const uint32_t p_addr = s_addr + kPfKeys + b * (kPfKeys / 2);
+                ok = __all_sync(0xffffffffu, wait(s_full(x), (uint32_t)(nj & 1)));
                 if (!ok) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    float o[32];
-                    tmem_ld32(o_addr + c * 32, o);
+                float xs[kPfKeys];
+                tmem_ld32(s_addr, xs);
+                tmem_ld32(s_addr + 32, xs + 32);
+                // S is in registers: the next S product may overwrite the buffer
+                tc_fence_before();
+                mbar_arrive(s_free(x));
+                // causal mask, only in tiles that reach past some row's position
+                const int lim = pos - j * kPfKeys;  // keys c <= lim are visible
+                if (!__all_sync(0xffffffffu, lim >= kPfKeys - 1)) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= corr;
-                    tmem_st32(o_addr + c * 32, o);
+                    for (int c = 0; c < kPfKeys; ++c) xs[c] = c <= lim ? xs[c] : -INFINITY;
                 }
+                // row max: four chains of three-input maxima
+                float pm[4] = {xs[0], xs[1], xs[2], xs[3]};
+#pragma unroll
+                for (int c = 4; c < kPfKeys; c += 8) {
+                    pm[0] = max3f(pm[0], xs[c], xs[c + 1]);
+                    pm[1] = max3f(pm[1], xs[c + 2], xs[c + 3]);
+                    pm[2] = max3f(pm[2], xs[c + 4], xs[c + 5]);
+                    pm[3] = max3f(pm[3], xs[c + 6], xs[c + 7]);
+                }
+                const float mx = fmaxf(max3f(pm[0], pm[1], pm[2]), pm[3]) * p.scale_log2;  // scale > 0: the max commutes with it
+                // lazily moved reference max (log2 units): weights stay <= 2^kPfRescaleSlack
+                const bool bump = mx > m + kPfRescaleSlack;
+                float corr = 1.f;
+                if (bump) {
+                    corr = fast_exp2(m - mx);  // 0 on the first tile (m = -inf)
+                    m = mx;
+                }
+                // weights (scaled by 2^kPfP16Shift) as fp16 pairs, the lower key in
+                // the low half: (logit scale, shift) on key pairs by packed fp32 FMAs;
+                // the row sum in four packed fp32 accumulators
+                const float mneg = kPfP16Shift - m;
+                const uint64_t scale2 = f32x2(p.scale_log2, p.scale_log2), shift2 = f32x2(mneg, mneg);
+                uint64_t ps[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) ps[u] = 0ull;
+                float pw[kPfKeys / 2];
+#pragma unroll
+                for (int e = 0; e < kPfKeys / 2; ++e) {
+                    const float2 y = f32x2_split(fma_f32x2(f32x2(xs[2 * e], xs[2 * e + 1]), scale2, shift2));
+                    const float p0 = fast_exp2(y.x);
+                    const float p1 = fast_exp2(y.y);
+                    ps[e & 3] = add_f32x2(ps[e & 3], f32x2(p0, p1));
+                    pw[e] = __uint_as_float(pack_f16x2(p0, p1));
+                }
+                const float2 q01 = f32x2_split(add_f32x2(ps[0], ps[1])), q23 = f32x2_split(add_f32x2(ps[2], ps[3]));
+                l = l * corr + ((q01.x + q01.y) + (q23.x + q23.y));
+                if (j >= 1 && __any_sync(0xffffffffu, bump)) {
+                    // O holds P_{<j} V: rescale it once P_{j-1} V has completed
+                    const int64_t jp = nj - 1;
+                    ok = __all_sync(0xffffffffu, wait(o_done(x, (int)(jp & 1)), (uint32_t)((jp >> 1) & 1)));
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(o_addr + c * 32, o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] *= corr;
+                        tmem_st32(o_addr + c * 32, o);
+                    }
+                }
+                // P into buffer b, once the P V product two tiles back has read it
+                if (nj >= 2) {
+                    ok = __all_sync(0xffffffffu, wait(o_done(x, b), (uint32_t)(((nj - 2) >> 1) & 1)));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                tmem_st32(p_addr, pw);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(p_full(x, b));
             }
-            // P into buffer b, once P_{j-2} V has read it
-            if (j >= 2) {
-                ok = __all_sync(0xffffffffu, wait(o_done(x, b), ((j >> 1) - 1) & 1));
-                if (!ok) break;
-                tc_fence_after();
-            }
-            tmem_st32(p_addr, pw);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(p_full(x, b));
-        }
-        if (active && ok) {
-            const int jl = nkx - 1;
-            ok = __all_sync(0xffffffffu, wait(o_done(x, jl & 1), (jl >> 1) & 1));
-        }
-        if (active && ok) {
+            if (!ok) break;
+            // epilogue: O / l once the item's last P V has completed
+            const int64_t nl = n + nkx - 1;
+            ok = __all_sync(0xffffffffu, wait(o_done(x, (int)(nl & 1)), (uint32_t)((nl >> 1) & 1)));
+            if (!ok) break;
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *dst =
-                p.out + ((int64_t)(q0 + (row_ok ? i : 0)) * p.num_heads + (int64_t)g * G + gi) * D;
+                p.out + ((int64_t)(it.q0 + (row_ok ? i : 0)) * p.num_heads + (int64_t)it.g * G + gi) * D;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 float o[32];
@@ -549,6 +608,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                 }
             }
+            // O is in registers (and stored): the next item's first P V may overwrite it
+            tc_fence_before();
+            mbar_arrive(o_free(x));
+            n += nkx;
         }
     }
 
