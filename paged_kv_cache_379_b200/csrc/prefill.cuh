@@ -66,7 +66,8 @@ constexpr int kPfConvWarp = 11;       // first of the 4 V-conversion warps
 constexpr int kPfThreads = 480;
 constexpr int kPfRows = 128;          // MMA M: query rows per tile
 constexpr int kPfKeys = 64;           // keys per K/V tile
-constexpr int kPfStages = 3;          // K/V ring stages (two query buffers take the rest)
+constexpr int kPfStages = 4;          // K/V ring stages
+constexpr int kPfQBufs = 1;           // query buffers (pairs of query tiles)
 constexpr uint32_t kPfTmemCols = 512;
 // A row's softmax reference max moves only when a logit exceeds it by more
 // than this (log2 units), so unnormalised weights stay below 2^8.
@@ -130,7 +131,7 @@ struct PfLayout {
     static constexpr int kKTile = kPlanes * kKPlane;       // K or V tile
     static constexpr int kQ = 0;                           // Q buffer qb: tile A, then tile B
     static constexpr int kQBuf = 2 * kQTile;
-    static constexpr int kStage0 = 2 * kQBuf;              // stage st: K tile, then V tile
+    static constexpr int kStage0 = kPfQBufs * kQBuf;       // stage st: K tile, then V tile
     static constexpr int kStageBytes = 2 * kKTile;
     static constexpr int kBar = kStage0 + kPfStages * kStageBytes;
     // q_full[2], q_free[2], drain[2], kv_full[S], kv_empty[S], then per query
@@ -155,13 +156,15 @@ struct PfItem {
     int endA, endB, nkA, nk;  // causal: key tiles of tile A, of the pair (>= nkA)
 };
 
-// Persistent: each CTA walks the work items w = blockIdx.x, + gridDim.x, ...
-// Item w = (r, s, g) with the KV head fastest, then the sequence, then r:
-// the r-th pair of sequence s counted from its end (its longest), so every
-// sequence's longest pairs come first and the CTAs share each length class.
-// Consecutive items of a CTA overlap: the next item's queries load into the
-// other query buffer, and its first S is issued as soon as the softmax has
-// read the last S of the previous item, under that item's epilogue.
+// Persistent: each CTA takes one work item of every round of gridDim.x items,
+// in snake order (see item_of).  Item w = (r, s, g) with the KV head fastest,
+// then the sequence, then r: the r-th pair of sequence s counted from its end
+// (its longest), so every sequence's longest pairs come first and the CTAs
+// share each length class.  Consecutive items of a CTA overlap: the next
+// item's first K/V tile loads while the current item runs, its queries as
+// soon as the current item's last S products have completed, and its first S
+// is issued once the softmax has read the last S of the previous item, under
+// that item's epilogue.
 template <int D, int BS>
 __global__ void __launch_bounds__(kPfThreads, 1)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
@@ -250,6 +253,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // The CTA's kr-th item: rounds of gridDim.x items, taken in snake order
+    // (odd rounds reversed), so that the CTAs that take a round's longer items
+    // take the next round's shorter ones
+    auto item_of = [&](int64_t kr) -> int64_t {
+        const int64_t b = (kr & 1) ? (int64_t)gridDim.x - 1 - blockIdx.x : (int64_t)blockIdx.x;
+        return kr * gridDim.x + b;
+    };
     // item w, or false if it holds no pair
     auto decode = [&](int64_t w, PfItem &it) -> bool {
         const int64_t per_r = (int64_t)B * Hkv;
@@ -288,24 +298,43 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             prefetch_tensormap(&tmap_v);
         }
         int k = 0;         // items taken
+        int kq_issued = 0; // query loads issued
         int64_t T = 0;     // ring tiles issued
         bool ok = true;
-        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+        for (int64_t kr = 0; ok && kr * gridDim.x < W; ++kr) {
+            const int64_t w = item_of(kr);
+            if (w >= W) break;
             PfItem it;
             if (!decode(w, it)) continue;
-            const int qb = k & 1;
-            // the query buffer is free once both MMA warps' last S of item k-2 completed
-            if (k >= 2 && !__all_sync(0xffffffffu, wait(q_free(qb), ((k >> 1) - 1) & 1))) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(q_full(qb), (uint32_t)(2 * kPlanes * G * p.q_box * 128));
-                for (int x = 0; x < 2; ++x)
-                    for (int pl = 0; pl < kPlanes; ++pl)
-                        tma_load_4d(base + Lay::kQ + qb * Lay::kQBuf + x * Lay::kQTile + pl * kQPlane, &tmap_q,
-                                    q_full(qb), 0, pl, it.g * G, it.q0 + it.tA + x * p.tq);
-            }
-            ++k;
+            const int qb = k % kPfQBufs;
+            // the item's queries: the buffer is free once both MMA warps' last S of
+            // item k - kPfQBufs completed; issued after the item's first K/V tile, so
+            // that tile's load does not wait for the previous item's last S
+            auto load_q = [&]() -> bool {
+                if (k >= kPfQBufs &&
+                    !__all_sync(0xffffffffu, wait(q_free(qb), (uint32_t)((k / kPfQBufs - 1) & 1))))
+                    return false;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(q_full(qb), (uint32_t)(2 * kPlanes * G * p.q_box * 128));
+                    for (int x = 0; x < 2; ++x)
+                        for (int pl = 0; pl < kPlanes; ++pl)
+                            tma_load_4d(base + Lay::kQ + qb * Lay::kQBuf + x * Lay::kQTile + pl * kQPlane,
+                                        &tmap_q, q_full(qb), 0, pl, it.g * G, it.q0 + it.tA + x * p.tq);
+                }
+                __syncwarp();
+                ++kq_issued;
+                return true;
+            };
+            bool q_done = false;
             const int32_t *table = p.block_tables + (int64_t)it.s * p.max_blocks;
             for (int t = 0; t < it.nk; ++t, ++T) {
+                if (t == 1) {
+                    if (!load_q()) {
+                        ok = false;
+                        break;
+                    }
+                    q_done = true;
+                }
                 const int st = (int)(T % S);
                 const int key0 = t * kPfKeys;
                 const int nblk = min(kPfKeys / BS, (it.L - key0 + BS - 1) / BS);
@@ -328,11 +357,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                 }
             }
+            if (ok && !q_done && !load_q()) ok = false;   // an item of one key tile
+            if (!ok) break;
+            ++k;
         }
         if (lane == 0 && *abort_flag) {
             // let the loads this CTA issued land before it exits: the last two
             // query loads and each stage's last tile
-            for (int kq = max(0, k - 2); kq < k; ++kq) mbar_wait_bounded(q_full(kq & 1), (kq >> 1) & 1);
+            for (int kq = max(0, kq_issued - kPfQBufs); kq < kq_issued; ++kq)
+                mbar_wait_bounded(q_full(kq % kPfQBufs), (uint32_t)((kq / kPfQBufs) & 1));
             for (int st = 0; st < S; ++st)
                 if (st < T) {
                     const int64_t last = T - 1 - (T - 1 - st) % S;
@@ -354,14 +387,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int64_t T = 0;      // ring tiles consumed
         int64_t n = 0;      // S products of this query tile issued (= its P products)
         bool ok = true;
-        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+        for (int64_t kr = 0; ok && kr * gridDim.x < W; ++kr) {
+            const int64_t w = item_of(kr);
+            if (w >= W) break;
             PfItem it;
             if (!decode(w, it)) continue;
-            const int qb = k & 1;
+            const int qb = k % kPfQBufs;
             const bool act = x == 0 || it.hasB;
             const int nkx = x == 0 ? it.nkA : it.nk;
             const uint32_t qt = base + Lay::kQ + qb * Lay::kQBuf + x * Lay::kQTile;
-            if (act) ok = __all_sync(0xffffffffu, wait(q_full(qb), (k >> 1) & 1));
+            if (act) ok = __all_sync(0xffffffffu, wait(q_full(qb), (uint32_t)((k / kPfQBufs) & 1)));
             // S product number nn (tile j of the item, ring tile T0 + j)
             auto issue_s = [&](int64_t nn, int64_t tr) -> bool {
                 const int st = (int)(tr % S);
@@ -443,7 +478,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         float amax = 0.f;
         int64_t T = 0;
         bool ok = true;
-        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+        for (int64_t kr = 0; ok && kr * gridDim.x < W; ++kr) {
+            const int64_t w = item_of(kr);
+            if (w >= W) break;
             PfItem it;
             if (!decode(w, it)) continue;
             for (int t = 0; t < it.nk; ++t, ++T) {
@@ -491,7 +528,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t s_addr = lane_addr + x * Lay::kTmemTile;
         int64_t n = 0;      // S tiles of this query tile consumed (= P tiles written)
         bool ok = true;
-        for (int64_t w = blockIdx.x; ok && w < W; w += gridDim.x) {
+        for (int64_t kr = 0; ok && kr * gridDim.x < W; ++kr) {
+            const int64_t w = item_of(kr);
+            if (w >= W) break;
             PfItem it;
             if (!decode(w, it)) continue;
             const bool active = x == 0 || it.hasB;
