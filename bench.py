@@ -383,14 +383,24 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if args.l2_flush else None
 
-    def step(i):
+    def step(i, events=False):
         if flush is not None:
             flush.fill_((0 if i is None else i) & 255)   # evicts the previous step's lines from L2
-        device_step(resident, None if i is None else evs[i])
+        device_step(resident, evs[i] if (events and i is not None) else None)
 
     sampler = ClockSampler(local_rank)
     sampler.start()
+    # The timed window runs the steps' kernels back to back, as a serving loop
+    # does (each kernel may start under the end of the one before it); a
+    # second pass of the same K steps with events between the kernels gives
+    # each stage's own duration (the roofline's kernel time) -- and, with the
+    # L2 flushed between steps, the step time as the sum of the event
+    # intervals, which leaves the flush writes out.
     total_ms, clocks, remeasured = _timed_loop(step, K, W, stream, dev, dist, sampler)
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        step(i, events=True)
+    torch.cuda.synchronize(dev)
     stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(K)])
     copy_ms, append_ms, dec_ms = (float(x) for x in stage.mean(axis=0))
     if flush is not None:
@@ -523,6 +533,7 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
         "algorithmic_bytes_per_step": step_bytes,
         "seqs_per_s": round(all_seqs * K / (total_ms * 1e-3), 1),
         "frac_of_spec_hbm": round(gbs / world / SPEC_HBM_GBS, 4),
+        "stage_ms_note": "each stage's own duration: a second pass of the K steps with events between the kernels",
         "stage_ms": ({"append_decode_kv_cow": round(append_ms, 5), "decode": round(dec_ms, 5)} if fused else
                      {"copy_blocks": round(copy_ms, 5) if n_pairs else None, "append_decode_kv": round(append_ms, 5),
                       "decode": round(dec_ms, 5)}),
