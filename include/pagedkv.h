@@ -33,10 +33,12 @@
  *   the device.
  * - Every kernel is launched with programmatic dependent launch and lets the
  *   next kernel of the stream start early.  The decode kernels read seq_lens,
- *   block_tables and query before waiting for the previous kernel of the
- *   stream to finish (everything else after it); no kernel of this library
- *   writes those, and a kernel launched without that attribute (or one that
- *   never triggers its dependents early) is waited for as usual.
+ *   block_tables and query, and the pa_append_decode_kv* kernels seq_lens,
+ *   block_tables, cow_src and the new key / value rows, before waiting for the
+ *   previous kernel of the stream to finish (everything else after it); no
+ *   kernel of this library writes those, and a kernel launched without that
+ *   attribute (or one that never triggers its dependents early) is waited for
+ *   as usual.
  * - Preconditions NOT checked in the launch path (pa_validate_tables checks
  *   them on the device): table entries below num_blocks for the blocks a
  *   sequence uses; ceil(seq_len/block_size) <= max_blocks_per_seq;

@@ -116,30 +116,47 @@ __global__ void append_kv_kernel(const uint4 *__restrict__ key, const uint4 *__r
                                  int64_t *__restrict__ slots_out, int num_seqs, int max_blocks,
                                  int chunks_per_token, int block_size, int64_t num_slots, float k_inv, float v_inv)
 {
-    pdl_wait();
-    pdl_launch_dependents();
+    // The lengths, the table and the new rows are inputs no kernel of this
+    // library writes: they are read before waiting for the previous kernel of
+    // the stream; the slot output and the cache are written after it.
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)num_seqs * chunks_per_token) return;
-    const int s = (int)(i / chunks_per_token);
-    const int c = (int)(i - (int64_t)s * chunks_per_token);
-    const int64_t pos = (int64_t)seq_lens[s] - 1;
+    const bool live = i < (int64_t)num_seqs * chunks_per_token;
+    int s = 0, c = 0;
     int64_t slot = -1;
-    if (pos >= 0) {
-        const int64_t block_number = pos / block_size;
-        if (block_number < max_blocks) {
-            const int32_t physical = block_tables[(int64_t)s * max_blocks + block_number];
-            if (physical >= 0) slot = (int64_t)physical * block_size + (pos - block_number * block_size);
+    uint4 k0 = make_uint4(0, 0, 0, 0), k1 = k0, v0 = k0, v1 = k0;
+    if (live) {
+        s = (int)(i / chunks_per_token);
+        c = (int)(i - (int64_t)s * chunks_per_token);
+        if constexpr (FP8) {
+            k0 = key[2 * i];
+            k1 = key[2 * i + 1];
+            v0 = value[2 * i];
+            v1 = value[2 * i + 1];
+        } else {
+            k0 = key[i];
+            v0 = value[i];
+        }
+        const int64_t pos = (int64_t)seq_lens[s] - 1;
+        if (pos >= 0) {
+            const int64_t block_number = pos / block_size;
+            if (block_number < max_blocks) {
+                const int32_t physical = block_tables[(int64_t)s * max_blocks + block_number];
+                if (physical >= 0) slot = (int64_t)physical * block_size + (pos - block_number * block_size);
+            }
         }
     }
+    pdl_wait();
+    pdl_launch_dependents();
+    if (!live) return;
     if (c == 0 && slots_out) slots_out[s] = slot;
     if (slot < 0 || slot >= num_slots) return;
     const int64_t dst = slot * chunks_per_token + c;
     if constexpr (FP8) {
-        key_cache[dst] = quantise16(key[2 * i], key[2 * i + 1], k_inv);
-        value_cache[dst] = quantise16(value[2 * i], value[2 * i + 1], v_inv);
+        key_cache[dst] = quantise16(k0, k1, k_inv);
+        value_cache[dst] = quantise16(v0, v1, v_inv);
     } else {
-        key_cache[dst] = key[i];
-        value_cache[dst] = value[i];
+        key_cache[dst] = k0;
+        value_cache[dst] = v0;
     }
 }
 
@@ -153,7 +170,7 @@ __global__ void append_kv_kernel(const uint4 *__restrict__ key, const uint4 *__r
 // receives the new K/V -- the bytes that a block copy followed by the cache
 // write leave, with no ordering between the two needed, as no byte is written
 // twice.  Grid: (row slices of the block, sequence); a CTA covers rows
-// [r0, r0 + rows_per_cta) of both caches, one thread per 16-byte chunk with two
+// [r0, r0 + rows_per_cta) of both caches, one thread per 16-byte chunk with four
 // chunks per cache in flight.  Sequences without a copy only run the CTA that
 // holds row o.
 __global__ void __launch_bounds__(256) append_kv_cow_kernel(
@@ -162,11 +179,13 @@ __global__ void __launch_bounds__(256) append_kv_cow_kernel(
     const int32_t *__restrict__ cow_src, int64_t *__restrict__ slots_out, int max_blocks, int chunks_per_token,
     int block_size, int rows_per_cta, int64_t num_blocks)
 {
-    pdl_wait();
-    pdl_launch_dependents();
+    // The lengths, the table and the copy sources are inputs no kernel of this
+    // library writes: they are read before waiting for the previous kernel of
+    // the stream; the caches and the slot output are touched after it.
     const int s = blockIdx.y;
     const int r0 = blockIdx.x * rows_per_cta;
     const int r1 = min(block_size, r0 + rows_per_cta);
+    const int32_t src = cow_src ? cow_src[s] : -1;
     const int64_t pos = (int64_t)seq_lens[s] - 1;
     int64_t dst = -1, slot = -1;
     int o = -1;
@@ -181,9 +200,10 @@ __global__ void __launch_bounds__(256) append_kv_cow_kernel(
             }
         }
     }
+    pdl_wait();
+    pdl_launch_dependents();
     if (blockIdx.x == 0 && threadIdx.x == 0 && slots_out) slots_out[s] = slot;
     if (dst < 0) return;
-    const int32_t src = cow_src ? cow_src[s] : -1;
     const bool copy = src >= 0 && src < num_blocks && src != dst;
     const bool has_row = o >= r0 && o < r1;
     if (!copy && !has_row) return;
@@ -198,7 +218,7 @@ __global__ void __launch_bounds__(256) append_kv_cow_kernel(
     const uint4 *vs = copy ? value_cache + (int64_t)src * chunks_per_block : vd;
     const uint4 *kn = key + (int64_t)s * chunks_per_token;
     const uint4 *vn = value + (int64_t)s * chunks_per_token;
-    constexpr int U = 2;
+    constexpr int U = 4;
     int64_t c = c_begin + threadIdx.x;
     for (; c + (U - 1) * blockDim.x < c_end; c += U * blockDim.x) {
         uint4 k[U], v[U];

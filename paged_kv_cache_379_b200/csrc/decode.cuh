@@ -421,6 +421,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
         // ... and the histogram of the rest keys, for the largest-first order
         int nrest = 0;
         for (int s = threadIdx.x; s < B; s += kDecodeThreads) {
+            // the start of every table row into L2: the first items' table
+            // loads come right after the enumeration
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.block_tables + (int64_t)s * p.max_blocks));
             const int L = min(p.seq_lens[s], Lcap);
             const int key = rest_key(L);
             keys[s] = (int16_t)key;
