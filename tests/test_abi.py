@@ -139,3 +139,50 @@ def test_prefill_argument_errors_without_gpu(lib):
     assert call(b=0) == 0
     assert call(out=None) == -1
     assert call(q=P(4100)) == -8       # misaligned query
+
+
+def test_shared_prefix_and_cow_argument_errors_without_gpu(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    # pa_decode_shared(out, q, kc, vc, bt, sl, scale, bs, Hkv, B, Hq, D, max_blocks, nb, max_len, part,
+    #                  group_start, group_parts, num_groups, ws, ws_bytes, st)
+    args = [fake, fake, fake, fake, fake, fake, 1.0, 16, 8, 4, 64, 128, 8, 100, 128, 512, fake, fake, 2, fake,
+            1 << 30, None]
+
+    def shared(changes):
+        a = list(args)
+        for i, v in changes.items():
+            a[i] = v
+        return lib.pa_decode_shared(*a)
+    assert shared({16: None}) == -1      # groups given without their starts
+    assert shared({18: 5}) == -2         # more groups than sequences
+    assert shared({18: -1}) == -2
+    assert shared({15: 100}) == -2       # partition size not a multiple of 16
+    assert shared({19: None, 20: 0}) == -4   # the split form needs a workspace
+    assert shared({11: 96}) == -3        # head_dim not compiled
+    # pa_append_decode_kv_cow(k, v, kc, vc, bt, sl, cow_src, slots, B, max_blocks, Hkv, D, bs, nb, st)
+    assert lib.pa_append_decode_kv_cow(None, None, None, None, None, None, None, None, 0, 8, 8, 128, 16, 10,
+                                       None) == 0
+    assert lib.pa_append_decode_kv_cow(fake, fake, fake, fake, fake, fake, None, None, 3, 8, 8, 128, 16, 0,
+                                       None) == -2
+    assert lib.pa_append_decode_kv_cow(None, fake, fake, fake, fake, fake, None, None, 3, 8, 8, 128, 16, 10,
+                                       None) == -1
+    assert lib.pa_append_decode_kv_cow(fake, fake, fake, fake, fake, fake, None, None, 70000, 8, 8, 128, 16, 10,
+                                       None) == -2   # one grid row per sequence
+    assert lib.pa_append_decode_kv_cow(P(4100), fake, fake, fake, fake, fake, None, None, 3, 8, 8, 128, 16, 10,
+                                       None) == -8
+
+
+def test_prefix_groups_argument_errors(lib):
+    import numpy as np
+    t = np.zeros((2, 4), np.int32)
+    lens = np.array([8, 8], np.int32)
+    out_s = np.zeros(3, np.int32)
+    out_p = np.zeros(2, np.int32)
+    n = ctypes.c_int(0)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    # partition size not a multiple of the block size
+    assert lib.pa_prefix_groups(ptr(t), 2, 4, ptr(lens), 4, 6, ptr(out_s), ptr(out_p), ctypes.byref(n)) == -2
+    assert lib.pa_prefix_groups(ptr(t), 2, 4, ptr(lens), 4, 8, None, ptr(out_p), ctypes.byref(n)) == -1
+    assert lib.pa_prefix_groups(ptr(t), 2, 4, ptr(lens), 4, 8, ptr(out_s), ptr(out_p), ctypes.byref(n)) == 0
+    assert n.value == 1 and out_s.tolist() == [0, 2, 0] and out_p[0] == 1
