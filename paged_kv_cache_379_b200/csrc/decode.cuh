@@ -188,9 +188,6 @@ struct MergeScratch {
     float m[kConsumerWarps][ROWS];         // reference max that o and l are relative to (log2 units)
     float mt[kConsumerWarps][ROWS];        // true max of the logits seen (log2 units), >= m
     float l[kConsumerWarps][ROWS];
-    float cw[kConsumerWarps][ROWS];        // merge weight of each warp's state
-    float den[ROWS];                       // merged sum of weights
-    float M[ROWS];                         // merged reference max (log2 units)
 };
 
 // A work item as the scheduler publishes it.
@@ -246,9 +243,13 @@ struct DecodeSmem {
     static constexpr int ROWS = MODE == 0 ? GC : (MODE == 1 ? 8 : 16);
     using Ring = std::conditional_t<FP8, TileGeom8<D, BS>, TileGeom<D, BS>>;
     using Merge = MergeScratch<D, ROWS>;
+    static_assert(ROWS <= 32, "one query row per scheduler lane");
     static constexpr int kMergeOff = Ring::kPipeSmem;
     static constexpr int kQOff = (kMergeOff + (int)sizeof(Merge) + 127) & ~127;
-    static constexpr int kQBytes = ROWS * D * 2;                  // one item's query rows
+    // one item's query rows, each padded by 16 bytes: the MMA consumers' fragment
+    // loads (8 rows x 4 words per instruction) then fall in 32 distinct banks
+    static constexpr int kQRow = D * 2 + 16;
+    static constexpr int kQBytes = ROWS * kQRow;
     static constexpr int kItemOff = kQOff + kItemSlots * kQBytes;
     static constexpr int kChunkOff = kItemOff + kItemSlots * (int)sizeof(ItemInfo);
     static constexpr int kBarOff = (kChunkOff + kChunkSlots * (int)sizeof(ChunkInfo) + 7) & ~7;
@@ -625,20 +626,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
             } else {
                 it.stop = 1;
             }
-            if (lane == 0) {
-                items[islot] = it;
+            {
+                // the G query rows of each of the item's sequences, one after another,
+                // one row per lane into the padded rows of the item's query slot
                 const uint32_t bar = ifull_bar + 8 * islot;
-                if (!it.stop) {
-                    // the G query rows of each of the item's sequences, one after another
-                    const uint32_t qbytes = (uint32_t)(G * D * 2);
-                    const int nq = it.nseq > 0 ? it.nseq : 1;
-                    mbar_arrive_expect_tx(bar, qbytes * (uint32_t)nq);
-                    for (int i = 0; i < nq; ++i)
-                        bulk_load(base + Lay::kQOff + islot * Lay::kQBytes + (uint32_t)i * qbytes,
-                                  p.query + ((int64_t)(it.s + i) * p.num_heads + (int64_t)it.g * G) * D, qbytes, bar);
-                } else {
-                    mbar_arrive(bar);
+                const int rows = it.stop ? 0 : (it.nseq > 0 ? it.nseq : 1) * G;
+                if (lane == 0) {
+                    items[islot] = it;
+                    if (rows > 0)
+                        mbar_arrive_expect_tx(bar, (uint32_t)(rows * D * 2));
+                    else
+                        mbar_arrive(bar);
                 }
+                __syncwarp();
+                if (lane < rows)
+                    bulk_load(base + Lay::kQOff + islot * Lay::kQBytes + (uint32_t)(lane * Lay::kQRow),
+                              p.query + ((int64_t)(it.s + lane / G) * p.num_heads + (int64_t)it.g * G + lane % G) * D,
+                              (uint32_t)(D * 2), bar);
             }
             // chunks of the item's block table (and a stop marker after the last item)
             for (int cb = first_blk; ok && (cb < end_blk || it.stop); cb += kChunkBlocks) {
@@ -849,7 +853,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 float q[GC][8];
 #pragma unroll
                 for (int h = 0; h < GC; ++h) {
-                    const uint4 rq = *reinterpret_cast<const uint4 *>(qsm + (h * D + qc * 8) * 2);
+                    const uint4 rq = *reinterpret_cast<const uint4 *>(qsm + h * Lay::kQRow + qc * 16);
                     const uint32_t w[4] = {rq.x, rq.y, rq.z, rq.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -959,7 +963,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 // then O^T[D x heads] += V^T P^T.  Tokens are the MMA's M dimension,
                 // so no accumulator row is wasted when G <= 8; P^T is taken from the
                 // S^T accumulators by an in-register 8x8 transpose (movmatrix).
-                constexpr int NH = (MODE == 2) ? 2 : 1;  // 8-head column tiles
+                // The body is compiled once per count of 8-column tiles (NH): an item
+                // of at most 8 query rows runs the one-tile body even in the
+                // 16-row kernel, with half the accumulators and no second softmax.
+                auto mma_item = [&](auto nh_tag) {
+                constexpr int NH = decltype(nh_tag)::value;  // 8-head column tiles
                 constexpr int KSTEPS = D / 16;           // k-steps of S^T = K Q^T
                 constexpr int MT = D / 16;               // 16-row d tiles of O^T
                 const int gq = lane >> 2;                // MMA groupID
@@ -990,7 +998,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             for (int hh = 0; hh < 2; ++hh) {
                                 const int col = 16 * (tq + 4 * (kk >> 1)) + 8 * (kk & 1) + 4 * hh;
                                 uint2 w = make_uint2(0u, 0u);
-                                if (head < it.ncols) w = *reinterpret_cast<const uint2 *>(qsm + (head * D + col) * 2);
+                                if (head < it.ncols) w = *reinterpret_cast<const uint2 *>(qsm + head * Lay::kQRow + col * 2);
                                 const float2 f0 = unpack_bf16x2(w.x), f1 = unpack_bf16x2(w.y);
                                 v[kk][hh][0] = f0.x;
                                 v[kk][hh][1] = f0.y;
@@ -1043,7 +1051,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             for (int hh = 0; hh < 2; ++hh) {
                                 const int col = kk * 16 + hh * 8 + tq * 2;
                                 qb[nh][kk][hh] =
-                                    head < it.ncols ? *reinterpret_cast<const uint32_t *>(qsm + (head * D + col) * 2) : 0u;
+                                    head < it.ncols ? *reinterpret_cast<const uint32_t *>(qsm + head * Lay::kQRow + col * 2) : 0u;
                             }
                         }
                         qscale[nh][0] = qscale[nh][1] = p.scale_log2;
@@ -1065,8 +1073,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 const int kpar = lane >> 4;
                 const int vtok = (lane & 7) + ((lane >> 4) << 3);
                 const int vpar = (lane >> 3) & 1;
-                // 8-column tiles with a query row (two only for items of more than 8)
-                const int nh_used = NH == 1 ? 1 : (it.ncols + 7) / 8;
+                (void)qb, (void)q8, (void)ktok, (void)kpar, (void)vtok, (void)vpar;  // each form uses some
 
                 for (int j = warp; j < it.n_tiles; j += kConsumerWarps) {
                     const int ring = it.ring_base + j;
@@ -1118,8 +1125,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             ldsm_x4(kt + Geo::chunk_offset(ktok, 2 * kk + kpar), a0, a1, a2, a3);
 #pragma unroll
                             for (int nh = 0; nh < NH; ++nh)
-                                if (nh < nh_used)
-                                    mma_bf16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
+                                mma_bf16_16816((kk & 1) ? sd[nh] : sc[nh], a0, a1, a2, a3, qb[nh][kk][0], qb[nh][kk][1]);
                         }
                     }
 #pragma unroll
@@ -1222,10 +1228,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                             ldsm_x4_trans(vt + Geo::chunk_offset(vtok, 2 * mt + vpar), a0, a1, a2, a3);
 #pragma unroll
                             for (int nh = 0; nh < NH; ++nh) {
-                                if (nh < nh_used) {
-                                    mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
-                                    mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
-                                }
+                                mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
+                                mma_bf16_16816(o[mt][nh], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
                             }
                         }
                     }
@@ -1264,40 +1268,41 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                         }
                     }
                 }
+                };
+                if constexpr (MODE == 2) {
+                    if (it.ncols > 8)
+                        mma_item(std::integral_constant<int, 2>{});
+                    else
+                        mma_item(std::integral_constant<int, 1>{});
+                } else {
+                    mma_item(std::integral_constant<int, 1>{});
+                }
             }
             consumer_bar();  // every warp's state is in the merge scratch
+            // the item's slot (its description and query rows) is read no more
+            if (threadIdx.x == 0) mbar_arrive(iempty_bar + 8 * islot);
             // ---- merge the four warps of this item (after an abort the values are
             // meaningless but harmless; the next item check stops every warp)
             const bool direct = p.direct_single && it.nparts == 1;
-            // per head row: the combined true max is the common reference (every
-            // warp's own reference is <= it, so the weights are <= 1)
             const int ncols = MODE == 0 ? G : it.ncols;
-            if (threadIdx.x < ncols) {
-                const int row = threadIdx.x;
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->mt[w][row]);
-                float den = 0.f;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = ms->m[w][row];
-                    const float c = (M != -INFINITY && mw != -INFINITY) ? exp2f(mw - M) : 0.f;
-                    ms->cw[w][row] = c;
-                    den = fmaf(c, ms->l[w][row], den);
-                }
-                ms->den[row] = den;
-                ms->M[row] = M;
-            }
-            consumer_bar();
-            // weighted sum of the four accumulators, 4 columns per thread
+            // weighted sum of the four accumulators, 4 columns per thread; each
+            // thread forms its row's weights itself: the combined true max is the
+            // common reference (every warp's own reference is <= it, so the
+            // weights are <= 1)
             constexpr int D4 = D / 4;
             for (int idx = threadIdx.x; idx < ncols * D4; idx += kConsumerWarps * 32) {
                 const int row = idx / D4;
                 const int d = (idx - row * D4) * 4;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ms->mt[w][row]);
+                float den = 0.f;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float c = ms->cw[w][row];
+                    const float mw = ms->m[w][row];
+                    const float c = (M != -INFINITY && mw != -INFINITY) ? exp2f(mw - M) : 0.f;
+                    den = fmaf(c, ms->l[w][row], den);
                     const float4 v = *reinterpret_cast<const float4 *>(&ms->o[w][row][d]);
                     acc.x = fmaf(c, v.x, acc.x);
                     acc.y = fmaf(c, v.y, acc.y);
@@ -1308,7 +1313,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                 // its sequence row / G
                 const int64_t hrow = (int64_t)(it.s + row / G) * p.num_heads + (int64_t)it.g * G + row % G;
                 const bool direct_row = direct || (p.direct_single && ((it.single_mask >> (row / G)) & 1));
-                const float den = ms->den[row];
                 acc.x *= p.v_scale;
                 acc.y *= p.v_scale;
                 acc.z *= p.v_scale;
@@ -1323,14 +1327,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
                     const int64_t wi = hrow * p.max_parts + it.part;
                     *reinterpret_cast<float4 *>(p.ws_o + wi * D + d) = acc;
                     if (d == 0) {
-                        const float M = ms->M[row];
                         p.ws_m[wi] = M == -INFINITY ? -INFINITY : M * kLn2;
                         p.ws_l[wi] = den;
                     }
                 }
             }
-            consumer_bar();  // merge scratch and the item slot may be reused
-            if (threadIdx.x == 0) mbar_arrive(iempty_bar + 8 * islot);
+            consumer_bar();  // the merge scratch may be reused
             ++item_seq;
         }
     }
