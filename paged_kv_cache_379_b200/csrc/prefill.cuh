@@ -14,23 +14,25 @@
 // them.  Keys are processed in tiles of 64.  Fifteen warps:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: warp w owns TMEM
 //              lanes 32(w % 4) .. +31, one row per thread; it reads S from
-//              TMEM, keeps a lazily moved reference max, writes P back over S
-//              as fp16 (rounded to nearest: 11 significant bits),
-//              rescales O in TMEM when a reference moves, and finally
-//              normalises O and stores the output rows;
-//   warp 8     producer: TMA loads of the two query tiles (once) and of 64-key
-//              K and V tiles, block by block through the table, into a 4-stage
-//              ring (a stage frees once both query tiles' P V have read it);
-//   warps 9-10 MMA: warp 9 allocates TMEM -- two 64-column S/P buffers per
-//              query tile (A: columns 0..127, B: 128..255), O of A from 256, O
-//              of B from 256 + D; one thread of warp 9 issues tile A's
-//              tcgen05.mma, one of warp 10 tile B's:
+//              TMEM (which frees the S buffer for the next S), keeps a lazily
+//              moved reference max, writes P as fp16 (rounded to nearest: 11
+//              significant bits) into one of two P buffers, rescales O in
+//              TMEM when a reference moves, and finally normalises O and
+//              stores the output rows;
+//   warp 8     producer: TMA loads of the two query tiles and of 64-key K and
+//              V tiles, block by block through the table, into a 4-stage ring
+//              (a stage frees once both query tiles' S and P V have read it);
+//   warps 9-10 MMA: warp 9 allocates TMEM -- per query tile a 64-column S
+//              buffer and two 32-column P buffers (A: columns 0..127, B:
+//              128..255), O of A from 256, O of B from 256 + D.  One thread of
+//              warp 9 issues both tiles' S products, one of warp 10 both
+//              tiles' P V products:
 //                S_X = Q_X K_j^T    (SS form, bf16: M 128, N 64, K D)
 //                O_X += P V_j       (TS form, fp16: P read from TMEM; V an
 //                                    MN-major shared-memory operand)
-//              S_X(j) goes to buffer j % 2, so it overlaps the softmax of
-//              S_X(j-1); completion is tracked by tcgen05.commit on mbarriers,
-//              one per buffer.  The two tiles' chains run independently;
+//              so S_X(j+1) is issued as soon as the softmax has read S_X(j) and
+//              is never queued behind a P V that waits for P; completion is
+//              tracked by tcgen05.commit on mbarriers;
 //   warps 11-14 convert every V tile in shared memory from bf16 to fp16 in
 //              place as soon as it lands (16 keys each), zeroing rows past the
 //              sequence end; the four quarters meet on a per-stage mbarrier
@@ -220,12 +222,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (threadIdx.x == 32) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(q_full(b), 1);
-            mbar_init(q_free(b), 2);  // one commit from each MMA warp after its last S of the item
+            mbar_init(q_free(b), 1);  // the S warp's commit after its last S of the item
             mbar_init(drain(b), 1);
         }
         for (int i = 0; i < S; ++i) {
             mbar_init(kv_full(i), 1);
-            mbar_init(kv_empty(i), 2);  // one commit from each MMA warp
+            mbar_init(kv_empty(i), 2);  // one commit from each MMA warp (K read by S, V by P V)
             mbar_init(v16(i), 4);       // one arrival per conversion warp
         }
         for (int x = 0; x < 2; ++x) {
@@ -372,20 +374,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     mbar_wait_bounded(kv_full(st), (uint32_t)((last / S) & 1));
                 }
         }
-    } else if (warp >= kPfMmaWarp && warp < kPfConvWarp) {
-        // ------------------------------------------------------------ MMA issue
-        // Warp 9 issues tile A's products, warp 10 tile B's.  Per key tile j of
-        // an item: S_X(j+1) (once the softmax has read S_X(j)) before waiting for
-        // P_X(j), then P_X(j) V once the softmax has written P and V(j) is fp16.
-        // Each warp releases every K/V stage with its own commit, also for key
-        // tiles its query tile skips, and the item's query buffer after its last S.
-        const int x = warp - kPfMmaWarp;
+    } else if (warp == kPfMmaWarp) {
+        // ------------------------------------------------------------ S products
+        // Warp 9 issues both query tiles' S = Q K^T: S_X(j) as soon as K/V tile j
+        // has landed and the softmax has read S_X(j-1), never behind a P V
+        // product (those come from warp 10), so the next S is ready when the
+        // softmax finishes the current tile.  After tile j's S products it
+        // commits once to the stage's release (the K half of its reads), and
+        // after the item's last S to the query buffer's.
         constexpr uint32_t kIdS = idesc_bf16_f32(kPfRows, kPfKeys, false, false);
-        constexpr uint32_t kIdO = idesc_f16_f32(kPfRows, D, false, true);
         int k = 0;          // items taken
-        int kx = 0;         // items with this query tile active
         int64_t T = 0;      // ring tiles consumed
-        int64_t n = 0;      // S products of this query tile issued (= its P products)
+        int64_t n[2] = {0, 0};  // S products issued per query tile
         bool ok = true;
         for (int64_t kr = 0; ok && kr * gridDim.x < W; ++kr) {
             const int64_t w = item_of(kr);
@@ -393,65 +393,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             PfItem it;
             if (!decode(w, it)) continue;
             const int qb = k % kPfQBufs;
-            const bool act = x == 0 || it.hasB;
-            const int nkx = x == 0 ? it.nkA : it.nk;
-            const uint32_t qt = base + Lay::kQ + qb * Lay::kQBuf + x * Lay::kQTile;
-            if (act) ok = __all_sync(0xffffffffu, wait(q_full(qb), (uint32_t)((k / kPfQBufs) & 1)));
-            // S product number nn (tile j of the item, ring tile T0 + j)
-            auto issue_s = [&](int64_t nn, int64_t tr) -> bool {
-                const int st = (int)(tr % S);
-                if (!__all_sync(0xffffffffu, wait(kv_full(st), (uint32_t)((tr / S) & 1)))) return false;
-                if (nn >= 1 && !__all_sync(0xffffffffu, wait(s_free(x), (uint32_t)((nn - 1) & 1)))) return false;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t kt = base + Lay::kStage0 + st * Lay::kStageBytes;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        tc_mma_bf16(tmem + x * Lay::kTmemTile,
-                                    desc_kmajor_sw128(qt + (kk >> 2) * kQPlane + (kk & 3) * 32),
-                                    desc_kmajor_sw128(kt + (kk >> 2) * kKPlane + (kk & 3) * 32), kIdS, kk > 0);
-                    }
-                    tc_commit(s_full(x));
-                }
-                __syncwarp();
-                return true;
-            };
-            if (ok && act && nkx > 0) ok = issue_s(n, T);
+            ok = __all_sync(0xffffffffu, wait(q_full(qb), (uint32_t)((k / kPfQBufs) & 1)));
             for (int j = 0; ok && j < it.nk; ++j) {
                 const int64_t tr = T + j;
                 const int st = (int)(tr % S);
-                if (act && j < nkx) {
-                    const int64_t nj = n + j;
-                    const int b = (int)(nj & 1);
-                    if (j + 1 < nkx) {
-                        ok = issue_s(nj + 1, tr + 1);
-                        if (!ok) break;
+                ok = __all_sync(0xffffffffu, wait(kv_full(st), (uint32_t)((tr / S) & 1)));
+                for (int x = 0; ok && x < 2; ++x) {
+                    if (j >= (x == 0 ? it.nkA : (it.hasB ? it.nk : 0))) continue;
+                    const int64_t nn = n[x] + j;
+                    if (nn >= 1 && !__all_sync(0xffffffffu, wait(s_free(x), (uint32_t)((nn - 1) & 1)))) {
+                        ok = false;
+                        break;
                     }
-                    ok = __all_sync(0xffffffffu, wait(p_full(x, b), (uint32_t)((nj >> 1) & 1)));
-                    if (ok) ok = __all_sync(0xffffffffu, wait(v16(st), (uint32_t)((tr / S) & 1)));
-                    // O of the previous item must have been read by its epilogue
-                    if (ok && j == 0 && kx >= 1) ok = __all_sync(0xffffffffu, wait(o_free(x), (uint32_t)((kx - 1) & 1)));
-                    if (!ok) break;
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t vt = base + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile;
-                        // P of the tile's 64 keys: fp16 pairs in kPfKeys / 2 columns; a K
-                        // step of 16 keys is 8 columns
+                        const uint32_t q_lo = desc_lo_sw128(base + Lay::kQ + qb * Lay::kQBuf + x * Lay::kQTile, 16);
+                        const uint32_t k_lo = desc_lo_sw128(base + Lay::kStage0 + st * Lay::kStageBytes, 16);
 #pragma unroll
-                        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-                            tc_mma_bf16_ts(tmem + Lay::kTmemO + x * D,
-                                           tmem + x * Lay::kTmemTile + kPfKeys + b * (kPfKeys / 2) + kk * 8,
-                                           desc_mnmajor_sw128(vt + kk * 16 * 128, kKPlane), kIdO, j > 0 || kk > 0);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            tc_mma_lo(tmem + x * Lay::kTmemTile, q_lo + (uint32_t)(((kk >> 2) * kQPlane + (kk & 3) * 32) >> 4),
+                                      k_lo + (uint32_t)(((kk >> 2) * kKPlane + (kk & 3) * 32) >> 4), kIdS, kk > 0);
                         }
-                        tc_commit(o_done(x, b));
+                        tc_commit(s_full(x));
                     }
                     __syncwarp();
-                } else {
-                    // a key tile this query tile does not need: wait for it to land so the
-                    // release below cannot run ahead of the load
-                    ok = __all_sync(0xffffffffu, wait(kv_full(st), (uint32_t)((tr / S) & 1)));
-                    if (!ok) break;
                 }
+                if (!ok) break;
                 if (lane == 0) tc_commit(kv_empty(st));
                 __syncwarp();
             }
@@ -461,11 +428,66 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (lane == 0) tc_commit(q_free(qb));
             __syncwarp();
             T += it.nk;
-            if (act) {
-                n += nkx;
-                ++kx;
-            }
+            n[0] += it.nkA;
+            if (it.hasB) n[1] += it.nk;
             ++k;
+        }
+    } else if (warp == kPfMmaWarp + 1) {
+        // ------------------------------------------------------------ P V products
+        // Warp 10 issues both query tiles' O += P V_j once the softmax has written
+        // P_X(j) and V_j is fp16 (which also means tile j has landed), the first
+        // of an item once the previous item's epilogue has read O; then commits
+        // once to the stage's release (the V half of its reads).
+        constexpr uint32_t kIdO = idesc_f16_f32(kPfRows, D, false, true);
+        int64_t T = 0;          // ring tiles consumed
+        int64_t n[2] = {0, 0};  // P V products issued per query tile
+        int kx[2] = {0, 0};     // items with query tile x active
+        bool ok = true;
+        for (int64_t kr = 0; ok && kr * gridDim.x < W; ++kr) {
+            const int64_t w = item_of(kr);
+            if (w >= W) break;
+            PfItem it;
+            if (!decode(w, it)) continue;
+            for (int j = 0; ok && j < it.nk; ++j) {
+                const int64_t tr = T + j;
+                const int st = (int)(tr % S);
+                ok = __all_sync(0xffffffffu, wait(v16(st), (uint32_t)((tr / S) & 1)));
+                for (int x = 0; ok && x < 2; ++x) {
+                    if (j >= (x == 0 ? it.nkA : (it.hasB ? it.nk : 0))) continue;
+                    const int64_t nj = n[x] + j;
+                    const int b = (int)(nj & 1);
+                    ok = __all_sync(0xffffffffu, wait(p_full(x, b), (uint32_t)((nj >> 1) & 1)));
+                    // O of the previous item must have been read by its epilogue
+                    if (ok && j == 0 && kx[x] >= 1)
+                        ok = __all_sync(0xffffffffu, wait(o_free(x), (uint32_t)((kx[x] - 1) & 1)));
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t v_lo = desc_lo_sw128(base + Lay::kStage0 + st * Lay::kStageBytes + Lay::kKTile, kKPlane);
+                        // P of the tile's 64 keys: fp16 pairs in kPfKeys / 2 columns; a K
+                        // step of 16 keys is 8 columns
+#pragma unroll
+                        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
+                            tc_mma_ts_lo(tmem + Lay::kTmemO + x * D,
+                                         tmem + x * Lay::kTmemTile + kPfKeys + b * (kPfKeys / 2) + kk * 8,
+                                         v_lo + (uint32_t)(kk * 16 * 128 / 16), kIdO, j > 0 || kk > 0);
+                        }
+                        tc_commit(o_done(x, b));
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (lane == 0) tc_commit(kv_empty(st));
+                __syncwarp();
+            }
+            if (!ok) break;
+            T += it.nk;
+            n[0] += it.nkA;
+            ++kx[0];
+            if (it.hasB) {
+                n[1] += it.nk;
+                ++kx[1];
+            }
         }
     } else if (warp >= kPfConvWarp) {
         // ------------------------------------------------------------ V to fp16

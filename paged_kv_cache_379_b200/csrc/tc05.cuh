@@ -45,7 +45,7 @@ constexpr uint64_t kDescVersion = 1ull << 46;
 // 8-row groups 1024 bytes apart (stride byte offset); the leading byte offset
 // is unused by swizzled K-major layouts and set to 16 bytes.  A K step of 16
 // bf16 elements inside the atom advances the start address by 32 bytes.
-__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr)
+__host__ __device__ constexpr uint64_t desc_kmajor_sw128(uint32_t saddr)
 {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | kDescVersion |
            kDescSw128;
@@ -54,11 +54,29 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr)
 // MN-major operand (rows = K, 64 contiguous MN elements per 128-byte row):
 // atoms of 8 K-rows 1024 bytes apart along K (stride byte offset), atoms along
 // MN `lbo` bytes apart (leading byte offset).
-__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo)
+__host__ __device__ constexpr uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo)
 {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)(1024 >> 4) << 32) | kDescVersion | kDescSw128;
 }
+
+// The two words of those descriptors apart: the high word (stride byte offset,
+// version, swizzle mode) is the same for every operand here, and the low word
+// (start address, leading byte offset) of an address plus a multiple of 16
+// bytes is the low word of the address plus that multiple / 16 (shared-memory
+// addresses stay below 2^18).  An MMA loop then derives each k-step's
+// descriptor with one add instead of rebuilding it.
+constexpr uint32_t kDescHiSw128 = (uint32_t)((((uint64_t)(1024 >> 4) << 32) | kDescVersion | kDescSw128) >> 32);
+__host__ __device__ constexpr uint32_t desc_lo_sw128(uint32_t saddr, uint32_t lbo)
+{
+    return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+
+static_assert(desc_kmajor_sw128(0x1C400u) == (((uint64_t)kDescHiSw128 << 32) | desc_lo_sw128(0x1C400u, 16)) &&
+                  desc_kmajor_sw128(0x1C400u + 96) == (((uint64_t)kDescHiSw128 << 32) | (desc_lo_sw128(0x1C400u, 16) + 6)) &&
+                  desc_mnmajor_sw128(0x30000u + 3 * 2048, 8192) ==
+                      (((uint64_t)kDescHiSw128 << 32) | (desc_lo_sw128(0x30000u, 8192) + 3 * 128)),
+              "split descriptor words");
 
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, dense:
 // D format (1 = f32) in bits [4,6), A format (1 = bf16) in [7,10), B format in
@@ -77,15 +95,18 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n, bool a_mn_maj
            ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
-__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            bool accumulate)
+// D[tmem] (+)= A[smem] * B[smem], issued by one thread, both descriptors given
+// by their low words over kDescHiSw128.
+__device__ __forceinline__ void tc_mma_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                          bool accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
         "setp.ne.u32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        "mov.b64 da, {%1, %5};\n\t"
+        "mov.b64 db, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"((uint32_t)accumulate), "r"(kDescHiSw128)
         : "memory");
 }
 
@@ -161,15 +182,17 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t *v)
 
 // D[tmem] (+)= A[tmem] * B[smem]: A (M x 16, K-major) read from TMEM -- lane =
 // row, two 16-bit K elements per 32-bit column, the lower K index in the low
-// half; issued by one thread.
-__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                               bool accumulate)
+// half; B's descriptor given by its low word over kDescHiSw128; issued by one
+// thread.
+__device__ __forceinline__ void tc_mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
+                                             bool accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
         "setp.ne.u32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        "mov.b64 db, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"((uint32_t)accumulate), "r"(kDescHiSw128)
         : "memory");
 }
 
