@@ -92,12 +92,14 @@ def test_variants_match_oracle(D, bs, Hq, Hkv):
         assert_close(_run(w, kind, part), ref, f"D{D} bs{bs} {Hq}/{Hkv} {kind}/{part}")
 
 
-@pytest.mark.parametrize("B", [256, 257, 600])
+@pytest.mark.parametrize("B", [256, 257, 600, 3000])
 def test_batch_sizes_around_the_rank_sort_limit(B):
-    """The work items of a launch are ordered largest first by a block-wide rank
-    sort for batches of up to 256 sequences and by the scheduler warp's
-    counting sort above that: both orders (and the items' split into
-    partitions) against the oracle, ragged lengths with empty sequences."""
+    """The work items of a launch are ordered largest first by a counting sort
+    over the remainders' tile counts (the first item of a CTA selected from the
+    histogram before the order is scattered), with every CTA's enumeration
+    tables in shared memory: batches around a warp multiple and one of 3000
+    sequences (tables of ~25 KB per CTA), in one pass, split and the plan's
+    choice, against the oracle, ragged lengths with empty sequences."""
     rng = np.random.default_rng(900 + B)
     lens = rng.integers(0, 700, B)
     lens[::37] = 0

@@ -127,3 +127,23 @@ def test_groups_that_compute_fewer_partitions_than_shared():
         assert np.array_equal(got, split), gp
     ref = oracle.paged_decode(w.query, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, w.scale)
     assert_close(got, ref, "groups computing fewer partitions")
+
+
+def test_many_groups_and_sequences():
+    """More groups than the kernel has threads (the enumeration's per-group
+    loop takes several rounds) and over a thousand sequences: 300 groups of
+    2-6 sequences sharing 1-3 partitions, against the oracle and bit for bit
+    against the split decode."""
+    part = 64
+    rng = np.random.default_rng(31)
+    sizes = rng.integers(2, 7, size=300).tolist()
+    shared = rng.integers(1, 4, size=300).tolist()
+    w = _grouped_case(909, 4, 2, 64, 16, part, sizes=sizes, shared_parts=shared, tails=[0, 3, 16, 40, 64, 70])
+    assert w.num_seqs > 1000
+    gs, gp = ops.prefix_groups(w.block_tables, w.seq_lens, w.block_size, part)
+    assert len(gp) == 300 and np.array_equal(np.diff(gs), sizes) and gp.tolist() == shared
+    got, split, _ = _decode_both(w, w.block_tables, part, (gs, gp))
+    ref = oracle.paged_decode(w.query, w.key_cache, w.value_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(got, ref, "300 groups, %d sequences" % w.num_seqs)
+    assert np.array_equal(got, split)
+    assert ops.device_status() == 0
