@@ -563,7 +563,14 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
                                  "fused_with_cache_write": fused,
                                  "ms": round(cow_ms, 5),
                                  "gbs": round(copy_bytes / (cow_ms * 1e-3) / 1e9, 2) if cow_ms > 0 else None,
-                                 "share_of_step": round(cow_ms / (copy_ms + append_ms + dec_ms), 4)}
+                                 "share_of_step": round(cow_ms / (copy_ms + append_ms + dec_ms), 4),
+                                 # back to back the copies overlap the decode's start: what they
+                                 # add to the step is the step minus the decode's own duration
+                                 "exposed_ms_back_to_back": round(max(0.0, total_ms / K - dec_ms), 5),
+                                 "exposed_share_back_to_back": round(max(0.0, total_ms / K - dec_ms) / (total_ms / K), 4),
+                                 "note": ("share_of_step: the copy launch's own duration (events between the "
+                                          "kernels) over the sum of the stages; exposed_*: the whole step back "
+                                          "to back minus the decode's own duration")}
     if remeasured:
         line["clocks_note"] = "first timed region saw a thermal/hw slowdown reason; re-measured once"
     if e2e:
