@@ -61,6 +61,8 @@ KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_379_b200", "csrc", f)
                   for f in ("decode.cuh", "common.cuh", "pagedkv.cu", "cache_ops.cuh", "prefill.cuh", "tc05.cuh")]
 PROFILE_FP8 = os.path.join(ROOT, "profiles", "paged_decode_fp8_gqa_ncu.md")
 PROFILE_PREFILL = os.path.join(ROOT, "profiles", "paged_prefill_prompt2k_ncu.md")
+PROFILE_SHARED = os.path.join(ROOT, "profiles", "paged_decode_shared_prefix_ncu.md")
+PROFILE_LONG = os.path.join(ROOT, "profiles", "paged_decode_long_ncu.md")
 METRIC_FP8 = "paged-decode KV GB/s, FP8 E4M3 KV cache (per-tensor scales), GQA 64q/8kv d128 b16"
 METRIC_PREFILL = "paged-prefill useful TFLOP/s (causal), 8 x 2048-token prompts, GQA 64q/8kv d128 b16"
 PREFILL_SHAPE = dict(num_seqs=8, prompt=2048, num_heads=64, num_kv_heads=8, head_dim=128, block_size=16)
@@ -505,7 +507,16 @@ def run_decode(args, rank: int, world: int, local_rank: int) -> dict | None:
     gbs = all_bytes * K / (total_ms * 1e-3) / 1e9
     achieved = roof_bytes / (dec_ms * 1e-3) / 1e9
     peak, peak_src = measured_peak()
-    traffic = profiled_traffic() if (name == "gqa" and not part) else None
+    # DRAM bytes per decode call from the committed ncu captures, for the
+    # configurations they were taken on (whole batch, no L2 flush)
+    traffic = None
+    if not args.num_seqs and not args.l2_flush:
+        if name == "gqa" and not part:
+            traffic = profiled_traffic()
+        elif name == "shared" and groups is not None and part == 1024:
+            traffic = profiled_traffic(PROFILE_SHARED)
+        elif name == "long" and not int(args.partition):
+            traffic = profiled_traffic(PROFILE_LONG)
     path = f"split, partition {plan} (partition kernel + LSE reduce)" if plan else "one pass"
     if groups is not None:
         path = (f"shared-prefix groups ({len(gp_h)} groups; the shared {int(gp_h.max())} x {part}-token "
