@@ -864,6 +864,143 @@ def run_cow(args, rank: int, world: int, local_rank: int) -> dict | None:
     return line
 
 
+def swap_row_plan(w):
+    """The swap row's host work: the pool adopts the batch's step tables, every
+    4th sequence is swapped out to a host pool sized for exactly those blocks,
+    then all of them back in.  Returns (tables, swapped sequences, host blocks,
+    swap-out pairs, swap-in pairs), the pairs int64 [P, 2]."""
+    from paged_kv_cache_379_b200.pool import BlockPool, swap_plan
+    from paged_kv_cache_379_b200.step import host_step
+
+    gpu_pool, tables, nblk, _, _ = host_step(w)
+    swapped = np.arange(0, w.num_seqs, 4)                  # a quarter of the batch
+    n_host = int(nblk[swapped].sum())
+    with BlockPool(n_host, w.block_size) as host_pool:
+        outs, ins, host_tables = [], [], []
+        for s in swapped:
+            host_table, po = swap_plan(gpu_pool, host_pool, tables[s, :nblk[s]])
+            host_tables.append(host_table)
+            outs.append(po)
+        for host_table in host_tables:
+            _, pi = swap_plan(host_pool, gpu_pool, host_table)
+            ins.append(pi)
+    gpu_pool.close()
+    return tables, swapped, n_host, np.concatenate(outs).astype(np.int64), np.concatenate(ins).astype(np.int64)
+
+
+def run_swap(args, rank: int, world: int, local_rank: int) -> dict | None:
+    """Preemption by swapping (the CPU-GPU block allocator of [深度解析
+    «BlockAllocator 源码核心»]): the blocks of a quarter of the GQA batch's
+    sequences move to a pinned host cache through the host pool's swap plan
+    (pa_pool_swap_plan) and back into the GPU pool (pa_swap_blocks both ways).
+    A step is the swap-out plus the swap-in; device time by events around each
+    launch.  The denominator is measured in the same run: the copy engines'
+    rate (cudaMemcpyAsync between a device buffer and pinned host memory) for
+    the same bytes, each direction."""
+    import torch
+
+    from paged_kv_cache_379_b200 import ops
+    from paged_kv_cache_379_b200 import workload as wlmod
+    from paged_kv_cache_379_b200.step import DecodeBatch
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    stream = torch.cuda.current_stream(dev)
+    K, W = args.steps, args.warmup
+    w = wlmod.make("gqa", seed=rank_seed(rank, "gqa"))
+    tables, swapped, n_host, out_pairs, in_pairs = swap_row_plan(w)
+    batch = DecodeBatch(w, dev, tables=tables)
+    shape = (n_host,) + tuple(batch.key_cache.shape[1:])
+    host_k = torch.zeros(shape, dtype=torch.bfloat16).pin_memory()
+    host_v = torch.zeros(shape, dtype=torch.bfloat16).pin_memory()
+    d_out = torch.from_numpy(out_pairs).to(dev)
+    d_in = torch.from_numpy(in_pairs).to(dev)
+    blk_bytes = w.block_size * w.num_kv_heads * w.head_dim * 2
+    bytes_out = int(out_pairs.shape[0]) * blk_bytes * 2     # K and V blocks over the link, GPU -> host
+    bytes_in = int(in_pairs.shape[0]) * blk_bytes * 2       # and back
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    def step(i):
+        if i is not None:
+            ev[i][0].record(stream)
+        ops.swap_blocks(host_k, host_v, batch.key_cache, batch.value_cache, d_out, stream=stream)
+        if i is not None:
+            ev[i][1].record(stream)
+        ops.swap_blocks(batch.key_cache, batch.value_cache, host_k, host_v, d_in, stream=stream)
+        if i is not None:
+            ev[i][2].record(stream)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    total_ms, clocks, remeasured = _timed_loop(step, K, W, stream, dev, dist, sampler)
+    sampler.stop()
+    out_ms = float(np.mean([ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]))
+    in_ms = float(np.mean([ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]))
+
+    # the copy engines on the same bytes, contiguous: the link's measured rate
+    dbuf = torch.empty(max(bytes_out, bytes_in), dtype=torch.uint8, device=dev)
+    hbuf = torch.empty(max(bytes_out, bytes_in), dtype=torch.uint8).pin_memory()
+    ce = []
+    for _ in range(3):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        hbuf[:bytes_out].copy_(dbuf[:bytes_out], non_blocking=True)
+        e[1].record(stream)
+        dbuf[:bytes_in].copy_(hbuf[:bytes_in], non_blocking=True)
+        e[2].record(stream)
+        torch.cuda.synchronize(dev)
+        ce.append((e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])))
+    ce_out_ms = float(np.median([c[0] for c in ce]))
+    ce_in_ms = float(np.median([c[1] for c in ce]))
+    vals = torch.tensor([out_ms, in_ms, total_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    out_ms, in_ms, total_ms = (float(v) for v in vals.tolist())
+    if rank != 0:
+        return None
+    ms_per_step = total_ms / K
+    step_bytes = bytes_out + bytes_in
+    achieved = step_bytes / ((out_ms + in_ms) * 1e-3) / 1e9
+    peak = step_bytes / ((ce_out_ms + ce_in_ms) * 1e-3) / 1e9
+    line = {
+        "metric": "block swap GB/s over the host link (GPU -> pinned host and back), preempting a quarter "
+                  "of the GQA batch",
+        "value": round(step_bytes * world / (ms_per_step * 1e-3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (bit copy)", "data": "synthetic (seeded)",
+        "config": {"workload": f"gqa: {workload_description(w)}; the blocks of {len(swapped)} of its "
+                               f"{w.num_seqs} sequences ({n_host} blocks of {blk_bytes} bytes per cache) "
+                               f"swapped out to a pinned host cache and back in",
+                   "step": "pa_swap_blocks GPU -> host (the pool's swap-out plan), then host -> GPU (its "
+                           "swap-in plan), K and V caches",
+                   "l2": "no flush: each step moves more than L2 (126 MB) each way"},
+        "stage_ms": {"swap_out": round(out_ms, 5), "swap_in": round(in_ms, 5)},
+        "clocks": clocks,
+        "gpu_launches": 2 * K,
+        "roofline": {"bound": "host link", "kernel": "pa_swap_blocks (swap_blocks_kernel), both directions",
+                     "achieved": round(achieved, 2), "peak": round(peak, 2), "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_source": "measured in this run: cudaMemcpyAsync of the same bytes, contiguous, "
+                                    f"device <-> pinned host ({ce_out_ms:.3f} ms out, {ce_in_ms:.3f} ms in)",
+                     "traffic": None, "avg_launch_ms": round((out_ms + in_ms) / 2, 5),
+                     "per_direction_gbs": {"out": round(bytes_out / (out_ms * 1e-3) / 1e9, 2),
+                                           "in": round(bytes_in / (in_ms * 1e-3) / 1e9, 2),
+                                           "copy_engine_out": round(bytes_out / (ce_out_ms * 1e-3) / 1e9, 2),
+                                           "copy_engine_in": round(bytes_in / (ce_in_ms * 1e-3) / 1e9, 2)}},
+        "e2e": None,
+        "e2e_note": "the swap already runs between device and host buffers; end-to-end host-buffer timing is "
+                    "measured on the decode rows",
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_swap(w, out_pairs, n_host, max(2.0, args.cpu_budget / 2))
+    if remeasured:
+        line["clocks_note"] = "first timed region saw a thermal/hw slowdown reason; re-measured once"
+    return line
+
+
 # ---------------------------------------------------------------- the oracle
 
 def _oracle_decode_rate(w, tables, threads: int, budget_s: float):
@@ -899,6 +1036,27 @@ def cpu_baseline(w, tables, budget_s: float = 15.0) -> dict:
             "single_thread": {"value": round(bps1 / 1e9, 4), "unit": "GB/s", "cores": 1,
                               "seqs_per_s": round(sps1, 3),
                               "sample": f"{n1} sequence decodes, {el1:.1f} s, fp64, one thread"}}
+
+
+def cpu_baseline_swap(w, out_pairs, n_host: int, budget_s: float) -> dict:
+    """The oracle's block copy (as it stands) between two host arrays of the
+    workload's caches, the swap-out pairs in chunks, until budget_s seconds."""
+    import oracle
+    hk = np.zeros((n_host,) + w.key_cache.shape[1:], dtype=np.uint16)
+    hv = np.zeros_like(hk)
+    blk_bytes = w.block_size * w.num_kv_heads * w.head_dim * 2
+    done, elapsed, i = 0, 0.0, 0
+    chunk = 64
+    while elapsed < budget_s:
+        idx = (np.arange(chunk) + i) % out_pairs.shape[0]
+        t = time.perf_counter()
+        oracle.swap_blocks(hk, hv, w.key_cache, w.value_cache, out_pairs[idx])
+        elapsed += time.perf_counter() - t
+        done += chunk * blk_bytes * 2
+        i += chunk
+    return {"value": round(done / elapsed / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done // (blk_bytes * 2)} block pairs of the swap-out plan, K and V, host to host, "
+                      f"{elapsed:.1f} s, one thread"}
 
 
 def cpu_baseline_fp8(w, kc, vc, ks, vs, budget_s: float) -> dict:
@@ -1003,7 +1161,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--workload", choices=list(DECODE_ROWS) + ["gqa-fp8", "prefill", "cow"], default="gqa")
+    ap.add_argument("--workload", choices=list(DECODE_ROWS) + ["gqa-fp8", "prefill", "cow", "swap"], default="gqa")
     ap.add_argument("--partition", type=int, default=0,
                     help="decode rows: force the split form with this many positions per partition "
                          "(0 = the library's plan)")
@@ -1051,6 +1209,8 @@ def main():
             line = run_decode(args, rank, world, local_rank)
         elif args.workload == "cow":
             line = run_cow(args, rank, world, local_rank)
+        elif args.workload == "swap":
+            line = run_swap(args, rank, world, local_rank)
         else:
             line = run_row(args, rank, world, local_rank)
     finally:

@@ -96,3 +96,19 @@ def _check_reference_line(r):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     return d
+
+
+def test_swap_row_plan_moves_each_swapped_block_out_and_back():
+    from paged_kv_cache_379_b200 import workload as wlmod
+    w = wlmod.make("gqa", seed=bench.rank_seed(0, "gqa"))
+    tables, swapped, n_host, out_pairs, in_pairs = bench.swap_row_plan(w)
+    # swap-out: the swapped sequences' blocks (distinct, none shared in this
+    # batch), each to its own host block
+    want = np.concatenate([tables[s][tables[s] >= 0] for s in swapped])
+    assert sorted(out_pairs[:, 0].tolist()) == sorted(want.tolist())
+    assert len(set(out_pairs[:, 1].tolist())) == out_pairs.shape[0] == n_host
+    assert out_pairs[:, 1].min() >= 0 and out_pairs[:, 1].max() < n_host
+    # swap-in: every host block back to a distinct GPU block of the pool
+    assert sorted(in_pairs[:, 0].tolist()) == sorted(out_pairs[:, 1].tolist())
+    assert len(set(in_pairs[:, 1].tolist())) == in_pairs.shape[0]
+    assert in_pairs[:, 1].min() >= 0 and in_pairs[:, 1].max() < w.num_blocks
