@@ -1001,6 +1001,88 @@ def run_swap(args, rank: int, world: int, local_rank: int) -> dict | None:
     return line
 
 
+def prefix_row_prompts(seed: int, prompts: int = 32, samples: int = 8, prompt_len: int = 1024):
+    """The prefix-cache row's requests: `prompts` seeded prompts of random token
+    ids, each requested `samples` times in a row (parallel sampling)."""
+    rng = np.random.default_rng(seed)
+    toks = rng.integers(0, 32000, size=(prompts, prompt_len), dtype=np.int32)
+    return [toks[p] for p in range(prompts) for _ in range(samples)]
+
+
+def prefix_step(pool, requests, free_table):
+    """One step of the prefix-cache row: every request's table through the
+    pool's prefix cache, then every table freed.  Returns (blocks, cached
+    tokens)."""
+    tables, cached, blocks = [], 0, 0
+    for toks in requests:
+        t, c = pool.allocate_prompt_cached(toks)
+        tables.append(t)
+        cached += c
+        blocks += len(t)
+    for t in tables:
+        free_table(t)
+    return blocks, cached
+
+
+def run_prefix(args, rank: int, world: int, local_rank: int) -> dict | None:
+    """Prefix-hash caching in the host pool ([深度解析 «Copy-on-Write 与 Prefix
+    Caching»]): 32 prompts of 1024 tokens, each requested by 8 samples in a row;
+    every request hashes its full blocks (chained FNV-1a) and reuses the live
+    blocks of an equal prefix, then all tables are freed.  Host code only: the
+    step is timed by the host clock, and no kernel runs."""
+    from paged_kv_cache_379_b200.pool import BlockPool
+
+    if rank != 0:
+        return None
+    K, W = args.steps, args.warmup
+    bs = 16
+    requests = prefix_row_prompts(rank_seed(rank, "shared"))
+    n_tokens = sum(len(t) for t in requests)
+    num_blocks = int(1.2 * n_tokens // bs)
+    with BlockPool(num_blocks, bs) as pool:
+        for _ in range(W):
+            prefix_step(pool, requests, pool.free_table)
+        t0 = time.perf_counter()
+        for _ in range(K):
+            blocks, cached = prefix_step(pool, requests, pool.free_table)
+        el = time.perf_counter() - t0
+    ms_per_step = el / K * 1e3
+    line = {
+        "metric": "prefix-cached prompt allocations per second (host block pool)",
+        "value": round(len(requests) * K / el, 1), "unit": "prompts/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int32 token ids, uint64 hashes", "data": "synthetic (seeded token ids)",
+        "config": {"workload": f"prefix: {len(requests) // 8} prompts of 1024 tokens x 8 samples in a row, "
+                               f"block_size {bs}, pool of {num_blocks} blocks",
+                   "step": "pa_pool_allocate_prompt_cached for every request, then pa_pool_free_table for "
+                           "every table"},
+        "tokens_hashed_per_s": round(n_tokens * K / el, 1),
+        "blocks_per_step": blocks,
+        "hit_rate": round(cached / n_tokens, 4),
+        "gpu_launches": 0,
+        "gpu_note": "host code: the pool is the C++ library's, called through its C ABI; no kernel runs",
+        "roofline": None,
+        "e2e": None,
+    }
+    if not args.no_cpu_baseline:
+        from oracle.pool import OraclePool
+        opool = OraclePool(num_blocks, bs)
+
+        def ofree(t):
+            for b in t:
+                opool.free(b)
+        sub = requests[:64]                    # 8 prompts x 8 samples
+        n, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < max(2.0, args.cpu_budget / 2):
+            prefix_step(opool, sub, ofree)
+            n += len(sub)
+        el_o = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": round(n / el_o, 1), "unit": "prompts/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} requests (8 of the prompts x 8 samples, repeated), {el_o:.1f} s, "
+                                          "pure Python, one thread"}
+    return line
+
+
 # ---------------------------------------------------------------- the oracle
 
 def _oracle_decode_rate(w, tables, threads: int, budget_s: float):
@@ -1161,7 +1243,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--workload", choices=list(DECODE_ROWS) + ["gqa-fp8", "prefill", "cow", "swap"], default="gqa")
+    ap.add_argument("--workload", choices=list(DECODE_ROWS) + ["gqa-fp8", "prefill", "cow", "swap", "prefix"],
+                    default="gqa")
     ap.add_argument("--partition", type=int, default=0,
                     help="decode rows: force the split form with this many positions per partition "
                          "(0 = the library's plan)")
@@ -1211,6 +1294,8 @@ def main():
             line = run_cow(args, rank, world, local_rank)
         elif args.workload == "swap":
             line = run_swap(args, rank, world, local_rank)
+        elif args.workload == "prefix":
+            line = run_prefix(args, rank, world, local_rank)
         else:
             line = run_row(args, rank, world, local_rank)
     finally:

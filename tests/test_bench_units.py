@@ -112,3 +112,20 @@ def test_swap_row_plan_moves_each_swapped_block_out_and_back():
     assert sorted(in_pairs[:, 0].tolist()) == sorted(out_pairs[:, 1].tolist())
     assert len(set(in_pairs[:, 1].tolist())) == in_pairs.shape[0]
     assert in_pairs[:, 1].min() >= 0 and in_pairs[:, 1].max() < w.num_blocks
+
+
+def test_prefix_row_reuses_the_full_blocks_of_every_later_sample():
+    from oracle.pool import OraclePool
+    from paged_kv_cache_379_b200.pool import BlockPool
+    # 3 prompts of 100 tokens (6 full blocks of 16 + 1 partial), 4 samples each
+    reqs = bench.prefix_row_prompts(5, prompts=3, samples=4, prompt_len=100)
+    with BlockPool(64, 16) as pool:
+        first = bench.prefix_step(pool, reqs, pool.free_table)
+        again = bench.prefix_step(pool, reqs, pool.free_table)   # everything was freed: the same again
+        assert pool.get_num_free_blocks() == 64
+    op = OraclePool(64, 16)
+
+    def ofree(t):
+        for b in t:
+            op.free(b)
+    assert first == again == bench.prefix_step(op, reqs, ofree) == (3 * 4 * 7, 3 * 3 * 6 * 16)
