@@ -9,7 +9,7 @@ lengths lognormal (median 1024, sigma 0.8) clipped to [16, 4096], shuffled
 block pool 1.2x.  Inputs are seeded synthetic data already resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload tiny|mha|gqa|long|shared|gqa-fp8|prefill|cow]
+                    [--workload tiny|mha|gqa|long|shared|gqa-fp8|prefill|cow|swap|prefix]
                     [--partition P] [--l2-flush]
 
 The default workload is the line above.  The other decode workloads run the
@@ -18,12 +18,15 @@ heads), `long` (8 sequences of 32K..128K positions; --partition 512 is the
 workload's stated split), `shared` (256 sequences forked from 32 shared
 1024-token prompts: the step starts with the copy-on-write block copies; its
 roofline counts every shared block once).  --l2-flush empties L2 before every
-step.  Three more rows of the path: `gqa-fp8` (the gqa batch with an FP8 E4M3
+step.  More rows of the path: `gqa-fp8` (the gqa batch with an FP8 E4M3
 cache: slot mapping + quantising cache write -> decode over codes; KV GB/s of
 1-byte elements), `prefill` (8 x 2048-token prompts with the gqa heads: slot
 mapping -> cache write of the prompts' K/V -> causal paged prefill on the
-tensor cores; useful TFLOP/s) and `cow` (the shared step's block copies
-alone).
+tensor cores; useful TFLOP/s), `cow` (the shared step's block copies alone),
+`swap` (a quarter of the gqa batch's blocks swapped out to pinned host memory
+and back through the host pool's plans; GB/s over the host link against the
+copy engines' rate for the same bytes) and `prefix` (host only: 32 prompts x
+8 samples through the pool's prefix cache; prompts/s).
 
 Prints ONE JSON line (rank 0).  `value` = KV GB/s: the decode's algorithmic
 bytes per step (KV blocks touched + queries + block tables + outputs) over the
