@@ -60,3 +60,35 @@ def test_swap_rejects_pageable_host_memory():
     assert rc == -11
     with pytest.raises(ValueError):
         ops.swap_blocks(host_k, host_v, dev_k, dev_v, pairs)
+
+
+def test_swap_bench_plan_round_trip_full_size():
+    """The bench's swap row at full size: a quarter of the GQA batch's blocks
+    out to pinned host memory and back into the GPU pool through the host
+    pool's plans, compared bit for bit with the oracle's copies applied to host
+    copies of the same caches (the host cache and the whole GPU cache after
+    each direction)."""
+    import bench
+    from paged_kv_cache_379_b200 import workload as wlmod
+    w = wlmod.make("gqa", seed=bench.rank_seed(0, "gqa"))
+    tables, swapped, n_host, out_pairs, in_pairs = bench.swap_row_plan(w)
+    gk, gv = w.key_cache.copy(), w.value_cache.copy()
+    dev_k, dev_v = _bf16(gk, "cuda"), _bf16(gv, "cuda")
+    hk = np.zeros((n_host,) + gk.shape[1:], np.uint16)
+    hv = np.zeros_like(hk)
+    host_k, host_v = _bf16(hk, pin=True), _bf16(hv, pin=True)
+    ops.swap_blocks(host_k, host_v, dev_k, dev_v, torch.from_numpy(out_pairs).cuda())
+    torch.cuda.synchronize()
+    oracle.swap_blocks(hk, hv, gk, gv, out_pairs)
+    assert np.array_equal(_bits(host_k), hk) and np.array_equal(_bits(host_v), hv)
+    ops.swap_blocks(dev_k, dev_v, host_k, host_v, torch.from_numpy(in_pairs).cuda())
+    torch.cuda.synchronize()
+    oracle.swap_blocks(gk, gv, hk, hv, in_pairs)
+    assert np.array_equal(_bits(dev_k), gk) and np.array_equal(_bits(dev_v), gv)
+    # every swapped sequence's blocks hold their content again, at the blocks
+    # the swap-in chose
+    moved = dict(zip(out_pairs[:, 0].tolist(), out_pairs[:, 1].tolist()))
+    back = dict(zip(in_pairs[:, 0].tolist(), in_pairs[:, 1].tolist()))
+    for s in swapped[:4]:
+        for b in tables[s][tables[s] >= 0]:
+            assert np.array_equal(gk[back[moved[int(b)]]], w.key_cache[b])
