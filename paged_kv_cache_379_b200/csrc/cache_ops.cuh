@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(256) append_kv_cow_kernel(
 }
 
 // One CTA per (pair, slice): copies `per_cta` 16-byte chunks of the source block
-// into the destination block, in both caches, with 4 loads in flight per thread.
+// into the destination block, in both caches, with 16 loads in flight per thread.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ key_cache,
                                                           uint4 *__restrict__ value_cache,
                                                           const int64_t *__restrict__ pairs,
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ ke
     const uint4 *vs = value_cache + src * chunks_per_block;
     uint4 *kd = key_cache + dst * chunks_per_block;
     uint4 *vd = value_cache + dst * chunks_per_block;
-    constexpr int U = 2;
+    constexpr int U = 8;
     int64_t c = begin + threadIdx.x;
     for (; c + (U - 1) * blockDim.x < end; c += U * blockDim.x) {
         uint4 k[U], v[U];
